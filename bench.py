@@ -1,0 +1,408 @@
+"""Benchmark of the RG-LRU block core on B200: prefill tokens/s and HBM GB/s
+against the measured roofline, plus batched decode tokens/s at B=256.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one rglru_prefill call over the whole workload (default: the
+2B-shaped block, B=8 T=4096 D=2560 bf16), inputs resident in HBM.  Inputs and
+outputs (x, g, y: 168 MB each) are larger than the 126 MB L2, so no flush is
+needed between steps.  With N>1 (torchrun, one rank per GPU) every rank runs
+the same workload on its own GPU with no data-path collective (weak scaling);
+the timed region is bracketed by a barrier and a device synchronize, and the
+time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from lm_causal_depthwise_b200 import workloads as W  # noqa: E402
+
+METRIC = "RG-LRU block prefill tokens/s & HBM GB/s vs peak; decode tok/s at B=256"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def _env_rank():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lm_causal_depthwise_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".h", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    only if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("source_digest") != source_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        self.max_mhz = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def cpu_sample_run(w: W.Workload, budget_s: float = 12.0):
+    """Times the float64 oracle (as it stands) on a bounded sample of workload
+    ``w``: whole sequences of the first rows, all heads.  Returns tokens/s,
+    threads used and a description of the sample."""
+    from oracle import oracle
+    inp = W.generate(w.scaled(B=1))
+    t0 = time.perf_counter()
+    oracle.prefill(**inp)
+    one = time.perf_counter() - t0
+    rows = int(max(1, min(w.B, budget_s // max(one, 1e-3))))
+    if rows > 1:
+        inp = W.generate(w.scaled(B=rows))
+        t0 = time.perf_counter()
+        oracle.prefill(**inp)
+        dt = time.perf_counter() - t0
+    else:
+        dt = one
+    tokens = rows * w.T
+    return tokens / dt, oracle.threads(), f"{rows} of {w.B} sequences x T={w.T} x D={w.D} " \
+                                          f"(all heads), float64 C oracle, {dt:.1f} s"
+
+
+def run_reference(args, w):
+    rank, world, _ = _env_rank()
+    if rank != 0:
+        return 0
+    from oracle import oracle
+    inp = W.generate(w.scaled(B=1))
+    cores = oracle.threads()
+    for _ in range(max(args.warmup, 0)):
+        oracle.prefill(**inp)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.prefill(**inp)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = args.steps * w.T / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.describe(), "sample": "1 sequence per step (all heads, full T)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"1 of {w.B} sequences x T={w.T} x D={w.D} per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- CUDA arm
+
+def count_launches(fn, prefix=("rglru",)):
+    """Kernels of this library launched by one call of ``fn`` (CUPTI via torch.profiler)."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = []
+    for e in prof.events():
+        if e.device_type is not None and str(e.device_type).endswith("CUDA"):
+            if any(p in e.name for p in prefix):
+                names.append(e.name)
+    return len(names), sorted(set(names))
+
+
+def run_cuda(args, w):
+    import torch
+    import torch.distributed as dist
+    from lm_causal_depthwise_b200 import api
+
+    rank, world, local = _env_rank()
+    distributed = world > 1
+    if distributed:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    api.load()
+
+    bf = torch.bfloat16 if w.io == "bf16" else torch.float32
+    inp = W.generate(w)
+    x = torch.from_numpy(inp["x"]).to(dev).to(bf)
+    g = torch.from_numpy(inp["g"]).to(dev).to(bf)
+    sp = torch.from_numpy(inp["segpos"]).to(dev)
+    cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
+    hs = torch.from_numpy(inp["h_state"]).to(dev)
+    p = api.Params.from_arrays(inp, bf, dev)
+    y = torch.empty_like(x)
+    ws = api.new_workspace(api.workspace_size(w.B, w.T, w.D, bf), dev)
+
+    def step():
+        api.prefill(x, g, p, sp, cs, hs, workspace=ws, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step, kernel_names = count_launches(step)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if distributed:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if distributed:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if distributed:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    per_step_ms = ms_max / args.steps
+    tokens = w.tokens * world
+    value = tokens / (per_step_ms * 1e-3)
+
+    # ---- end to end through the public API: pinned host inputs in, y back to host
+    hx = torch.from_numpy(inp["x"]).to(bf).pin_memory()
+    hg = torch.from_numpy(inp["g"]).to(bf).pin_memory()
+    hsp = torch.from_numpy(inp["segpos"]).pin_memory()
+    hy = torch.empty(tuple(y.shape), dtype=bf).pin_memory()
+    e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        x.copy_(hx, non_blocking=True)
+        g.copy_(hg, non_blocking=True)
+        sp.copy_(hsp, non_blocking=True)
+        api.prefill(x, g, p, sp, cs, hs, workspace=ws, y=y)
+        hy.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if distributed:
+        dist.barrier()
+    ev0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = torch.tensor([ev0.elapsed_time(ev1)], device=dev, dtype=torch.float64)
+    if distributed:
+        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e_value = tokens / (float(e_ms.item()) / e_steps * 1e-3)
+    h2d = hx.numel() * hx.element_size() + hg.numel() * hg.element_size() + hsp.numel() * 4
+    d2h = hy.numel() * hy.element_size()
+
+    # ---- batched decode at B=256 (a separate timed loop of single-token steps)
+    dec = None
+    if not args.no_decode:
+        dec = run_decode(args, dev, stream, distributed)
+
+    del hx, hg, hy, hsp
+    if distributed:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = measured_peaks()
+    alg_bytes = W.algorithmic_bytes(w)
+    achieved = alg_bytes / (per_step_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.io == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.describe(), "B": w.B, "T": w.T, "D": w.D,
+                   "tokens_per_gpu": w.tokens, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "no flush: x, g, y are each larger than L2 (126 MB)"},
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "peak_source": f"{peak_kind} copy bandwidth",
+                     "frac_of_nominal_8tbs": achieved / 8000.0,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "kernel": kernel_names},
+        "e2e": {"value": e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "source_digest": source_digest(),
+    }
+    if dec is not None:
+        line["decode"] = dec
+    if world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_sample_run(w)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args, dev, stream, distributed):
+    import torch
+    import torch.distributed as dist
+    from lm_causal_depthwise_b200 import api
+
+    w = W.DECODE_2B
+    steps = args.decode_steps or w.decode_steps
+    inp = W.generate(w.scaled(T=steps))
+    bf = torch.bfloat16
+    xs = torch.from_numpy(inp["x"]).to(dev).to(bf).transpose(0, 1).contiguous()
+    gs = torch.from_numpy(inp["g"]).to(dev).to(bf).transpose(0, 1).contiguous()
+    ss = torch.from_numpy(inp["segpos"]).to(dev).t().contiguous()
+    cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
+    hs = torch.from_numpy(inp["h_state"]).to(dev)
+    p = api.Params.from_arrays(inp, bf, dev)
+    ys = torch.empty_like(xs)
+    ws = api.new_workspace(api.decode_workspace_size(w.B, w.D, bf), dev)
+
+    def loop():
+        for t in range(steps):
+            api.decode_step(xs[t], gs[t], p, ss[t], cs, hs, workspace=ws, y=ys[t])
+
+    loop()
+    torch.cuda.synchronize()
+    n_launch, names = count_launches(lambda: api.decode_step(xs[0], gs[0], p, ss[0], cs, hs,
+                                                             workspace=ws, y=ys[0]))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if distributed:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    loop()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = torch.tensor([ev0.elapsed_time(ev1)], device=dev, dtype=torch.float64)
+    if distributed:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms = float(ms.item())
+    world = dist.get_world_size() if distributed else 1
+    per_step_us = 1e3 * ms / steps
+    step_bytes = W.decode_step_bytes(w)
+    return {"workload": w.scaled(T=steps).describe(), "value": world * w.B * steps / (ms * 1e-3),
+            "unit": "tokens/s", "us_per_step": per_step_us, "steps": steps,
+            "algorithmic_gbs": step_bytes / (per_step_us * 1e-6) / 1e9,
+            "algorithmic_bytes_per_step": step_bytes, "gpu_launches": n_launch * steps,
+            "kernel": names}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=W.PREFILL_2B.name, choices=sorted(W.ALL))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=0)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "cuda":
+        args.warmup = 3
+    w = W.ALL[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_cuda(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,174 @@
+/*
+ * rglru.h -- C ABI of the B200 RG-LRU recurrent-block core (librglru.so).
+ *
+ * One call computes the core of a RecurrentGemma recurrent temporal block,
+ * from the input of the causal depthwise conv to the product with the GELU
+ * branch.  Structure: "Gemma explained: RecurrentGemma architecture"
+ * (gemma.gh.miniasp.com), the RecurrentGemmaRecurrentBlock module printout
+ * (Conv1d(D, D, kernel_size=4, padding=3, groups=D), RecurrentGemmaRglru,
+ * PytorchGELUTanh) and the section "Residual block with recurrent block"
+ * (conv then RG-LRU on one branch, GELU on the other, elementwise product).
+ * The RG-LRU equations are those of Griffin / RecurrentGemma
+ * ("RecurrentGemma: Moving Past Transformers for Efficient Open Language
+ * Models", arXiv 2404.07839), which the pages name but do not print:
+ *
+ *   xc_t = conv_b + sum_{k=0..3} conv_w[k] * x_{t-3+k} * [3-k <= segpos_t]
+ *   r_t  = sigmoid(W_a[h] xc_t + b_a),   i_t = sigmoid(W_x[h] xc_t + b_x)
+ *   a_t  = sigmoid(Lambda)^(8 r_t)
+ *   h_t  = a_t h_{t-1} + sqrt(1 - a_t^2) (i_t xc_t)      (segpos_t > 0)
+ *   h_t  = i_t xc_t                                      (segpos_t == 0)
+ *   y_t  = GELU_tanh(g_t) h_t
+ *
+ * Conventions for every call below
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd, or managed),
+ *     owned by the caller, 16-byte aligned.  The library allocates nothing,
+ *     keeps no global state and never synchronises the stream (except
+ *     rglru_get_device_status).  Work is enqueued on `stream`.
+ *   - Layouts are row-major with the channel index fastest:
+ *       x, gate_branch, y     [B, T, D]  io dtype
+ *       conv_w [4, D] fp32    tap k multiplies the input 3-k steps back
+ *       conv_b, b_a, b_x, lambda [D] fp32
+ *       W_a, W_x [H, 256, 256] with H = D/256, index [head][out][in];
+ *                 bf16 in RGLRU_IO_BF16 mode, fp32 in RGLRU_IO_F32 mode
+ *       segment_pos [B, T] int32: position inside the current document;
+ *                 0 marks a document start (resets h, masks conv taps);
+ *                 values < 0 are not allowed; >= 3 means all taps valid
+ *       conv_state [B, 3, D] io dtype, the last three raw inputs, oldest
+ *                 first; read and overwritten in place
+ *       h_state   [B, D] fp32; read and overwritten in place
+ *   - D must be a multiple of 256 (heads of 256 channels).
+ *   - y must not overlap any input.  The states are updated in place.
+ *   - Argument errors are reported synchronously, before anything is
+ *     enqueued.  A failed launch returns RGLRU_ERR_CUDA.  A device-side
+ *     bounded wait that gave up is recorded in the workspace and read back
+ *     by rglru_get_device_status.
+ *   - The workspace is caller-owned device memory of at least the size the
+ *     matching *_workspace_size call returns, zero-filled once before its
+ *     first use (the calls leave it valid for the next one).  It may be
+ *     reused across calls on the same stream but not shared by calls that
+ *     can overlap on the GPU.
+ */
+#ifndef RGLRU_H
+#define RGLRU_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define RGLRU_API __attribute__((visibility("default")))
+#else
+#define RGLRU_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RGLRU_OK = 0,
+    RGLRU_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, overlap */
+    RGLRU_ERR_UNSUPPORTED = 2,  /* shape or dtype this build does not handle */
+    RGLRU_ERR_WORKSPACE = 3,    /* workspace missing or too small */
+    RGLRU_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    RGLRU_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
+} rglru_status;
+
+typedef enum {
+    RGLRU_IO_F32 = 0,   /* x, gate_branch, y, conv_state, W_a, W_x in fp32 */
+    RGLRU_IO_BF16 = 1   /* the same tensors in bf16 (the state h stays fp32) */
+} rglru_io_dtype;
+
+/* Library ABI version (major * 100 + minor). */
+RGLRU_API int rglru_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+RGLRU_API const char *rglru_status_string(rglru_status status);
+
+/*
+ * Workspace bytes rglru_prefill needs for these sizes (0 on bad sizes).
+ * Holds the device status word and the cross-chunk scan carry (per chunk,
+ * flags and (prod a, h) aggregates).
+ */
+RGLRU_API size_t rglru_workspace_size(int B, int T, int D, rglru_io_dtype dt);
+
+/*
+ * Prefill: runs the block core over T tokens of B sequences.
+ * bf16 mode runs one fused kernel (conv, tensor-core gate projections,
+ * chunked fp32 scan with a cross-chunk carry, GELU product); fp32 mode runs
+ * the plain SIMT kernels of rglru_prefill_simt.
+ * Outputs: y [B,T,D]; conv_state and h_state updated to their values after
+ * token T-1.
+ */
+RGLRU_API rglru_status rglru_prefill(int B, int T, int D, rglru_io_dtype dt,
+                           const void *x, const void *gate_branch,
+                           const float *conv_w, const float *conv_b,
+                           const void *W_a, const float *b_a,
+                           const void *W_x, const float *b_x,
+                           const float *lambda, const int32_t *segment_pos,
+                           void *conv_state, float *h_state, void *y,
+                           void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/*
+ * Workspace bytes rglru_prefill_simt needs (0 on bad sizes): the device
+ * status word plus three fp32 [B,T,D] intermediates (conv output and the
+ * two gate pre-activations).
+ */
+RGLRU_API size_t rglru_simt_workspace_size(int B, int T, int D, rglru_io_dtype dt);
+
+/*
+ * The same computation as rglru_prefill on plain SIMT kernels (CUDA cores
+ * only, fp32 arithmetic with accurate transcendentals), in either dtype.
+ * It is the fp32-mode path and an independent second implementation for
+ * cross-checks.  Same arguments and semantics as rglru_prefill.
+ */
+RGLRU_API rglru_status rglru_prefill_simt(int B, int T, int D, rglru_io_dtype dt,
+                                const void *x, const void *gate_branch,
+                                const float *conv_w, const float *conv_b,
+                                const void *W_a, const float *b_a,
+                                const void *W_x, const float *b_x,
+                                const float *lambda, const int32_t *segment_pos,
+                                void *conv_state, float *h_state, void *y,
+                                void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
+/* Workspace bytes rglru_decode_step needs for B sequences of width D. */
+RGLRU_API size_t rglru_decode_workspace_size(int B, int D, rglru_io_dtype dt);
+
+/*
+ * Decode: one token for each of B sequences (the prefill recurrence with
+ * T = 1).  x, gate_branch, y are [B, D]; segment_pos is [B]; conv_state and
+ * h_state are updated in place.  Other arguments as rglru_prefill.
+ */
+RGLRU_API rglru_status rglru_decode_step(int B, int D, rglru_io_dtype dt,
+                               const void *x, const void *gate_branch,
+                               const float *conv_w, const float *conv_b,
+                               const void *W_a, const float *b_a,
+                               const void *W_x, const float *b_x,
+                               const float *lambda, const int32_t *segment_pos,
+                               void *conv_state, float *h_state, void *y,
+                               void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, returns the device status recorded in `workspace`
+ * by the calls enqueued so far (RGLRU_OK or RGLRU_ERR_TIMEOUT) and clears it.
+ * RGLRU_ERR_CUDA if the synchronisation or the read fails.
+ */
+RGLRU_API rglru_status rglru_get_device_status(void *workspace, cudaStream_t stream);
+
+/*
+ * Test hook for the bounded waits (never used by a normal call): makes chunk
+ * `unit` of the next rglru_prefill calls on this workspace skip publishing
+ * its scan carry, so that its successor's wait runs out and records
+ * RGLRU_ERR_TIMEOUT instead of hanging.  unit = -1 turns it off.  The flag
+ * lives in the workspace header and is enqueued on `stream`.
+ */
+RGLRU_API rglru_status rglru_debug_suppress_publish(void *workspace, int unit, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RGLRU_H */

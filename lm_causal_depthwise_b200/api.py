@@ -1,0 +1,224 @@
+"""Python binding of librglru (include/rglru.h): argument marshalling only.
+
+Every step of the block core runs in the CUDA library; this module checks
+tensor dtypes, shapes, devices and contiguity, passes raw pointers and the
+current CUDA stream through ctypes, and turns a non-OK status into an
+exception.  PyTorch provides device memory and streams, nothing else.  If
+the library is missing or cannot be loaded, every call raises: there is no
+fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librglru.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+IO_F32, IO_BF16 = 0, 1
+
+SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglru_prefill",
+           "rglru_simt_workspace_size", "rglru_prefill_simt", "rglru_decode_workspace_size",
+           "rglru_decode_step", "rglru_get_device_status", "rglru_debug_suppress_publish")
+
+_lib = None
+
+
+class RGLRUError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load librglru.so (built in-tree by lm_causal_depthwise_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing; build it with "
+                           "`python -m lm_causal_depthwise_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    prefill_args = [i, i, i, i] + [vp] * 14 + [sz, vp]
+    decode_args = [i, i, i] + [vp] * 14 + [sz, vp]
+    lib.rglru_version.restype = i
+    lib.rglru_version.argtypes = []
+    lib.rglru_status_string.restype = ctypes.c_char_p
+    lib.rglru_status_string.argtypes = [i]
+    for n in ("rglru_workspace_size", "rglru_simt_workspace_size"):
+        getattr(lib, n).restype = sz
+        getattr(lib, n).argtypes = [i, i, i, i]
+    lib.rglru_decode_workspace_size.restype = sz
+    lib.rglru_decode_workspace_size.argtypes = [i, i, i]
+    for n in ("rglru_prefill", "rglru_prefill_simt"):
+        getattr(lib, n).restype = i
+        getattr(lib, n).argtypes = prefill_args
+    lib.rglru_decode_step.restype = i
+    lib.rglru_decode_step.argtypes = decode_args
+    lib.rglru_get_device_status.restype = i
+    lib.rglru_get_device_status.argtypes = [vp, vp]
+    lib.rglru_debug_suppress_publish.restype = i
+    lib.rglru_debug_suppress_publish.argtypes = [vp, i, vp]
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().rglru_status_string(int(status)).decode()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return IO_BF16
+    if t.dtype == torch.float32:
+        return IO_F32
+    raise TypeError(f"io tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+@dataclass
+class Params:
+    """Block parameters on the device.  conv_w [4,D], conv_b/b_a/b_x/lam [D]
+    are fp32; W_a, W_x [H,256,256] are in the io dtype."""
+    conv_w: torch.Tensor
+    conv_b: torch.Tensor
+    W_a: torch.Tensor
+    b_a: torch.Tensor
+    W_x: torch.Tensor
+    b_x: torch.Tensor
+    lam: torch.Tensor
+
+    @staticmethod
+    def from_arrays(inp: dict, io_dtype: torch.dtype, device="cuda") -> "Params":
+        def f32(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).contiguous()
+
+        def io(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).to(io_dtype).contiguous()
+        return Params(f32(inp["conv_w"]), f32(inp["conv_b"]), io(inp["W_a"]), f32(inp["b_a"]),
+                      io(inp["W_x"]), f32(inp["b_x"]), f32(inp["lam"]))
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def workspace_size(B: int, T: int, D: int, io_dtype: torch.dtype, simt: bool = False) -> int:
+    dt = IO_BF16 if io_dtype == torch.bfloat16 else IO_F32
+    fn = load().rglru_simt_workspace_size if simt else load().rglru_workspace_size
+    n = int(fn(B, T, D, dt))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "workspace_size")
+    return n
+
+
+def decode_workspace_size(B: int, D: int, io_dtype: torch.dtype) -> int:
+    dt = IO_BF16 if io_dtype == torch.bfloat16 else IO_F32
+    n = int(load().rglru_decode_workspace_size(B, D, dt))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "decode_workspace_size")
+    return n
+
+
+def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled device workspace (the valid initial state)."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def _common(x, g, p: Params, segpos, conv_state, h_state, y, lead):
+    dev = x.device
+    dt = _dt(x)
+    D = x.shape[-1]
+    H = D // 256
+    _check(g, "gate_branch", x.shape, x.dtype, dev)
+    _check(x, "x", x.shape, x.dtype, dev)
+    _check(p.conv_w, "conv_w", (4, D), torch.float32, dev)
+    for n in ("conv_b", "b_a", "b_x", "lam"):
+        _check(getattr(p, n), n, (D,), torch.float32, dev)
+    _check(p.W_a, "W_a", (H, 256, 256), x.dtype, dev)
+    _check(p.W_x, "W_x", (H, 256, 256), x.dtype, dev)
+    _check(segpos, "segment_pos", lead, torch.int32, dev)
+    B = x.shape[0]
+    _check(conv_state, "conv_state", (B, 3, D), x.dtype, dev)
+    _check(h_state, "h_state", (B, D), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", x.shape, x.dtype, dev)
+    return dt, y
+
+
+def prefill(x, gate_branch, p: Params, segment_pos, conv_state, h_state, workspace=None,
+            y=None, simt: bool = False) -> torch.Tensor:
+    """y = block core over x, gate_branch [B,T,D]; conv_state [B,3,D] and
+    h_state [B,D] are updated in place.  Enqueued on the current stream."""
+    if x.dim() != 3:
+        raise ValueError("x must be [B,T,D]")
+    B, T, D = x.shape
+    dt, y = _common(x, gate_branch, p, segment_pos, conv_state, h_state, y, (B, T))
+    need = workspace_size(B, T, D, x.dtype, simt=simt)
+    if workspace is None:
+        workspace = new_workspace(need, x.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise RGLRUError(ERR_WORKSPACE, "prefill")
+    fn = load().rglru_prefill_simt if simt else load().rglru_prefill
+    st = fn(B, T, D, dt, _ptr(x), _ptr(gate_branch), _ptr(p.conv_w), _ptr(p.conv_b), _ptr(p.W_a),
+            _ptr(p.b_a), _ptr(p.W_x), _ptr(p.b_x), _ptr(p.lam), _ptr(segment_pos),
+            _ptr(conv_state), _ptr(h_state), _ptr(y), _ptr(workspace),
+            ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(x.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_prefill_simt" if simt else "rglru_prefill")
+    return y
+
+
+def decode_step(x, gate_branch, p: Params, segment_pos, conv_state, h_state, workspace=None,
+                y=None) -> torch.Tensor:
+    """One token per sequence: x, gate_branch [B,D]; segment_pos [B]."""
+    if x.dim() != 2:
+        raise ValueError("x must be [B,D]")
+    B, D = x.shape
+    dt, y = _common(x, gate_branch, p, segment_pos, conv_state, h_state, y, (B,))
+    need = decode_workspace_size(B, D, x.dtype)
+    if workspace is None:
+        workspace = new_workspace(need, x.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise RGLRUError(ERR_WORKSPACE, "decode_step")
+    st = load().rglru_decode_step(
+        B, D, dt, _ptr(x), _ptr(gate_branch), _ptr(p.conv_w), _ptr(p.conv_b), _ptr(p.W_a),
+        _ptr(p.b_a), _ptr(p.W_x), _ptr(p.b_x), _ptr(p.lam), _ptr(segment_pos), _ptr(conv_state),
+        _ptr(h_state), _ptr(y), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(x.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_decode_step")
+    return y
+
+
+def device_status(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream and read (and clear) the device status word."""
+    return int(load().rglru_get_device_status(_ptr(workspace), _stream(workspace.device)))
+
+
+def debug_suppress_publish(workspace: torch.Tensor, unit: int) -> None:
+    st = load().rglru_debug_suppress_publish(_ptr(workspace), int(unit), _stream(workspace.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_debug_suppress_publish")

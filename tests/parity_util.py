@@ -1,0 +1,96 @@
+"""Helpers shared by the GPU parity tests: upload seeded inputs, run the CUDA
+library, run the oracle on the same arrays, compare with the stated bars.
+
+Tolerances (fixed here, used by every parity test):
+  fp32 I/O : max_e |got - ref| / max(|ref_e|, 1e-3 * rms(ref)) <= 1e-5
+  bf16 I/O : every element |got - ref| <= 2e-2 + 1e-2 * |ref|
+             (atol 2e-2, rtol 1e-2; bf16 output rounding alone is 2^-9 relative)
+  integer / copied state (conv_state): bit-exact.
+"""
+from __future__ import annotations
+
+import concurrent.futures as cf
+
+import numpy as np
+import torch
+
+from oracle import oracle
+from lm_causal_depthwise_b200 import api
+
+F32_RTOL = 1e-5
+BF16_ATOL = 2e-2
+BF16_RTOL = 1e-2
+
+
+def io_dtype(io: str) -> torch.dtype:
+    return torch.bfloat16 if io == "bf16" else torch.float32
+
+
+def to_device(inp: dict, io: str, device="cuda") -> dict:
+    dt = io_dtype(io)
+    d = {
+        "x": torch.from_numpy(inp["x"]).to(device).to(dt).contiguous(),
+        "g": torch.from_numpy(inp["g"]).to(device).to(dt).contiguous(),
+        "segpos": torch.from_numpy(inp["segpos"]).to(device).contiguous(),
+        "conv_state": torch.from_numpy(inp["conv_state"]).to(device).to(dt).contiguous(),
+        "h_state": torch.from_numpy(inp["h_state"]).to(device).contiguous(),
+        "params": api.Params.from_arrays(inp, dt, device),
+    }
+    return d
+
+
+def run_gpu(dev: dict, simt: bool = False, workspace=None):
+    y = api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"],
+                    dev["h_state"], workspace=workspace, simt=simt)
+    torch.cuda.synchronize()
+    return {"y": y.float().cpu().numpy(), "conv_state": dev["conv_state"].float().cpu().numpy(),
+            "h_state": dev["h_state"].cpu().numpy()}
+
+
+def run_oracle(inp: dict, nthreads: int = 0):
+    return oracle.prefill(**inp, nthreads=nthreads)
+
+
+def oracle_units(inp: dict, units, t_end=None):
+    """Oracle outputs of several (b, head) units, run concurrently (the C
+    oracle releases the GIL)."""
+    with cf.ThreadPoolExecutor(max_workers=min(len(units), 16)) as ex:
+        futs = {u: ex.submit(oracle.prefill_unit, inp, u[0], u[1], t_end, 8.0, 1) for u in units}
+        return {u: f.result() for u, f in futs.items()}
+
+
+def check_f32(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
+    den = np.maximum(np.abs(ref), 1e-3 * rms + 1e-300)
+    err = np.max(np.abs(got - ref) / den) if ref.size else 0.0
+    assert err <= F32_RTOL, f"{what}: max scaled error {err:.3e} > {F32_RTOL}"
+    return err
+
+
+def check_bf16(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = np.abs(got - ref)
+    bad = diff > BF16_ATOL + BF16_RTOL * np.abs(ref)
+    if bad.any():
+        idx = np.argwhere(bad)[0]
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} elements outside atol {BF16_ATOL} + rtol "
+            f"{BF16_RTOL}; first at {tuple(idx)}: got {got[tuple(idx)]!r} ref {ref[tuple(idx)]!r}; "
+            f"max abs {diff.max():.3e}")
+    big = np.abs(ref) >= 1.0
+    max_rel = float((diff[big] / np.abs(ref[big])).max()) if big.any() else 0.0
+    return float(diff.max()), max_rel
+
+
+def check(io: str, got, ref, what=""):
+    return check_bf16(got, ref, what) if io == "bf16" else check_f32(got, ref, what)
+
+
+def check_state(io: str, got: dict, ref: dict, what=""):
+    check(io, got["h_state"], ref["h_state"], f"{what} h_state")
+    np.testing.assert_array_equal(np.asarray(got["conv_state"], np.float64),
+                                  np.asarray(ref["conv_state"], np.float64),
+                                  err_msg=f"{what} conv_state")

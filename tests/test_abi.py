@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every symbol include/rglru.h declares, and
+rejects bad arguments synchronously.  No call here reaches a kernel launch:
+every case fails validation first (on a host without a GPU a launch could
+only fail with 'no device', never touch memory)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lm_causal_depthwise_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rglru.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RGLRU_API\s+[\w\s\*]+?\b(rglru_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert sorted(api.SYMBOLS) == declared_symbols()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.rglru_version() == 100
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert api.status_string(s)
+    assert api.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("B,T,D", [(0, 4, 256), (1, 0, 256), (1, 4, 255), (1, 4, 384), (1, 4, 0),
+                                   (70000, 1, 256)])
+def test_workspace_size_rejects_bad_sizes(lib, B, T, D):
+    for dt in (api.IO_F32, api.IO_BF16):
+        assert lib.rglru_workspace_size(B, T, D, dt) == 0
+        assert lib.rglru_simt_workspace_size(B, T, D, dt) == 0
+    assert lib.rglru_workspace_size(1, 4, 256, 7) == 0
+
+
+def test_workspace_size_positive(lib):
+    for dt in (api.IO_F32, api.IO_BF16):
+        assert lib.rglru_workspace_size(8, 4096, 2560, dt) >= 4096
+        assert lib.rglru_decode_workspace_size(256, 2560, dt) >= 4096
+    # the SIMT path keeps three fp32 [B,T,D] intermediates
+    assert lib.rglru_simt_workspace_size(2, 8, 256, api.IO_BF16) >= 3 * 2 * 8 * 256 * 4
+
+
+def _call(lib, fn="rglru_prefill", B=1, T=4, D=256, dt=api.IO_BF16, ptrs=None, ws=None, wsb=None):
+    base = 1 << 20
+    if ptrs is None:
+        # distinct, aligned, non-overlapping fake addresses (validation must stop before use)
+        ptrs = [base * (k + 1) for k in range(13)]
+    if ws is None:
+        ws = base * 64
+    if wsb is None:
+        wsb = lib.rglru_workspace_size(B, T, D, dt) or 1 << 20
+    args = [ctypes.c_void_p(p) if p else None for p in ptrs]
+    if fn == "rglru_decode_step":
+        return getattr(lib, fn)(B, D, dt, *args, ctypes.c_void_p(ws) if ws else None,
+                                ctypes.c_size_t(wsb), None)
+    return getattr(lib, fn)(B, T, D, dt, *args, ctypes.c_void_p(ws) if ws else None,
+                            ctypes.c_size_t(wsb), None)
+
+
+@pytest.mark.parametrize("fn", ["rglru_prefill", "rglru_prefill_simt"])
+def test_rejects_before_launch(lib, fn):
+    assert _call(lib, fn, D=300) == api.ERR_INVALID_ARG
+    assert _call(lib, fn, T=0) == api.ERR_INVALID_ARG
+    assert _call(lib, fn, dt=5) == api.ERR_INVALID_ARG
+    for k in range(13):
+        p = [(1 << 20) * (j + 1) for j in range(13)]
+        p[k] = 0
+        assert _call(lib, fn, ptrs=p) == api.ERR_INVALID_ARG, f"null pointer {k}"
+        p[k] = (1 << 20) * (k + 1) + 4
+        assert _call(lib, fn, ptrs=p) == api.ERR_INVALID_ARG, f"misaligned pointer {k}"
+    assert _call(lib, fn, ws=0) == api.ERR_WORKSPACE
+    assert _call(lib, fn, ws=(1 << 20) * 64 + 8) == api.ERR_WORKSPACE
+    assert _call(lib, fn, wsb=16) == api.ERR_WORKSPACE
+    # y overlapping x
+    p = [(1 << 20) * (j + 1) for j in range(13)]
+    p[12] = p[0]
+    assert _call(lib, fn, ptrs=p) == api.ERR_INVALID_ARG
+    # conv_state overlapping h_state
+    p = [(1 << 20) * (j + 1) for j in range(13)]
+    p[10] = p[11]
+    assert _call(lib, fn, ptrs=p) == api.ERR_INVALID_ARG
+
+
+def test_decode_rejects_before_launch(lib):
+    f = "rglru_decode_step"
+    wsb = lib.rglru_decode_workspace_size(4, 256, api.IO_BF16)
+    assert _call(lib, f, B=4, D=512 + 3, wsb=wsb) == api.ERR_INVALID_ARG
+    assert _call(lib, f, B=0, wsb=wsb) == api.ERR_INVALID_ARG
+    assert _call(lib, f, B=4, wsb=8) == api.ERR_WORKSPACE
+    p = [(1 << 20) * (j + 1) for j in range(13)]
+    p[9] = 0
+    assert _call(lib, f, B=4, ptrs=p, wsb=wsb) == api.ERR_INVALID_ARG
+
+
+def test_status_calls_reject_null_workspace(lib):
+    assert lib.rglru_get_device_status(None, None) == api.ERR_WORKSPACE
+    assert lib.rglru_debug_suppress_publish(None, 0, None) == api.ERR_WORKSPACE
+    assert lib.rglru_debug_suppress_publish(ctypes.c_void_p(1 << 20), -2, None) == api.ERR_INVALID_ARG

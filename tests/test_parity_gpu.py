@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA library against the float64 oracle on the same seeded inputs.
+
+Small cases compare every element; the full-size workloads compare every
+output of sampled (batch row, head) units, whole sequences long, computed by
+the oracle unit by unit (heads and batch rows are independent).
+"""
+import numpy as np
+import pytest
+import torch
+
+from lm_causal_depthwise_b200 import api, workloads as W
+
+from parity_util import (check, check_bf16, check_f32, check_state, oracle_units, run_gpu,
+                         run_oracle, to_device)
+
+pytestmark = pytest.mark.gpu
+
+PATHS = [False, True]  # rglru_prefill, rglru_prefill_simt
+
+
+def _case(B, T, D, io="bf16", seed=21, doc_len=None, reset_at=(0,), continue_doc=False,
+          init_state="random"):
+    w = W.Workload("case", B=B, T=T, D=D, io=io, seed=seed, doc_len=doc_len, reset_at=reset_at,
+                   continue_doc=continue_doc, init_state=init_state)
+    return w, W.generate(w)
+
+
+@pytest.mark.parametrize("simt", PATHS)
+def test_tiny_f32_full(simt):
+    inp = W.generate(W.TINY_F32)
+    got = run_gpu(to_device(inp, "f32"), simt=simt)
+    ref = run_oracle(inp)
+    check_f32(got["y"], ref["y"], "y")
+    check_state("f32", got, ref, "tiny")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+@pytest.mark.parametrize("B,T,D,kw", [
+    (2, 1000, 512, dict(doc_len=300)),            # several chunks, ragged tail, mid resets
+    (1, 2053, 256, dict(continue_doc=True)),      # no reset: initial state carried through chunks
+    (3, 515, 768, dict(reset_at=(0, 1, 2, 3, 64, 65, 511))),  # resets near chunk edges
+    (1, 4096, 512, dict(doc_len=1024)),
+])
+def test_bf16_full_tensor(simt, B, T, D, kw):
+    _, inp = _case(B, T, D, **kw)
+    got = run_gpu(to_device(inp, "bf16"), simt=simt)
+    ref = run_oracle(inp)
+    check_bf16(got["y"], ref["y"], "y")
+    check_state("bf16", got, ref, "state")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 31, 32, 33, 127, 128, 129])
+def test_edge_lengths(simt, io, T):
+    _, inp = _case(2, T, 256, io=io, continue_doc=True, seed=T)
+    got = run_gpu(to_device(inp, io), simt=simt)
+    ref = run_oracle(inp)
+    check(io, got["y"], ref["y"], f"y T={T}")
+    check_state(io, got, ref, f"T={T}")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+def test_every_token_a_reset(simt):
+    w, inp = _case(2, 300, 256)
+    inp["segpos"][:] = 0
+    got = run_gpu(to_device(inp, "bf16"), simt=simt)
+    ref = run_oracle(inp)
+    check_bf16(got["y"], ref["y"], "y")
+    check_state("bf16", got, ref, "state")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+def test_short_documents(simt):
+    _, inp = _case(2, 400, 256, continue_doc=True)
+    inp["segpos"][:] = np.arange(400)[None, :] % 2   # a reset every other token
+    got = run_gpu(to_device(inp, "bf16"), simt=simt)
+    ref = run_oracle(inp)
+    check_bf16(got["y"], ref["y"], "y")
+
+
+def test_write_coverage_and_canaries():
+    """Every output element is written (NaN sentinels gone) and nothing past
+    the end of y is touched."""
+    _, inp = _case(2, 777, 512, doc_len=200)
+    dev = to_device(inp, "bf16")
+    B, T, D = 2, 777, 512
+    buf = torch.full((B * T * D + 4096,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y = buf[:B * T * D].view(B, T, D)
+    api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"],
+                dev["h_state"], y=y)
+    torch.cuda.synchronize()
+    assert not torch.isnan(y).any()
+    assert torch.isnan(buf[B * T * D:]).all()
+
+
+@pytest.mark.parametrize("simt", PATHS)
+def test_split_with_carried_state_equals_whole(simt):
+    _, inp = _case(2, 1500, 512, continue_doc=True)
+    whole = run_gpu(to_device(inp, "bf16"), simt=simt)
+    tau = 613
+    a = {**inp, "x": inp["x"][:, :tau], "g": inp["g"][:, :tau], "segpos": inp["segpos"][:, :tau]}
+    dev_a = to_device(a, "bf16")
+    o1 = run_gpu(dev_a, simt=simt)
+    b = {**inp, "x": inp["x"][:, tau:], "g": inp["g"][:, tau:], "segpos": inp["segpos"][:, tau:]}
+    dev_b = to_device(b, "bf16")
+    dev_b["conv_state"].copy_(dev_a["conv_state"])
+    dev_b["h_state"].copy_(dev_a["h_state"])
+    o2 = run_gpu(dev_b, simt=simt)
+    y = np.concatenate([o1["y"], o2["y"]], axis=1)
+    check_bf16(y, whole["y"], "split y")
+    np.testing.assert_array_equal(o2["conv_state"], whole["conv_state"])
+    check_bf16(o2["h_state"], whole["h_state"], "split h")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+def test_reset_makes_output_independent_of_earlier_tokens(simt):
+    s = 700
+    _, inp = _case(1, 1200, 512, reset_at=(0, s))
+    base = run_gpu(to_device(inp, "bf16"), simt=simt)
+    pert = {k: v.copy() for k, v in inp.items()}
+    rng = np.random.default_rng(9)
+    pert["x"][:, :s] = W.round_bf16(rng.standard_normal(pert["x"][:, :s].shape).astype(np.float32))
+    pert["g"][:, :s] = W.round_bf16(rng.standard_normal(pert["g"][:, :s].shape).astype(np.float32))
+    pert["h_state"] += 1.0
+    alt = run_gpu(to_device(pert, "bf16"), simt=simt)
+    np.testing.assert_array_equal(alt["y"][:, s:], base["y"][:, s:])
+    np.testing.assert_array_equal(alt["h_state"], base["h_state"])
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_decode_steps_match_oracle(io):
+    B, T, D = 64, 40, 512
+    _, inp = _case(B, T, D, io=io, reset_at=(0, 17))
+    dev = to_device(inp, io)
+    ys = []
+    for t in range(T):
+        y = api.decode_step(dev["x"][:, t].contiguous(), dev["g"][:, t].contiguous(), dev["params"],
+                            dev["segpos"][:, t].contiguous(), dev["conv_state"], dev["h_state"])
+        ys.append(y.float().cpu().numpy())
+    torch.cuda.synchronize()
+    ref = run_oracle(inp)
+    check(io, np.stack(ys, axis=1), ref["y"], "decode y")
+    got = {"h_state": dev["h_state"].cpu().numpy(), "conv_state": dev["conv_state"].float().cpu().numpy()}
+    check_state(io, got, ref, "decode")
+
+
+# ------------------------------------------------------------- full-size workloads
+
+def _full_size(w, units, simt=False):
+    inp = W.generate(w)
+    dev = to_device(inp, w.io)
+    y = api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"],
+                    dev["h_state"], simt=simt)
+    torch.cuda.synchronize()
+    ref = oracle_units(inp, units)
+    for (b, h), r in ref.items():
+        s = slice(h * 256, (h + 1) * 256)
+        check_bf16(y[b, :, s].float().cpu().numpy(), r["y"], f"{w.name} y unit {(b, h)}")
+        check_bf16(dev["h_state"][b, s].cpu().numpy(), r["h_state"], f"{w.name} h unit {(b, h)}")
+        np.testing.assert_array_equal(dev["conv_state"][b, :, s].float().cpu().numpy(),
+                                      r["conv_state"])
+    return y
+
+
+@pytest.mark.parametrize("wname,units", [
+    ("prefill-2b", [(0, 0), (3, 4), (7, 9)]),
+    ("prefill-long", [(0, 0), (0, 9)]),
+    ("prefill-long-carry", [(0, 3)]),
+    ("prefill-9b", [(0, 0), (15, 15), (9, 7)]),
+])
+def test_full_size_sampled_units(wname, units):
+    _full_size(W.ALL[wname], units)
+
+
+def test_full_size_decode_sampled_units():
+    w = W.DECODE_2B
+    inp = W.generate(w)
+    dev = to_device(inp, w.io)
+    ys = torch.empty((w.T, w.B, w.D), dtype=torch.bfloat16, device="cuda")
+    ws = api.new_workspace(api.decode_workspace_size(w.B, w.D, torch.bfloat16))
+    xs = dev["x"].transpose(0, 1).contiguous()
+    gs = dev["g"].transpose(0, 1).contiguous()
+    ss = dev["segpos"].t().contiguous()
+    for t in range(w.decode_steps):
+        api.decode_step(xs[t], gs[t], dev["params"], ss[t], dev["conv_state"], dev["h_state"],
+                        workspace=ws, y=ys[t])
+    torch.cuda.synchronize()
+    ref = oracle_units(inp, [(0, 0), (100, 5), (255, 9)])
+    for (b, h), r in ref.items():
+        s = slice(h * 256, (h + 1) * 256)
+        check_bf16(ys[:, b, s].float().cpu().numpy(), r["y"], f"decode y unit {(b, h)}")
+        check_bf16(dev["h_state"][b, s].cpu().numpy(), r["h_state"], "decode h")
