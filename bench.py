@@ -188,20 +188,33 @@ def run_reference(args, w):
 
 # ----------------------------------------------------------------------------- CUDA arm
 
-def count_launches(fn, prefix=("rglru",)):
-    """Kernels of this library launched by one call of ``fn`` (CUPTI via torch.profiler)."""
+def count_launches(fns, prefix=("rglru",)):
+    """Kernels of this library launched by each function in ``fns`` (one
+    profiler session, CUPTI via torch.profiler).  A marker kernel launched
+    between the calls splits the device timeline."""
     import torch
     from torch.profiler import ProfilerActivity, profile
+    marker = torch.zeros(1, device="cuda")
     torch.cuda.synchronize()
     with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        fn()
-        torch.cuda.synchronize()
-    names = []
-    for e in prof.events():
-        if e.device_type is not None and str(e.device_type).endswith("CUDA"):
-            if any(p in e.name for p in prefix):
-                names.append(e.name)
-    return len(names), sorted(set(names))
+        for fn in fns:
+            fn()
+            torch.cuda.synchronize()
+            marker.add_(1.0)
+            torch.cuda.synchronize()
+    kern = [e for e in prof.events()
+            if e.device_type is not None and str(e.device_type).endswith("CUDA")]
+    kern.sort(key=lambda e: e.time_range.start)
+    groups, cur = [], []
+    for e in kern:
+        if any(p in e.name for p in prefix):
+            cur.append(e.name)
+        elif "add" in e.name.lower() or "elementwise" in e.name.lower():
+            groups.append(cur)
+            cur = []
+    while len(groups) < len(fns):
+        groups.append([])
+    return [(len(g), sorted(set(g))) for g in groups[:len(fns)]]
 
 
 def run_cuda(args, w):
@@ -236,7 +249,10 @@ def run_cuda(args, w):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    launches_per_step, kernel_names = count_launches(step)
+    dec_setup = None if args.no_decode else setup_decode(args, dev)
+    fns = [step] + ([dec_setup["one"]] if dec_setup else [])
+    counts = count_launches(fns)
+    launches_per_step, kernel_names = counts[0]
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if distributed:
@@ -292,8 +308,8 @@ def run_cuda(args, w):
 
     # ---- batched decode at B=256 (a separate timed loop of single-token steps)
     dec = None
-    if not args.no_decode:
-        dec = run_decode(args, dev, stream, distributed)
+    if dec_setup is not None:
+        dec = run_decode(dec_setup, counts[1], stream, distributed)
 
     del hx, hg, hy, hsp
     if distributed:
@@ -337,47 +353,60 @@ def run_cuda(args, w):
     return 0
 
 
-def run_decode(args, dev, stream, distributed):
+def setup_decode(args, dev):
+    """Device buffers of the batched decode workload: B=256 sequences, one
+    token per step, inputs of every step resident in HBM."""
     import torch
-    import torch.distributed as dist
     from lm_causal_depthwise_b200 import api
 
     w = W.DECODE_2B
     steps = args.decode_steps or w.decode_steps
     inp = W.generate(w.scaled(T=steps))
     bf = torch.bfloat16
-    xs = torch.from_numpy(inp["x"]).to(dev).to(bf).transpose(0, 1).contiguous()
-    gs = torch.from_numpy(inp["g"]).to(dev).to(bf).transpose(0, 1).contiguous()
-    ss = torch.from_numpy(inp["segpos"]).to(dev).t().contiguous()
-    cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
-    hs = torch.from_numpy(inp["h_state"]).to(dev)
-    p = api.Params.from_arrays(inp, bf, dev)
-    ys = torch.empty_like(xs)
-    ws = api.new_workspace(api.decode_workspace_size(w.B, w.D, bf), dev)
+    d = dict(w=w, steps=steps)
+    d["xs"] = torch.from_numpy(inp["x"]).to(dev).to(bf).transpose(0, 1).contiguous()
+    d["gs"] = torch.from_numpy(inp["g"]).to(dev).to(bf).transpose(0, 1).contiguous()
+    d["ss"] = torch.from_numpy(inp["segpos"]).to(dev).t().contiguous()
+    d["cs"] = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
+    d["hs"] = torch.from_numpy(inp["h_state"]).to(dev)
+    d["p"] = api.Params.from_arrays(inp, bf, dev)
+    d["ys"] = torch.empty_like(d["xs"])
+    d["ws"] = api.new_workspace(api.decode_workspace_size(w.B, w.D, bf), dev)
+
+    def one(t=0):
+        api.decode_step(d["xs"][t], d["gs"][t], d["p"], d["ss"][t], d["cs"], d["hs"],
+                        workspace=d["ws"], y=d["ys"][t])
 
     def loop():
         for t in range(steps):
-            api.decode_step(xs[t], gs[t], p, ss[t], cs, hs, workspace=ws, y=ys[t])
+            one(t)
+    d["one"], d["loop"] = one, loop
+    return d
 
-    loop()
+
+def run_decode(d, launch_count, stream, distributed):
+    import torch
+    import torch.distributed as dist
+
+    w, steps = d["w"], d["steps"]
+    d["loop"]()
     torch.cuda.synchronize()
-    n_launch, names = count_launches(lambda: api.decode_step(xs[0], gs[0], p, ss[0], cs, hs,
-                                                             workspace=ws, y=ys[0]))
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if distributed:
         dist.barrier()
     torch.cuda.synchronize()
     ev0.record(stream)
-    loop()
+    d["loop"]()
     ev1.record(stream)
     torch.cuda.synchronize()
-    ms = torch.tensor([ev0.elapsed_time(ev1)], device=dev, dtype=torch.float64)
+    ms = torch.tensor([ev0.elapsed_time(ev1)], device=stream.device, dtype=torch.float64)
     if distributed:
         dist.all_reduce(ms, op=dist.ReduceOp.MAX)
     ms = float(ms.item())
     world = dist.get_world_size() if distributed else 1
     per_step_us = 1e3 * ms / steps
     step_bytes = W.decode_step_bytes(w)
+    n_launch, names = launch_count
     return {"workload": w.scaled(T=steps).describe(), "value": world * w.B * steps / (ms * 1e-3),
             "unit": "tokens/s", "us_per_step": per_step_us, "steps": steps,
             "algorithmic_gbs": step_bytes / (per_step_us * 1e-6) / 1e9,

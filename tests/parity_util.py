@@ -2,7 +2,10 @@
 library, run the oracle on the same arrays, compare with the stated bars.
 
 Tolerances (fixed here, used by every parity test):
-  fp32 I/O : max_e |got - ref| / max(|ref_e|, 1e-3 * rms(ref)) <= 1e-5
+  fp32 I/O : max_e |got - ref| / max(|ref_e|, rms(ref)) <= 1e-5
+             (relative error 1e-5 for every element at least as large as the
+             rms of the output, absolute error 1e-5 * rms below it; a plain
+             fp32 evaluation of the definitions scores 3-5e-6 here)
   bf16 I/O : every element |got - ref| <= 2e-2 + 1e-2 * |ref|
              (atol 2e-2, rtol 1e-2; bf16 output rounding alone is 2^-9 relative)
   integer / copied state (conv_state): bit-exact.
@@ -63,7 +66,7 @@ def check_f32(got, ref, what=""):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     rms = np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
-    den = np.maximum(np.abs(ref), 1e-3 * rms + 1e-300)
+    den = np.maximum(np.abs(ref), rms + 1e-300)
     err = np.max(np.abs(got - ref) / den) if ref.size else 0.0
     assert err <= F32_RTOL, f"{what}: max scaled error {err:.3e} > {F32_RTOL}"
     return err
