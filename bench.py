@@ -249,6 +249,20 @@ def run_cuda(args, w):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    if args.profile_run:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        st = api.device_status(ws)
+        if rank == 0:
+            print(json.dumps({"profile_run": w.describe(), "steps": args.steps,
+                              "ms_per_step": ev0.elapsed_time(ev1) / args.steps, "device_status": st}))
+        if distributed:
+            dist.destroy_process_group()
+        return 0 if st == 0 else 1
     dec_setup = None if args.no_decode else setup_decode(args, dev)
     fns = [step] + ([dec_setup["one"]] if dec_setup else [])
     counts = count_launches(fns)
@@ -424,6 +438,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="only the warm-up and timed prefill steps (no profiler, e2e, decode or "
+                         "CPU legs): the command an ncu capture wraps")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "cuda":
         args.warmup = 3

@@ -19,7 +19,7 @@ struct WsHeader {
     int detail;            // first chunk index whose wait gave up (+1), 0 = none
     int debug_unit_plus1;  // test hook: chunk that skips publishing (+1), 0 = off
     int pad0;
-    unsigned int ticket[64];  // per-group work counters of the fused prefill kernel
+    unsigned int ticket[1000];  // per-group work counters of the fused prefill kernel
 };
 constexpr size_t kWsHeaderBytes = 4096;
 static_assert(sizeof(WsHeader) <= kWsHeaderBytes, "header too large");

@@ -1,10 +1,805 @@
-// prefill_fused.cu -- bf16 prefill entry (fused sm_100a kernel goes here).
+// prefill_fused.cu -- fused sm_100a prefill of the RG-LRU block core (bf16 I/O, fp32 state).
+//
+// One persistent kernel does, per tile of 32 tokens of one (sequence, head, half
+// of the head's 256 channels):
+//   conv warps   causal depthwise conv (k=4, document mask) of all 256 input
+//                channels of the head, in fp32; bf16 copy into the MMA B tile
+//                (128-byte swizzled, K-major), fp32 copy of this half's channels
+//                for the scan.
+//   MMA thread   both block-diagonal gate projections on the tensor cores:
+//                D[128 out x 32 tok] = W[128 x 256] (A, resident in TMEM) * xc^T
+//                (B, shared memory), fp32 accumulators in TMEM.
+//   scan warps   one thread per output channel (= TMEM lane).  Pass 1: sigmoid
+//                gates, a = sigmoid(Lambda)^(8 r), sqrt(1-a^2) normaliser,
+//                resets; local scan from h = 0 gives the tile aggregate
+//                (prod a, h_end); (a, v) are written back over the
+//                accumulators.  Pass 2 (two tiles later): re-run the scan from
+//                the carried-in state, multiply by GELU_tanh(g), store y.
+//   look-back    publishes the tile aggregate, walks back over predecessor
+//   warp         tiles of the same sequence (decoupled look-back; (A,h) o
+//                (A',h') = (A A', A' h + h'), a reset makes A = 0 and ends the
+//                walk) to get the carried-in state, publishes the tile's
+//                inclusive prefix.
+//   producer     claims tiles in order from a per-(head, half) ticket counter,
+//                TMA-loads the GELU-branch tile, issues the MMAs.
+// Every wait is bounded: a wait that runs out records RGLRU_ERR_TIMEOUT in the
+// workspace header and the CTA unwinds (waiting, bounded, for its own copies
+// and MMAs in flight) and frees its TMEM.
+//
+// Block structure: "Gemma explained: RecurrentGemma architecture",
+// RecurrentGemmaRecurrentBlock printout (Conv1d k=4, padding=3, groups=D; GELU
+// tanh) and section "Residual block with recurrent block"; RG-LRU equations of
+// Griffin / RecurrentGemma (arXiv 2404.07839).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <mutex>
+
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace rglru {
+namespace {
 
-size_t fused_workspace_bytes(int B, int T, int D) { return simt_workspace_bytes(B, T, D); }
+using namespace sm100;
 
-rglru_status fused_prefill(const PrefillArgs &a) { return simt_prefill(a); }
+constexpr int NT = 32;       // tokens per tile (MMA N)
+constexpr int SLOTS = 4;     // tiles in flight per CTA
+constexpr int LAG = 2;       // pass 2 runs this many tiles behind pass 1
+constexpr int kHalf = 128;   // output channels per CTA (MMA M, TMEM lanes)
+constexpr int kScanWarps = 4, kConvWarps = 4;
+constexpr int kProdWarp = 8, kLbWarp = 9;
+constexpr int kThreads = 320;
+
+// TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
+// [pre_r | pre_i] accumulators that pass 1 overwrites with [a | v].
+constexpr uint32_t kColWa = 0, kColWx = 128, kColSlot0 = 256, kColPerSlot = 2 * NT;
+
+// Shared memory map (offsets from a 1024-byte aligned base)
+constexpr int kBTile = NT * 256 * 2;            // bf16 xc, 4 K-blocks of 64 channels
+constexpr int kBBlock = NT * 128;               // one K-block: NT rows x 128 B
+constexpr int kXcsTile = NT * kHalf * 4;        // fp32 xc of this half
+constexpr int kGTile = NT * kHalf * 2;          // bf16 gate-branch tile (TMA box)
+constexpr int OFF_B = 0;
+constexpr int OFF_XCS = OFF_B + SLOTS * kBTile;
+constexpr int OFF_G = OFF_XCS + SLOTS * kXcsTile;
+constexpr int OFF_AGG = OFF_G + SLOTS * kGTile;
+constexpr int OFF_HIN = OFF_AGG + SLOTS * kHalf * 8;
+constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
+constexpr int OFF_BAR = OFF_INFO + SLOTS * 32;
+enum { BAR_INFO, BAR_CONV, BAR_MMA, BAR_PASS1, BAR_LB, BAR_G, BAR_FREE, BAR_KINDS };
+constexpr int OFF_MISC = OFF_BAR + BAR_KINDS * SLOTS * 8;
+constexpr int kSmemUsed = OFF_MISC + 16;
+constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+
+struct TileInfo {
+    int u;        // tile index inside the (head, half) group, -1 = no more work
+    int b, t0, valid;
+    uint32_t reset_mask;  // bit t: segment_pos == 0 at token t0 + t
+    int first, last, pad;
+};
+static_assert(sizeof(TileInfo) == 32, "TileInfo size");
+
+struct FusedParams {
+    int B, T, D, C, G, tiles_per_group;
+    const __nv_bfloat16 *x;
+    const float *conv_w, *conv_b;
+    const __nv_bfloat16 *W_a;
+    const float *b_a;
+    const __nv_bfloat16 *W_x;
+    const float *b_x, *lambda;
+    const int32_t *segpos;
+    __nv_bfloat16 *conv_state;
+    float *h_state;
+    __nv_bfloat16 *y;
+    WsHeader *hdr;
+    uint32_t *flags;   // [G][tiles_per_group]
+    float2 *agg;       // [G][tiles_per_group][128]  (prod a, h_end) from h = 0
+    float *prefix;     // [G][tiles_per_group][128]  h after the tile
+};
+
+constexpr uint32_t F_AGG = 1u, F_PREFIX = 2u, F_RESET = 4u;
+
+__device__ __forceinline__ void raise_timeout(volatile int *abort_flag, WsHeader *hdr, int where)
+{
+    atomicCAS(&hdr->status, 0, (int)RGLRU_ERR_TIMEOUT);
+    atomicCAS(&hdr->detail, 0, where + 1);
+    *abort_flag = 1;
+}
+
+// Bounded wait on an mbarrier phase; false on timeout or when the CTA is aborting.
+__device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
+                                      int where)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (*(volatile int *)&hdr->status != 0) {
+                *abort_flag = 1;
+                return false;
+            }
+            if (globaltimer() - t0 > kTimeoutNs) {
+                raise_timeout(abort_flag, hdr, where);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded spin on a global flag by one thread; 0 on timeout/abort.
+__device__ __noinline__ uint32_t wait_flag(const uint32_t *f, uint32_t need, volatile int *abort_flag,
+                                           WsHeader *hdr, int where)
+{
+    uint32_t v = ld_acquire_u32(f);
+    if (v & need) return v;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        v = ld_acquire_u32(f);
+        if (v & need) return v;
+        if ((it & 31u) == 0) {
+            if (*abort_flag) return 0;
+            if (*(volatile int *)&hdr->status != 0) {
+                *abort_flag = 1;
+                return 0;
+            }
+            if (globaltimer() - t0 > kTimeoutNs) {
+                raise_timeout(abort_flag, hdr, where);
+                return 0;
+            }
+        }
+    }
+}
+
+// Warp-collective forms: lane 0 waits, the result is broadcast, then every lane
+// performs its own (already satisfied) acquire so that the warp stays converged
+// for the .sync.aligned tcgen05 instructions that follow.
+__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              WsHeader *hdr, int where)
+{
+    uint32_t ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, hdr, where) ? 1u : 0u;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) {
+        while (!mbar_try_wait(bar, parity)) {
+        }
+    }
+    return ok != 0;
+}
+
+// Flags only gain bits during a launch; the value lane 0 saw drives every lane's
+// control flow, each lane's own acquire load orders its later data loads.
+__device__ __forceinline__ uint32_t warp_wait_flag(const uint32_t *f, uint32_t need, volatile int *abort_flag,
+                                                   WsHeader *hdr, int where)
+{
+    uint32_t v = 0;
+    if ((threadIdx.x & 31) == 0) v = wait_flag(f, need, abort_flag, hdr, where);
+    v = __shfl_sync(0xffffffffu, v, 0);
+    if (v) (void)ld_acquire_u32(f);
+    return v;
+}
+
+// Decoupled look-back, first half: walking back from tile `hi` (>= seq_first),
+// find the nearest anchor -- a tile whose inclusive prefix is published, or a
+// tile holding a reset (A = 0: its prefix is its own H) -- such that every tile
+// between the anchor and `hi` has published its aggregate.  Lane l examines
+// tile hi - l, so 32 flags cost one round trip.  The first tile of the
+// sequence is an anchor only once its prefix (or its reset) is out.
+// Warp-collective; false on timeout or abort.
+__device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_first, int &anchor,
+                                         uint32_t &anchor_flag, volatile int *abort_flag, WsHeader *hdr)
+{
+    const int lane = threadIdx.x & 31;
+    uint64_t t0 = 0;
+    for (uint32_t spins = 0;;) {
+        const int pu = hi - lane;
+        const bool in = pu >= seq_first;
+        const uint32_t f = in ? ld_acquire_u32(flags + pu) : 0u;
+        const uint32_t anchors = __ballot_sync(0xffffffffu, in && (f & (F_PREFIX | F_RESET)));
+        const uint32_t ready = __ballot_sync(0xffffffffu, in && (f & F_AGG));
+        if (anchors) {
+            const int la = __ffs(anchors) - 1;
+            const uint32_t span = la ? ((1u << la) - 1u) : 0u;
+            if ((ready & span) == span) {
+                anchor = hi - la;
+                anchor_flag = __shfl_sync(0xffffffffu, f, la);
+                return true;
+            }
+        } else if (ready == 0xffffffffu) {
+            hi -= 32;  // 32 aggregates, no anchor yet: look further back
+            continue;
+        }
+        if (t0 == 0) t0 = globaltimer();
+        __nanosleep(64);
+        if ((++spins & 31u) == 0) {
+            uint32_t stop = 0;
+            if (lane == 0) {
+                if (*abort_flag) {
+                    stop = 1;
+                } else if (*(volatile int *)&hdr->status != 0) {
+                    *abort_flag = 1;
+                    stop = 1;
+                } else if (globaltimer() - t0 > kTimeoutNs) {
+                    raise_timeout(abort_flag, hdr, 12);
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        f[2 * k] = __uint_as_float(w[k] << 16);
+        f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// -(exp(2l) - 1) for small |l| by its Taylor series: -2l (1 + l + 2/3 l^2 + 1/3 l^3 + 2/15 l^4)
+__device__ __forceinline__ float one_minus_exp2l_small(float l)
+{
+    float s = fmaf(l, 2.f / 15.f, 1.f / 3.f);
+    s = fmaf(l, s, 2.f / 3.f);
+    s = fmaf(l, s, 1.f);
+    s = fmaf(l, s, 1.f);
+    return -2.f * l * s;
+}
+
+__device__ __forceinline__ float gelu_tanh_fast(float g)
+{
+    const float k0 = 0.7978845608028654f, k1 = 0.7978845608028654f * 0.044715f;
+    const float u = g * fmaf(k1 * g, g, k0);
+    const float hg = 0.5f * g;
+    return fmaf(hg, tanh_approx(u), hg);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap tmap_g)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int group = blockIdx.x % p.G;
+    const int head = group >> 1, half = group & 1;
+    TileInfo *info = reinterpret_cast<TileInfo *>(smem + OFF_INFO);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    auto bar = [&](int kind, int s) { return bars + kind * SLOTS + s; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    WsHeader *hdr = p.hdr;
+
+    // ------------------------------------------------------------------ setup
+    if (warp == kProdWarp) {
+        tmem_alloc(tmem_holder, 512);
+        if (lane == 0) {
+            for (int s = 0; s < SLOTS; ++s) {
+                mbar_init(bar(BAR_INFO, s), 1);
+                mbar_init(bar(BAR_CONV, s), kConvWarps * 32);
+                mbar_init(bar(BAR_MMA, s), 1);
+                mbar_init(bar(BAR_PASS1, s), kScanWarps * 32);
+                mbar_init(bar(BAR_LB, s), 32);
+                mbar_init(bar(BAR_G, s), 1);
+                mbar_init(bar(BAR_FREE, s), kScanWarps * 32);
+            }
+            *abort_flag = 0;
+            mbar_fence_init();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp < kScanWarps) {
+        // this thread's TMEM lane = output channel c of the half: rows of W_a and W_x
+        const int c = threadIdx.x;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const size_t row = (size_t)head * 256 + half * kHalf + c;
+#pragma unroll 1
+        for (int gate = 0; gate < 2; ++gate) {
+            const uint4 *src = reinterpret_cast<const uint4 *>((gate == 0 ? p.W_a : p.W_x) + row * 256);
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 v = src[q * 8 + k];
+                    r[4 * k] = v.x;
+                    r[4 * k + 1] = v.y;
+                    r[4 * k + 2] = v.z;
+                    r[4 * k + 3] = v.w;
+                }
+                tmem_st32(tmem + lane_off + (gate == 0 ? kColWa : kColWx) + q * 32, r);
+            }
+        }
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int debug_unit = *(volatile int *)&hdr->debug_unit_plus1 - 1;
+
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------ producer / MMA issuer
+        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
+        int issued = 0;  // tiles whose TMA and MMAs were issued
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            bool ok = true;
+            if (j >= SLOTS) ok = warp_wait_bar(bar(BAR_FREE, s), ph ^ 1u, abort_flag, hdr, 1);
+            int u = -1;
+            if (lane == 0 && ok && !*abort_flag) {
+                u = (int)atomicAdd(&hdr->ticket[group], 1u);
+                if (u >= p.tiles_per_group) u = -1;
+            }
+            u = __shfl_sync(0xffffffffu, u, 0);
+            TileInfo ti{};
+            ti.u = u;
+            if (u >= 0) {
+                ti.b = u / p.C;
+                const int c = u % p.C;
+                ti.t0 = c * NT;
+                ti.valid = min(NT, p.T - ti.t0);
+                ti.first = c == 0;
+                ti.last = c == p.C - 1;
+                const int t = ti.t0 + lane;
+                const int sp = lane < ti.valid ? p.segpos[(size_t)ti.b * p.T + t] : 1;
+                ti.reset_mask = __ballot_sync(0xffffffffu, sp == 0);
+            }
+            if (lane == 0) {
+                info[s] = ti;
+                mbar_arrive(bar(BAR_INFO, s));
+            }
+            if (u < 0) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(BAR_G, s), kGTile);
+                tma_load_3d(smem + OFF_G + s * kGTile, &tmap_g, bar(BAR_G, s), head * 256 + half * kHalf, ti.t0,
+                            ti.b);
+            }
+            ++issued;
+            if (!warp_wait_bar(bar(BAR_CONV, s), ph, abort_flag, hdr, 2)) {
+                // the TMA is in flight; the MMAs of this tile were never issued
+                break;
+            }
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t b_base = smem_u32(smem + OFF_B + s * kBTile);
+                const uint32_t d_r = tmem + kColSlot0 + s * kColPerSlot;
+                const uint32_t d_i = d_r + NT;
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const uint64_t bd = umma_desc_sw128(b_base + (kk >> 2) * kBBlock + (kk & 3) * 32);
+                    umma_ts(d_r, tmem + kColWa + kk * 8, bd, idesc, kk > 0);
+                    umma_ts(d_i, tmem + kColWx + kk * 8, bd, idesc, kk > 0);
+                }
+                umma_commit(bar(BAR_MMA, s));
+            }
+            __syncwarp();
+        }
+        // drain: this thread's last commit covers every MMA it issued; each slot's
+        // last TMA load is waited on (bounded) so that nothing lands after exit.
+        if (lane == 0 && *abort_flag) {
+            for (int k = max(0, issued - SLOTS); k < issued; ++k) {
+                const int s = k % SLOTS;
+                const uint32_t ph = (uint32_t)(k / SLOTS) & 1u;
+                uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(bar(BAR_G, s), ph) && globaltimer() - t0 < kTimeoutNs) {
+                }
+                t0 = globaltimer();
+                while (!mbar_try_wait(bar(BAR_MMA, s), ph) && globaltimer() - t0 < kTimeoutNs / 4) {
+                }
+            }
+        }
+    } else if (warp >= kScanWarps && warp < kScanWarps + kConvWarps) {
+        // ------------------------------------------------------------ conv warps
+        const int kb = warp - kScanWarps;  // K-block: channels [64 kb, 64 kb + 64) of the head
+        const int cg = lane & 7;           // 8 channels per lane
+        const int q = lane >> 3;           // token quarter of the tile
+        const int dl = kb * 64 + cg * 8;   // channel within the head
+        const size_t d0 = (size_t)head * 256 + dl;
+        float w[4][8], cb[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[k][e] = p.conv_w[(size_t)k * p.D + d0 + e];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cb[e] = p.conv_b[d0 + e];
+        const bool own = (kb >> 1) == half;
+        const int xcs_col = (kb & 1) * 64 + cg * 8;
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            if (!warp_wait_bar(bar(BAR_INFO, s), ph, abort_flag, hdr, 3)) break;
+            const TileInfo ti = info[s];
+            if (ti.u < 0) break;
+            const int n0 = q * 8;
+            const int tb = ti.t0 + n0;
+            const size_t rowB = (size_t)ti.b * p.T;
+            uint4 raw[11];
+            int pos[8];
+#pragma unroll
+            for (int r = 0; r < 11; ++r) {
+                const int t = tb - 3 + r;
+                raw[r] = make_uint4(0, 0, 0, 0);
+                if (t >= 0 && t < p.T)
+                    raw[r] = *reinterpret_cast<const uint4 *>(p.x + (rowB + t) * p.D + d0);
+                else if (t < 0)
+                    raw[r] = *reinterpret_cast<const uint4 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + t) * p.D + d0);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int t = tb + i;
+                pos[i] = t < p.T ? p.segpos[rowB + t] : 0;
+            }
+            float xm3[8], xm2[8], xm1[8];
+            unpack8(raw[0], xm3);
+            unpack8(raw[1], xm2);
+            unpack8(raw[2], xm1);
+            uint8_t *btile = smem + OFF_B + s * kBTile + kb * kBBlock;
+            float *xcs = reinterpret_cast<float *>(smem + OFF_XCS + s * kXcsTile);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float x0[8];
+                unpack8(raw[3 + i], x0);
+                const int n = n0 + i;
+                const int ps = pos[i];
+                float xc[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float acc = cb[e];
+                    if (ps >= 3) acc = fmaf(w[0][e], xm3[e], acc);
+                    if (ps >= 2) acc = fmaf(w[1][e], xm2[e], acc);
+                    if (ps >= 1) acc = fmaf(w[2][e], xm1[e], acc);
+                    acc = fmaf(w[3][e], x0[e], acc);
+                    xc[e] = n < ti.valid ? acc : 0.f;
+                }
+                uint4 pk;
+                pk.x = pack_bf16x2(xc[0], xc[1]);
+                pk.y = pack_bf16x2(xc[2], xc[3]);
+                pk.z = pack_bf16x2(xc[4], xc[5]);
+                pk.w = pack_bf16x2(xc[6], xc[7]);
+                *reinterpret_cast<uint4 *>(btile + n * 128 + ((cg ^ (n & 7)) << 4)) = pk;
+                if (own) {
+                    float4 *dst = reinterpret_cast<float4 *>(xcs + n * kHalf + xcs_col);
+                    dst[0] = make_float4(xc[0], xc[1], xc[2], xc[3]);
+                    dst[1] = make_float4(xc[4], xc[5], xc[6], xc[7]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    xm3[e] = xm2[e];
+                    xm2[e] = xm1[e];
+                    xm1[e] = x0[e];
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(BAR_CONV, s));
+        }
+    } else if (warp < kScanWarps) {
+        // ------------------------------------------------------------ scan warps
+        const int c = threadIdx.x;
+        const int d = head * 256 + half * kHalf + c;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float ba = p.b_a[d], bx = p.b_x[d];
+        const float lam = p.lambda[d];
+        const float ls = lam >= 0.f ? -log1pf(expf(-lam)) : lam - log1pf(expf(lam));  // log sigmoid(Lambda)
+        const float kl = kC * ls;                       // log a per unit r
+        const float kl2 = kl * 1.4426950408889634f;     // log2 a per unit r
+
+        auto pass1 = [&](int j) -> bool {
+            const int s = j % SLOTS;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            const TileInfo ti = info[s];
+            if (!warp_wait_bar(bar(BAR_MMA, s), ph, abort_flag, hdr, 4)) return false;
+            tc_fence_after();
+            uint32_t ar[32], ai[32];
+            const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
+            tmem_ld32(col, ar);
+            tmem_ld32(col + NT, ai);
+            tmem_wait_ld();
+            const float *xcs = reinterpret_cast<const float *>(smem + OFF_XCS + s * kXcsTile);
+            float hl = 0.f, P = 1.f;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const float xc = xcs[t * kHalf + c];
+                const float r = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ar[t]) + ba)), 0.5f);
+                const float ig = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ai[t]) + bx)), 0.5f);
+                const float ell = r * kl;
+                float a = ex2_approx(r * kl2);
+                const float om = ell > -0.125f ? one_minus_exp2l_small(ell) : fmaf(-a, a, 1.f);
+                const float uu = ig * xc;
+                float v = sqrt_approx(om) * uu;
+                if ((ti.reset_mask >> t) & 1u) {
+                    a = 0.f;
+                    v = uu;
+                }
+                if (t >= ti.valid) {
+                    a = 1.f;
+                    v = 0.f;
+                }
+                hl = fmaf(a, hl, v);
+                P *= a;
+                ar[t] = __float_as_uint(a);
+                ai[t] = __float_as_uint(v);
+            }
+            tmem_st32(col, ar);
+            tmem_st32(col + NT, ai);
+            tmem_wait_st();
+            reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = make_float2(P, hl);
+            mbar_arrive(bar(BAR_PASS1, s));
+            return true;
+        };
+
+        auto pass2 = [&](int j) -> bool {
+            const int s = j % SLOTS;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            const TileInfo ti = info[s];
+            if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 5)) return false;
+            float h = reinterpret_cast<const float *>(smem + OFF_HIN + s * kHalf * 4)[c];
+            if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 6)) return false;
+            tc_fence_after();
+            uint32_t aa[32], vv[32];
+            const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
+            tmem_ld32(col, aa);
+            tmem_ld32(col + NT, vv);
+            tmem_wait_ld();
+            const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile);
+            __nv_bfloat16 *yp = p.y + ((size_t)ti.b * p.T + ti.t0) * p.D + d;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                h = fmaf(__uint_as_float(aa[t]), h, __uint_as_float(vv[t]));
+                if (t < ti.valid) {
+                    const float gv = __bfloat162float(gs[t * kHalf + c]);
+                    yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                }
+            }
+            if (ti.last) {
+                // The old states are read by the first tile of this sequence (its
+                // conv in both halves of the head, its look-back for h): wait until
+                // those reads are published before overwriting the states.
+                const size_t u0 = (size_t)ti.b * p.C;
+                const uint32_t *f_own = p.flags + (size_t)group * p.tiles_per_group + u0;
+                const uint32_t *f_oth = p.flags + (size_t)(group ^ 1) * p.tiles_per_group + u0;
+                if (warp_wait_flag(f_own, F_PREFIX, abort_flag, hdr, 7) == 0) return false;
+                if (warp_wait_flag(f_oth, F_AGG, abort_flag, hdr, 8) == 0) return false;
+                p.h_state[(size_t)ti.b * p.D + d] = h;
+                __nv_bfloat16 ncs[3];
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int ts = p.T - 3 + k;
+                    ncs[k] = ts >= 0 ? p.x[((size_t)ti.b * p.T + ts) * p.D + d]
+                                     : p.conv_state[((size_t)ti.b * 3 + 3 + ts) * p.D + d];
+                }
+#pragma unroll
+                for (int k = 0; k < 3; ++k) p.conv_state[((size_t)ti.b * 3 + k) * p.D + d] = ncs[k];
+            }
+            tc_fence_before();
+            mbar_arrive(bar(BAR_FREE, s));
+            return true;
+        };
+
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            bool end = !warp_wait_bar(bar(BAR_INFO, s), ph, abort_flag, hdr, 9);
+            if (!end) end = info[s].u < 0;
+            bool ok = true;
+            if (!end) ok = pass1(j);
+            if (ok && j >= LAG) ok = pass2(j - LAG);
+            if (!ok) break;
+            if (end) {
+                for (int k = max(0, j - LAG + 1); k < j && ok; ++k) ok = pass2(k);
+                break;
+            }
+        }
+    } else if (warp == kLbWarp) {
+        // ------------------------------------------------------------ look-back warp
+        const int ch = lane * 4;  // 4 channels per lane
+        const size_t dch = (size_t)head * 256 + half * kHalf + ch;
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            if (!warp_wait_bar(bar(BAR_INFO, s), ph, abort_flag, hdr, 10)) break;
+            const TileInfo ti = info[s];
+            if (ti.u < 0) break;
+            if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 11)) break;
+            const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
+            const float4 g01 = sagg[lane * 2], g23 = sagg[lane * 2 + 1];  // (A,H) of 4 channels
+            const float A[4] = {g01.x, g01.z, g23.x, g23.z};
+            const float Hh[4] = {g01.y, g01.w, g23.y, g23.w};
+            const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
+            const uint32_t rbit = ti.reset_mask ? F_RESET : 0u;
+            const bool suppress = (int)gu == debug_unit;
+            if (!suppress) {
+                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf + ch);
+                dst[0] = g01;
+                dst[1] = g23;
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_u32(p.flags + gu, F_AGG | rbit);
+            }
+            float hin[4];
+            bool ok = true;
+            if (ti.first) {
+                const float4 hs = *reinterpret_cast<const float4 *>(p.h_state + (size_t)ti.b * p.D + dch);
+                hin[0] = hs.x; hin[1] = hs.y; hin[2] = hs.z; hin[3] = hs.w;
+            } else {
+                const size_t gbase = (size_t)group * p.tiles_per_group;
+                int anchor = -1;
+                uint32_t aflag = 0;
+                ok = find_anchor(p.flags + gbase, ti.u - 1, ti.b * p.C, anchor, aflag, abort_flag, hdr);
+                if (ok) {
+                    // carried-in state = the chain h <- A h + H folded forward in
+                    // sequence order from the anchor, the same order whichever
+                    // prefixes happened to be published (bit-reproducible)
+                    if (aflag & F_PREFIX) {
+                        const float4 pr = ld_relaxed_f4(reinterpret_cast<const float4 *>(p.prefix + (gbase + anchor) * kHalf + ch));
+                        hin[0] = pr.x; hin[1] = pr.y; hin[2] = pr.z; hin[3] = pr.w;
+                    } else {  // a tile holding a reset: A = 0, its prefix is its H
+                        const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + anchor) * kHalf + ch);
+                        const float4 a01 = ld_relaxed_f4(src), a23 = ld_relaxed_f4(src + 1);
+                        hin[0] = a01.y; hin[1] = a01.w; hin[2] = a23.y; hin[3] = a23.w;
+                    }
+#pragma unroll 1
+                    for (int p0 = anchor + 1; p0 < ti.u; p0 += 8) {
+                        float4 dd[8][2];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (p0 + q < ti.u) {
+                                const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + p0 + q) * kHalf + ch);
+                                dd[q][0] = ld_relaxed_f4(src);
+                                dd[q][1] = ld_relaxed_f4(src + 1);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (p0 + q < ti.u) {
+                                hin[0] = fmaf(dd[q][0].x, hin[0], dd[q][0].y);
+                                hin[1] = fmaf(dd[q][0].z, hin[1], dd[q][0].w);
+                                hin[2] = fmaf(dd[q][1].x, hin[2], dd[q][1].y);
+                                hin[3] = fmaf(dd[q][1].z, hin[3], dd[q][1].w);
+                            }
+                        }
+                    }
+                }
+            }
+            if (!ok) break;
+            float pre[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
+            if (!suppress) {
+                *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
+            }
+            *reinterpret_cast<float4 *>(smem + OFF_HIN + s * kHalf * 4 + ch * 4) =
+                make_float4(hin[0], hin[1], hin[2], hin[3]);
+            mbar_arrive(bar(BAR_LB, s));
+        }
+    }
+
+    // ------------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kProdWarp) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+struct Layout {
+    int C, G, tpg;
+    size_t flags_off, flags_bytes, agg_off, prefix_off, total;
+};
+
+Layout layout_of(int B, int T, int D)
+{
+    Layout L;
+    L.C = (T + NT - 1) / NT;
+    L.G = 2 * (D / kHead);
+    L.tpg = B * L.C;
+    const size_t tiles = (size_t)L.G * L.tpg;
+    L.flags_off = kWsHeaderBytes;
+    L.flags_bytes = align_up(tiles * 4, 256);
+    L.agg_off = L.flags_off + L.flags_bytes;
+    L.prefix_off = L.agg_off + align_up(tiles * kHalf * 8, 256);
+    L.total = L.prefix_off + align_up(tiles * kHalf * 4, 256);
+    return L;
+}
+
+}  // namespace
+
+size_t fused_workspace_bytes(int B, int T, int D) { return layout_of(B, T, D).total; }
+
+rglru_status fused_prefill(const PrefillArgs &a)
+{
+    const Layout L = layout_of(a.B, a.T, a.D);
+    if ((size_t)L.tpg > 0x7fffffffu / 2 || L.G > (int)(sizeof(WsHeader::ticket) / sizeof(unsigned int)))
+        return RGLRU_ERR_UNSUPPORTED;
+    auto encode = encode_fn();
+    if (!encode) return RGLRU_ERR_CUDA;
+
+    CUtensorMap tmap;
+    const cuuint64_t gdim[3] = {(cuuint64_t)a.D, (cuuint64_t)a.T, (cuuint64_t)a.B};
+    const cuuint64_t gstride[2] = {(cuuint64_t)a.D * 2, (cuuint64_t)a.T * a.D * 2};
+    const cuuint32_t box[3] = {kHalf, NT, 1};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.g), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RGLRU_ERR_CUDA;
+
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return RGLRU_ERR_CUDA;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(rglru_prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return RGLRU_ERR_CUDA;
+
+    char *ws = static_cast<char *>(a.ws);
+    // tickets and flags start at zero; the status word and the test hook are kept
+    if (cudaMemsetAsync(ws + offsetof(WsHeader, ticket), 0,
+                        L.flags_off - offsetof(WsHeader, ticket) + L.flags_bytes, a.stream) != cudaSuccess)
+        return RGLRU_ERR_CUDA;
+
+    FusedParams p;
+    p.B = a.B; p.T = a.T; p.D = a.D; p.C = L.C; p.G = L.G; p.tiles_per_group = L.tpg;
+    p.x = static_cast<const __nv_bfloat16 *>(a.x);
+    p.conv_w = a.conv_w; p.conv_b = a.conv_b;
+    p.W_a = static_cast<const __nv_bfloat16 *>(a.W_a); p.b_a = a.b_a;
+    p.W_x = static_cast<const __nv_bfloat16 *>(a.W_x); p.b_x = a.b_x;
+    p.lambda = a.lambda; p.segpos = a.segpos;
+    p.conv_state = static_cast<__nv_bfloat16 *>(a.conv_state);
+    p.h_state = a.h_state;
+    p.y = static_cast<__nv_bfloat16 *>(a.y);
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    p.flags = reinterpret_cast<uint32_t *>(ws + L.flags_off);
+    p.agg = reinterpret_cast<float2 *>(ws + L.agg_off);
+    p.prefix = reinterpret_cast<float *>(ws + L.prefix_off);
+
+    const int per_group = max(1, sms / L.G);
+    const int grid = per_group * L.G;
+    rglru_prefill_fused_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(p, tmap);
+    return cuda_status(cudaGetLastError());
+}
 
 }  // namespace rglru

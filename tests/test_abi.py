@@ -66,7 +66,8 @@ def _call(lib, fn="rglru_prefill", B=1, T=4, D=256, dt=api.IO_BF16, ptrs=None, w
     if ws is None:
         ws = base * 64
     if wsb is None:
-        wsb = lib.rglru_workspace_size(B, T, D, dt) or 1 << 20
+        q = lib.rglru_simt_workspace_size if fn == "rglru_prefill_simt" else lib.rglru_workspace_size
+        wsb = q(B, T, D, dt) or 1 << 20
     args = [ctypes.c_void_p(p) if p else None for p in ptrs]
     if fn == "rglru_decode_step":
         return getattr(lib, fn)(B, D, dt, *args, ctypes.c_void_p(ws) if ws else None,

@@ -191,3 +191,58 @@ def test_full_size_decode_sampled_units():
         s = slice(h * 256, (h + 1) * 256)
         check_bf16(ys[:, b, s].float().cpu().numpy(), r["y"], f"decode y unit {(b, h)}")
         check_bf16(dev["h_state"][b, s].cpu().numpy(), r["h_state"], "decode h")
+
+
+# ------------------------------------------------------------- bounded waits and cross-checks
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A tile that never publishes its scan carry (host-set test hook) makes its
+    successor's look-back wait run out: the call ends with RGLRU_ERR_TIMEOUT in
+    the device status, within seconds, and the next call on the same context
+    and workspace is correct."""
+    import time
+    _, inp = _case(1, 256, 256, continue_doc=True)
+    dev = to_device(inp, "bf16")
+    ws = api.new_workspace(api.workspace_size(1, 256, 256, torch.bfloat16))
+    api.debug_suppress_publish(ws, 3)
+    t0 = time.time()
+    api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"], dev["h_state"],
+                workspace=ws)
+    assert api.device_status(ws) == api.ERR_TIMEOUT
+    assert time.time() - t0 < 60
+    api.debug_suppress_publish(ws, -1)
+    dev = to_device(inp, "bf16")
+    got = run_gpu(dev, workspace=ws)
+    assert api.device_status(ws) == api.OK
+    ref = run_oracle(inp)
+    check_bf16(got["y"], ref["y"], "y after timeout")
+
+
+@pytest.mark.parametrize("wname", ["prefill-2b", "prefill-long-carry"])
+def test_full_size_fused_matches_simt_everywhere(wname):
+    """Whole-tensor check at full size: the fused kernel against the plain SIMT
+    kernels (fp32, accurate transcendentals), every element."""
+    w = W.ALL[wname]
+    inp = W.generate(w)
+    a = to_device(inp, w.io)
+    b = to_device(inp, w.io)
+    ya = api.prefill(a["x"], a["g"], a["params"], a["segpos"], a["conv_state"], a["h_state"])
+    yb = api.prefill(b["x"], b["g"], b["params"], b["segpos"], b["conv_state"], b["h_state"], simt=True)
+    torch.cuda.synchronize()
+    diff = (ya.float() - yb.float()).abs()
+    bound = 2e-2 + 1e-2 * yb.float().abs()
+    assert bool((diff <= bound).all()), f"max diff {diff.max().item():.3e}"
+    hb = b["h_state"]
+    assert bool(((a["h_state"] - hb).abs() <= 2e-2 + 1e-2 * hb.abs()).all())
+    assert torch.equal(a["conv_state"], b["conv_state"])
+
+
+def test_fused_prefill_is_bit_reproducible():
+    """The cross-tile carry is folded in sequence order from its anchor, so two
+    runs on the same inputs give identical bits whatever the scheduling."""
+    _, inp = _case(2, 3000, 512, doc_len=800)
+    a = run_gpu(to_device(inp, "bf16"))
+    for _ in range(3):
+        b = run_gpu(to_device(inp, "bf16"))
+        np.testing.assert_array_equal(a["y"], b["y"])
+        np.testing.assert_array_equal(a["h_state"], b["h_state"])
