@@ -12,14 +12,16 @@
 //   scan warps   one thread per output channel (= TMEM lane).  Pass 1: sigmoid
 //                gates, a = sigmoid(Lambda)^(8 r), sqrt(1-a^2) normaliser,
 //                resets; local scan from h = 0 gives the tile aggregate
-//                (prod a, h_end); (a, v) are written back over the
-//                accumulators.  Pass 2 (two tiles later): re-run the scan from
-//                the carried-in state, multiply by GELU_tanh(g), store y.
-//   look-back    publishes the tile aggregate, walks back over predecessor
-//   warp         tiles of the same sequence (decoupled look-back; (A,h) o
-//                (A',h') = (A A', A' h + h'), a reset makes A = 0 and ends the
-//                walk) to get the carried-in state, publishes the tile's
-//                inclusive prefix.
+//                (prod a, h_end), published at once; (a, v) are written back
+//                over the accumulators.  Pass 2 (two tiles later): re-run the
+//                scan from the carried-in state, multiply by GELU_tanh(g),
+//                store y.
+//   look-back    walks back over predecessor tiles of the same sequence to the
+//   warp         nearest anchor (a published inclusive prefix, or a tile that
+//                holds a reset: A = 0), folds h <- A h + H forward from it in
+//                sequence order (decoupled look-back with a fixed combination
+//                order, so results are bit-reproducible), hands the carried-in
+//                state to pass 2 and publishes the tile's inclusive prefix.
 //   producer     claims tiles in order from a per-(head, half) ticket counter,
 //                TMA-loads the GELU-branch tile, issues the MMAs.
 // Every wait is bounded: a wait that runs out records RGLRU_ERR_TIMEOUT in the
@@ -68,7 +70,7 @@ constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
 constexpr int OFF_BAR = OFF_INFO + SLOTS * 32;
 enum { BAR_INFO, BAR_CONV, BAR_MMA, BAR_PASS1, BAR_LB, BAR_G, BAR_FREE, BAR_KINDS };
 constexpr int OFF_MISC = OFF_BAR + BAR_KINDS * SLOTS * 8;
-constexpr int kSmemUsed = OFF_MISC + 16;
+constexpr int kSmemUsed = OFF_MISC + 16 + SLOTS * 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
@@ -210,8 +212,8 @@ __device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_
                 anchor_flag = __shfl_sync(0xffffffffu, f, la);
                 return true;
             }
-        } else if (ready == 0xffffffffu) {
-            hi -= 32;  // 32 aggregates, no anchor yet: look further back
+        } else if (ready == 0xffffffffu && hi - 31 > seq_first) {
+            hi -= 32;  // 32 aggregates, no anchor yet, the sequence start not reached: look further back
             continue;
         }
         if (t0 == 0) t0 = globaltimer();
@@ -281,6 +283,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     auto bar = [&](int kind, int s) { return bars + kind * SLOTS + s; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    int *agg_count = reinterpret_cast<int *>(smem + OFF_MISC + 16);  // per slot: scan warps done with pass 1
     WsHeader *hdr = p.hdr;
 
     // ------------------------------------------------------------------ setup
@@ -297,6 +300,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 mbar_init(bar(BAR_FREE, s), kScanWarps * 32);
             }
             *abort_flag = 0;
+            for (int s = 0; s < SLOTS; ++s) agg_count[s] = 0;
             mbar_fence_init();
         }
     }
@@ -543,7 +547,27 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             tmem_st32(col, ar);
             tmem_st32(col + NT, ai);
             tmem_wait_st();
-            reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = make_float2(P, hl);
+            const float2 agg = make_float2(P, hl);
+            reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = agg;
+            // Publish the tile aggregate right away (decoupled look-back): later
+            // tiles of the sequence may combine it before this tile's own
+            // look-back has finished.
+            const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
+            const bool suppress = (int)gu == debug_unit;
+            if (!suppress) {
+                p.agg[gu * kHalf + c] = agg;
+                __threadfence();
+            }
+            // the last scan warp to finish publishes the flag; nobody waits here
+            __syncwarp();
+            if (lane == 0) {
+                const int prev = atomicAdd(agg_count + s, 1);
+                if (prev == kScanWarps - 1) {
+                    agg_count[s] = 0;
+                    __threadfence();
+                    if (!suppress) st_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
+                }
+            }
             mbar_arrive(bar(BAR_PASS1, s));
             return true;
         };
@@ -630,14 +654,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
             const uint32_t rbit = ti.reset_mask ? F_RESET : 0u;
             const bool suppress = (int)gu == debug_unit;
-            if (!suppress) {
-                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf + ch);
-                dst[0] = g01;
-                dst[1] = g23;
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release_u32(p.flags + gu, F_AGG | rbit);
-            }
             float hin[4];
             bool ok = true;
             if (ti.first) {

@@ -43,9 +43,14 @@ def to_device(inp: dict, io: str, device="cuda") -> dict:
 
 
 def run_gpu(dev: dict, simt: bool = False, workspace=None):
+    """Run the library on device inputs; fails if the device status is not OK."""
+    x = dev["x"]
+    if workspace is None:
+        workspace = api.new_workspace(api.workspace_size(*x.shape, x.dtype, simt=simt), x.device)
     y = api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"],
                     dev["h_state"], workspace=workspace, simt=simt)
-    torch.cuda.synchronize()
+    st = api.device_status(workspace)
+    assert st == api.OK, f"device status {api.status_string(st)}"
     return {"y": y.float().cpu().numpy(), "conv_state": dev["conv_state"].float().cpu().numpy(),
             "h_state": dev["h_state"].cpu().numpy()}
 
