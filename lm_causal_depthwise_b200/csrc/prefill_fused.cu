@@ -48,9 +48,10 @@ constexpr int NT = 32;       // tokens per tile (MMA N)
 constexpr int SLOTS = 4;     // tiles in flight per CTA
 constexpr int LAG = 2;       // pass 2 runs this many tiles behind pass 1
 constexpr int kHalf = 128;   // output channels per CTA (MMA M, TMEM lanes)
+constexpr int INFO_RING = 8; // tile descriptors in flight (claimed ahead)
 constexpr int kScanWarps = 4, kConvWarps = 4;
-constexpr int kProdWarp = 8, kLbWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8, kLbWarp = 9, kSchedWarp = 10;
+constexpr int kThreads = 352;
 
 // TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
 // [pre_r | pre_i] accumulators that pass 1 overwrites with [a | v].
@@ -67,9 +68,11 @@ constexpr int OFF_G = OFF_XCS + SLOTS * kXcsTile;
 constexpr int OFF_AGG = OFF_G + SLOTS * kGTile;
 constexpr int OFF_HIN = OFF_AGG + SLOTS * kHalf * 8;
 constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
-constexpr int OFF_BAR = OFF_INFO + SLOTS * 32;
-enum { BAR_INFO, BAR_CONV, BAR_MMA, BAR_PASS1, BAR_LB, BAR_G, BAR_FREE, BAR_KINDS };
-constexpr int OFF_MISC = OFF_BAR + BAR_KINDS * SLOTS * 8;
+constexpr int OFF_BAR = OFF_INFO + INFO_RING * 32;
+// per-slot barriers (slot = tile % SLOTS)
+enum { BAR_CONV, BAR_SMEM_FREE, BAR_MMA, BAR_TMEM_FREE, BAR_PASS1, BAR_LB, BAR_G, BAR_KINDS };
+constexpr int OFF_RING_BAR = OFF_BAR + BAR_KINDS * SLOTS * 8;  // INFO_FULL[8], INFO_EMPTY[8]
+constexpr int OFF_MISC = OFF_RING_BAR + 2 * INFO_RING * 8;
 constexpr int kSmemUsed = OFF_MISC + 16 + SLOTS * 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -83,6 +86,7 @@ struct TileInfo {
     int first, last, pad;
 };
 static_assert(sizeof(TileInfo) == 32, "TileInfo size");
+static_assert(SLOTS * 2 == INFO_RING, "ring sizes");
 
 struct FusedParams {
     int B, T, D, C, G, tiles_per_group;
@@ -280,24 +284,31 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     const int head = group >> 1, half = group & 1;
     TileInfo *info = reinterpret_cast<TileInfo *>(smem + OFF_INFO);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *ring_bars = reinterpret_cast<uint64_t *>(smem + OFF_RING_BAR);
     auto bar = [&](int kind, int s) { return bars + kind * SLOTS + s; };
+    auto info_full = [&](int i) { return ring_bars + i; };
+    auto info_empty = [&](int i) { return ring_bars + INFO_RING + i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
     int *agg_count = reinterpret_cast<int *>(smem + OFF_MISC + 16);  // per slot: scan warps done with pass 1
     WsHeader *hdr = p.hdr;
 
     // ------------------------------------------------------------------ setup
-    if (warp == kProdWarp) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_holder, 512);
         if (lane == 0) {
             for (int s = 0; s < SLOTS; ++s) {
-                mbar_init(bar(BAR_INFO, s), 1);
                 mbar_init(bar(BAR_CONV, s), kConvWarps * 32);
+                mbar_init(bar(BAR_SMEM_FREE, s), kScanWarps * 32);
                 mbar_init(bar(BAR_MMA, s), 1);
+                mbar_init(bar(BAR_TMEM_FREE, s), kScanWarps * 32);
                 mbar_init(bar(BAR_PASS1, s), kScanWarps * 32);
                 mbar_init(bar(BAR_LB, s), 32);
                 mbar_init(bar(BAR_G, s), 1);
-                mbar_init(bar(BAR_FREE, s), kScanWarps * 32);
+            }
+            for (int i = 0; i < INFO_RING; ++i) {
+                mbar_init(info_full(i), 1);
+                mbar_init(info_empty(i), kScanWarps * 32);
             }
             *abort_flag = 0;
             for (int s = 0; s < SLOTS; ++s) agg_count[s] = 0;
@@ -339,18 +350,14 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 
     const int debug_unit = *(volatile int *)&hdr->debug_unit_plus1 - 1;
 
-    if (warp == kProdWarp) {
-        // ------------------------------------------------------------ producer / MMA issuer
-        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
-        int issued = 0;  // tiles whose TMA and MMAs were issued
-#pragma unroll 1
-        for (int j = 0;; ++j) {
-            const int s = j % SLOTS;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            bool ok = true;
-            if (j >= SLOTS) ok = warp_wait_bar(bar(BAR_FREE, s), ph ^ 1u, abort_flag, hdr, 1);
+    if (warp == kSchedWarp) {
+        // ------------------------------------------------------------ scheduler
+        // Claims tiles in order from this group's ticket counter, one tile ahead
+        // of the ring, so that the atomic and the segment_pos read overlap the
+        // wait for a free ring entry.
+        auto claim = [&]() -> TileInfo {
             int u = -1;
-            if (lane == 0 && ok && !*abort_flag) {
+            if (lane == 0 && !*abort_flag) {
                 u = (int)atomicAdd(&hdr->ticket[group], 1u);
                 if (u >= p.tiles_per_group) u = -1;
             }
@@ -364,25 +371,45 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 ti.valid = min(NT, p.T - ti.t0);
                 ti.first = c == 0;
                 ti.last = c == p.C - 1;
-                const int t = ti.t0 + lane;
-                const int sp = lane < ti.valid ? p.segpos[(size_t)ti.b * p.T + t] : 1;
+                const int sp = lane < ti.valid ? p.segpos[(size_t)ti.b * p.T + ti.t0 + lane] : 1;
                 ti.reset_mask = __ballot_sync(0xffffffffu, sp == 0);
             }
+            return ti;
+        };
+        TileInfo next = claim();
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int ir = j % INFO_RING;
+            bool ok = true;
+            if (j >= INFO_RING)
+                ok = warp_wait_bar(info_empty(ir), (uint32_t)((j / INFO_RING) - 1) & 1u, abort_flag, hdr, 1);
+            if (!ok) next.u = -1;
             if (lane == 0) {
-                info[s] = ti;
-                mbar_arrive(bar(BAR_INFO, s));
+                info[ir] = next;
+                mbar_arrive(info_full(ir));
             }
-            if (u < 0) break;
+            if (next.u < 0) break;
+            next = claim();
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer (+ GELU-branch TMA)
+        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
+        int issued = 0;
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS, ir = j % INFO_RING;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 2)) break;
+            const TileInfo ti = info[ir];
+            if (ti.u < 0) break;
+            if (j >= SLOTS && !warp_wait_bar(bar(BAR_TMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 3)) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(BAR_G, s), kGTile);
                 tma_load_3d(smem + OFF_G + s * kGTile, &tmap_g, bar(BAR_G, s), head * 256 + half * kHalf, ti.t0,
                             ti.b);
             }
             ++issued;
-            if (!warp_wait_bar(bar(BAR_CONV, s), ph, abort_flag, hdr, 2)) {
-                // the TMA is in flight; the MMAs of this tile were never issued
-                break;
-            }
+            if (!warp_wait_bar(bar(BAR_CONV, s), ph, abort_flag, hdr, 4)) break;
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t b_base = smem_u32(smem + OFF_B + s * kBTile);
@@ -398,8 +425,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             __syncwarp();
         }
-        // drain: this thread's last commit covers every MMA it issued; each slot's
-        // last TMA load is waited on (bounded) so that nothing lands after exit.
+        // on abort, wait (bounded) for this CTA's copies and MMAs in flight
         if (lane == 0 && *abort_flag) {
             for (int k = max(0, issued - SLOTS); k < issued; ++k) {
                 const int s = k % SLOTS;
@@ -430,14 +456,15 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const int xcs_col = (kb & 1) * 64 + cg * 8;
 #pragma unroll 1
         for (int j = 0;; ++j) {
-            const int s = j % SLOTS;
+            const int s = j % SLOTS, ir = j % INFO_RING;
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(bar(BAR_INFO, s), ph, abort_flag, hdr, 3)) break;
-            const TileInfo ti = info[s];
+            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 5)) break;
+            const TileInfo ti = info[ir];
             if (ti.u < 0) break;
             const int n0 = q * 8;
             const int tb = ti.t0 + n0;
             const size_t rowB = (size_t)ti.b * p.T;
+            // loads first (registers), then wait for the slot's shared memory
             uint4 raw[11];
             int pos[8];
 #pragma unroll
@@ -454,6 +481,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 const int t = tb + i;
                 pos[i] = t < p.T ? p.segpos[rowB + t] : 0;
             }
+            if (j >= SLOTS && !warp_wait_bar(bar(BAR_SMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
             float xm3[8], xm2[8], xm1[8];
             unpack8(raw[0], xm3);
             unpack8(raw[1], xm2);
@@ -511,8 +539,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         auto pass1 = [&](int j) -> bool {
             const int s = j % SLOTS;
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            const TileInfo ti = info[s];
-            if (!warp_wait_bar(bar(BAR_MMA, s), ph, abort_flag, hdr, 4)) return false;
+            const TileInfo ti = info[j % INFO_RING];
+            if (!warp_wait_bar(bar(BAR_MMA, s), ph, abort_flag, hdr, 7)) return false;
             tc_fence_after();
             uint32_t ar[32], ai[32];
             const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
@@ -544,6 +572,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 ar[t] = __float_as_uint(a);
                 ai[t] = __float_as_uint(v);
             }
+            mbar_arrive(bar(BAR_SMEM_FREE, s));  // xcs (and, via the MMA wait, the B tile) consumed
             tmem_st32(col, ar);
             tmem_st32(col + NT, ai);
             tmem_wait_st();
@@ -551,14 +580,14 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = agg;
             // Publish the tile aggregate right away (decoupled look-back): later
             // tiles of the sequence may combine it before this tile's own
-            // look-back has finished.
+            // look-back has finished.  The last scan warp to get here sets the
+            // flag; nobody waits.
             const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
             const bool suppress = (int)gu == debug_unit;
             if (!suppress) {
                 p.agg[gu * kHalf + c] = agg;
                 __threadfence();
             }
-            // the last scan warp to finish publishes the flag; nobody waits here
             __syncwarp();
             if (lane == 0) {
                 const int prev = atomicAdd(agg_count + s, 1);
@@ -573,12 +602,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         };
 
         auto pass2 = [&](int j) -> bool {
-            const int s = j % SLOTS;
+            const int s = j % SLOTS, ir = j % INFO_RING;
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            const TileInfo ti = info[s];
-            if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 5)) return false;
+            const TileInfo ti = info[ir];
+            if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 8)) return false;
             float h = reinterpret_cast<const float *>(smem + OFF_HIN + s * kHalf * 4)[c];
-            if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 6)) return false;
+            if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 9)) return false;
             tc_fence_after();
             uint32_t aa[32], vv[32];
             const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
@@ -602,8 +631,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 const size_t u0 = (size_t)ti.b * p.C;
                 const uint32_t *f_own = p.flags + (size_t)group * p.tiles_per_group + u0;
                 const uint32_t *f_oth = p.flags + (size_t)(group ^ 1) * p.tiles_per_group + u0;
-                if (warp_wait_flag(f_own, F_PREFIX, abort_flag, hdr, 7) == 0) return false;
-                if (warp_wait_flag(f_oth, F_AGG, abort_flag, hdr, 8) == 0) return false;
+                if (warp_wait_flag(f_own, F_PREFIX, abort_flag, hdr, 10) == 0) return false;
+                if (warp_wait_flag(f_oth, F_AGG, abort_flag, hdr, 11) == 0) return false;
                 p.h_state[(size_t)ti.b * p.D + d] = h;
                 __nv_bfloat16 ncs[3];
 #pragma unroll
@@ -616,16 +645,16 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 for (int k = 0; k < 3; ++k) p.conv_state[((size_t)ti.b * 3 + k) * p.D + d] = ncs[k];
             }
             tc_fence_before();
-            mbar_arrive(bar(BAR_FREE, s));
+            mbar_arrive(bar(BAR_TMEM_FREE, s));
+            mbar_arrive(info_empty(ir));
             return true;
         };
 
 #pragma unroll 1
         for (int j = 0;; ++j) {
-            const int s = j % SLOTS;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            bool end = !warp_wait_bar(bar(BAR_INFO, s), ph, abort_flag, hdr, 9);
-            if (!end) end = info[s].u < 0;
+            const int ir = j % INFO_RING;
+            bool end = !warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 12);
+            if (!end) end = info[ir].u < 0;
             bool ok = true;
             if (!end) ok = pass1(j);
             if (ok && j >= LAG) ok = pass2(j - LAG);
@@ -641,12 +670,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const size_t dch = (size_t)head * 256 + half * kHalf + ch;
 #pragma unroll 1
         for (int j = 0;; ++j) {
-            const int s = j % SLOTS;
+            const int s = j % SLOTS, ir = j % INFO_RING;
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(bar(BAR_INFO, s), ph, abort_flag, hdr, 10)) break;
-            const TileInfo ti = info[s];
+            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 13)) break;
+            const TileInfo ti = info[ir];
             if (ti.u < 0) break;
-            if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 11)) break;
+            if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 14)) break;
             const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
             const float4 g01 = sagg[lane * 2], g23 = sagg[lane * 2 + 1];  // (A,H) of 4 channels
             const float A[4] = {g01.x, g01.z, g23.x, g23.z};
@@ -680,20 +709,20 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     for (int p0 = anchor + 1; p0 < ti.u; p0 += 8) {
                         float4 dd[8][2];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            if (p0 + q < ti.u) {
-                                const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + p0 + q) * kHalf + ch);
-                                dd[q][0] = ld_relaxed_f4(src);
-                                dd[q][1] = ld_relaxed_f4(src + 1);
+                        for (int k = 0; k < 8; ++k) {
+                            if (p0 + k < ti.u) {
+                                const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + p0 + k) * kHalf + ch);
+                                dd[k][0] = ld_relaxed_f4(src);
+                                dd[k][1] = ld_relaxed_f4(src + 1);
                             }
                         }
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            if (p0 + q < ti.u) {
-                                hin[0] = fmaf(dd[q][0].x, hin[0], dd[q][0].y);
-                                hin[1] = fmaf(dd[q][0].z, hin[1], dd[q][0].w);
-                                hin[2] = fmaf(dd[q][1].x, hin[2], dd[q][1].y);
-                                hin[3] = fmaf(dd[q][1].z, hin[3], dd[q][1].w);
+                        for (int k = 0; k < 8; ++k) {
+                            if (p0 + k < ti.u) {
+                                hin[0] = fmaf(dd[k][0].x, hin[0], dd[k][0].y);
+                                hin[1] = fmaf(dd[k][0].z, hin[1], dd[k][0].w);
+                                hin[2] = fmaf(dd[k][1].x, hin[2], dd[k][1].y);
+                                hin[3] = fmaf(dd[k][1].z, hin[3], dd[k][1].w);
                             }
                         }
                     }
@@ -719,7 +748,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kProdWarp) tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- host side
