@@ -49,28 +49,41 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and up_to_date():
+TRACE_LIB = os.path.join(PKG, "librglru_trace.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str = LIB) -> str:
+    """Compile every csrc/*.cu for sm_100a and link ``out``.  ``build_trace()``
+    makes the per-role timeline variant (-DRGLRU_TRACE) used for kernel studies."""
+    if not force and up_to_date() and out == LIB:
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
     objs = []
+    tag = "" if out == LIB else os.path.splitext(os.path.basename(out))[0] + "."
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(BUILD_DIR, tag + os.path.basename(src) + ".o")
         cmd = [_nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
            "-Xcompiler", "-fPIC"]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
+
+
+def build_trace(verbose: bool = False) -> str:
+    return build(force=True, verbose=verbose, extra_flags=("-DRGLRU_TRACE",), out=TRACE_LIB)
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    if "--trace" in sys.argv:
+        print(build_trace(verbose=True))
+    else:
+        build(force="--force" in sys.argv, verbose=True)
+        print(LIB)

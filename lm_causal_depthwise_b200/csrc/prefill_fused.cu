@@ -46,12 +46,14 @@ using namespace sm100;
 
 constexpr int NT = 32;       // tokens per tile (MMA N)
 constexpr int SLOTS = 4;     // tiles in flight per CTA
-constexpr int LAG = 2;       // pass 2 runs this many tiles behind pass 1
 constexpr int kHalf = 128;   // output channels per CTA (MMA M, TMEM lanes)
 constexpr int INFO_RING = 8; // tile descriptors in flight (claimed ahead)
-constexpr int kScanWarps = 4, kConvWarps = 4;
-constexpr int kMmaWarp = 8, kLbWarp = 9, kSchedWarp = 10;
-constexpr int kThreads = 352;
+constexpr int kScanGroups = 2;  // scan warp groups, alternate tiles
+constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
+constexpr int kConvWarp0 = kScanWarps;
+constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kLbWarp = kMmaWarp + 1, kSchedWarp = kMmaWarp + 2;
+constexpr int kThreads = 32 * (kSchedWarp + 1);
+constexpr int kGroupThreads = 128;  // threads of one scan group (one per channel)
 
 // TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
 // [pre_r | pre_i] accumulators that pass 1 overwrites with [a | v].
@@ -104,7 +106,28 @@ struct FusedParams {
     uint32_t *flags;   // [G][tiles_per_group]
     float2 *agg;       // [G][tiles_per_group][128]  (prod a, h_end) from h = 0
     float *prefix;     // [G][tiles_per_group][128]  h after the tile
+    unsigned long long *trace;  // RGLRU_TRACE builds only: per-role timestamps
 };
+
+// Tracing (compiled in with -DRGLRU_TRACE only): CTAs below kTraceCtas record
+// %globaltimer at each role's milestones for their first kTraceTiles tiles,
+// into trace[(cta * kTraceTiles + tile) * kTraceEvents + event].
+enum TraceEvent {
+    TR_SCHED_INFO, TR_CONV_START, TR_CONV_DONE, TR_MMA_ISSUED, TR_P1_START, TR_P1_END, TR_LB_START,
+    TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, kTraceEvents
+};
+constexpr int kTraceCtas = 4, kTraceTiles = 128;
+#ifdef RGLRU_TRACE
+#define RGLRU_TR(ev, j, val)                                                                                   \
+    do {                                                                                                      \
+        if (p.trace != nullptr && blockIdx.x < kTraceCtas && (j) < kTraceTiles)                               \
+            p.trace[((size_t)blockIdx.x * kTraceTiles + (j)) * kTraceEvents + (ev)] = (val);                  \
+    } while (0)
+#else
+#define RGLRU_TR(ev, j, val) \
+    do {                     \
+    } while (0)
+#endif
 
 constexpr uint32_t F_AGG = 1u, F_PREFIX = 2u, F_RESET = 4u;
 
@@ -123,6 +146,7 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile i
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(it < 16 ? 16 : 64);
         if ((it & 63u) == 0) {
             if (*abort_flag) return false;
             if (*(volatile int *)&hdr->status != 0) {
@@ -299,16 +323,16 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         if (lane == 0) {
             for (int s = 0; s < SLOTS; ++s) {
                 mbar_init(bar(BAR_CONV, s), kConvWarps * 32);
-                mbar_init(bar(BAR_SMEM_FREE, s), kScanWarps * 32);
+                mbar_init(bar(BAR_SMEM_FREE, s), kGroupThreads);
                 mbar_init(bar(BAR_MMA, s), 1);
-                mbar_init(bar(BAR_TMEM_FREE, s), kScanWarps * 32);
-                mbar_init(bar(BAR_PASS1, s), kScanWarps * 32);
+                mbar_init(bar(BAR_TMEM_FREE, s), kGroupThreads);
+                mbar_init(bar(BAR_PASS1, s), kGroupThreads);
                 mbar_init(bar(BAR_LB, s), 32);
                 mbar_init(bar(BAR_G, s), 1);
             }
             for (int i = 0; i < INFO_RING; ++i) {
                 mbar_init(info_full(i), 1);
-                mbar_init(info_empty(i), kScanWarps * 32);
+                mbar_init(info_empty(i), kGroupThreads);
             }
             *abort_flag = 0;
             for (int s = 0; s < SLOTS; ++s) agg_count[s] = 0;
@@ -321,12 +345,13 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     const uint32_t tmem = *tmem_holder;
 
     if (warp < kScanWarps) {
-        // this thread's TMEM lane = output channel c of the half: rows of W_a and W_x
-        const int c = threadIdx.x;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // TMEM lane = output channel c of the half; scan group g loads the rows
+        // of gate g (W_a, W_x) for its channel
+        const int c = threadIdx.x % kGroupThreads;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const size_t row = (size_t)head * 256 + half * kHalf + c;
 #pragma unroll 1
-        for (int gate = 0; gate < 2; ++gate) {
+        for (int gate = warp / 4; gate < 2; gate += kScanGroups) {
             const uint4 *src = reinterpret_cast<const uint4 *>((gate == 0 ? p.W_a : p.W_x) + row * 256);
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
@@ -377,6 +402,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             return ti;
         };
         TileInfo next = claim();
+        int ends = 0;  // end markers written: one per scan group (each reads its own tiles)
 #pragma unroll 1
         for (int j = 0;; ++j) {
             const int ir = j % INFO_RING;
@@ -387,8 +413,13 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (lane == 0) {
                 info[ir] = next;
                 mbar_arrive(info_full(ir));
+                RGLRU_TR(TR_SCHED_INFO, j, globaltimer());
+                RGLRU_TR(TR_TILE_U, j, (unsigned long long)(unsigned)next.u);
             }
-            if (next.u < 0) break;
+            if (next.u < 0) {
+                if (++ends == kScanGroups || !ok) break;
+                continue;
+            }
             next = claim();
         }
     } else if (warp == kMmaWarp) {
@@ -422,6 +453,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     umma_ts(d_i, tmem + kColWx + kk * 8, bd, idesc, kk > 0);
                 }
                 umma_commit(bar(BAR_MMA, s));
+                RGLRU_TR(TR_MMA_ISSUED, j, globaltimer());
             }
             __syncwarp();
         }
@@ -438,9 +470,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 }
             }
         }
-    } else if (warp >= kScanWarps && warp < kScanWarps + kConvWarps) {
+    } else if (warp >= kConvWarp0 && warp < kConvWarp0 + kConvWarps) {
         // ------------------------------------------------------------ conv warps
-        const int kb = warp - kScanWarps;  // K-block: channels [64 kb, 64 kb + 64) of the head
+        const int kb = warp - kConvWarp0;  // K-block: channels [64 kb, 64 kb + 64) of the head
         const int cg = lane & 7;           // 8 channels per lane
         const int q = lane >> 3;           // token quarter of the tile
         const int dl = kb * 64 + cg * 8;   // channel within the head
@@ -461,6 +493,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 5)) break;
             const TileInfo ti = info[ir];
             if (ti.u < 0) break;
+            if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_START, j, globaltimer());
             const int n0 = q * 8;
             const int tb = ti.t0 + n0;
             const size_t rowB = (size_t)ti.b * p.T;
@@ -524,12 +557,14 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(BAR_CONV, s));
+            if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_DONE, j, globaltimer());
         }
     } else if (warp < kScanWarps) {
         // ------------------------------------------------------------ scan warps
-        const int c = threadIdx.x;
+        const int sg = warp / 4;                 // scan group: tiles j with j % kScanGroups == sg
+        const int c = threadIdx.x % kGroupThreads;
         const int d = head * 256 + half * kHalf + c;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float ba = p.b_a[d], bx = p.b_x[d];
         const float lam = p.lambda[d];
         const float ls = lam >= 0.f ? -log1pf(expf(-lam)) : lam - log1pf(expf(lam));  // log sigmoid(Lambda)
@@ -541,47 +576,52 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
             const TileInfo ti = info[j % INFO_RING];
             if (!warp_wait_bar(bar(BAR_MMA, s), ph, abort_flag, hdr, 7)) return false;
+            if (c == 0) RGLRU_TR(TR_P1_START, j, globaltimer());
             tc_fence_after();
-            uint32_t ar[32], ai[32];
             const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
-            tmem_ld32(col, ar);
-            tmem_ld32(col + NT, ai);
-            tmem_wait_ld();
             const float *xcs = reinterpret_cast<const float *>(smem + OFF_XCS + s * kXcsTile);
             float hl = 0.f, P = 1.f;
+#pragma unroll 1
+            for (int t8 = 0; t8 < NT; t8 += 8) {
+                uint32_t ar[8], ai[8];
+                tmem_ld8(col + t8, ar);
+                tmem_ld8(col + NT + t8, ai);
+                tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const float xc = xcs[t * kHalf + c];
-                const float r = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ar[t]) + ba)), 0.5f);
-                const float ig = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ai[t]) + bx)), 0.5f);
-                const float ell = r * kl;
-                float a = ex2_approx(r * kl2);
-                const float om = ell > -0.125f ? one_minus_exp2l_small(ell) : fmaf(-a, a, 1.f);
-                const float uu = ig * xc;
-                float v = sqrt_approx(om) * uu;
-                if ((ti.reset_mask >> t) & 1u) {
-                    a = 0.f;
-                    v = uu;
+                for (int k = 0; k < 8; ++k) {
+                    const int t = t8 + k;
+                    const float xc = xcs[t * kHalf + c];
+                    const float r = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ar[k]) + ba)), 0.5f);
+                    const float ig = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ai[k]) + bx)), 0.5f);
+                    const float ell = r * kl;
+                    float a = ex2_approx(r * kl2);
+                    const float om = ell > -0.125f ? one_minus_exp2l_small(ell) : fmaf(-a, a, 1.f);
+                    const float uu = ig * xc;
+                    float v = sqrt_approx(om) * uu;
+                    if ((ti.reset_mask >> t) & 1u) {
+                        a = 0.f;
+                        v = uu;
+                    }
+                    if (t >= ti.valid) {
+                        a = 1.f;
+                        v = 0.f;
+                    }
+                    hl = fmaf(a, hl, v);
+                    P *= a;
+                    ar[k] = __float_as_uint(a);
+                    ai[k] = __float_as_uint(v);
                 }
-                if (t >= ti.valid) {
-                    a = 1.f;
-                    v = 0.f;
-                }
-                hl = fmaf(a, hl, v);
-                P *= a;
-                ar[t] = __float_as_uint(a);
-                ai[t] = __float_as_uint(v);
+                tmem_st8(col + t8, ar);
+                tmem_st8(col + NT + t8, ai);
             }
             mbar_arrive(bar(BAR_SMEM_FREE, s));  // xcs (and, via the MMA wait, the B tile) consumed
-            tmem_st32(col, ar);
-            tmem_st32(col + NT, ai);
             tmem_wait_st();
             const float2 agg = make_float2(P, hl);
             reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = agg;
             // Publish the tile aggregate right away (decoupled look-back): later
             // tiles of the sequence may combine it before this tile's own
-            // look-back has finished.  The last scan warp to get here sets the
-            // flag; nobody waits.
+            // look-back has finished.  The last warp of the group to get here
+            // sets the flag; nobody waits.
             const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
             const bool suppress = (int)gu == debug_unit;
             if (!suppress) {
@@ -591,13 +631,14 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             __syncwarp();
             if (lane == 0) {
                 const int prev = atomicAdd(agg_count + s, 1);
-                if (prev == kScanWarps - 1) {
+                if (prev == 3) {
                     agg_count[s] = 0;
                     __threadfence();
                     if (!suppress) st_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
                 }
             }
             mbar_arrive(bar(BAR_PASS1, s));
+            if (c == 0) RGLRU_TR(TR_P1_END, j, globaltimer());
             return true;
         };
 
@@ -608,20 +649,25 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 8)) return false;
             float h = reinterpret_cast<const float *>(smem + OFF_HIN + s * kHalf * 4)[c];
             if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 9)) return false;
+            if (c == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
             tc_fence_after();
-            uint32_t aa[32], vv[32];
             const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
-            tmem_ld32(col, aa);
-            tmem_ld32(col + NT, vv);
-            tmem_wait_ld();
             const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile);
             __nv_bfloat16 *yp = p.y + ((size_t)ti.b * p.T + ti.t0) * p.D + d;
+#pragma unroll 1
+            for (int t8 = 0; t8 < NT; t8 += 8) {
+                uint32_t aa[8], vv[8];
+                tmem_ld8(col + t8, aa);
+                tmem_ld8(col + NT + t8, vv);
+                tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                h = fmaf(__uint_as_float(aa[t]), h, __uint_as_float(vv[t]));
-                if (t < ti.valid) {
-                    const float gv = __bfloat162float(gs[t * kHalf + c]);
-                    yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                for (int k = 0; k < 8; ++k) {
+                    const int t = t8 + k;
+                    h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
+                    if (t < ti.valid) {
+                        const float gv = __bfloat162float(gs[t * kHalf + c]);
+                        yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                    }
                 }
             }
             if (ti.last) {
@@ -647,22 +693,21 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             tc_fence_before();
             mbar_arrive(bar(BAR_TMEM_FREE, s));
             mbar_arrive(info_empty(ir));
+            if (c == 0) RGLRU_TR(TR_P2_END, j, globaltimer());
             return true;
         };
 
+        // this group's tiles: j = sg, sg + kScanGroups, ...; pass 2 of a tile runs
+        // after pass 1 of the group's next tile (the look-back has that long)
 #pragma unroll 1
-        for (int j = 0;; ++j) {
+        for (int j = sg;; j += kScanGroups) {
             const int ir = j % INFO_RING;
             bool end = !warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 12);
             if (!end) end = info[ir].u < 0;
             bool ok = true;
             if (!end) ok = pass1(j);
-            if (ok && j >= LAG) ok = pass2(j - LAG);
-            if (!ok) break;
-            if (end) {
-                for (int k = max(0, j - LAG + 1); k < j && ok; ++k) ok = pass2(k);
-                break;
-            }
+            if (ok && j >= kScanGroups) ok = pass2(j - kScanGroups);
+            if (!ok || end) break;
         }
     } else if (warp == kLbWarp) {
         // ------------------------------------------------------------ look-back warp
@@ -676,6 +721,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const TileInfo ti = info[ir];
             if (ti.u < 0) break;
             if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 14)) break;
+            if (lane == 0) RGLRU_TR(TR_LB_START, j, globaltimer());
             const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
             const float4 g01 = sagg[lane * 2], g23 = sagg[lane * 2 + 1];  // (A,H) of 4 channels
             const float A[4] = {g01.x, g01.z, g23.x, g23.z};
@@ -729,6 +775,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 }
             }
             if (!ok) break;
+            if (lane == 0) RGLRU_TR(TR_LB_HIN, j, globaltimer());
             float pre[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
@@ -741,6 +788,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             *reinterpret_cast<float4 *>(smem + OFF_HIN + s * kHalf * 4 + ch * 4) =
                 make_float4(hin[0], hin[1], hin[2], hin[3]);
             mbar_arrive(bar(BAR_LB, s));
+            if (lane == 0) RGLRU_TR(TR_LB_DONE, j, globaltimer());
         }
     }
 
@@ -769,7 +817,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 struct Layout {
     int C, G, tpg;
-    size_t flags_off, flags_bytes, agg_off, prefix_off, total;
+    size_t flags_off, flags_bytes, agg_off, prefix_off, trace_off, total;
 };
 
 Layout layout_of(int B, int T, int D)
@@ -784,6 +832,12 @@ Layout layout_of(int B, int T, int D)
     L.agg_off = L.flags_off + L.flags_bytes;
     L.prefix_off = L.agg_off + align_up(tiles * kHalf * 8, 256);
     L.total = L.prefix_off + align_up(tiles * kHalf * 4, 256);
+#ifdef RGLRU_TRACE
+    L.trace_off = L.total;
+    L.total += align_up((size_t)kTraceCtas * kTraceTiles * kTraceEvents * 8, 256);
+#else
+    L.trace_off = 0;
+#endif
     return L;
 }
 
@@ -840,6 +894,7 @@ rglru_status fused_prefill(const PrefillArgs &a)
     p.flags = reinterpret_cast<uint32_t *>(ws + L.flags_off);
     p.agg = reinterpret_cast<float2 *>(ws + L.agg_off);
     p.prefix = reinterpret_cast<float *>(ws + L.prefix_off);
+    p.trace = L.trace_off ? reinterpret_cast<unsigned long long *>(ws + L.trace_off) : nullptr;
 
     const int per_group = max(1, sms / L.G);
     const int grid = per_group * L.G;
