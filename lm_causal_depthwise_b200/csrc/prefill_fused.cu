@@ -64,17 +64,22 @@ constexpr int kBTile = NT * 256 * 2;            // bf16 xc, 4 K-blocks of 64 cha
 constexpr int kBBlock = NT * 128;               // one K-block: NT rows x 128 B
 constexpr int kXcsTile = NT * kHalf * 4;        // fp32 xc of this half
 constexpr int kGTile = NT * kHalf * 2;          // bf16 gate-branch tile (TMA box)
+constexpr int XRING = 3;                         // x tiles (32 rows + 3 halo rows) in flight
+constexpr int kXRows = NT + 3;
+constexpr int kXTile = kXRows * 256 * 2;         // bf16, all 256 channels of the head
 constexpr int OFF_B = 0;
 constexpr int OFF_XCS = OFF_B + SLOTS * kBTile;
 constexpr int OFF_G = OFF_XCS + SLOTS * kXcsTile;
-constexpr int OFF_AGG = OFF_G + SLOTS * kGTile;
+constexpr int OFF_X = OFF_G + SLOTS * kGTile;
+constexpr int OFF_AGG = OFF_X + XRING * kXTile;
 constexpr int OFF_HIN = OFF_AGG + SLOTS * kHalf * 8;
 constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
 constexpr int OFF_BAR = OFF_INFO + INFO_RING * 32;
 // per-slot barriers (slot = tile % SLOTS)
 enum { BAR_CONV, BAR_SMEM_FREE, BAR_MMA, BAR_TMEM_FREE, BAR_PASS1, BAR_LB, BAR_G, BAR_KINDS };
 constexpr int OFF_RING_BAR = OFF_BAR + BAR_KINDS * SLOTS * 8;  // INFO_FULL[8], INFO_EMPTY[8]
-constexpr int OFF_MISC = OFF_RING_BAR + 2 * INFO_RING * 8;
+constexpr int OFF_XBAR = OFF_RING_BAR + 2 * INFO_RING * 8;         // X_FULL[3], X_EMPTY[3]
+constexpr int OFF_MISC = OFF_XBAR + 2 * XRING * 8;
 constexpr int kSmemUsed = OFF_MISC + 16 + SLOTS * 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -84,8 +89,9 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 struct TileInfo {
     int u;        // tile index inside the (head, half) group, -1 = no more work
     int b, t0, valid;
-    uint32_t reset_mask;  // bit t: segment_pos == 0 at token t0 + t
-    int first, last, pad;
+    uint32_t reset_mask;  // bit t: segment_pos == 0 at token t0 + t (conv tap of lag 1 dropped, h reset)
+    uint32_t m2, m3;      // bit t: segment_pos < 2 (< 3): conv tap of lag 2 (3) dropped
+    int first_last;       // bit 0: first tile of the sequence, bit 1: last tile
 };
 static_assert(sizeof(TileInfo) == 32, "TileInfo size");
 static_assert(SLOTS * 2 == INFO_RING, "ring sizes");
@@ -299,7 +305,8 @@ __device__ __forceinline__ float gelu_tanh_fast(float g)
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap tmap_g)
+rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap tmap_g,
+                           const __grid_constant__ CUtensorMap tmap_x)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -312,6 +319,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     auto bar = [&](int kind, int s) { return bars + kind * SLOTS + s; };
     auto info_full = [&](int i) { return ring_bars + i; };
     auto info_empty = [&](int i) { return ring_bars + INFO_RING + i; };
+    uint64_t *xbars = reinterpret_cast<uint64_t *>(smem + OFF_XBAR);
+    auto x_full = [&](int i) { return xbars + i; };
+    auto x_empty = [&](int i) { return xbars + XRING + i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
     int *agg_count = reinterpret_cast<int *>(smem + OFF_MISC + 16);  // per slot: scan warps done with pass 1
@@ -333,6 +343,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             for (int i = 0; i < INFO_RING; ++i) {
                 mbar_init(info_full(i), 1);
                 mbar_init(info_empty(i), kGroupThreads);
+            }
+            for (int i = 0; i < XRING; ++i) {
+                mbar_init(x_full(i), 1);
+                mbar_init(x_empty(i), kConvWarps * 32);
             }
             *abort_flag = 0;
             for (int s = 0; s < SLOTS; ++s) agg_count[s] = 0;
@@ -394,15 +408,17 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 const int c = u % p.C;
                 ti.t0 = c * NT;
                 ti.valid = min(NT, p.T - ti.t0);
-                ti.first = c == 0;
-                ti.last = c == p.C - 1;
-                const int sp = lane < ti.valid ? p.segpos[(size_t)ti.b * p.T + ti.t0 + lane] : 1;
-                ti.reset_mask = __ballot_sync(0xffffffffu, sp == 0);
+                ti.first_last = (c == 0 ? 1 : 0) | (c == p.C - 1 ? 2 : 0);
+                const int sp = lane < ti.valid ? p.segpos[(size_t)ti.b * p.T + ti.t0 + lane] : 3;
+                ti.reset_mask = __ballot_sync(0xffffffffu, sp < 1);
+                ti.m2 = __ballot_sync(0xffffffffu, sp < 2);
+                ti.m3 = __ballot_sync(0xffffffffu, sp < 3);
             }
             return ti;
         };
         TileInfo next = claim();
-        int ends = 0;  // end markers written: one per scan group (each reads its own tiles)
+        int ends = 0;      // end markers written: one per scan group (each reads its own tiles)
+        int x_issued = 0;  // x-tile TMA loads issued
 #pragma unroll 1
         for (int j = 0;; ++j) {
             const int ir = j % INFO_RING;
@@ -420,7 +436,27 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 if (++ends == kScanGroups || !ok) break;
                 continue;
             }
+            // x rows t0-3 .. t0+31 of all 256 channels of the head into the x ring
+            // (rows before t = 0 arrive zero-filled; the conv reads conv_state there)
+            const int xr = j % XRING;
+            if (j >= XRING && !warp_wait_bar(x_empty(xr), (uint32_t)((j / XRING) - 1) & 1u, abort_flag, hdr, 15)) {
+                next.u = -1;
+                continue;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(x_full(xr), kXTile);
+                tma_load_3d(smem + OFF_X + xr * kXTile, &tmap_x, x_full(xr), head * 256, next.t0 - 3, next.b);
+            }
+            ++x_issued;
             next = claim();
+        }
+        // on abort, wait (bounded) for the x loads still in flight
+        if (lane == 0 && *abort_flag) {
+            for (int k = max(0, x_issued - XRING); k < x_issued; ++k) {
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(x_full(k % XRING), (uint32_t)(k / XRING) & 1u) && globaltimer() - t0 < kTimeoutNs) {
+                }
+            }
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (+ GELU-branch TMA)
@@ -494,46 +530,39 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const TileInfo ti = info[ir];
             if (ti.u < 0) break;
             if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_START, j, globaltimer());
-            const int n0 = q * 8;
-            const int tb = ti.t0 + n0;
-            const size_t rowB = (size_t)ti.b * p.T;
-            // loads first (registers), then wait for the slot's shared memory
-            uint4 raw[11];
-            int pos[8];
-#pragma unroll
-            for (int r = 0; r < 11; ++r) {
-                const int t = tb - 3 + r;
-                raw[r] = make_uint4(0, 0, 0, 0);
-                if (t >= 0 && t < p.T)
-                    raw[r] = *reinterpret_cast<const uint4 *>(p.x + (rowB + t) * p.D + d0);
-                else if (t < 0)
-                    raw[r] = *reinterpret_cast<const uint4 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + t) * p.D + d0);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = tb + i;
-                pos[i] = t < p.T ? p.segpos[rowB + t] : 0;
-            }
+            const int xr = j % XRING;
+            if (!warp_wait_bar(x_full(xr), (uint32_t)(j / XRING) & 1u, abort_flag, hdr, 16)) break;
             if (j >= SLOTS && !warp_wait_bar(bar(BAR_SMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
+            const int n0 = q * 8;
+            const uint8_t *xt = smem + OFF_X + xr * kXTile + dl * 2;  // row r = token t0 - 3 + r
+            auto xrow = [&](int r, float (&f)[8]) {
+                const int t = ti.t0 - 3 + r;
+                uint4 v;
+                if (t >= 0)
+                    v = *reinterpret_cast<const uint4 *>(xt + r * 512);
+                else
+                    v = *reinterpret_cast<const uint4 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + t) * p.D + d0);
+                unpack8(v, f);
+            };
             float xm3[8], xm2[8], xm1[8];
-            unpack8(raw[0], xm3);
-            unpack8(raw[1], xm2);
-            unpack8(raw[2], xm1);
+            xrow(n0, xm3);
+            xrow(n0 + 1, xm2);
+            xrow(n0 + 2, xm1);
             uint8_t *btile = smem + OFF_B + s * kBTile + kb * kBBlock;
             float *xcs = reinterpret_cast<float *>(smem + OFF_XCS + s * kXcsTile);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float x0[8];
-                unpack8(raw[3 + i], x0);
+                xrow(n0 + i + 3, x0);
                 const int n = n0 + i;
-                const int ps = pos[i];
+                const bool k1 = !((ti.reset_mask >> n) & 1u), k2 = !((ti.m2 >> n) & 1u), k3 = !((ti.m3 >> n) & 1u);
                 float xc[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     float acc = cb[e];
-                    if (ps >= 3) acc = fmaf(w[0][e], xm3[e], acc);
-                    if (ps >= 2) acc = fmaf(w[1][e], xm2[e], acc);
-                    if (ps >= 1) acc = fmaf(w[2][e], xm1[e], acc);
+                    if (k3) acc = fmaf(w[0][e], xm3[e], acc);
+                    if (k2) acc = fmaf(w[1][e], xm2[e], acc);
+                    if (k1) acc = fmaf(w[2][e], xm1[e], acc);
                     acc = fmaf(w[3][e], x0[e], acc);
                     xc[e] = n < ti.valid ? acc : 0.f;
                 }
@@ -555,6 +584,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     xm1[e] = x0[e];
                 }
             }
+            mbar_arrive(x_empty(xr));
             fence_proxy_async_smem();
             mbar_arrive(bar(BAR_CONV, s));
             if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_DONE, j, globaltimer());
@@ -670,7 +700,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     }
                 }
             }
-            if (ti.last) {
+            if (ti.first_last & 2) {
                 // The old states are read by the first tile of this sequence (its
                 // conv in both halves of the head, its look-back for h): wait until
                 // those reads are published before overwriting the states.
@@ -731,7 +761,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const bool suppress = (int)gu == debug_unit;
             float hin[4];
             bool ok = true;
-            if (ti.first) {
+            if (ti.first_last & 1) {
                 const float4 hs = *reinterpret_cast<const float4 *>(p.h_state + (size_t)ti.b * p.D + dch);
                 hin[0] = hs.x; hin[1] = hs.y; hin[2] = hs.z; hin[3] = hs.w;
             } else {
@@ -862,6 +892,12 @@ rglru_status fused_prefill(const PrefillArgs &a)
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RGLRU_ERR_CUDA;
+    CUtensorMap tmap_x;
+    const cuuint32_t xbox[3] = {256, kXRows, 1};
+    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.x), gdim, gstride, xbox, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RGLRU_ERR_CUDA;
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
@@ -898,7 +934,7 @@ rglru_status fused_prefill(const PrefillArgs &a)
 
     const int per_group = max(1, sms / L.G);
     const int grid = per_group * L.G;
-    rglru_prefill_fused_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(p, tmap);
+    rglru_prefill_fused_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(p, tmap, tmap_x);
     return cuda_status(cudaGetLastError());
 }
 
