@@ -62,7 +62,7 @@ constexpr uint32_t kColWa = 0, kColWx = 128, kColSlot0 = 256, kColPerSlot = 2 * 
 // Shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kBTile = NT * 256 * 2;            // bf16 xc, 4 K-blocks of 64 channels
 constexpr int kBBlock = NT * 128;               // one K-block: NT rows x 128 B
-constexpr int kXcsTile = NT * kHalf * 4;        // fp32 xc of this half
+constexpr int kXcsTile = NT * kHalf * 4;        // fp32 xc / 2 of this half
 constexpr int kGTile = NT * kHalf * 2;          // bf16 gate-branch tile (TMA box)
 constexpr int XRING = 3;                         // x tiles (32 rows + 3 halo rows) in flight
 constexpr int kXRows = NT + 3;
@@ -286,14 +286,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// -(exp(2l) - 1) for small |l| by its Taylor series: -2l (1 + l + 2/3 l^2 + 1/3 l^3 + 2/15 l^4)
+// 1 - exp(2l) = -(exp(2l) - 1) for -1/8 < l <= 0 by its Taylor series
+// -2l (1 + l + 2/3 l^2 + 1/3 l^3 + ...), cut after l^3: the first term left
+// out is 2/15 l^4, under 3.3e-5 relative for |l| < 1/8.
 __device__ __forceinline__ float one_minus_exp2l_small(float l)
 {
-    float s = fmaf(l, 2.f / 15.f, 1.f / 3.f);
-    s = fmaf(l, s, 2.f / 3.f);
+    float s = fmaf(l, 1.f / 3.f, 2.f / 3.f);
     s = fmaf(l, s, 1.f);
     s = fmaf(l, s, 1.f);
-    return -2.f * l * s;
+    return (-2.f * l) * s;
 }
 
 __device__ __forceinline__ float gelu_tanh_fast(float g)
@@ -513,13 +514,16 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const int q = lane >> 3;           // token quarter of the tile
         const int dl = kb * 64 + cg * 8;   // channel within the head
         const size_t d0 = (size_t)head * 256 + dl;
+        // The conv produces xh = xc / 2 (halving is exact): the MMA then yields
+        // half pre-activations, which is what sigmoid(z) = (1 + tanh(z/2)) / 2
+        // needs, and the scan's i*xc becomes one FMA on xh.
         float w[4][8], cb[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[k][e] = p.conv_w[(size_t)k * p.D + d0 + e];
+            for (int e = 0; e < 8; ++e) w[k][e] = 0.5f * p.conv_w[(size_t)k * p.D + d0 + e];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) cb[e] = p.conv_b[d0 + e];
+        for (int e = 0; e < 8; ++e) cb[e] = 0.5f * p.conv_b[d0 + e];
         const bool own = (kb >> 1) == half;
         const int xcs_col = (kb & 1) * 64 + cg * 8;
 #pragma unroll 1
@@ -595,11 +599,16 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const int c = threadIdx.x % kGroupThreads;
         const int d = head * 256 + half * kHalf + c;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const float ba = p.b_a[d], bx = p.b_x[d];
+        const float hba = 0.5f * p.b_a[d], hbx = 0.5f * p.b_x[d];
         const float lam = p.lambda[d];
         const float ls = lam >= 0.f ? -log1pf(expf(-lam)) : lam - log1pf(expf(lam));  // log sigmoid(Lambda)
-        const float kl = kC * ls;                       // log a per unit r
-        const float kl2 = kl * 1.4426950408889634f;     // log2 a per unit r
+        const float kl = kC * ls;                       // log a per unit r (<= 0)
+        // r = (1 + tr) / 2 with tr = tanh(half pre-activation): log a = tr * hkl + hkl
+        const float hkl = 0.5f * kl;
+        const float hkl2 = hkl * 1.4426950408889634f;  // same in log2
+        // every log a of this channel lies in [kl, 0]: the short series for
+        // 1 - a^2 applies to all of them when kl > -1/8
+        const bool series_ok = kl > -0.125f;
 
         auto pass1 = [&](int j) -> bool {
             const int s = j % SLOTS;
@@ -617,29 +626,46 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 tmem_ld8(col + t8, ar);
                 tmem_ld8(col + NT + t8, ai);
                 tmem_wait_ld();
+                const bool clean = ((ti.reset_mask >> t8) & 0xffu) == 0u && t8 + 8 <= ti.valid && series_ok;
+                if (clean) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int t = t8 + k;
-                    const float xc = xcs[t * kHalf + c];
-                    const float r = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ar[k]) + ba)), 0.5f);
-                    const float ig = fmaf(0.5f, tanh_approx(0.5f * (__uint_as_float(ai[k]) + bx)), 0.5f);
-                    const float ell = r * kl;
-                    float a = ex2_approx(r * kl2);
-                    const float om = ell > -0.125f ? one_minus_exp2l_small(ell) : fmaf(-a, a, 1.f);
-                    const float uu = ig * xc;
-                    float v = sqrt_approx(om) * uu;
-                    if ((ti.reset_mask >> t) & 1u) {
-                        a = 0.f;
-                        v = uu;
+                    for (int k = 0; k < 8; ++k) {
+                        const float xh = xcs[(t8 + k) * kHalf + c];
+                        const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
+                        const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
+                        const float ell = fmaf(tr, hkl, hkl);
+                        const float a = ex2_approx(fmaf(tr, hkl2, hkl2));
+                        const float v = sqrt_approx(one_minus_exp2l_small(ell)) * fmaf(tg, xh, xh);
+                        hl = fmaf(a, hl, v);
+                        P *= a;
+                        ar[k] = __float_as_uint(a);
+                        ai[k] = __float_as_uint(v);
                     }
-                    if (t >= ti.valid) {
-                        a = 1.f;
-                        v = 0.f;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int t = t8 + k;
+                        const float xh = xcs[t * kHalf + c];
+                        const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
+                        const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
+                        const float ell = fmaf(tr, hkl, hkl);
+                        float a = ex2_approx(fmaf(tr, hkl2, hkl2));
+                        const float om = ell > -0.125f ? one_minus_exp2l_small(ell) : fmaf(-a, a, 1.f);
+                        const float uu = fmaf(tg, xh, xh);  // i * xc
+                        float v = sqrt_approx(om) * uu;
+                        if ((ti.reset_mask >> t) & 1u) {
+                            a = 0.f;
+                            v = uu;
+                        }
+                        if (t >= ti.valid) {
+                            a = 1.f;
+                            v = 0.f;
+                        }
+                        hl = fmaf(a, hl, v);
+                        P *= a;
+                        ar[k] = __float_as_uint(a);
+                        ai[k] = __float_as_uint(v);
                     }
-                    hl = fmaf(a, hl, v);
-                    P *= a;
-                    ar[k] = __float_as_uint(a);
-                    ai[k] = __float_as_uint(v);
                 }
                 tmem_st8(col + t8, ar);
                 tmem_st8(col + NT + t8, ai);
@@ -690,13 +716,22 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 tmem_ld8(col + t8, aa);
                 tmem_ld8(col + NT + t8, vv);
                 tmem_wait_ld();
+                if (t8 + 8 <= ti.valid) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int t = t8 + k;
-                    h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
-                    if (t < ti.valid) {
-                        const float gv = __bfloat162float(gs[t * kHalf + c]);
-                        yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                    for (int k = 0; k < 8; ++k) {
+                        h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
+                        const float gv = __bfloat162float(gs[(t8 + k) * kHalf + c]);
+                        yp[(size_t)(t8 + k) * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int t = t8 + k;
+                        h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
+                        if (t < ti.valid) {
+                            const float gv = __bfloat162float(gs[t * kHalf + c]);
+                            yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                        }
                     }
                 }
             }
