@@ -52,7 +52,8 @@ constexpr int kScanGroups = 2;  // scan warp groups, alternate tiles
 constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
 constexpr int kConvWarp0 = kScanWarps;
 constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kLbWarp = kMmaWarp + 1, kSchedWarp = kMmaWarp + 2;
-constexpr int kThreads = 32 * (kSchedWarp + 1);
+constexpr int kPubWarp = kMmaWarp + 3;
+constexpr int kThreads = 32 * (kPubWarp + 1);
 constexpr int kGroupThreads = 128;  // threads of one scan group (one per channel)
 
 // TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
@@ -76,7 +77,7 @@ constexpr int OFF_HIN = OFF_AGG + SLOTS * kHalf * 8;
 constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
 constexpr int OFF_BAR = OFF_INFO + INFO_RING * 32;
 // per-slot barriers (slot = tile % SLOTS)
-enum { BAR_CONV, BAR_SMEM_FREE, BAR_MMA, BAR_TMEM_FREE, BAR_PASS1, BAR_LB, BAR_G, BAR_KINDS };
+enum { BAR_CONV, BAR_SMEM_FREE, BAR_MMA, BAR_TMEM_FREE, BAR_PASS1, BAR_LB, BAR_G, BAR_PUB, BAR_KINDS };
 constexpr int OFF_RING_BAR = OFF_BAR + BAR_KINDS * SLOTS * 8;  // INFO_FULL[8], INFO_EMPTY[8]
 constexpr int OFF_XBAR = OFF_RING_BAR + 2 * INFO_RING * 8;         // X_FULL[3], X_EMPTY[3]
 constexpr int OFF_MISC = OFF_XBAR + 2 * XRING * 8;
@@ -151,9 +152,9 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile i
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        __nanosleep(it < 16 ? 16 : 64);
-        if ((it & 63u) == 0) {
+        // suspended in hardware until the phase completes (or 20 us pass)
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        {
             if (*abort_flag) return false;
             if (*(volatile int *)&hdr->status != 0) {
                 *abort_flag = 1;
@@ -325,7 +326,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     auto x_empty = [&](int i) { return xbars + XRING + i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-    int *agg_count = reinterpret_cast<int *>(smem + OFF_MISC + 16);  // per slot: scan warps done with pass 1
     WsHeader *hdr = p.hdr;
 
     // ------------------------------------------------------------------ setup
@@ -340,6 +340,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 mbar_init(bar(BAR_PASS1, s), kGroupThreads);
                 mbar_init(bar(BAR_LB, s), 32);
                 mbar_init(bar(BAR_G, s), 1);
+                mbar_init(bar(BAR_PUB, s), 32);
             }
             for (int i = 0; i < INFO_RING; ++i) {
                 mbar_init(info_full(i), 1);
@@ -350,7 +351,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 mbar_init(x_empty(i), kConvWarps * 32);
             }
             *abort_flag = 0;
-            for (int s = 0; s < SLOTS; ++s) agg_count[s] = 0;
             mbar_fence_init();
         }
     }
@@ -672,27 +672,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             mbar_arrive(bar(BAR_SMEM_FREE, s));  // xcs (and, via the MMA wait, the B tile) consumed
             tmem_wait_st();
-            const float2 agg = make_float2(P, hl);
-            reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = agg;
-            // Publish the tile aggregate right away (decoupled look-back): later
-            // tiles of the sequence may combine it before this tile's own
-            // look-back has finished.  The last warp of the group to get here
-            // sets the flag; nobody waits.
-            const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
-            const bool suppress = (int)gu == debug_unit;
-            if (!suppress) {
-                p.agg[gu * kHalf + c] = agg;
-                __threadfence();
-            }
-            __syncwarp();
-            if (lane == 0) {
-                const int prev = atomicAdd(agg_count + s, 1);
-                if (prev == 3) {
-                    agg_count[s] = 0;
-                    __threadfence();
-                    if (!suppress) st_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
-                }
-            }
+            // the publisher warp must have copied out this slot's previous aggregate
+            if (j >= SLOTS && !warp_wait_bar(bar(BAR_PUB, s), ph ^ 1u, abort_flag, hdr, 17)) return false;
+            reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = make_float2(P, hl);
             mbar_arrive(bar(BAR_PASS1, s));
             if (c == 0) RGLRU_TR(TR_P1_END, j, globaltimer());
             return true;
@@ -773,6 +755,32 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (!end) ok = pass1(j);
             if (ok && j >= kScanGroups) ok = pass2(j - kScanGroups);
             if (!ok || end) break;
+        }
+    } else if (warp == kPubWarp) {
+        // ------------------------------------------------------------ publisher
+        // Publishes each tile aggregate as soon as pass 1 ends (decoupled
+        // look-back: later tiles of the sequence may combine it before this
+        // tile's own look-back has finished).  It is the only warp that fences
+        // for the aggregates, and it has no other global stores in flight.
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS, ir = j % INFO_RING;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 18)) break;
+            const TileInfo ti = info[ir];
+            if (ti.u < 0) break;
+            if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 19)) break;
+            const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
+            if ((int)gu != debug_unit) {
+                const float4 *src = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
+                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf);
+                dst[lane] = src[lane];
+                dst[lane + 32] = src[lane + 32];
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
+            }
+            mbar_arrive(bar(BAR_PUB, s));
         }
     } else if (warp == kLbWarp) {
         // ------------------------------------------------------------ look-back warp
