@@ -16,7 +16,7 @@ constexpr float kC = 8.0f;      // exponent scale in a = sigmoid(Lambda)^(c r)
 // Workspace header.  A zero-filled header is the valid initial state.
 struct WsHeader {
     int status;            // rglru_status recorded by device code (0 = OK)
-    int detail;            // first chunk index whose wait gave up (+1), 0 = none
+    int detail;            // first wait that gave up: (CTA << 8) | (wait site + 1), 0 = none
     int debug_unit_plus1;  // test hook: chunk that skips publishing (+1), 0 = off
     int pad0;
     unsigned int ticket[1000];  // per-group work counters of the fused prefill kernel

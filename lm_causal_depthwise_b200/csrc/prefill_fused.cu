@@ -141,7 +141,7 @@ constexpr uint32_t F_AGG = 1u, F_PREFIX = 2u, F_RESET = 4u;
 __device__ __forceinline__ void raise_timeout(volatile int *abort_flag, WsHeader *hdr, int where)
 {
     atomicCAS(&hdr->status, 0, (int)RGLRU_ERR_TIMEOUT);
-    atomicCAS(&hdr->detail, 0, where + 1);
+    atomicCAS(&hdr->detail, 0, (int)(blockIdx.x << 8) | (where + 1));
     *abort_flag = 1;
 }
 
@@ -778,7 +778,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 dst[lane + 32] = src[lane + 32];
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
+                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
             }
             mbar_arrive(bar(BAR_PUB, s));
         }
@@ -856,7 +856,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
+                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
             }
             *reinterpret_cast<float4 *>(smem + OFF_HIN + s * kHalf * 4 + ch * 4) =
                 make_float4(hin[0], hin[1], hin[2], hin[3]);

@@ -83,6 +83,14 @@ __device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v)
 {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Sets bits of a flag word with release semantics (several writers may set
+// different bits of the same word; none can erase another's).
+__device__ __forceinline__ void atom_or_release_u32(uint32_t *p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.or.release.gpu.global.b32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    (void)old;
+}
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
 {
     uint32_t v;
