@@ -121,7 +121,8 @@ struct FusedParams {
 // into trace[(cta * kTraceTiles + tile) * kTraceEvents + event].
 enum TraceEvent {
     TR_SCHED_INFO, TR_CONV_START, TR_CONV_DONE, TR_MMA_ISSUED, TR_P1_START, TR_P1_END, TR_LB_START,
-    TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, kTraceEvents
+    TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, TR_MMA_TFREE, TR_MMA_TMA, TR_MMA_CONV,
+    kTraceEvents
 };
 constexpr int kTraceCtas = 4, kTraceTiles = 128;
 #ifdef RGLRU_TRACE
@@ -471,13 +472,16 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const TileInfo ti = info[ir];
             if (ti.u < 0) break;
             if (j >= SLOTS && !warp_wait_bar(bar(BAR_TMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 3)) break;
+            if (lane == 0) RGLRU_TR(TR_MMA_TFREE, j, globaltimer());
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(BAR_G, s), kGTile);
                 tma_load_3d(smem + OFF_G + s * kGTile, &tmap_g, bar(BAR_G, s), head * 256 + half * kHalf, ti.t0,
                             ti.b);
             }
+            if (lane == 0) RGLRU_TR(TR_MMA_TMA, j, globaltimer());
             ++issued;
             if (!warp_wait_bar(bar(BAR_CONV, s), ph, abort_flag, hdr, 4)) break;
+            if (lane == 0) RGLRU_TR(TR_MMA_CONV, j, globaltimer());
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t b_base = smem_u32(smem + OFF_B + s * kBTile);
