@@ -124,8 +124,8 @@ enum TraceEvent {
     TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, TR_MMA_TFREE, TR_MMA_TMA, TR_MMA_CONV,
     kTraceEvents
 };
-constexpr int kTraceCtas = 4, kTraceTiles = 128;
 #ifdef RGLRU_TRACE
+constexpr int kTraceCtas = 4, kTraceTiles = 128;
 #define RGLRU_TR(ev, j, val)                                                                                   \
     do {                                                                                                      \
         if (p.trace != nullptr && blockIdx.x < kTraceCtas && (j) < kTraceTiles)                               \

@@ -87,9 +87,7 @@ __device__ __forceinline__ void st_release_u32(uint32_t *p, uint32_t v)
 // different bits of the same word; none can erase another's).
 __device__ __forceinline__ void atom_or_release_u32(uint32_t *p, uint32_t v)
 {
-    uint32_t old;
-    asm volatile("atom.or.release.gpu.global.b32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    (void)old;
+    asm volatile("red.release.gpu.global.or.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
 {
