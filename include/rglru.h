@@ -167,6 +167,35 @@ RGLRU_API rglru_status rglru_get_device_status(void *workspace, cudaStream_t str
  */
 RGLRU_API rglru_status rglru_debug_suppress_publish(void *workspace, int unit, cudaStream_t stream);
 
+/*
+ * rglru_prefill without a workspace argument, for callers that cannot
+ * allocate device memory where they run the block (a serving loop whose
+ * device memory is fixed at start-up, a plug-in handed tensors but no
+ * allocator).  The pages have no counterpart to this call; it only changes
+ * where the scratch lives.  It allocates nothing: the caller passes inputs
+ * and outputs as for rglru_prefill, and the scratch is a library-owned device
+ * array of 8 MiB per GPU, held from library load until the process exits.
+ *   - bf16 only (RGLRU_ERR_UNSUPPORTED otherwise); shapes whose
+ *     rglru_workspace_size exceeds 8 MiB are rejected with
+ *     RGLRU_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the array and zeroes what must start at zero; calls
+ *     that can overlap on the GPU (other streams, other host threads) race
+ *     on it, so the caller must serialise them.
+ *   - A device-side wait that runs out cannot be read back (there is no
+ *     workspace handle); the next call clears the record.
+ * Other arguments, layouts and semantics as rglru_prefill.
+ */
+RGLRU_API rglru_status rglru_prefill_noalloc(int B, int T, int D, rglru_io_dtype dt,
+                                             const void *x, const void *gate_branch,
+                                             const float *conv_w, const float *conv_b,
+                                             const void *W_a, const float *b_a,
+                                             const void *W_x, const float *b_x,
+                                             const float *lambda, const int32_t *segment_pos,
+                                             void *conv_state, float *h_state, void *y,
+                                             cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

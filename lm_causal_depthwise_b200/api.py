@@ -23,7 +23,8 @@ IO_F32, IO_BF16 = 0, 1
 
 SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglru_prefill",
            "rglru_simt_workspace_size", "rglru_prefill_simt", "rglru_decode_workspace_size",
-           "rglru_decode_step", "rglru_get_device_status", "rglru_debug_suppress_publish")
+           "rglru_decode_step", "rglru_get_device_status", "rglru_debug_suppress_publish",
+           "rglru_prefill_noalloc")
 
 _lib = None
 
@@ -64,6 +65,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_get_device_status.argtypes = [vp, vp]
     lib.rglru_debug_suppress_publish.restype = i
     lib.rglru_debug_suppress_publish.argtypes = [vp, i, vp]
+    lib.rglru_prefill_noalloc.restype = i
+    lib.rglru_prefill_noalloc.argtypes = [i, i, i, i] + [vp] * 13 + [vp]
     _lib = lib
     return lib
 
@@ -188,6 +191,24 @@ def prefill(x, gate_branch, p: Params, segment_pos, conv_state, h_state, workspa
             ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(x.device))
     if st != OK:
         raise RGLRUError(st, "rglru_prefill_simt" if simt else "rglru_prefill")
+    return y
+
+
+def prefill_noalloc(x, gate_branch, p: Params, segment_pos, conv_state, h_state, y=None) -> torch.Tensor:
+    """rglru_prefill_noalloc: the bf16 prefill with the library's own fixed
+    scratch (no workspace, nothing allocated by the library).  Same tensors
+    and semantics as :func:`prefill`; shapes whose workspace would exceed the
+    library's 8 MiB scratch raise RGLRUError(ERR_WORKSPACE)."""
+    if x.dim() != 3:
+        raise ValueError("x must be [B,T,D]")
+    B, T, D = x.shape
+    dt, y = _common(x, gate_branch, p, segment_pos, conv_state, h_state, y, (B, T))
+    st = load().rglru_prefill_noalloc(
+        B, T, D, dt, _ptr(x), _ptr(gate_branch), _ptr(p.conv_w), _ptr(p.conv_b), _ptr(p.W_a),
+        _ptr(p.b_a), _ptr(p.W_x), _ptr(p.b_x), _ptr(p.lam), _ptr(segment_pos), _ptr(conv_state),
+        _ptr(h_state), _ptr(y), _stream(x.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_prefill_noalloc")
     return y
 
 
