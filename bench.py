@@ -281,6 +281,9 @@ def run_cuda(args, w):
     if distributed:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
+    st = api.device_status(ws)
+    if st != api.OK:
+        raise RuntimeError(f"prefill reported device status {api.status_string(st)}: no valid timing")
     ms_t = torch.tensor([ms], device=dev, dtype=torch.float64)
     if distributed:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
@@ -317,6 +320,9 @@ def run_cuda(args, w):
     if distributed:
         dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
     e_value = tokens / (float(e_ms.item()) / e_steps * 1e-3)
+    st = api.device_status(ws)
+    if st != api.OK:
+        raise RuntimeError(f"prefill reported device status {api.status_string(st)} in the e2e loop")
     h2d = hx.numel() * hx.element_size() + hg.numel() * hg.element_size() + hsp.numel() * 4
     d2h = hy.numel() * hy.element_size()
 

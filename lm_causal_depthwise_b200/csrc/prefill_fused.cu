@@ -34,7 +34,6 @@
 // Griffin / RecurrentGemma (arXiv 2404.07839).
 #include <cuda.h>
 #include <cudaTypedefs.h>
-#include <cuda_fp16.h>
 #include <mutex>
 
 #include "internal.h"
@@ -57,17 +56,13 @@ constexpr int kPubWarp = kMmaWarp + 3;
 constexpr int kThreads = 32 * (kPubWarp + 1);
 constexpr int kGroupThreads = 128;  // threads of one scan group (one per channel)
 
-// TMEM columns (512 allocated): W_a half-head rows, W_x rows (the MMA A
-// operands), then the pre-activation accumulators of the SLOTS tiles: r-gate
-// block [256, 384) and i-gate block [384, 512), NT columns per slot.  Slots
-// 2m and 2m+1 are adjacent in both blocks, so one N = 2 NT MMA covers a pair
-// of tiles (an M=128 tcgen05.mma costs ~45 cycles for any N <= 64).
-constexpr uint32_t kColWa = 0, kColWx = 128, kColPreR = 256, kColPreI = 384;
+// TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
+// [pre_r | pre_i] accumulators that pass 1 overwrites with [a | v].
+constexpr uint32_t kColWa = 0, kColWx = 128, kColSlot0 = 256, kColPerSlot = 2 * NT;
 
 // Shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kBTile = NT * 256 * 2;            // bf16 xc/2 of one tile, 4 K-blocks of 64 channels
-constexpr int kBBlock = NT * 128;               // one K-block of one tile: NT rows x 128 B
-constexpr int kBKStride = SLOTS * kBBlock;      // K-block kb of slot s at kb * kBKStride + s * kBBlock
+constexpr int kBTile = NT * 256 * 2;            // bf16 xc, 4 K-blocks of 64 channels
+constexpr int kBBlock = NT * 128;               // one K-block: NT rows x 128 B
 constexpr int kXcsTile = NT * kHalf * 4;        // fp32 xc / 2 of this half
 constexpr int kGTile = NT * kHalf * 2;          // bf16 gate-branch tile (TMA box)
 constexpr int XRING = 3;                         // x tiles (32 rows + 3 halo rows) in flight
@@ -82,8 +77,7 @@ constexpr int OFF_HIN = OFF_AGG + SLOTS * kHalf * 8;
 constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
 constexpr int OFF_BAR = OFF_INFO + INFO_RING * 32;
 // per-slot barriers (slot = tile % SLOTS)
-// BAR_MMA is per tile pair (entries 0 and 1 used: pair index % 2)
-enum { BAR_CONV, BAR_SLOT_FREE, BAR_MMA, BAR_PASS1, BAR_LB, BAR_G, BAR_PUB, BAR_KINDS };
+enum { BAR_CONV, BAR_SMEM_FREE, BAR_MMA, BAR_TMEM_FREE, BAR_PASS1, BAR_LB, BAR_G, BAR_PUB, BAR_KINDS };
 constexpr int OFF_RING_BAR = OFF_BAR + BAR_KINDS * SLOTS * 8;  // INFO_FULL[8], INFO_EMPTY[8]
 constexpr int OFF_XBAR = OFF_RING_BAR + 2 * INFO_RING * 8;         // X_FULL[3], X_EMPTY[3]
 constexpr int OFF_MISC = OFF_XBAR + 2 * XRING * 8;
@@ -118,7 +112,7 @@ struct FusedParams {
     WsHeader *hdr;
     uint32_t *flags;   // [G][tiles_per_group]
     float2 *agg;       // [G][tiles_per_group][128]  (prod a, h_end) from h = 0
-    float *prefix;     // [G][tiles_per_group][128]  h after the tile (A h_in + H)
+    float *prefix;     // [G][tiles_per_group][128]  h after the tile
     unsigned long long *trace;  // RGLRU_TRACE builds only: per-role timestamps
 };
 
@@ -288,17 +282,6 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
     }
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
-{
-    __half2 v = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
-__device__ __forceinline__ float2 unpack_half2(uint32_t u)
-{
-    return __half22float2(*reinterpret_cast<__half2 *>(&u));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -352,8 +335,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         if (lane == 0) {
             for (int s = 0; s < SLOTS; ++s) {
                 mbar_init(bar(BAR_CONV, s), kConvWarps * 32);
-                mbar_init(bar(BAR_SLOT_FREE, s), kGroupThreads);
+                mbar_init(bar(BAR_SMEM_FREE, s), kGroupThreads);
                 mbar_init(bar(BAR_MMA, s), 1);
+                mbar_init(bar(BAR_TMEM_FREE, s), kGroupThreads);
                 mbar_init(bar(BAR_PASS1, s), kGroupThreads);
                 mbar_init(bar(BAR_LB, s), 32);
                 mbar_init(bar(BAR_G, s), 1);
@@ -411,7 +395,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // ------------------------------------------------------------ scheduler
         // Claims tiles in order from this group's ticket counter, one tile ahead
         // of the ring, so that the atomic and the segment_pos read overlap the
-        // wait for a free ring entry; starts the x-tile TMA of each tile.
+        // wait for a free ring entry.
         auto claim = [&]() -> TileInfo {
             int u = -1;
             if (lane == 0 && !*abort_flag) {
@@ -478,70 +462,52 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (+ GELU-branch TMA)
-        // Tiles go in pairs (2m, 2m+1) through one N = 2 NT MMA per K step;
-        // a lone last tile takes an N = NT MMA.
-        const uint32_t idesc2 = umma_idesc_bf16(kHalf, 2 * NT), idesc1 = umma_idesc_bf16(kHalf, NT);
-        int g_issued = 0, pairs = 0;
+        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
+        int issued = 0;
 #pragma unroll 1
-        for (int m = 0;; ++m) {
-            const int j0 = 2 * m, j1 = 2 * m + 1;
-            if (!warp_wait_bar(info_full(j0 % INFO_RING), (uint32_t)(j0 / INFO_RING) & 1u, abort_flag, hdr, 2)) break;
-            const TileInfo t0i = info[j0 % INFO_RING];
-            if (t0i.u < 0) break;
-            if (!warp_wait_bar(info_full(j1 % INFO_RING), (uint32_t)(j1 / INFO_RING) & 1u, abort_flag, hdr, 2)) break;
-            const TileInfo t1i = info[j1 % INFO_RING];
-            const int n_tiles = t1i.u >= 0 ? 2 : 1;
-            const int s0 = j0 % SLOTS;
-            const uint32_t ph = (uint32_t)(j0 / SLOTS) & 1u;
-            // TMEM columns, B tile and g tile of both slots free (pass 1 of tiles j-4 done)
-            bool ok = true;
-            for (int k = 0; k < n_tiles && ok; ++k)
-                if (j0 >= SLOTS) ok = warp_wait_bar(bar(BAR_SLOT_FREE, s0 + k), ph ^ 1u, abort_flag, hdr, 3);
-            if (!ok) break;
-            if (lane == 0) RGLRU_TR(TR_MMA_TFREE, j0, globaltimer());
+        for (int j = 0;; ++j) {
+            const int s = j % SLOTS, ir = j % INFO_RING;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 2)) break;
+            const TileInfo ti = info[ir];
+            if (ti.u < 0) break;
+            if (j >= SLOTS && !warp_wait_bar(bar(BAR_TMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 3)) break;
+            if (lane == 0) RGLRU_TR(TR_MMA_TFREE, j, globaltimer());
             if (lane == 0) {
-                for (int k = 0; k < n_tiles; ++k) {
-                    const TileInfo &ti = k == 0 ? t0i : t1i;
-                    mbar_arrive_expect_tx(bar(BAR_G, s0 + k), kGTile);
-                    tma_load_3d(smem + OFF_G + (s0 + k) * kGTile, &tmap_g, bar(BAR_G, s0 + k),
-                                head * 256 + half * kHalf, ti.t0, ti.b);
-                }
+                mbar_arrive_expect_tx(bar(BAR_G, s), kGTile);
+                tma_load_3d(smem + OFF_G + s * kGTile, &tmap_g, bar(BAR_G, s), head * 256 + half * kHalf, ti.t0,
+                            ti.b);
             }
-            g_issued += n_tiles;
-            if (lane == 0) RGLRU_TR(TR_MMA_TMA, j0, globaltimer());
-            for (int k = 0; k < n_tiles && ok; ++k) ok = warp_wait_bar(bar(BAR_CONV, s0 + k), ph, abort_flag, hdr, 4);
-            if (!ok) break;
-            if (lane == 0) RGLRU_TR(TR_MMA_CONV, j0, globaltimer());
+            if (lane == 0) RGLRU_TR(TR_MMA_TMA, j, globaltimer());
+            ++issued;
+            if (!warp_wait_bar(bar(BAR_CONV, s), ph, abort_flag, hdr, 4)) break;
+            if (lane == 0) RGLRU_TR(TR_MMA_CONV, j, globaltimer());
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t b_base = smem_u32(smem + OFF_B + s0 * kBBlock);
-                const uint32_t d_r = tmem + kColPreR + s0 * NT;
-                const uint32_t d_i = tmem + kColPreI + s0 * NT;
-                const uint32_t idesc = n_tiles == 2 ? idesc2 : idesc1;
+                const uint32_t b_base = smem_u32(smem + OFF_B + s * kBTile);
+                const uint32_t d_r = tmem + kColSlot0 + s * kColPerSlot;
+                const uint32_t d_i = d_r + NT;
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk) {
-                    const uint64_t bd = umma_desc_sw128(b_base + (kk >> 2) * kBKStride + (kk & 3) * 32);
+                    const uint64_t bd = umma_desc_sw128(b_base + (kk >> 2) * kBBlock + (kk & 3) * 32);
                     umma_ts(d_r, tmem + kColWa + kk * 8, bd, idesc, kk > 0);
                     umma_ts(d_i, tmem + kColWx + kk * 8, bd, idesc, kk > 0);
                 }
-                umma_commit(bar(BAR_MMA, m & 1));
-                RGLRU_TR(TR_MMA_ISSUED, j0, globaltimer());
+                umma_commit(bar(BAR_MMA, s));
+                RGLRU_TR(TR_MMA_ISSUED, j, globaltimer());
             }
-            ++pairs;
             __syncwarp();
-            if (n_tiles == 1) break;
         }
         // on abort, wait (bounded) for this CTA's copies and MMAs in flight
         if (lane == 0 && *abort_flag) {
-            for (int k = max(0, g_issued - SLOTS); k < g_issued; ++k) {
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(bar(BAR_G, k % SLOTS), (uint32_t)(k / SLOTS) & 1u) && globaltimer() - t0 < kTimeoutNs) {
+            for (int k = max(0, issued - SLOTS); k < issued; ++k) {
+                const int s = k % SLOTS;
+                const uint32_t ph = (uint32_t)(k / SLOTS) & 1u;
+                uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(bar(BAR_G, s), ph) && globaltimer() - t0 < kTimeoutNs) {
                 }
-            }
-            if (pairs > 0) {
-                const int m = pairs - 1;
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(bar(BAR_MMA, m & 1), (uint32_t)(m >> 1) & 1u) && globaltimer() - t0 < kTimeoutNs / 4) {
+                t0 = globaltimer();
+                while (!mbar_try_wait(bar(BAR_MMA, s), ph) && globaltimer() - t0 < kTimeoutNs / 4) {
                 }
             }
         }
@@ -574,7 +540,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_START, j, globaltimer());
             const int xr = j % XRING;
             if (!warp_wait_bar(x_full(xr), (uint32_t)(j / XRING) & 1u, abort_flag, hdr, 16)) break;
-            if (j >= SLOTS && !warp_wait_bar(bar(BAR_SLOT_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
+            if (j >= SLOTS && !warp_wait_bar(bar(BAR_SMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
             const int n0 = q * 8;
             const uint8_t *xt = smem + OFF_X + xr * kXTile + dl * 2;  // row r = token t0 - 3 + r
             auto xrow = [&](int r, float (&f)[8]) {
@@ -590,7 +556,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             xrow(n0, xm3);
             xrow(n0 + 1, xm2);
             xrow(n0 + 2, xm1);
-            uint8_t *btile = smem + OFF_B + kb * kBKStride + s * kBBlock;
+            uint8_t *btile = smem + OFF_B + s * kBTile + kb * kBBlock;
             float *xcs = reinterpret_cast<float *>(smem + OFF_XCS + s * kXcsTile);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -648,38 +614,27 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // 1 - a^2 applies to all of them when kl > -1/8
         const bool series_ok = kl > -0.125f;
 
-#pragma unroll 1
-        for (int j = sg;; j += kScanGroups) {
-            const int s = j % SLOTS, ir = j % INFO_RING;
+        auto pass1 = [&](int j) -> bool {
+            const int s = j % SLOTS;
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 12)) break;
-            const TileInfo ti = info[ir];
-            if (ti.u < 0) break;
-
-            // ---- pass 1: gates, decay, normaliser, local scan from h = 0, GELU branch.
-            // Per token the tile keeps y_loc = G h_loc and q = G prod(a) (f16 pair in
-            // one register): after the carried-in state h_in arrives,
-            // y = y_loc + q h_in.  TMEM and shared memory are released right away.
-            if (!warp_wait_bar(bar(BAR_MMA, (j >> 1) & 1), (uint32_t)(j >> 2) & 1u, abort_flag, hdr, 7)) break;
-            if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 9)) break;
+            const TileInfo ti = info[j % INFO_RING];
+            if (!warp_wait_bar(bar(BAR_MMA, s), ph, abort_flag, hdr, 7)) return false;
             if (c == 0) RGLRU_TR(TR_P1_START, j, globaltimer());
             tc_fence_after();
+            const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
             const float *xcs = reinterpret_cast<const float *>(smem + OFF_XCS + s * kXcsTile);
-            const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile);
-            uint32_t stash[NT];
             float hl = 0.f, P = 1.f;
-#pragma unroll
+#pragma unroll 1
             for (int t8 = 0; t8 < NT; t8 += 8) {
                 uint32_t ar[8], ai[8];
-                tmem_ld8(tmem + lane_off + kColPreR + s * NT + t8, ar);
-                tmem_ld8(tmem + lane_off + kColPreI + s * NT + t8, ai);
+                tmem_ld8(col + t8, ar);
+                tmem_ld8(col + NT + t8, ai);
                 tmem_wait_ld();
                 const bool clean = ((ti.reset_mask >> t8) & 0xffu) == 0u && t8 + 8 <= ti.valid && series_ok;
                 if (clean) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        const int t = t8 + k;
-                        const float xh = xcs[t * kHalf + c];
+                        const float xh = xcs[(t8 + k) * kHalf + c];
                         const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
                         const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
                         const float ell = fmaf(tr, hkl, hkl);
@@ -687,8 +642,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const float v = sqrt_approx(one_minus_exp2l_small(ell)) * fmaf(tg, xh, xh);
                         hl = fmaf(a, hl, v);
                         P *= a;
-                        const float G = gelu_tanh_fast(__bfloat162float(gs[t * kHalf + c]));
-                        stash[t] = pack_half2(G * hl, G * P);
+                        ar[k] = __float_as_uint(a);
+                        ai[k] = __float_as_uint(v);
                     }
                 } else {
 #pragma unroll
@@ -712,36 +667,57 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         }
                         hl = fmaf(a, hl, v);
                         P *= a;
-                        const float G = gelu_tanh_fast(__bfloat162float(gs[t * kHalf + c]));
-                        stash[t] = pack_half2(G * hl, G * P);
+                        ar[k] = __float_as_uint(a);
+                        ai[k] = __float_as_uint(v);
                     }
                 }
+                tmem_st8(col + t8, ar);
+                tmem_st8(col + NT + t8, ai);
             }
-            tc_fence_before();
-            mbar_arrive(bar(BAR_SLOT_FREE, s));  // TMEM columns, B tile, xc and g tiles of this slot
+            mbar_arrive(bar(BAR_SMEM_FREE, s));  // xcs (and, via the MMA wait, the B tile) consumed
+            tmem_wait_st();
             // the publisher warp must have copied out this slot's previous aggregate
-            if (j >= SLOTS && !warp_wait_bar(bar(BAR_PUB, s), ph ^ 1u, abort_flag, hdr, 17)) break;
+            if (j >= SLOTS && !warp_wait_bar(bar(BAR_PUB, s), ph ^ 1u, abort_flag, hdr, 17)) return false;
             reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = make_float2(P, hl);
             mbar_arrive(bar(BAR_PASS1, s));
             if (c == 0) RGLRU_TR(TR_P1_END, j, globaltimer());
+            return true;
+        };
 
-            // ---- pass 2: y = y_loc + q h_in as soon as the carried-in state is known
-            if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 8)) break;
-            const float h_in = reinterpret_cast<const float *>(smem + OFF_HIN + s * kHalf * 4)[c];
+        auto pass2 = [&](int j) -> bool {
+            const int s = j % SLOTS, ir = j % INFO_RING;
+            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            const TileInfo ti = info[ir];
+            if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 8)) return false;
+            float h = reinterpret_cast<const float *>(smem + OFF_HIN + s * kHalf * 4)[c];
+            if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 9)) return false;
             if (c == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
+            tc_fence_after();
+            const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
+            const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile);
             __nv_bfloat16 *yp = p.y + ((size_t)ti.b * p.T + ti.t0) * p.D + d;
-            if (ti.valid == NT) {
+#pragma unroll 1
+            for (int t8 = 0; t8 < NT; t8 += 8) {
+                uint32_t aa[8], vv[8];
+                tmem_ld8(col + t8, aa);
+                tmem_ld8(col + NT + t8, vv);
+                tmem_wait_ld();
+                if (t8 + 8 <= ti.valid) {
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    const float2 f = unpack_half2(stash[t]);
-                    yp[(size_t)t * p.D] = __float2bfloat16_rn(fmaf(f.y, h_in, f.x));
-                }
-            } else {
+                    for (int k = 0; k < 8; ++k) {
+                        h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
+                        const float gv = __bfloat162float(gs[(t8 + k) * kHalf + c]);
+                        yp[(size_t)(t8 + k) * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                    }
+                } else {
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (t < ti.valid) {
-                        const float2 f = unpack_half2(stash[t]);
-                        yp[(size_t)t * p.D] = __float2bfloat16_rn(fmaf(f.y, h_in, f.x));
+                    for (int k = 0; k < 8; ++k) {
+                        const int t = t8 + k;
+                        h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
+                        if (t < ti.valid) {
+                            const float gv = __bfloat162float(gs[t * kHalf + c]);
+                            yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                        }
                     }
                 }
             }
@@ -752,9 +728,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 const size_t u0 = (size_t)ti.b * p.C;
                 const uint32_t *f_own = p.flags + (size_t)group * p.tiles_per_group + u0;
                 const uint32_t *f_oth = p.flags + (size_t)(group ^ 1) * p.tiles_per_group + u0;
-                if (warp_wait_flag(f_own, F_PREFIX, abort_flag, hdr, 10) == 0) break;
-                if (warp_wait_flag(f_oth, F_AGG, abort_flag, hdr, 11) == 0) break;
-                p.h_state[(size_t)ti.b * p.D + d] = fmaf(P, h_in, hl);  // the tile's inclusive prefix
+                if (warp_wait_flag(f_own, F_PREFIX, abort_flag, hdr, 10) == 0) return false;
+                if (warp_wait_flag(f_oth, F_AGG, abort_flag, hdr, 11) == 0) return false;
+                p.h_state[(size_t)ti.b * p.D + d] = h;
                 __nv_bfloat16 ncs[3];
 #pragma unroll
                 for (int k = 0; k < 3; ++k) {
@@ -765,8 +741,24 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 #pragma unroll
                 for (int k = 0; k < 3; ++k) p.conv_state[((size_t)ti.b * 3 + k) * p.D + d] = ncs[k];
             }
+            tc_fence_before();
+            mbar_arrive(bar(BAR_TMEM_FREE, s));
             mbar_arrive(info_empty(ir));
             if (c == 0) RGLRU_TR(TR_P2_END, j, globaltimer());
+            return true;
+        };
+
+        // this group's tiles: j = sg, sg + kScanGroups, ...; pass 2 of a tile runs
+        // after pass 1 of the group's next tile (the look-back has that long)
+#pragma unroll 1
+        for (int j = sg;; j += kScanGroups) {
+            const int ir = j % INFO_RING;
+            bool end = !warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 12);
+            if (!end) end = info[ir].u < 0;
+            bool ok = true;
+            if (!end) ok = pass1(j);
+            if (ok && j >= kScanGroups) ok = pass2(j - kScanGroups);
+            if (!ok || end) break;
         }
     } else if (warp == kPubWarp) {
         // ------------------------------------------------------------ publisher
