@@ -16,12 +16,15 @@
 //                over the accumulators.  Pass 2 (two tiles later): re-run the
 //                scan from the carried-in state, multiply by GELU_tanh(g),
 //                store y.
-//   look-back    walks back over predecessor tiles of the same sequence to the
-//   warp         nearest anchor (a published inclusive prefix, or a tile that
-//                holds a reset: A = 0), folds h <- A h + H forward from it in
-//                sequence order (decoupled look-back with a fixed combination
-//                order, so results are bit-reproducible), hands the carried-in
-//                state to pass 2 and publishes the tile's inclusive prefix.
+//   look-back    one warp per slot, so that the look-backs of consecutive
+//   warps        tiles overlap.  Publishes the tile aggregate as soon as pass 1
+//                ends, walks back over predecessor tiles of the same sequence
+//                to the nearest anchor (a published inclusive prefix, or a tile
+//                that holds a reset: A = 0), folds h <- A h + H forward from it
+//                in sequence order (decoupled look-back with a fixed
+//                combination order, so results are bit-reproducible), hands
+//                the carried-in state to pass 2, then publishes the tile's
+//                inclusive prefix.
 //   producer     claims tiles in order from a per-(head, half) ticket counter,
 //                TMA-loads the GELU-branch tile, issues the MMAs.
 // Every wait is bounded: a wait that runs out records RGLRU_ERR_TIMEOUT in the
@@ -35,6 +38,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -51,9 +55,9 @@ constexpr int INFO_RING = 8; // tile descriptors in flight (claimed ahead)
 constexpr int kScanGroups = 2;  // scan warp groups, alternate tiles
 constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
 constexpr int kConvWarp0 = kScanWarps;
-constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kLbWarp = kMmaWarp + 1, kSchedWarp = kMmaWarp + 2;
-constexpr int kPubWarp = kMmaWarp + 3;
-constexpr int kThreads = 32 * (kPubWarp + 1);
+constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kSchedWarp = kMmaWarp + 1;
+constexpr int kLbWarp0 = kMmaWarp + 2, kLbWarps = SLOTS;  // look-back warp s serves slot s
+constexpr int kThreads = 32 * (kLbWarp0 + kLbWarps);
 constexpr int kGroupThreads = 128;  // threads of one scan group (one per channel)
 
 // TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
@@ -122,7 +126,7 @@ struct FusedParams {
 enum TraceEvent {
     TR_SCHED_INFO, TR_CONV_START, TR_CONV_DONE, TR_MMA_ISSUED, TR_P1_START, TR_P1_END, TR_LB_START,
     TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, TR_MMA_TFREE, TR_MMA_TMA, TR_MMA_CONV,
-    kTraceEvents
+    TR_CONV_GO, kTraceEvents
 };
 #ifdef RGLRU_TRACE
 constexpr int kTraceCtas = 4, kTraceTiles = 128;
@@ -204,7 +208,15 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, vo
     if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, hdr, where) ? 1u : 0u;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) {
-        while (!mbar_try_wait(bar, parity)) {
+        // the phase is complete, so each lane's own test passes at once unless
+        // the barrier had already moved on a further phase (a logic error,
+        // reported rather than waited on)
+        bool seen = false;
+        for (uint32_t it = 0; it < (1u << 20) && !(seen = mbar_try_wait(bar, parity)); ++it) {
+        }
+        if (!__all_sync(0xffffffffu, seen)) {
+            if ((threadIdx.x & 31) == 0) raise_timeout(abort_flag, hdr, where + 32);
+            ok = 0;
         }
     }
     return ok != 0;
@@ -272,22 +284,6 @@ __device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_
     }
 }
 
-__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
-{
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        f[2 * k] = __uint_as_float(w[k] << 16);
-        f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
 // 1 - exp(2l) = -(exp(2l) - 1) for -1/8 < l <= 0 by its Taylor series
 // -2l (1 + l + 2/3 l^2 + 1/3 l^3 + ...), cut after l^3: the first term left
 // out is 2/15 l^4, under 3.3e-5 relative for |l| < 1/8.
@@ -297,6 +293,19 @@ __device__ __forceinline__ float one_minus_exp2l_small(float l)
     s = fmaf(l, s, 1.f);
     s = fmaf(l, s, 1.f);
     return (-2.f * l) * s;
+}
+
+// GELU_tanh of two values: the polynomial argument in fp32 pairs, the tanh on
+// the f16x2 unit (its error, under 2^-10 relative, is well below the bf16
+// rounding of the product the result feeds)
+__device__ __forceinline__ f2_t gelu2(f2_t g)
+{
+    const f2_t k0 = f2_splat(0.7978845608028654f), k1 = f2_splat(0.7978845608028654f * 0.044715f);
+    const f2_t u = f2_mul(g, f2_fma(f2_mul(k1, g), g, k0));
+    float t0, t1;
+    tanh2_f16(f2_lo(u), f2_hi(u), t0, t1);
+    const f2_t hg = f2_mul(f2_splat(0.5f), g);
+    return f2_fma(hg, f2_make(t0, t1), hg);
 }
 
 __device__ __forceinline__ float gelu_tanh_fast(float g)
@@ -419,7 +428,11 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             return ti;
         };
         TileInfo next = claim();
-        int ends = 0;      // end markers written: one per scan group (each reads its own tiles)
+        // end markers: one per scan group and one per look-back warp (each of
+        // those reads only its own residue class of tiles)
+        constexpr int kEndMarkers = kScanGroups > kLbWarps ? kScanGroups : kLbWarps;
+        static_assert(kEndMarkers <= INFO_RING, "end markers fit the ring");
+        int ends = 0;
         int x_issued = 0;  // x-tile TMA loads issued
 #pragma unroll 1
         for (int j = 0;; ++j) {
@@ -435,7 +448,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 RGLRU_TR(TR_TILE_U, j, (unsigned long long)(unsigned)next.u);
             }
             if (next.u < 0) {
-                if (++ends == kScanGroups || !ok) break;
+                if (++ends == kEndMarkers || !ok) break;
                 continue;
             }
             // x rows t0-3 .. t0+31 of all 256 channels of the head into the x ring
@@ -513,23 +526,28 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         }
     } else if (warp >= kConvWarp0 && warp < kConvWarp0 + kConvWarps) {
         // ------------------------------------------------------------ conv warps
-        const int kb = warp - kConvWarp0;  // K-block: channels [64 kb, 64 kb + 64) of the head
-        const int cg = lane & 7;           // 8 channels per lane
-        const int q = lane >> 3;           // token quarter of the tile
-        const int dl = kb * 64 + cg * 8;   // channel within the head
+        // Warp kb covers the head's channels [64 kb, 64 kb + 64) (one K-block of
+        // the B tile); lane = (token half q, group of 4 channels cg), so each
+        // lane runs 16 consecutive tokens of 4 channels, in fp32 pairs.
+        const int kb = warp - kConvWarp0;
+        const int cg = lane & 15;
+        const int q = lane >> 4;
+        const int dl = kb * 64 + cg * 4;  // channel within the head
         const size_t d0 = (size_t)head * 256 + dl;
         // The conv produces xh = xc / 2 (halving is exact): the MMA then yields
         // half pre-activations, which is what sigmoid(z) = (1 + tanh(z/2)) / 2
         // needs, and the scan's i*xc becomes one FMA on xh.
-        float w[4][8], cb[8];
+        f2_t w2[4][2], cb2[2];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[k][e] = 0.5f * p.conv_w[(size_t)k * p.D + d0 + e];
+            for (int e = 0; e < 2; ++e)
+                w2[k][e] = f2_make(0.5f * p.conv_w[(size_t)k * p.D + d0 + 2 * e],
+                                   0.5f * p.conv_w[(size_t)k * p.D + d0 + 2 * e + 1]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) cb[e] = 0.5f * p.conv_b[d0 + e];
+        for (int e = 0; e < 2; ++e) cb2[e] = f2_make(0.5f * p.conv_b[d0 + 2 * e], 0.5f * p.conv_b[d0 + 2 * e + 1]);
         const bool own = (kb >> 1) == half;
-        const int xcs_col = (kb & 1) * 64 + cg * 8;
+        const int xcs_c = (kb & 1) * 64 + cg * 4;  // channel within this half
 #pragma unroll 1
         for (int j = 0;; ++j) {
             const int s = j % SLOTS, ir = j % INFO_RING;
@@ -541,57 +559,72 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const int xr = j % XRING;
             if (!warp_wait_bar(x_full(xr), (uint32_t)(j / XRING) & 1u, abort_flag, hdr, 16)) break;
             if (j >= SLOTS && !warp_wait_bar(bar(BAR_SMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
-            const int n0 = q * 8;
+            if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_GO, j, globaltimer());
+            const int n0 = q * 16;
             const uint8_t *xt = smem + OFF_X + xr * kXTile + dl * 2;  // row r = token t0 - 3 + r
-            auto xrow = [&](int r, float (&f)[8]) {
+            auto xrow = [&](int r, f2_t (&f)[2]) {
                 const int t = ti.t0 - 3 + r;
-                uint4 v;
+                uint2 v;
                 if (t >= 0)
-                    v = *reinterpret_cast<const uint4 *>(xt + r * 512);
+                    v = *reinterpret_cast<const uint2 *>(xt + r * 512);
                 else
-                    v = *reinterpret_cast<const uint4 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + t) * p.D + d0);
-                unpack8(v, f);
+                    v = *reinterpret_cast<const uint2 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + t) * p.D + d0);
+                f[0] = f2_from_bf16x2(v.x);
+                f[1] = f2_from_bf16x2(v.y);
             };
-            float xm3[8], xm2[8], xm1[8];
-            xrow(n0, xm3);
-            xrow(n0 + 1, xm2);
-            xrow(n0 + 2, xm1);
             uint8_t *btile = smem + OFF_B + s * kBTile + kb * kBBlock;
+            // fp32 xh of this half, token pairs interleaved: [t / 2][channel][t % 2]
             float *xcs = reinterpret_cast<float *>(smem + OFF_XCS + s * kXcsTile);
+            // a tile with no document start and all 32 tokens valid needs no masks
+            const bool clean = (ti.reset_mask | ti.m2 | ti.m3) == 0u && ti.valid == NT;
+            auto run = [&](auto clean_tag) {
+                constexpr bool kClean = decltype(clean_tag)::value;
+                f2_t xm3[2], xm2[2], xm1[2], prev[2];
+                xrow(n0, xm3);
+                xrow(n0 + 1, xm2);
+                xrow(n0 + 2, xm1);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float x0[8];
-                xrow(n0 + i + 3, x0);
-                const int n = n0 + i;
-                const bool k1 = !((ti.reset_mask >> n) & 1u), k2 = !((ti.m2 >> n) & 1u), k3 = !((ti.m3 >> n) & 1u);
-                float xc[8];
+                for (int i = 0; i < 16; ++i) {
+                    f2_t x0[2];
+                    xrow(n0 + i + 3, x0);
+                    const int n = n0 + i;
+                    f2_t acc[2];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float acc = cb[e];
-                    if (k3) acc = fmaf(w[0][e], xm3[e], acc);
-                    if (k2) acc = fmaf(w[1][e], xm2[e], acc);
-                    if (k1) acc = fmaf(w[2][e], xm1[e], acc);
-                    acc = fmaf(w[3][e], x0[e], acc);
-                    xc[e] = n < ti.valid ? acc : 0.f;
-                }
-                uint4 pk;
-                pk.x = pack_bf16x2(xc[0], xc[1]);
-                pk.y = pack_bf16x2(xc[2], xc[3]);
-                pk.z = pack_bf16x2(xc[4], xc[5]);
-                pk.w = pack_bf16x2(xc[6], xc[7]);
-                *reinterpret_cast<uint4 *>(btile + n * 128 + ((cg ^ (n & 7)) << 4)) = pk;
-                if (own) {
-                    float4 *dst = reinterpret_cast<float4 *>(xcs + n * kHalf + xcs_col);
-                    dst[0] = make_float4(xc[0], xc[1], xc[2], xc[3]);
-                    dst[1] = make_float4(xc[4], xc[5], xc[6], xc[7]);
-                }
+                    for (int e = 0; e < 2; ++e) {
+                        if constexpr (kClean) {
+                            acc[e] = f2_fma(w2[3][e], x0[e],
+                                            f2_fma(w2[2][e], xm1[e], f2_fma(w2[1][e], xm2[e], f2_fma(w2[0][e], xm3[e], cb2[e]))));
+                        } else {
+                            // tap of lag k dropped when segment_pos < k (document start)
+                            f2_t v = cb2[e];
+                            if (!((ti.m3 >> n) & 1u)) v = f2_fma(w2[0][e], xm3[e], v);
+                            if (!((ti.m2 >> n) & 1u)) v = f2_fma(w2[1][e], xm2[e], v);
+                            if (!((ti.reset_mask >> n) & 1u)) v = f2_fma(w2[2][e], xm1[e], v);
+                            v = f2_fma(w2[3][e], x0[e], v);
+                            acc[e] = n < ti.valid ? v : 0ull;
+                        }
+                    }
+                    // B tile row n: 4 channels = the (cg & 1) half of 16-byte chunk cg >> 1
+                    *reinterpret_cast<uint2 *>(btile + n * 128 + (((cg >> 1) ^ (n & 7)) << 4) + (cg & 1) * 8) =
+                        make_uint2(f2_to_bf16x2(acc[0]), f2_to_bf16x2(acc[1]));
+                    if ((i & 1) && own) {
+                        float4 *dst = reinterpret_cast<float4 *>(xcs + ((n >> 1) * kHalf + xcs_c) * 2);
+                        dst[0] = make_float4(f2_lo(prev[0]), f2_lo(acc[0]), f2_hi(prev[0]), f2_hi(acc[0]));
+                        dst[1] = make_float4(f2_lo(prev[1]), f2_lo(acc[1]), f2_hi(prev[1]), f2_hi(acc[1]));
+                    }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    xm3[e] = xm2[e];
-                    xm2[e] = xm1[e];
-                    xm1[e] = x0[e];
+                    for (int e = 0; e < 2; ++e) {
+                        prev[e] = acc[e];
+                        xm3[e] = xm2[e];
+                        xm2[e] = xm1[e];
+                        xm1[e] = x0[e];
+                    }
                 }
-            }
+            };
+            if (clean)
+                run(std::true_type{});
+            else
+                run(std::false_type{});
             mbar_arrive(x_empty(xr));
             fence_proxy_async_smem();
             mbar_arrive(bar(BAR_CONV, s));
@@ -613,6 +646,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // every log a of this channel lies in [kl, 0]: the short series for
         // 1 - a^2 applies to all of them when kl > -1/8
         const bool series_ok = kl > -0.125f;
+        const f2_t hba2 = f2_splat(hba), hbx2 = f2_splat(hbx), hkl_2 = f2_splat(hkl), hkl2_2 = f2_splat(hkl2);
+        const f2_t c13_2 = f2_splat(1.f / 3.f), c23_2 = f2_splat(2.f / 3.f), one_2 = f2_splat(1.f),
+                   mtwo_2 = f2_splat(-2.f);
 
         auto pass1 = [&](int j) -> bool {
             const int s = j % SLOTS;
@@ -622,8 +658,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (c == 0) RGLRU_TR(TR_P1_START, j, globaltimer());
             tc_fence_after();
             const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
-            const float *xcs = reinterpret_cast<const float *>(smem + OFF_XCS + s * kXcsTile);
+            // xh of tokens (2m, 2m + 1) of this channel: one 8-byte load
+            const float2 *xcs2 = reinterpret_cast<const float2 *>(smem + OFF_XCS + s * kXcsTile) + c;
             float hl = 0.f, P = 1.f;
+            f2_t lsum = 0ull;  // clean chunks: sum of log2 a (P = 2^sum at the end)
 #pragma unroll 1
             for (int t8 = 0; t8 < NT; t8 += 8) {
                 uint32_t ar[8], ai[8];
@@ -633,23 +671,36 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 const bool clean = ((ti.reset_mask >> t8) & 0xffu) == 0u && t8 + 8 <= ti.valid && series_ok;
                 if (clean) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float xh = xcs[(t8 + k) * kHalf + c];
-                        const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
-                        const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
-                        const float ell = fmaf(tr, hkl, hkl);
-                        const float a = ex2_approx(fmaf(tr, hkl2, hkl2));
-                        const float v = sqrt_approx(one_minus_exp2l_small(ell)) * fmaf(tg, xh, xh);
-                        hl = fmaf(a, hl, v);
-                        P *= a;
-                        ar[k] = __float_as_uint(a);
-                        ai[k] = __float_as_uint(v);
+                    for (int k = 0; k < 8; k += 2) {
+                        const float2 xh = xcs2[((t8 + k) >> 1) * kHalf];
+                        const f2_t zr = f2_add(f2_make(__uint_as_float(ar[k]), __uint_as_float(ar[k + 1])), hba2);
+                        const f2_t zi = f2_add(f2_make(__uint_as_float(ai[k]), __uint_as_float(ai[k + 1])), hbx2);
+                        const f2_t tr = f2_make(tanh_approx(f2_lo(zr)), tanh_approx(f2_hi(zr)));
+                        const f2_t tg = f2_make(tanh_approx(f2_lo(zi)), tanh_approx(f2_hi(zi)));
+                        const f2_t ell = f2_fma(tr, hkl_2, hkl_2);    // log a
+                        const f2_t la = f2_fma(tr, hkl2_2, hkl2_2);  // log2 a
+                        lsum = f2_add(lsum, la);
+                        const float a0 = ex2_approx(f2_lo(la)), a1 = ex2_approx(f2_hi(la));
+                        // 1 - exp(2 ell) by its series (see one_minus_exp2l_small)
+                        f2_t sr = f2_fma(ell, c13_2, c23_2);
+                        sr = f2_fma(ell, sr, one_2);
+                        sr = f2_fma(ell, sr, one_2);
+                        const f2_t om = f2_mul(f2_mul(ell, mtwo_2), sr);
+                        const f2_t nrm = f2_make(sqrt_approx(f2_lo(om)), sqrt_approx(f2_hi(om)));
+                        const f2_t xh2 = f2_make(xh.x, xh.y);
+                        const f2_t v = f2_mul(nrm, f2_fma(tg, xh2, xh2));  // sqrt(1-a^2) * i * xc
+                        hl = fmaf(a0, hl, f2_lo(v));
+                        hl = fmaf(a1, hl, f2_hi(v));
+                        ar[k] = __float_as_uint(a0);
+                        ar[k + 1] = __float_as_uint(a1);
+                        ai[k] = __float_as_uint(f2_lo(v));
+                        ai[k + 1] = __float_as_uint(f2_hi(v));
                     }
                 } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int t = t8 + k;
-                        const float xh = xcs[t * kHalf + c];
+                        const float xh = reinterpret_cast<const float *>(xcs2 + (t >> 1) * kHalf)[t & 1];
                         const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
                         const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
                         const float ell = fmaf(tr, hkl, hkl);
@@ -674,9 +725,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 tmem_st8(col + t8, ar);
                 tmem_st8(col + NT + t8, ai);
             }
+            P *= ex2_approx(f2_lo(lsum) + f2_hi(lsum));
             mbar_arrive(bar(BAR_SMEM_FREE, s));  // xcs (and, via the MMA wait, the B tile) consumed
             tmem_wait_st();
-            // the publisher warp must have copied out this slot's previous aggregate
+            // the look-back warp must have copied out this slot's previous aggregate
             if (j >= SLOTS && !warp_wait_bar(bar(BAR_PUB, s), ph ^ 1u, abort_flag, hdr, 17)) return false;
             reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = make_float2(P, hl);
             mbar_arrive(bar(BAR_PASS1, s));
@@ -694,8 +746,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (c == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
             tc_fence_after();
             const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
-            const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile);
+            const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile) + c;
             __nv_bfloat16 *yp = p.y + ((size_t)ti.b * p.T + ti.t0) * p.D + d;
+            const size_t ystep = p.D;
 #pragma unroll 1
             for (int t8 = 0; t8 < NT; t8 += 8) {
                 uint32_t aa[8], vv[8];
@@ -704,10 +757,15 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 tmem_wait_ld();
                 if (t8 + 8 <= ti.valid) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
+                    for (int k = 0; k < 8; k += 2) {
                         h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
-                        const float gv = __bfloat162float(gs[(t8 + k) * kHalf + c]);
-                        yp[(size_t)(t8 + k) * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                        const float h0 = h;
+                        h = fmaf(__uint_as_float(aa[k + 1]), h, __uint_as_float(vv[k + 1]));
+                        const f2_t gv = f2_make(__bfloat162float(gs[(t8 + k) * kHalf]), __bfloat162float(gs[(t8 + k + 1) * kHalf]));
+                        const uint32_t yy = f2_to_bf16x2(f2_mul(gelu2(gv), f2_make(h0, h)));
+                        const __nv_bfloat162 y2 = *reinterpret_cast<const __nv_bfloat162 *>(&yy);
+                        yp[(size_t)(t8 + k) * ystep] = y2.x;
+                        yp[(size_t)(t8 + k + 1) * ystep] = y2.y;
                     }
                 } else {
 #pragma unroll
@@ -715,8 +773,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const int t = t8 + k;
                         h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
                         if (t < ti.valid) {
-                            const float gv = __bfloat162float(gs[t * kHalf + c]);
-                            yp[(size_t)t * p.D] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
+                            const float gv = __bfloat162float(gs[t * kHalf]);
+                            yp[(size_t)t * ystep] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
                         }
                     }
                 }
@@ -760,39 +818,22 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (ok && j >= kScanGroups) ok = pass2(j - kScanGroups);
             if (!ok || end) break;
         }
-    } else if (warp == kPubWarp) {
-        // ------------------------------------------------------------ publisher
-        // Publishes each tile aggregate as soon as pass 1 ends (decoupled
-        // look-back: later tiles of the sequence may combine it before this
-        // tile's own look-back has finished).  It is the only warp that fences
-        // for the aggregates, and it has no other global stores in flight.
-#pragma unroll 1
-        for (int j = 0;; ++j) {
-            const int s = j % SLOTS, ir = j % INFO_RING;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 18)) break;
-            const TileInfo ti = info[ir];
-            if (ti.u < 0) break;
-            if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 19)) break;
-            const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
-            if ((int)gu != debug_unit) {
-                const float4 *src = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
-                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf);
-                dst[lane] = src[lane];
-                dst[lane + 32] = src[lane + 32];
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | (ti.reset_mask ? F_RESET : 0u));
-            }
-            mbar_arrive(bar(BAR_PUB, s));
-        }
-    } else if (warp == kLbWarp) {
-        // ------------------------------------------------------------ look-back warp
+    } else if (warp >= kLbWarp0) {
+        // ------------------------------------------------------------ look-back warps
+        // Warp s serves the tiles of slot s (j = s, s + SLOTS, ...), so it waits on
+        // its slot's barriers one phase at a time.  Per tile: publish the
+        // aggregate (later tiles of the sequence may combine it before this
+        // tile's own look-back has finished), find the anchor, fold, hand the
+        // carried-in state to pass 2, publish the inclusive prefix.  These warps
+        // are the only ones that fence for the aggregates and prefixes.
+        const int s = warp - kLbWarp0;
         const int ch = lane * 4;  // 4 channels per lane
         const size_t dch = (size_t)head * 256 + half * kHalf + ch;
+        const size_t gbase = (size_t)group * p.tiles_per_group;
+        constexpr int kFoldBatch = 4;  // aggregates loaded per round trip
 #pragma unroll 1
-        for (int j = 0;; ++j) {
-            const int s = j % SLOTS, ir = j % INFO_RING;
+        for (int j = s;; j += SLOTS) {
+            const int ir = j % INFO_RING;
             const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
             if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 13)) break;
             const TileInfo ti = info[ir];
@@ -801,18 +842,26 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (lane == 0) RGLRU_TR(TR_LB_START, j, globaltimer());
             const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
             const float4 g01 = sagg[lane * 2], g23 = sagg[lane * 2 + 1];  // (A,H) of 4 channels
+            mbar_arrive(bar(BAR_PUB, s));  // the slot's aggregate buffer is free again
             const float A[4] = {g01.x, g01.z, g23.x, g23.z};
             const float Hh[4] = {g01.y, g01.w, g23.y, g23.w};
-            const size_t gu = (size_t)group * p.tiles_per_group + ti.u;
+            const size_t gu = gbase + ti.u;
             const uint32_t rbit = ti.reset_mask ? F_RESET : 0u;
             const bool suppress = (int)gu == debug_unit;
+            if (!suppress) {
+                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf + ch);
+                dst[0] = g01;
+                dst[1] = g23;
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | rbit);
+            }
             float hin[4];
             bool ok = true;
             if (ti.first_last & 1) {
                 const float4 hs = *reinterpret_cast<const float4 *>(p.h_state + (size_t)ti.b * p.D + dch);
                 hin[0] = hs.x; hin[1] = hs.y; hin[2] = hs.z; hin[3] = hs.w;
             } else {
-                const size_t gbase = (size_t)group * p.tiles_per_group;
                 int anchor = -1;
                 uint32_t aflag = 0;
                 ok = find_anchor(p.flags + gbase, ti.u - 1, ti.b * p.C, anchor, aflag, abort_flag, hdr);
@@ -829,10 +878,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         hin[0] = a01.y; hin[1] = a01.w; hin[2] = a23.y; hin[3] = a23.w;
                     }
 #pragma unroll 1
-                    for (int p0 = anchor + 1; p0 < ti.u; p0 += 8) {
-                        float4 dd[8][2];
+                    for (int p0 = anchor + 1; p0 < ti.u; p0 += kFoldBatch) {
+                        float4 dd[kFoldBatch][2];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
+                        for (int k = 0; k < kFoldBatch; ++k) {
                             if (p0 + k < ti.u) {
                                 const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + p0 + k) * kHalf + ch);
                                 dd[k][0] = ld_relaxed_f4(src);
@@ -840,7 +889,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                             }
                         }
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
+                        for (int k = 0; k < kFoldBatch; ++k) {
                             if (p0 + k < ti.u) {
                                 hin[0] = fmaf(dd[k][0].x, hin[0], dd[k][0].y);
                                 hin[1] = fmaf(dd[k][0].z, hin[1], dd[k][0].w);
@@ -853,18 +902,19 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             if (!ok) break;
             if (lane == 0) RGLRU_TR(TR_LB_HIN, j, globaltimer());
-            float pre[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
+            // pass 2 needs only the carried-in state: hand it over before publishing
+            *reinterpret_cast<float4 *>(smem + OFF_HIN + s * kHalf * 4 + ch * 4) =
+                make_float4(hin[0], hin[1], hin[2], hin[3]);
+            mbar_arrive(bar(BAR_LB, s));
             if (!suppress) {
+                float pre[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
                 *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
             }
-            *reinterpret_cast<float4 *>(smem + OFF_HIN + s * kHalf * 4 + ch * 4) =
-                make_float4(hin[0], hin[1], hin[2], hin[3]);
-            mbar_arrive(bar(BAR_LB, s));
             if (lane == 0) RGLRU_TR(TR_LB_DONE, j, globaltimer());
         }
     }

@@ -128,9 +128,11 @@ def test_reset_makes_output_independent_of_earlier_tokens(simt):
     np.testing.assert_array_equal(alt["h_state"], base["h_state"])
 
 
-@pytest.mark.parametrize("io", ["bf16", "f32"])
-def test_decode_steps_match_oracle(io):
-    B, T, D = 64, 40, 512
+@pytest.mark.parametrize("io,B", [("bf16", 64), ("f32", 64), ("bf16", 100), ("bf16", 3)])
+def test_decode_steps_match_oracle(io, B):
+    """B = 100 leaves the second 64-row block of the bf16 decode kernel partial;
+    B = 3 is a single, mostly empty block."""
+    T, D = 40, 512
     _, inp = _case(B, T, D, io=io, reset_at=(0, 17))
     dev = to_device(inp, io)
     ys = []
