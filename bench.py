@@ -232,6 +232,8 @@ def run_cuda(args, w):
     stream = torch.cuda.current_stream(dev)
     api.load()
 
+    if args.profile_run and w.decode_steps:
+        return profile_decode(args, w, dev, rank, distributed)
     bf = torch.bfloat16 if w.io == "bf16" else torch.float32
     inp = W.generate(w)
     x = torch.from_numpy(inp["x"]).to(dev).to(bf)
@@ -371,6 +373,32 @@ def run_cuda(args, w):
                                 "sample": sample}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def profile_decode(args, w, dev, rank, distributed):
+    """--profile-run on a decode workload: warm-up and timed single-token steps
+    launched one by one (the command an ncu capture of the decode kernel wraps)."""
+    import torch
+    import torch.distributed as dist
+    args.decode_steps = args.decode_steps or (args.warmup + args.steps)
+    d = setup_decode(args, dev)
+    for t in range(args.warmup):
+        d["one"](t % d["steps"])
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for t in range(args.steps):
+        d["one"]((args.warmup + t) % d["steps"])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    st = d["status"]()
+    if rank == 0:
+        print(json.dumps({"profile_run": w.describe(), "steps": args.steps,
+                          "us_per_step": 1e3 * ev0.elapsed_time(ev1) / args.steps, "device_status": st}))
+    if distributed:
+        dist.destroy_process_group()
+    return 0 if st == 0 else 1
 
 
 def setup_decode(args, dev):

@@ -8,22 +8,23 @@
 // a head are the token dimension of its gate GEMM.
 //
 // Grid: one cluster of two CTAs per (head, block of kTok batch rows); CTA rank r
-// owns channels [128 r, 128 r + 128) of the head:
-//   1. every thread prefetches the h_state and GELU-branch values its epilogue
-//      needs (independent of everything else, so their latency overlaps the rest);
-//   2. one thread TMA-loads this half's 128 rows of W_a and W_x (128-byte
-//      swizzled, K-major: the tensor core's A operands);
-//   3. all threads run the conv of this half's channels for the block's rows,
-//      keep xc / 2 in fp32 for the epilogue, write its bf16 copy into the B
-//      tile of both CTAs of the cluster (this half's two K-blocks), and shift
-//      this half's conv_state rows; a cluster barrier completes both B tiles;
-//   4. one thread issues the 2 x 16 MMAs D[128 out x kTok rows] = W * xc^T;
-//   5. every warp reads its TMEM lane quarter for half of the rows and applies
-//      the gates, a = sigmoid(Lambda)^(8 r), the normalised one-step update (a
-//      reset when segment_pos == 0) and the GELU product.
+// owns channels [128 r, 128 r + 128) of the head.  Thread = one channel (its
+// TMEM lane) and 16 rows, for the conv and the epilogue alike:
+//   1. one thread TMA-loads this half's x and conv_state tiles and its 128 rows
+//      of W_a and W_x (128-byte swizzled, K-major: the tensor core's A
+//      operands); every thread prefetches the h_state and GELU-branch values
+//      of its rows into registers;
+//   2. the conv of the thread's channel keeps xc / 2 in registers, writes its
+//      bf16 copy into the B tile of both CTAs of the cluster, and shifts the
+//      conv_state tile in shared memory (rows 1, 2, x become rows 0, 1, 2),
+//      which a TMA store writes back; a cluster barrier completes both B tiles;
+//   3. one thread issues the 2 x 16 MMAs D[128 out x kTok rows] = W * xc^T;
+//   4. the epilogue applies the gates, a = sigmoid(Lambda)^(8 r), the
+//      normalised one-step update (a reset when segment_pos == 0) and the GELU
+//      product; y goes out through shared memory and a TMA store, h directly.
 // Each CTA reads and writes only its own channels of the states, so the two
 // CTAs never race.  Waits on mbarriers are bounded (RGLRU_ERR_TIMEOUT in the
-// workspace header); the cluster barrier is reached exactly once by every
+// workspace header); the two cluster barriers are reached exactly once by every
 // thread of both CTAs.
 //
 // Block structure: "Gemma explained: RecurrentGemma architecture",
@@ -44,18 +45,21 @@ using namespace sm100;
 
 constexpr int kTok = 64;        // batch rows per cluster: the MMA N
 constexpr int kHalfCh = 128;    // channels per CTA: the MMA M and TMEM lanes
-constexpr int kThreads = 256;   // 8 warps
-constexpr int kRowsPerWarp = kTok / 2;  // epilogue: warps w and w + 4 share a lane quarter
+constexpr int kThreads = 512;   // 16 warps: lane quarter (warp & 3), row group (warp >> 2)
+constexpr int kRows = kTok / 4;  // rows per thread
 
 constexpr int kWBlock = kHalfCh * 128;          // 128 weight rows x 64 channels (bf16): 16 KB
 constexpr int kWGate = 4 * kWBlock;             // one gate, K = 256: 64 KB
 constexpr int kBBlock = kTok * 128;             // kTok rows x 64 channels (bf16): 8 KB
+constexpr int kXTile = kTok * kHalfCh * 2;      // [kTok][128] bf16: 16 KB
+constexpr int kCsTile = 3 * kXTile;             // [kTok][3][128] bf16: 48 KB
 constexpr int OFF_W = 0;                        // W_a rows, then W_x rows
 constexpr int OFF_B = OFF_W + 2 * kWGate;       // B tile: 4 K-blocks (all 256 channels of the head)
-constexpr int OFF_XC = OFF_B + 4 * kBBlock;     // fp32 xc / 2 of this half: [kTok][128]
-constexpr int OFF_SP = OFF_XC + kTok * kHalfCh * 4;  // segment_pos of the block's rows
-constexpr int OFF_BAR = OFF_SP + kTok * 4;      // W loaded, MMA done
-constexpr int OFF_MISC = OFF_BAR + 2 * 8;       // TMEM base address
+constexpr int OFF_X = OFF_B + 4 * kBBlock;      // x tile, later the y tile
+constexpr int OFF_CS = OFF_X + kXTile;          // conv_state tile
+constexpr int OFF_SP = OFF_CS + kCsTile;        // segment_pos of the block's rows
+constexpr int OFF_BAR = OFF_SP + kTok * 4;      // x and conv_state loaded, W loaded, MMA done
+constexpr int OFF_MISC = OFF_BAR + 4 * 8;       // TMEM base address
 constexpr int kSmemUsed = OFF_MISC + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -64,13 +68,17 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 struct DecodeParams {
     int B, D, nblk;
-    const __nv_bfloat16 *x, *g;
+    const __nv_bfloat16 *g;
     const float *conv_w, *conv_b, *b_a, *b_x, *lambda;
     const int32_t *segpos;
-    __nv_bfloat16 *conv_state;
     float *h_state;
-    __nv_bfloat16 *y;
     WsHeader *hdr;
+};
+
+struct DecodeMaps {
+    CUtensorMap wa, wx;  // [D rows, 256] bf16, 64 x 128 boxes, 128-byte swizzle
+    CUtensorMap x, y;    // [B, D] bf16, 128 x kTok boxes
+    CUtensorMap cs;      // conv_state [B, 3, D] bf16, 128 x 3 x kTok boxes
 };
 
 // Bounded wait on an mbarrier phase by every lane of a warp; false (and the
@@ -111,9 +119,11 @@ __device__ __forceinline__ float gelu_tanh(float g)
     return fmaf(hg, tanh_approx(u), hg);
 }
 
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_wa,
-                    const __grid_constant__ CUtensorMap tmap_wx)
+rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_wa,
+                    const __grid_constant__ CUtensorMap tm_wx, const __grid_constant__ CUtensorMap tm_x,
+                    const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_cs)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -122,22 +132,42 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const int cluster = blockIdx.x >> 1;
     const int head = cluster / p.nblk, blk = cluster % p.nblk;
     const int b0 = blk * kTok;
-    const int nb = min(kTok, p.B - b0);  // valid rows of this block
+    const int nb = min(kTok, p.B - b0);                // valid rows of this block
     const int ch0 = head * 256 + (int)half * kHalfCh;  // first channel of this CTA
-    uint64_t *bar_w = reinterpret_cast<uint64_t *>(smem + OFF_BAR), *bar_mma = bar_w + 1;
+    uint64_t *bar_in = reinterpret_cast<uint64_t *>(smem + OFF_BAR), *bar_w = bar_in + 1, *bar_mma = bar_in + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     int32_t *sp_s = reinterpret_cast<int32_t *>(smem + OFF_SP);
-    float *xcs = reinterpret_cast<float *>(smem + OFF_XC);
+    const __nv_bfloat16 *x_s = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_X);  // [kTok][128]
+    __nv_bfloat16 *cs_s = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_CS);            // [kTok][3][128]
 
-    // ---- 1. epilogue operands: lane quarter (warp & 3) = channels, rows [32 (warp >> 2), +32)
+    // thread = channel c of this half (TMEM lane c) and rows [n0, n0 + kRows)
     const int c = (warp & 3) * 32 + lane;
     const int d = ch0 + c;
-    const int n_base = (warp >> 2) * kRowsPerWarp;
-    float hprev[kRowsPerWarp];
-    uint32_t graw[kRowsPerWarp / 2];  // bf16 pairs of consecutive rows
+    const int n0 = (warp >> 2) * kRows;
+
+    // ---- 1. loads
+    if (tid == 32) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_w, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        mbar_arrive_expect_tx(bar_in, kXTile + kCsTile);  // whole boxes: rows past B arrive zero-filled
+        tma_load_2d(smem + OFF_X, &tm_x, bar_in, ch0, b0);
+        tma_load_3d(smem + OFF_CS, &tm_cs, bar_in, ch0, 0, b0);
+        mbar_arrive_expect_tx(bar_w, 2 * kWGate);
 #pragma unroll
-    for (int k = 0; k < kRowsPerWarp; k += 2) {
-        const int n = n_base + k;
+        for (int kb = 0; kb < 4; ++kb) {
+            tma_load_2d(smem + OFF_W + kb * kWBlock, &tm_wa, bar_w, kb * 64, ch0);
+            tma_load_2d(smem + OFF_W + kWGate + kb * kWBlock, &tm_wx, bar_w, kb * 64, ch0);
+        }
+    }
+    if (tid < kTok) sp_s[tid] = tid < nb ? p.segpos[b0 + tid] : 3;
+    if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
+    float hprev[kRows];
+    uint32_t graw[kRows / 2];  // bf16 pairs of consecutive rows
+#pragma unroll
+    for (int k = 0; k < kRows; k += 2) {
+        const int n = n0 + k;
         const size_t e0 = (size_t)(b0 + n) * p.D + d, e1 = e0 + p.D;
         const uint32_t g0 = n < nb ? (uint32_t)__bfloat16_as_ushort(p.g[e0]) : 0u;
         const uint32_t g1 = n + 1 < nb ? (uint32_t)__bfloat16_as_ushort(p.g[e1]) : 0u;
@@ -145,91 +175,60 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         hprev[k] = n < nb ? p.h_state[e0] : 0.f;
         hprev[k + 1] = n + 1 < nb ? p.h_state[e1] : 0.f;
     }
-
-    // ---- 2. TMEM, barriers, weights
-    if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
-    if (tid == 32) {
-        mbar_init(bar_w, 1);
-        mbar_init(bar_mma, 1);
-        mbar_fence_init();
-        mbar_arrive_expect_tx(bar_w, 2 * kWGate);
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-            tma_load_2d(smem + OFF_W + kb * kWBlock, &tmap_wa, bar_w, kb * 64, ch0);
-            tma_load_2d(smem + OFF_W + kWGate + kb * kWBlock, &tmap_wx, bar_w, kb * 64, ch0);
-        }
-    }
-
+    const float w0 = 0.5f * p.conv_w[d], w1 = 0.5f * p.conv_w[(size_t)p.D + d],
+                w2 = 0.5f * p.conv_w[2 * (size_t)p.D + d], w3 = 0.5f * p.conv_w[3 * (size_t)p.D + d];
+    const float cb = 0.5f * p.conv_b[d];
     // the peer CTA must be running before its shared memory is written
     tc_fence_before();
     cluster_sync();
-
-    // ---- 3. conv of this half: lane = 4 channels, warp = 8 rows
-    {
-        const int cg = lane;                 // channels ch0 + 4 cg .. + 3
-        const size_t dc = (size_t)ch0 + cg * 4;
-        f2_t w2[4][2], cb2[2];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                w2[k][e] = f2_make(0.5f * p.conv_w[(size_t)k * p.D + dc + 2 * e],
-                                   0.5f * p.conv_w[(size_t)k * p.D + dc + 2 * e + 1]);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) cb2[e] = f2_make(0.5f * p.conv_b[dc + 2 * e], 0.5f * p.conv_b[dc + 2 * e + 1]);
-        // this half's channels are K-blocks 2 half + (cg >> 4) of the B tile
-        const int kb = 2 * (int)half + (cg >> 4);
-        const uint32_t b_local = smem_u32(smem + OFF_B + kb * kBBlock);
-        const uint32_t b_peer = mapa_shared(b_local, half ^ 1u);
-        const int chunk = (cg & 15) >> 1;
-#pragma unroll 2
-        for (int i = 0; i < kTok / 8; ++i) {
-            const int n = warp * (kTok / 8) + i;
-            const int b = b0 + n;
-            f2_t acc[2] = {0ull, 0ull};
-            if (n < nb) {
-                const int sp = p.segpos[b];
-                const uint2 xv = *reinterpret_cast<const uint2 *>(p.x + (size_t)b * p.D + dc);
-                __nv_bfloat16 *cs = p.conv_state + (size_t)b * 3 * p.D + dc;
-                const uint2 s0 = *reinterpret_cast<const uint2 *>(cs);
-                const uint2 s1 = *reinterpret_cast<const uint2 *>(cs + p.D);
-                const uint2 s2 = *reinterpret_cast<const uint2 *>(cs + 2 * (size_t)p.D);
-                const uint32_t xw[2] = {xv.x, xv.y}, w0[2] = {s0.x, s0.y}, w1[2] = {s1.x, s1.y},
-                               w2r[2] = {s2.x, s2.y};
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    // tap of lag k dropped when segment_pos < k (document start)
-                    f2_t v = cb2[e];
-                    if (sp >= 3) v = f2_fma(w2[0][e], f2_from_bf16x2(w0[e]), v);
-                    if (sp >= 2) v = f2_fma(w2[1][e], f2_from_bf16x2(w1[e]), v);
-                    if (sp >= 1) v = f2_fma(w2[2][e], f2_from_bf16x2(w2r[e]), v);
-                    acc[e] = f2_fma(w2[3][e], f2_from_bf16x2(xw[e]), v);
-                }
-                // the window moves one step: rows (1, 2, x) become rows (0, 1, 2)
-                *reinterpret_cast<uint2 *>(cs) = s1;
-                *reinterpret_cast<uint2 *>(cs + p.D) = s2;
-                *reinterpret_cast<uint2 *>(cs + 2 * (size_t)p.D) = xv;
-                if (cg == 0) sp_s[n] = sp;
-            }
-            *reinterpret_cast<float4 *>(xcs + n * kHalfCh + cg * 4) =
-                make_float4(f2_lo(acc[0]), f2_hi(acc[0]), f2_lo(acc[1]), f2_hi(acc[1]));
-            const uint32_t off = n * 128 + ((chunk ^ (n & 7)) << 4) + (cg & 1) * 8;
-            const uint32_t lo = f2_to_bf16x2(acc[0]), hi = f2_to_bf16x2(acc[1]);
-            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(b_local + off), "r"(lo), "r"(hi) : "memory");
-            st_cluster_v2(b_peer + off, lo, hi);
-        }
-    }
-    fence_proxy_async_cluster();
-    cluster_sync();  // both halves of both B tiles written
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    // ---- 4. gate projections
-    bool ok = true;
+    // ---- 2. conv: xh = xc / 2 (halving is exact: the MMA then gives half
+    // pre-activations for sigmoid(z) = (1 + tanh(z / 2)) / 2)
+    bool ok = dec_wait(bar_in, 0, p.hdr, 0);
+    float xh[kRows];
+    {
+        const int k = (int)half * kHalfCh + c;  // channel within the head = K index of the B tile
+        const uint32_t b_local = smem_u32(smem + OFF_B + (k >> 6) * kBBlock);
+        const uint32_t b_peer = mapa_shared(b_local, half ^ 1u);
+        const int j = k & 63;
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+            const int n = n0 + i;
+            const int sp = sp_s[n];
+            __nv_bfloat16 *cr = cs_s + n * 3 * kHalfCh + c;
+            const __nv_bfloat16 xr = x_s[n * kHalfCh + c], c1 = cr[kHalfCh], c2 = cr[2 * kHalfCh];
+            // tap of lag k dropped when segment_pos < k (document start)
+            float v = cb;
+            if (sp >= 3) v = fmaf(w0, __bfloat162float(cr[0]), v);
+            if (sp >= 2) v = fmaf(w1, __bfloat162float(c1), v);
+            if (sp >= 1) v = fmaf(w2, __bfloat162float(c2), v);
+            v = fmaf(w3, __bfloat162float(xr), v);
+            xh[i] = v;
+            // the window moves one step: rows (1, 2, x) become rows (0, 1, 2)
+            cr[0] = c1;
+            cr[kHalfCh] = c2;
+            cr[2 * kHalfCh] = xr;
+            const uint32_t off = n * 128 + (((j >> 3) ^ (n & 7)) << 4) + (j & 7) * 2;
+            const uint16_t bv = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(b_local + off), "h"(bv) : "memory");
+            asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(b_peer + off), "h"(bv) : "memory");
+        }
+    }
+    fence_proxy_async_cluster();  // B tiles (both CTAs) and the conv_state tile, for the async proxy
+    tc_fence_before();
+    cluster_sync();               // both halves of both B tiles written
+    tc_fence_after();
+
+    // ---- 3. conv_state write-back and the gate projections
     if (warp == 1) {
-        ok = dec_wait(bar_w, 0, p.hdr, 0);
+        if (lane == 0) {
+            tma_store_3d(&tm_cs, smem + OFF_CS, ch0, 0, b0);  // rows past B are clipped
+            bulk_commit();
+        }
+        ok = dec_wait(bar_w, 0, p.hdr, 1) && ok;
         if (ok && lane == 0) {
-            fence_proxy_async_smem();
             tc_fence_after();
             const uint32_t idesc = umma_idesc_bf16(kHalfCh, kTok);
             const uint32_t wa = smem_u32(smem + OFF_W), wx = wa + kWGate, bt = smem_u32(smem + OFF_B);
@@ -245,48 +244,51 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         __syncwarp();
     }
 
-    // ---- 5. epilogue: thread = channel d (its TMEM lane), rows n_base .. n_base + 31
-    ok = dec_wait(bar_mma, 0, p.hdr, 1) && ok;
+    // ---- 4. epilogue
+    ok = dec_wait(bar_mma, 0, p.hdr, 2) && ok;
     tc_fence_after();
+    __nv_bfloat16 *y_s = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_X);  // the x tile is dead
     if (ok) {
         const float hba = 0.5f * p.b_a[d], hbx = 0.5f * p.b_x[d];
         const float lam = p.lambda[d];
         const float ls = lam >= 0.f ? -log1pf(expf(-lam)) : lam - log1pf(expf(lam));  // log sigmoid(Lambda)
         const float hkl = 0.5f * kC * ls;               // log a = (1 + tr) * hkl, tr = tanh(half pre-activation)
         const float hkl2 = hkl * 1.4426950408889634f;  // the same in log2
-        const uint32_t lane_col = tmem + ((uint32_t)((warp & 3) * 32) << 16) + n_base;
+        const uint32_t lane_col = tmem + ((uint32_t)((warp & 3) * 32) << 16) + n0;
 #pragma unroll
-        for (int k8 = 0; k8 < kRowsPerWarp; k8 += 8) {
+        for (int k8 = 0; k8 < kRows; k8 += 8) {
             uint32_t ar[8], ai[8];
             tmem_ld8(lane_col + k8, ar);
             tmem_ld8(lane_col + kTok + k8, ai);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const int n = n_base + k8 + k;
-                if (n < nb) {
-                    const float xh = xcs[n * kHalfCh + c];
-                    const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
-                    const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
-                    const float ell = fmaf(tr, hkl, hkl);
-                    const float a = ex2_approx(fmaf(tr, hkl2, hkl2));
-                    const float om = ell > -0.125f ? one_minus_exp2l(ell) : fmaf(-a, a, 1.f);
-                    const float uu = fmaf(tg, xh, xh);  // i * xc
-                    const float h = sp_s[n] == 0 ? uu : fmaf(a, hprev[k8 + k], sqrt_approx(om) * uu);
-                    const uint32_t gw = graw[(k8 + k) / 2];
-                    const float gv = __uint_as_float(((k8 + k) & 1) ? (gw & 0xffff0000u) : (gw << 16));
-                    const size_t e = (size_t)(b0 + n) * p.D + d;
-                    p.y[e] = __float2bfloat16_rn(gelu_tanh(gv) * h);
-                    p.h_state[e] = h;
-                }
+                const int i = k8 + k, n = n0 + i;
+                const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
+                const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
+                const float ell = fmaf(tr, hkl, hkl);
+                const float a = ex2_approx(fmaf(tr, hkl2, hkl2));
+                const float om = ell > -0.125f ? one_minus_exp2l(ell) : fmaf(-a, a, 1.f);
+                const float uu = fmaf(tg, xh[i], xh[i]);  // i * xc
+                const float h = sp_s[n] == 0 ? uu : fmaf(a, hprev[i], sqrt_approx(om) * uu);
+                const uint32_t gw = graw[i / 2];
+                const float gv = __uint_as_float((i & 1) ? (gw & 0xffff0000u) : (gw << 16));
+                y_s[n * kHalfCh + c] = __float2bfloat16_rn(gelu_tanh(gv) * h);
+                if (n < nb) p.h_state[(size_t)(b0 + n) * p.D + d] = h;
             }
         }
     }
-
-    // ---- teardown: TMEM reads done (or abandoned after a timeout) before the free
+    fence_proxy_async_smem();  // y tile, for the async proxy
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == 32) {
+        if (ok) {
+            tma_store_2d(&tm_y, smem + OFF_X, ch0, b0);  // rows past B are clipped
+            bulk_commit();
+        }
+        bulk_wait_read_all();  // shared memory stays valid until the stores have read it
+    }
     if (warp == 0) {
         if (!ok) {
             // a timed-out wait: give the MMAs in flight a bounded time to finish first
@@ -312,18 +314,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// [H * 256 rows, 256 channels] bf16 gate matrix, loaded as 128-row x 64-channel
-// boxes in the 128-byte swizzle the tensor core's K-major operand expects
-bool encode_weights(CUtensorMap *m, const void *W, int D)
+bool encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *m, const void *base, int rank,
+                 const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle sw)
 {
-    auto encode = encode_fn();
-    if (!encode) return false;
-    const cuuint64_t gdim[2] = {256, (cuuint64_t)D};
-    const cuuint64_t gstride[1] = {256 * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kHalfCh};
-    const cuuint32_t estride[2] = {1, 1};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(W), gdim, gstride, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const cuuint32_t estride[3] = {1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -333,8 +329,26 @@ size_t decode_workspace_bytes(int, int) { return kWsHeaderBytes; }
 
 rglru_status decode_step(const PrefillArgs &a)
 {
-    CUtensorMap tmap_wa, tmap_wx;
-    if (!encode_weights(&tmap_wa, a.W_a, a.D) || !encode_weights(&tmap_wx, a.W_x, a.D)) return RGLRU_ERR_CUDA;
+    auto encode = encode_fn();
+    if (!encode) return RGLRU_ERR_CUDA;
+    CUtensorMap tm_wa, tm_wx, tm_x, tm_y, tm_cs;
+    // gate matrices [D rows, 256]: 128-row x 64-channel boxes in the 128-byte
+    // swizzle of the tensor core's K-major operand
+    const cuuint64_t wdim[2] = {256, (cuuint64_t)a.D}, wstride[1] = {256 * 2};
+    const cuuint32_t wbox[2] = {64, (cuuint32_t)kHalfCh};
+    // [B, D] rows: 128 channels x kTok rows
+    const cuuint64_t rdim[2] = {(cuuint64_t)a.D, (cuuint64_t)a.B}, rstride[1] = {(cuuint64_t)a.D * 2};
+    const cuuint32_t rbox[2] = {(cuuint32_t)kHalfCh, (cuuint32_t)kTok};
+    // conv_state [B, 3, D]: 128 channels x 3 rows x kTok sequences
+    const cuuint64_t cdim[3] = {(cuuint64_t)a.D, 3, (cuuint64_t)a.B};
+    const cuuint64_t cstride[2] = {(cuuint64_t)a.D * 2, (cuuint64_t)a.D * 6};
+    const cuuint32_t cbox[3] = {(cuuint32_t)kHalfCh, 3, (cuuint32_t)kTok};
+    if (!encode_bf16(encode, &tm_wa, a.W_a, 2, wdim, wstride, wbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_bf16(encode, &tm_wx, a.W_x, 2, wdim, wstride, wbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_bf16(encode, &tm_x, a.x, 2, rdim, rstride, rbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_bf16(encode, &tm_y, a.y, 2, rdim, rstride, rbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_bf16(encode, &tm_cs, a.conv_state, 3, cdim, cstride, cbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return RGLRU_ERR_CUDA;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -346,7 +360,6 @@ rglru_status decode_step(const PrefillArgs &a)
     p.B = a.B;
     p.D = a.D;
     p.nblk = (a.B + kTok - 1) / kTok;
-    p.x = static_cast<const __nv_bfloat16 *>(a.x);
     p.g = static_cast<const __nv_bfloat16 *>(a.g);
     p.conv_w = a.conv_w;
     p.conv_b = a.conv_b;
@@ -354,13 +367,12 @@ rglru_status decode_step(const PrefillArgs &a)
     p.b_x = a.b_x;
     p.lambda = a.lambda;
     p.segpos = a.segpos;
-    p.conv_state = static_cast<__nv_bfloat16 *>(a.conv_state);
     p.h_state = a.h_state;
-    p.y = static_cast<__nv_bfloat16 *>(a.y);
     p.hdr = reinterpret_cast<WsHeader *>(a.ws);
     const long long clusters = (long long)(a.D / kHead) * p.nblk;
     if (clusters * 2 > 0x7fffffffLL) return RGLRU_ERR_UNSUPPORTED;
-    rglru_decode_kernel<<<(unsigned)(clusters * 2), kThreads, kSmemBytes, a.stream>>>(p, tmap_wa, tmap_wx);
+    rglru_decode_kernel<<<(unsigned)(clusters * 2), kThreads, kSmemBytes, a.stream>>>(p, tm_wa, tm_wx, tm_x, tm_y,
+                                                                                     tm_cs);
     return cuda_status(cudaGetLastError());
 }
 
