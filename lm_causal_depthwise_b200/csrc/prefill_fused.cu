@@ -201,8 +201,8 @@ __device__ __noinline__ uint32_t wait_flag(const uint32_t *f, uint32_t need, vol
 // Warp-collective forms: lane 0 waits, the result is broadcast, then every lane
 // performs its own (already satisfied) acquire so that the warp stays converged
 // for the .sync.aligned tcgen05 instructions that follow.
-__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                              WsHeader *hdr, int where)
+__device__ __noinline__ bool warp_wait_bar_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                WsHeader *hdr, int where)
 {
     uint32_t ok = 1;
     if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, hdr, where) ? 1u : 0u;
@@ -220,6 +220,14 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, vo
         }
     }
     return ok != 0;
+}
+
+// Fast path: a phase that is already complete costs one test per lane and a vote.
+__device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              WsHeader *hdr, int where)
+{
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    return warp_wait_bar_slow(bar, parity, abort_flag, hdr, where);
 }
 
 // Flags only gain bits during a launch; the value lane 0 saw drives every lane's
@@ -561,14 +569,18 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (j >= SLOTS && !warp_wait_bar(bar(BAR_SMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
             if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_GO, j, globaltimer());
             const int n0 = q * 16;
-            const uint8_t *xt = smem + OFF_X + xr * kXTile + dl * 2;  // row r = token t0 - 3 + r
+            uint8_t *xt = smem + OFF_X + xr * kXTile + dl * 2;  // row r = token t0 - 3 + r
+            if (ti.t0 == 0 && q == 0) {
+                // sequence start: rows 0..2 (tokens -3..-1, zero-filled by the
+                // load) are the carried conv state; each lane patches the 4
+                // channels it reads itself
+#pragma unroll
+                for (int r = 0; r < 3; ++r)
+                    *reinterpret_cast<uint2 *>(xt + r * 512) =
+                        *reinterpret_cast<const uint2 *>(p.conv_state + ((size_t)ti.b * 3 + r) * p.D + d0);
+            }
             auto xrow = [&](int r, f2_t (&f)[2]) {
-                const int t = ti.t0 - 3 + r;
-                uint2 v;
-                if (t >= 0)
-                    v = *reinterpret_cast<const uint2 *>(xt + r * 512);
-                else
-                    v = *reinterpret_cast<const uint2 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + t) * p.D + d0);
+                const uint2 v = *reinterpret_cast<const uint2 *>(xt + r * 512);
                 f[0] = f2_from_bf16x2(v.x);
                 f[1] = f2_from_bf16x2(v.y);
             };
@@ -583,7 +595,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 xrow(n0, xm3);
                 xrow(n0 + 1, xm2);
                 xrow(n0 + 2, xm1);
-#pragma unroll
+#pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
                     f2_t x0[2];
                     xrow(n0 + i + 3, x0);
@@ -625,8 +637,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 run(std::true_type{});
             else
                 run(std::false_type{});
-            mbar_arrive(x_empty(xr));
+            // generic writes (B tile, patched x rows) before the async proxy's
+            // next accesses (the MMA, the next load into this x slot)
             fence_proxy_async_smem();
+            mbar_arrive(x_empty(xr));
             mbar_arrive(bar(BAR_CONV, s));
             if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_DONE, j, globaltimer());
         }
