@@ -1,35 +1,40 @@
 // prefill_fused.cu -- fused sm_100a prefill of the RG-LRU block core (bf16 I/O, fp32 state).
 //
-// One persistent kernel does, per tile of 32 tokens of one (sequence, head, half
-// of the head's 256 channels):
-//   conv warps   causal depthwise conv (k=4, document mask) of all 256 input
-//                channels of the head, in fp32; bf16 copy into the MMA B tile
-//                (128-byte swizzled, K-major), fp32 copy of this half's channels
-//                for the scan.
+// One persistent kernel, launched as clusters of two CTAs per head: CTA rank r
+// owns channels [128 r, 128 r + 128) of the head (one TMEM lane per channel).
+// Both CTAs of a cluster walk the same sequence of tiles (32 tokens of one
+// sequence, claimed in order from the head's ticket counter by rank 0, which
+// writes each tile descriptor into both CTAs).  Per tile:
+//   conv warps   thread = channel: causal depthwise conv (k=4, document mask)
+//                of its channel over the tile in fp32; xc / 2 goes to TMEM (f16
+//                pairs) for the scan, its bf16 copy into the MMA B tile of BOTH
+//                CTAs (the two halves of the head's 256 input channels meet in
+//                each CTA's shared memory through the cluster).
 //   MMA thread   both block-diagonal gate projections on the tensor cores:
-//                D[128 out x 32 tok] = W[128 x 256] (A, resident in TMEM) * xc^T
-//                (B, shared memory), fp32 accumulators in TMEM.
-//   scan warps   one thread per output channel (= TMEM lane).  Pass 1: sigmoid
-//                gates, a = sigmoid(Lambda)^(8 r), sqrt(1-a^2) normaliser,
-//                resets; local scan from h = 0 gives the tile aggregate
-//                (prod a, h_end), published at once; (a, v) are written back
-//                over the accumulators.  Pass 2 (two tiles later): re-run the
-//                scan from the carried-in state, multiply by GELU_tanh(g),
-//                store y.
-//   look-back    one warp per slot, so that the look-backs of consecutive
-//   warps        tiles overlap.  Publishes the tile aggregate as soon as pass 1
-//                ends, walks back over predecessor tiles of the same sequence
-//                to the nearest anchor (a published inclusive prefix, or a tile
-//                that holds a reset: A = 0), folds h <- A h + H forward from it
-//                in sequence order (decoupled look-back with a fixed
-//                combination order, so results are bit-reproducible), hands
-//                the carried-in state to pass 2, then publishes the tile's
-//                inclusive prefix.
-//   producer     claims tiles in order from a per-(head, half) ticket counter,
-//                TMA-loads the GELU-branch tile, issues the MMAs.
+//                D[128 out x 32 tok] = W[128 x 256] * xc^T, A (this half's rows
+//                of W_a or W_x, TMA-loaded once, 128-byte swizzled) and B in
+//                shared memory, fp32 accumulators in TMEM.
+//   scan warps   thread = channel, two groups taking alternate tiles.  Pass 1:
+//                sigmoid gates, a = sigmoid(Lambda)^(8 r), sqrt(1-a^2)
+//                normaliser, resets, GELU_tanh(g); the local scan from h = 0
+//                gives the tile aggregate (prod a, h_end) and, per token, the
+//                output without the carried-in state, y_loc = G h_loc, and its
+//                coefficient q = G prod a, kept in TMEM as f16 pairs (the
+//                accumulators are free again at once).  Pass 2 (two tiles
+//                later): y = y_loc + q h_in.
+//   look-back    publish each tile aggregate as soon as pass 1 ends, walk back
+//   warps        over predecessor tiles of the sequence to the nearest anchor
+//                (a published inclusive prefix, or a tile holding a reset: A =
+//                0), fold h <- A h + H forward from it in sequence order
+//                (decoupled look-back with a fixed combination order, so
+//                results are bit-reproducible), hand h_in to pass 2, publish
+//                the inclusive prefix.
+//   scheduler    rank 0 claims tiles and fills both CTAs' descriptor rings;
+//                each CTA TMA-loads its own channels of x (tile + 3 halo rows).
 // Every wait is bounded: a wait that runs out records RGLRU_ERR_TIMEOUT in the
 // workspace header and the CTA unwinds (waiting, bounded, for its own copies
-// and MMAs in flight) and frees its TMEM.
+// and MMAs in flight), meets its peer at the final cluster barrier and frees
+// its TMEM.
 //
 // Block structure: "Gemma explained: RecurrentGemma architecture",
 // RecurrentGemmaRecurrentBlock printout (Conv1d k=4, padding=3, groups=D; GELU
@@ -48,75 +53,106 @@ namespace {
 
 using namespace sm100;
 
-constexpr int NT = 32;       // tokens per tile (MMA N)
-constexpr int SLOTS = 4;     // tiles in flight per CTA
-constexpr int kHalf = 128;   // output channels per CTA (MMA M, TMEM lanes)
-constexpr int INFO_RING = 8; // tile descriptors in flight (claimed ahead)
+constexpr int NT = 32;          // tokens per tile (MMA N)
+constexpr int kHalf = 128;      // channels per CTA (MMA M, TMEM lanes)
+constexpr int NX = 4;           // xc/2 slots in TMEM (conv -> pass 1)
+constexpr int NA = 4;           // accumulator slots in TMEM (MMA -> pass 1)
+constexpr int NS = 6;           // stash slots in TMEM (pass 1 -> pass 2)
+constexpr int NB = 2;           // B tiles in shared memory (conv -> MMA, both CTAs)
+constexpr int XRING = 2;        // x tiles in shared memory (TMA -> conv)
+constexpr int INFO_RING = 16;   // tile descriptors in flight
 constexpr int kScanGroups = 2;  // scan warp groups, alternate tiles
+constexpr int kP2Lag = 2;       // a group runs pass 2 of its tile kP2Lag tiles back
 constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
 constexpr int kConvWarp0 = kScanWarps;
 constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kSchedWarp = kMmaWarp + 1;
-constexpr int kLbWarp0 = kMmaWarp + 2, kLbWarps = SLOTS;  // look-back warp s serves slot s
+constexpr int kLbWarp0 = kMmaWarp + 2, kLbWarps = 3;
 constexpr int kThreads = 32 * (kLbWarp0 + kLbWarps);
-constexpr int kGroupThreads = 128;  // threads of one scan group (one per channel)
+constexpr int kGroupThreads = 128;  // threads of one scan group or of the conv warps (one per channel)
+constexpr int kEndMarkers = kLbWarps > kScanGroups ? kLbWarps : kScanGroups;
+// every barrier array is visited one phase at a time by each waiter: a scan
+// group's tiles use only its own accumulator and stash slots, a look-back
+// warp's tiles revisit a stash slot every lcm(kLbWarps, NS) = NS tiles
+static_assert(NA % kScanGroups == 0 && NS % kScanGroups == 0 && NS % kLbWarps == 0, "slot residues");
+static_assert(NS == kScanGroups * (kP2Lag + 1), "stash slots cover the pass-2 lag");
+static_assert(kEndMarkers <= INFO_RING, "end markers fit the ring");
 
-// TMEM columns (512 allocated): W_a half-head rows, W_x rows, then per slot
-// [pre_r | pre_i] accumulators that pass 1 overwrites with [a | v].
-constexpr uint32_t kColWa = 0, kColWx = 128, kColSlot0 = 256, kColPerSlot = 2 * NT;
+// TMEM columns (512): xc/2 f16 pairs, accumulators [pre_r | pre_i], stash f16 pairs
+constexpr uint32_t kColXh = 0, kColsXh = NT / 2;
+constexpr uint32_t kColAcc = kColXh + NX * kColsXh, kColsAcc = 2 * NT;
+constexpr uint32_t kColStash = kColAcc + NA * kColsAcc, kColsStash = NT;
+static_assert(kColStash + NS * kColsStash <= 512, "TMEM budget");
 
 // Shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kBTile = NT * 256 * 2;            // bf16 xc, 4 K-blocks of 64 channels
-constexpr int kBBlock = NT * 128;               // one K-block: NT rows x 128 B
-constexpr int kXcsTile = NT * kHalf * 4;        // fp32 xc / 2 of this half
-constexpr int kGTile = NT * kHalf * 2;          // bf16 gate-branch tile (TMA box)
-constexpr int XRING = 3;                         // x tiles (32 rows + 3 halo rows) in flight
+constexpr int kWBlock = kHalf * 128;            // 128 weight rows x 64 channels (bf16)
+constexpr int kWGate = 4 * kWBlock;             // one gate, K = 256
+constexpr int kBBlock = NT * 128;               // one K-block of the B tile: NT rows x 128 B
+constexpr int kBTile = 4 * kBBlock;             // bf16 xc of all 256 channels of the head
 constexpr int kXRows = NT + 3;
-constexpr int kXTile = kXRows * 256 * 2;         // bf16, all 256 channels of the head
-constexpr int OFF_B = 0;
-constexpr int OFF_XCS = OFF_B + SLOTS * kBTile;
-constexpr int OFF_G = OFF_XCS + SLOTS * kXcsTile;
-constexpr int OFF_X = OFF_G + SLOTS * kGTile;
-constexpr int OFF_AGG = OFF_X + XRING * kXTile;
-constexpr int OFF_HIN = OFF_AGG + SLOTS * kHalf * 8;
-constexpr int OFF_INFO = OFF_HIN + SLOTS * kHalf * 4;
+constexpr int kXTile = kXRows * kHalf * 2;      // bf16 x of this half, 3 halo rows first
+constexpr int OFF_W = 0;                        // W_a rows, then W_x rows of this half
+constexpr int OFF_B = OFF_W + 2 * kWGate;
+constexpr int OFF_X = OFF_B + NB * kBTile;
+constexpr int kGTile = NT * kHalf * 2;          // bf16 GELU branch of this half: [token][channel]
+constexpr int OFF_G = OFF_X + XRING * kXTile;   // one per scan group
+constexpr int OFF_Y = OFF_G + kScanGroups * kGTile;  // bf16 y of a tile, one per scan group
+// per stash slot: (prod a, h_end) per channel from pass 1; the look-back then
+// leaves the state after the tile (per channel) in the first half
+constexpr int OFF_AGG = OFF_Y + kScanGroups * kGTile;
+constexpr int OFF_HIN = OFF_AGG + NS * kHalf * 8;         // per stash slot: carried-in h per channel
+constexpr int OFF_INFO = OFF_HIN + NS * kHalf * 4;
 constexpr int OFF_BAR = OFF_INFO + INFO_RING * 32;
-// per-slot barriers (slot = tile % SLOTS)
-enum { BAR_CONV, BAR_SMEM_FREE, BAR_MMA, BAR_TMEM_FREE, BAR_PASS1, BAR_LB, BAR_G, BAR_PUB, BAR_KINDS };
-constexpr int OFF_RING_BAR = OFF_BAR + BAR_KINDS * SLOTS * 8;  // INFO_FULL[8], INFO_EMPTY[8]
-constexpr int OFF_XBAR = OFF_RING_BAR + 2 * INFO_RING * 8;         // X_FULL[3], X_EMPTY[3]
-constexpr int OFF_MISC = OFF_XBAR + 2 * XRING * 8;
-constexpr int kSmemUsed = OFF_MISC + 16 + SLOTS * 4;
+// barrier arrays: [first index, count]
+enum {
+    B_INFO_FULL = 0,
+    B_INFO_EMPTY = B_INFO_FULL + INFO_RING,
+    B_X_FULL = B_INFO_EMPTY + INFO_RING,
+    B_X_EMPTY = B_X_FULL + XRING,
+    B_XH_FREE = B_X_EMPTY + XRING,
+    B_BCONV = B_XH_FREE + NX,
+    B_BFREE = B_BCONV + NB,
+    B_MMA = B_BFREE + NB,
+    B_ACC_FREE = B_MMA + NA,
+    B_PASS1 = B_ACC_FREE + NA,
+    B_PUB = B_PASS1 + NS,
+    B_LB = B_PUB + NS,
+    B_STASH_FREE = B_LB + NS,
+    B_BHALF = B_STASH_FREE + NS,   // this CTA's half of a B tile written (before the copy to the peer)
+    B_YFULL = B_BHALF + NB,        // per scan group: its y tile written (before the tensor store)
+    B_YFREE = B_YFULL + kScanGroups,  // per scan group: the previous tensor store has read its y tile
+    B_W_FULL = B_YFREE + kScanGroups,
+    B_COUNT
+};
+constexpr int OFF_MISC = OFF_BAR + B_COUNT * 8;
+constexpr int kSmemUsed = OFF_MISC + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(OFF_B % 1024 == 0 && kBTile % 1024 == 0 && kXTile % 128 == 0, "alignment");
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 
 struct TileInfo {
-    int u;        // tile index inside the (head, half) group, -1 = no more work
+    int u;        // tile index inside the head's sequence of tiles, -1 = no more work
     int b, t0, valid;
     uint32_t reset_mask;  // bit t: segment_pos == 0 at token t0 + t (conv tap of lag 1 dropped, h reset)
     uint32_t m2, m3;      // bit t: segment_pos < 2 (< 3): conv tap of lag 2 (3) dropped
     int first_last;       // bit 0: first tile of the sequence, bit 1: last tile
 };
 static_assert(sizeof(TileInfo) == 32, "TileInfo size");
-static_assert(SLOTS * 2 == INFO_RING, "ring sizes");
 
 struct FusedParams {
-    int B, T, D, C, G, tiles_per_group;
-    const __nv_bfloat16 *x;
+    int B, T, D, C, tiles_per_head;
+    const __nv_bfloat16 *x, *g;
     const float *conv_w, *conv_b;
-    const __nv_bfloat16 *W_a;
-    const float *b_a;
-    const __nv_bfloat16 *W_x;
-    const float *b_x, *lambda;
+    const float *b_a, *b_x, *lambda;
     const int32_t *segpos;
     __nv_bfloat16 *conv_state;
     float *h_state;
     __nv_bfloat16 *y;
     WsHeader *hdr;
-    uint32_t *flags;   // [G][tiles_per_group]
-    float2 *agg;       // [G][tiles_per_group][128]  (prod a, h_end) from h = 0
-    float *prefix;     // [G][tiles_per_group][128]  h after the tile
+    uint32_t *flags;   // [2 H][tiles_per_head]: one scan chain per (head, half)
+    float2 *agg;       // [2 H][tiles_per_head][128]  (prod a, h_end) from h = 0
+    float *prefix;     // [2 H][tiles_per_head][128]  h after the tile
     unsigned long long *trace;  // RGLRU_TRACE builds only: per-role timestamps
 };
 
@@ -126,7 +162,7 @@ struct FusedParams {
 enum TraceEvent {
     TR_SCHED_INFO, TR_CONV_START, TR_CONV_DONE, TR_MMA_ISSUED, TR_P1_START, TR_P1_END, TR_LB_START,
     TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, TR_MMA_TFREE, TR_MMA_TMA, TR_MMA_CONV,
-    TR_CONV_GO, kTraceEvents
+    TR_CONV_GO, TR_P2_LD, TR_P2_ST, TR_CONV_LOOP, kTraceEvents
 };
 #ifdef RGLRU_TRACE
 constexpr int kTraceCtas = 4, kTraceTiles = 128;
@@ -154,11 +190,11 @@ __device__ __forceinline__ void raise_timeout(volatile int *abort_flag, WsHeader
 __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
                                       int where)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_cl(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         // suspended in hardware until the phase completes (or 20 us pass)
-        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (mbar_try_wait_sleep_cl(bar, parity, 20000u)) return true;
         {
             if (*abort_flag) return false;
             if (*(volatile int *)&hdr->status != 0) {
@@ -212,7 +248,7 @@ __device__ __noinline__ bool warp_wait_bar_slow(uint64_t *bar, uint32_t parity, 
         // the barrier had already moved on a further phase (a logic error,
         // reported rather than waited on)
         bool seen = false;
-        for (uint32_t it = 0; it < (1u << 20) && !(seen = mbar_try_wait(bar, parity)); ++it) {
+        for (uint32_t it = 0; it < (1u << 20) && !(seen = mbar_try_wait_cl(bar, parity)); ++it) {
         }
         if (!__all_sync(0xffffffffu, seen)) {
             if ((threadIdx.x & 31) == 0) raise_timeout(abort_flag, hdr, where + 32);
@@ -226,7 +262,7 @@ __device__ __noinline__ bool warp_wait_bar_slow(uint64_t *bar, uint32_t parity, 
 __device__ __forceinline__ bool warp_wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                               WsHeader *hdr, int where)
 {
-    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__all_sync(0xffffffffu, mbar_try_wait_cl(bar, parity))) return true;
     return warp_wait_bar_slow(bar, parity, abort_flag, hdr, where);
 }
 
@@ -324,24 +360,24 @@ __device__ __forceinline__ float gelu_tanh_fast(float g)
     return fmaf(hg, tanh_approx(u), hg);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap tmap_g,
-                           const __grid_constant__ CUtensorMap tmap_x)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap tmap_x,
+                           const __grid_constant__ CUtensorMap tmap_g, const __grid_constant__ CUtensorMap tmap_y,
+                           const __grid_constant__ CUtensorMap tmap_wa, const __grid_constant__ CUtensorMap tmap_wx)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int group = blockIdx.x % p.G;
-    const int head = group >> 1, half = group & 1;
+    const uint32_t half = cluster_ctarank(), peer = half ^ 1u;
+    const int nheads = p.D / 256;
+    const int head = (int)(blockIdx.x >> 1) % nheads;
+    const int group = 2 * head + (int)half;  // scan chain of this CTA: (head, half)
+    const int ch0 = head * 256 + (int)half * kHalf;  // first channel of this CTA
     TileInfo *info = reinterpret_cast<TileInfo *>(smem + OFF_INFO);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *ring_bars = reinterpret_cast<uint64_t *>(smem + OFF_RING_BAR);
-    auto bar = [&](int kind, int s) { return bars + kind * SLOTS + s; };
-    auto info_full = [&](int i) { return ring_bars + i; };
-    auto info_empty = [&](int i) { return ring_bars + INFO_RING + i; };
-    uint64_t *xbars = reinterpret_cast<uint64_t *>(smem + OFF_XBAR);
-    auto x_full = [&](int i) { return xbars + i; };
-    auto x_empty = [&](int i) { return xbars + XRING + i; };
+    auto bar = [&](int kind, int i) { return bars + kind + i; };
+    // the peer CTA's barrier at the same offset, for remote arrivals
+    auto peer_bar = [&](int kind, int i) { return mapa_shared(smem_u32(bars + kind + i), peer); };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
     WsHeader *hdr = p.hdr;
@@ -350,74 +386,58 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_holder, 512);
         if (lane == 0) {
-            for (int s = 0; s < SLOTS; ++s) {
-                mbar_init(bar(BAR_CONV, s), kConvWarps * 32);
-                mbar_init(bar(BAR_SMEM_FREE, s), kGroupThreads);
-                mbar_init(bar(BAR_MMA, s), 1);
-                mbar_init(bar(BAR_TMEM_FREE, s), kGroupThreads);
-                mbar_init(bar(BAR_PASS1, s), kGroupThreads);
-                mbar_init(bar(BAR_LB, s), 32);
-                mbar_init(bar(BAR_G, s), 1);
-                mbar_init(bar(BAR_PUB, s), 32);
-            }
             for (int i = 0; i < INFO_RING; ++i) {
-                mbar_init(info_full(i), 1);
-                mbar_init(info_empty(i), kGroupThreads);
+                mbar_init(bar(B_INFO_FULL, i), 1);
+                mbar_init(bar(B_INFO_EMPTY, i), 2 * 4);  // pass-2 warps of both CTAs (rank 0's ring only)
             }
             for (int i = 0; i < XRING; ++i) {
-                mbar_init(x_full(i), 1);
-                mbar_init(x_empty(i), kConvWarps * 32);
+                mbar_init(bar(B_X_FULL, i), 1);
+                mbar_init(bar(B_X_EMPTY, i), kGroupThreads);
             }
+            for (int i = 0; i < NX; ++i) mbar_init(bar(B_XH_FREE, i), kGroupThreads);
+            for (int i = 0; i < NB; ++i) {
+                // this CTA's conv threads (one of them also expects the peer's half
+                // of the tile: a bulk copy that completes the transaction count)
+                mbar_init(bar(B_BCONV, i), kGroupThreads);
+                mbar_init(bar(B_BFREE, i), 2);                  // MMA commits of both CTAs
+                mbar_init(bar(B_BHALF, i), kGroupThreads);
+            }
+            for (int i = 0; i < NA; ++i) {
+                mbar_init(bar(B_MMA, i), 1);
+                mbar_init(bar(B_ACC_FREE, i), kGroupThreads);
+            }
+            for (int i = 0; i < NS; ++i) {
+                mbar_init(bar(B_PASS1, i), kGroupThreads);
+                mbar_init(bar(B_PUB, i), 32);
+                mbar_init(bar(B_LB, i), 32);
+                mbar_init(bar(B_STASH_FREE, i), kGroupThreads);
+            }
+            for (int i = 0; i < kScanGroups; ++i) {
+                mbar_init(bar(B_YFULL, i), kGroupThreads);
+                mbar_init(bar(B_YFREE, i), 1);
+            }
+            mbar_init(bar(B_W_FULL, 0), 1);
             *abort_flag = 0;
             mbar_fence_init();
         }
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-
-    if (warp < kScanWarps) {
-        // TMEM lane = output channel c of the half; scan group g loads the rows
-        // of gate g (W_a, W_x) for its channel
-        const int c = threadIdx.x % kGroupThreads;
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const size_t row = (size_t)head * 256 + half * kHalf + c;
-#pragma unroll 1
-        for (int gate = warp / 4; gate < 2; gate += kScanGroups) {
-            const uint4 *src = reinterpret_cast<const uint4 *>((gate == 0 ? p.W_a : p.W_x) + row * 256);
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t r[32];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint4 v = src[q * 8 + k];
-                    r[4 * k] = v.x;
-                    r[4 * k + 1] = v.y;
-                    r[4 * k + 2] = v.z;
-                    r[4 * k + 3] = v.w;
-                }
-                tmem_st32(tmem + lane_off + (gate == 0 ? kColWa : kColWx) + q * 32, r);
-            }
-        }
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
     const int debug_unit = *(volatile int *)&hdr->debug_unit_plus1 - 1;
 
     if (warp == kSchedWarp) {
         // ------------------------------------------------------------ scheduler
-        // Claims tiles in order from this group's ticket counter, one tile ahead
-        // of the ring, so that the atomic and the segment_pos read overlap the
-        // wait for a free ring entry.
+        // Rank 0 claims the head's tiles in order, one ahead of the ring, and
+        // writes each descriptor into both CTAs; each CTA then loads its own
+        // channels of x: rows t0 - 3 .. t0 + 31 (rows before t = 0 arrive
+        // zero-filled; the conv reads conv_state there).
         auto claim = [&]() -> TileInfo {
             int u = -1;
             if (lane == 0 && !*abort_flag) {
-                u = (int)atomicAdd(&hdr->ticket[group], 1u);
-                if (u >= p.tiles_per_group) u = -1;
+                u = (int)atomicAdd(&hdr->ticket[head], 1u);
+                if (u >= p.tiles_per_head) u = -1;
             }
             u = __shfl_sync(0xffffffffu, u, 0);
             TileInfo ti{};
@@ -435,220 +455,240 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             return ti;
         };
-        TileInfo next = claim();
-        // end markers: one per scan group and one per look-back warp (each of
-        // those reads only its own residue class of tiles)
-        constexpr int kEndMarkers = kScanGroups > kLbWarps ? kScanGroups : kLbWarps;
-        static_assert(kEndMarkers <= INFO_RING, "end markers fit the ring");
-        int ends = 0;
-        int x_issued = 0;  // x-tile TMA loads issued
+        TileInfo next{};
+        if (half == 0) next = claim();
+        int ends = 0, x_issued = 0;
 #pragma unroll 1
         for (int j = 0;; ++j) {
             const int ir = j % INFO_RING;
             bool ok = true;
-            if (j >= INFO_RING)
-                ok = warp_wait_bar(info_empty(ir), (uint32_t)((j / INFO_RING) - 1) & 1u, abort_flag, hdr, 1);
-            if (!ok) next.u = -1;
-            if (lane == 0) {
-                info[ir] = next;
-                mbar_arrive(info_full(ir));
-                RGLRU_TR(TR_SCHED_INFO, j, globaltimer());
-                RGLRU_TR(TR_TILE_U, j, (unsigned long long)(unsigned)next.u);
+            TileInfo ti;
+            if (half == 0) {
+                if (j >= INFO_RING)
+                    ok = warp_wait_bar(bar(B_INFO_EMPTY, ir), (uint32_t)((j / INFO_RING) - 1) & 1u, abort_flag, hdr, 1);
+                if (!ok) next.u = -1;
+                ti = next;
+                if (lane == 0) {
+                    const uint4 *w = reinterpret_cast<const uint4 *>(&ti);
+                    reinterpret_cast<uint4 *>(info + ir)[0] = w[0];
+                    reinterpret_cast<uint4 *>(info + ir)[1] = w[1];
+                    const uint32_t remote = mapa_shared(smem_u32(info + ir), peer);
+                    st_cluster_v4(remote, w[0]);
+                    st_cluster_v4(remote + 16, w[1]);
+                    mbar_arrive(bar(B_INFO_FULL, ir));
+                    mbar_arrive_cluster(peer_bar(B_INFO_FULL, ir));
+                    RGLRU_TR(TR_SCHED_INFO, j, globaltimer());
+                    RGLRU_TR(TR_TILE_U, j, (unsigned long long)(unsigned)ti.u);
+                }
+                if (ti.u < 0) {
+                    if (++ends == kEndMarkers || !ok) break;
+                    continue;
+                }
+            } else {
+                if (!warp_wait_bar(bar(B_INFO_FULL, ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 2)) break;
+                ti = info[ir];
+                if (ti.u < 0) break;
             }
-            if (next.u < 0) {
-                if (++ends == kEndMarkers || !ok) break;
-                continue;
-            }
-            // x rows t0-3 .. t0+31 of all 256 channels of the head into the x ring
-            // (rows before t = 0 arrive zero-filled; the conv reads conv_state there)
             const int xr = j % XRING;
-            if (j >= XRING && !warp_wait_bar(x_empty(xr), (uint32_t)((j / XRING) - 1) & 1u, abort_flag, hdr, 15)) {
-                next.u = -1;
-                continue;
+            if (j >= XRING && !warp_wait_bar(bar(B_X_EMPTY, xr), (uint32_t)((j / XRING) - 1) & 1u, abort_flag, hdr, 3)) {
+                if (half == 0) {
+                    next.u = -1;
+                    continue;  // still write the end markers
+                }
+                break;
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(x_full(xr), kXTile);
-                tma_load_3d(smem + OFF_X + xr * kXTile, &tmap_x, x_full(xr), head * 256, next.t0 - 3, next.b);
+                mbar_arrive_expect_tx(bar(B_X_FULL, xr), kXTile);
+                tma_load_3d(smem + OFF_X + xr * kXTile, &tmap_x, bar(B_X_FULL, xr), ch0, ti.t0 - 3, ti.b);
+                // the GELU branch of this tile, read by pass 1 some microseconds later
+                tma_prefetch_l2_3d(&tmap_g, ch0, ti.t0, ti.b);
             }
             ++x_issued;
-            next = claim();
+            if (half == 0) next = claim();
         }
         // on abort, wait (bounded) for the x loads still in flight
         if (lane == 0 && *abort_flag) {
             for (int k = max(0, x_issued - XRING); k < x_issued; ++k) {
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(x_full(k % XRING), (uint32_t)(k / XRING) & 1u) && globaltimer() - t0 < kTimeoutNs) {
-                }
-            }
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer (+ GELU-branch TMA)
-        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
-        int issued = 0;
-#pragma unroll 1
-        for (int j = 0;; ++j) {
-            const int s = j % SLOTS, ir = j % INFO_RING;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 2)) break;
-            const TileInfo ti = info[ir];
-            if (ti.u < 0) break;
-            if (j >= SLOTS && !warp_wait_bar(bar(BAR_TMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 3)) break;
-            if (lane == 0) RGLRU_TR(TR_MMA_TFREE, j, globaltimer());
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar(BAR_G, s), kGTile);
-                tma_load_3d(smem + OFF_G + s * kGTile, &tmap_g, bar(BAR_G, s), head * 256 + half * kHalf, ti.t0,
-                            ti.b);
-            }
-            if (lane == 0) RGLRU_TR(TR_MMA_TMA, j, globaltimer());
-            ++issued;
-            if (!warp_wait_bar(bar(BAR_CONV, s), ph, abort_flag, hdr, 4)) break;
-            if (lane == 0) RGLRU_TR(TR_MMA_CONV, j, globaltimer());
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t b_base = smem_u32(smem + OFF_B + s * kBTile);
-                const uint32_t d_r = tmem + kColSlot0 + s * kColPerSlot;
-                const uint32_t d_i = d_r + NT;
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint64_t bd = umma_desc_sw128(b_base + (kk >> 2) * kBBlock + (kk & 3) * 32);
-                    umma_ts(d_r, tmem + kColWa + kk * 8, bd, idesc, kk > 0);
-                    umma_ts(d_i, tmem + kColWx + kk * 8, bd, idesc, kk > 0);
-                }
-                umma_commit(bar(BAR_MMA, s));
-                RGLRU_TR(TR_MMA_ISSUED, j, globaltimer());
-            }
-            __syncwarp();
-        }
-        // on abort, wait (bounded) for this CTA's copies and MMAs in flight
-        if (lane == 0 && *abort_flag) {
-            for (int k = max(0, issued - SLOTS); k < issued; ++k) {
-                const int s = k % SLOTS;
-                const uint32_t ph = (uint32_t)(k / SLOTS) & 1u;
-                uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(bar(BAR_G, s), ph) && globaltimer() - t0 < kTimeoutNs) {
-                }
-                t0 = globaltimer();
-                while (!mbar_try_wait(bar(BAR_MMA, s), ph) && globaltimer() - t0 < kTimeoutNs / 4) {
+                while (!mbar_try_wait(bar(B_X_FULL, k % XRING), (uint32_t)(k / XRING) & 1u) &&
+                       globaltimer() - t0 < kTimeoutNs) {
                 }
             }
         }
     } else if (warp >= kConvWarp0 && warp < kConvWarp0 + kConvWarps) {
         // ------------------------------------------------------------ conv warps
-        // Warp kb covers the head's channels [64 kb, 64 kb + 64) (one K-block of
-        // the B tile); lane = (token half q, group of 4 channels cg), so each
-        // lane runs 16 consecutive tokens of 4 channels, in fp32 pairs.
-        const int kb = warp - kConvWarp0;
-        const int cg = lane & 15;
-        const int q = lane >> 4;
-        const int dl = kb * 64 + cg * 4;  // channel within the head
-        const size_t d0 = (size_t)head * 256 + dl;
+        // thread = channel c of this half (its TMEM lane); 32 tokens in order.
         // The conv produces xh = xc / 2 (halving is exact): the MMA then yields
         // half pre-activations, which is what sigmoid(z) = (1 + tanh(z/2)) / 2
         // needs, and the scan's i*xc becomes one FMA on xh.
-        f2_t w2[4][2], cb2[2];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                w2[k][e] = f2_make(0.5f * p.conv_w[(size_t)k * p.D + d0 + 2 * e],
-                                   0.5f * p.conv_w[(size_t)k * p.D + d0 + 2 * e + 1]);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) cb2[e] = f2_make(0.5f * p.conv_b[d0 + 2 * e], 0.5f * p.conv_b[d0 + 2 * e + 1]);
-        const bool own = (kb >> 1) == half;
-        const int xcs_c = (kb & 1) * 64 + cg * 4;  // channel within this half
+        const int c = (warp - kConvWarp0) * 32 + lane;
+        const int d = ch0 + c;
+        const float w0 = 0.5f * p.conv_w[d], w1 = 0.5f * p.conv_w[(size_t)p.D + d];
+        const float w2 = 0.5f * p.conv_w[2 * (size_t)p.D + d], w3 = 0.5f * p.conv_w[3 * (size_t)p.D + d];
+        const float cb = 0.5f * p.conv_b[d];
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        // B tile: row n = token, K index = channel within the head (K-major,
+        // 128-byte swizzle: 16-byte chunk (k & 63) >> 3 of row n sits at chunk ^ (n & 7))
+        const int kidx = (int)half * kHalf + c;
+        const uint32_t b_local = smem_u32(smem + OFF_B + (kidx >> 6) * kBBlock);
+        const uint32_t chunk = (uint32_t)((kidx & 63) >> 3), sub = (uint32_t)(kidx & 7) * 2;
+        // this half's two K-blocks of a B tile: 8 KB, contiguous, sent to the peer in one copy
+        const int half_off = (int)half * 2 * kBBlock;
+        const bool sender = warp == kConvWarp0 && lane == 0;
 #pragma unroll 1
         for (int j = 0;; ++j) {
-            const int s = j % SLOTS, ir = j % INFO_RING;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 5)) break;
+            const int ir = j % INFO_RING, xr = j % XRING, sx = j % NX, sb = j % NB;
+            if (!warp_wait_bar(bar(B_INFO_FULL, ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 4)) break;
             const TileInfo ti = info[ir];
             if (ti.u < 0) break;
-            if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_START, j, globaltimer());
-            const int xr = j % XRING;
-            if (!warp_wait_bar(x_full(xr), (uint32_t)(j / XRING) & 1u, abort_flag, hdr, 16)) break;
-            if (j >= SLOTS && !warp_wait_bar(bar(BAR_SMEM_FREE, s), ph ^ 1u, abort_flag, hdr, 6)) break;
-            if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_GO, j, globaltimer());
-            const int n0 = q * 16;
-            uint8_t *xt = smem + OFF_X + xr * kXTile + dl * 2;  // row r = token t0 - 3 + r
-            if (ti.t0 == 0 && q == 0) {
-                // sequence start: rows 0..2 (tokens -3..-1, zero-filled by the
-                // load) are the carried conv state; each lane patches the 4
-                // channels it reads itself
-#pragma unroll
-                for (int r = 0; r < 3; ++r)
-                    *reinterpret_cast<uint2 *>(xt + r * 512) =
-                        *reinterpret_cast<const uint2 *>(p.conv_state + ((size_t)ti.b * 3 + r) * p.D + d0);
+            if (lane == 0 && warp == kConvWarp0) RGLRU_TR(TR_CONV_START, j, globaltimer());
+            if (!warp_wait_bar(bar(B_X_FULL, xr), (uint32_t)(j / XRING) & 1u, abort_flag, hdr, 5)) break;
+            if (j >= NX && !warp_wait_bar(bar(B_XH_FREE, sx), (uint32_t)((j / NX) - 1) & 1u, abort_flag, hdr, 6)) break;
+            if (j >= NB && !warp_wait_bar(bar(B_BFREE, sb), (uint32_t)((j / NB) - 1) & 1u, abort_flag, hdr, 7)) break;
+            if (lane == 0 && warp == kConvWarp0) RGLRU_TR(TR_CONV_GO, j, globaltimer());
+            const __nv_bfloat16 *xs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_X + xr * kXTile) + c;
+            float xm3, xm2, xm1;  // tokens t - 3, t - 2, t - 1
+            if (ti.t0 == 0) {     // sequence start: the carried conv state
+                const __nv_bfloat16 *cs = p.conv_state + (size_t)ti.b * 3 * p.D + d;
+                xm3 = __bfloat162float(cs[0]);
+                xm2 = __bfloat162float(cs[p.D]);
+                xm1 = __bfloat162float(cs[2 * (size_t)p.D]);
+            } else {
+                xm3 = __bfloat162float(xs[0]);
+                xm2 = __bfloat162float(xs[kHalf]);
+                xm1 = __bfloat162float(xs[2 * kHalf]);
             }
-            auto xrow = [&](int r, f2_t (&f)[2]) {
-                const uint2 v = *reinterpret_cast<const uint2 *>(xt + r * 512);
-                f[0] = f2_from_bf16x2(v.x);
-                f[1] = f2_from_bf16x2(v.y);
-            };
-            uint8_t *btile = smem + OFF_B + s * kBTile + kb * kBBlock;
-            // fp32 xh of this half, token pairs interleaved: [t / 2][channel][t % 2]
-            float *xcs = reinterpret_cast<float *>(smem + OFF_XCS + s * kXcsTile);
+            const uint32_t bl = b_local + sb * kBTile;
+            const uint32_t xh_col = tmem + lane_off + kColXh + sx * kColsXh;
             // a tile with no document start and all 32 tokens valid needs no masks
             const bool clean = (ti.reset_mask | ti.m2 | ti.m3) == 0u && ti.valid == NT;
             auto run = [&](auto clean_tag) {
                 constexpr bool kClean = decltype(clean_tag)::value;
-                f2_t xm3[2], xm2[2], xm1[2], prev[2];
-                xrow(n0, xm3);
-                xrow(n0 + 1, xm2);
-                xrow(n0 + 2, xm1);
-#pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    f2_t x0[2];
-                    xrow(n0 + i + 3, x0);
-                    const int n = n0 + i;
-                    f2_t acc[2];
+#pragma unroll 1
+                for (int t8 = 0; t8 < NT; t8 += 8) {
+                    uint32_t xq[4];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
+                    for (int k = 0; k < 8; ++k) {
+                        const int t = t8 + k;
+                        const float x0 = __bfloat162float(xs[(t + 3) * kHalf]);
+                        float v;
                         if constexpr (kClean) {
-                            acc[e] = f2_fma(w2[3][e], x0[e],
-                                            f2_fma(w2[2][e], xm1[e], f2_fma(w2[1][e], xm2[e], f2_fma(w2[0][e], xm3[e], cb2[e]))));
+                            v = fmaf(w3, x0, fmaf(w2, xm1, fmaf(w1, xm2, fmaf(w0, xm3, cb))));
                         } else {
                             // tap of lag k dropped when segment_pos < k (document start)
-                            f2_t v = cb2[e];
-                            if (!((ti.m3 >> n) & 1u)) v = f2_fma(w2[0][e], xm3[e], v);
-                            if (!((ti.m2 >> n) & 1u)) v = f2_fma(w2[1][e], xm2[e], v);
-                            if (!((ti.reset_mask >> n) & 1u)) v = f2_fma(w2[2][e], xm1[e], v);
-                            v = f2_fma(w2[3][e], x0[e], v);
-                            acc[e] = n < ti.valid ? v : 0ull;
+                            v = cb;
+                            if (!((ti.m3 >> t) & 1u)) v = fmaf(w0, xm3, v);
+                            if (!((ti.m2 >> t) & 1u)) v = fmaf(w1, xm2, v);
+                            if (!((ti.reset_mask >> t) & 1u)) v = fmaf(w2, xm1, v);
+                            v = fmaf(w3, x0, v);
+                            if (t >= ti.valid) v = 0.f;
                         }
+                        const uint32_t off = (uint32_t)t * 128 + ((chunk ^ (uint32_t)(t & 7)) << 4) + sub;
+                        const uint16_t bv = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(bl + off), "h"(bv) : "memory");
+                        const __half hv = __float2half_rn(v);
+                        if (k & 1)
+                            xq[k >> 1] |= (uint32_t)__half_as_ushort(hv) << 16;
+                        else
+                            xq[k >> 1] = (uint32_t)__half_as_ushort(hv);
+                        xm3 = xm2;
+                        xm2 = xm1;
+                        xm1 = x0;
                     }
-                    // B tile row n: 4 channels = the (cg & 1) half of 16-byte chunk cg >> 1
-                    *reinterpret_cast<uint2 *>(btile + n * 128 + (((cg >> 1) ^ (n & 7)) << 4) + (cg & 1) * 8) =
-                        make_uint2(f2_to_bf16x2(acc[0]), f2_to_bf16x2(acc[1]));
-                    if ((i & 1) && own) {
-                        float4 *dst = reinterpret_cast<float4 *>(xcs + ((n >> 1) * kHalf + xcs_c) * 2);
-                        dst[0] = make_float4(f2_lo(prev[0]), f2_lo(acc[0]), f2_hi(prev[0]), f2_hi(acc[0]));
-                        dst[1] = make_float4(f2_lo(prev[1]), f2_lo(acc[1]), f2_hi(prev[1]), f2_hi(acc[1]));
-                    }
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        prev[e] = acc[e];
-                        xm3[e] = xm2[e];
-                        xm2[e] = xm1[e];
-                        xm1[e] = x0[e];
-                    }
+                    tmem_st4(xh_col + (uint32_t)(t8 >> 1), xq);
                 }
             };
             if (clean)
                 run(std::true_type{});
             else
                 run(std::false_type{});
-            // generic writes (B tile, patched x rows) before the async proxy's
-            // next accesses (the MMA, the next load into this x slot)
+            if (lane == 0 && warp == kConvWarp0) RGLRU_TR(TR_CONV_LOOP, j, globaltimer());
+            tmem_wait_st();
+            tc_fence_before();
+            // this half of the B tile before the async proxy's reads (the MMA,
+            // the copy to the peer)
             fence_proxy_async_smem();
-            mbar_arrive(x_empty(xr));
-            mbar_arrive(bar(BAR_CONV, s));
-            if (lane == 0 && kb == 0) RGLRU_TR(TR_CONV_DONE, j, globaltimer());
+            mbar_arrive(bar(B_X_EMPTY, xr));
+            if (sender)
+                mbar_arrive_expect_tx(bar(B_BCONV, sb), 2 * kBBlock);  // the peer's half, arriving by copy
+            else
+                mbar_arrive(bar(B_BCONV, sb));
+            mbar_arrive(bar(B_BHALF, sb));
+            if (warp == kConvWarp0) {
+                // all of this half written: one bulk copy into the peer's tile
+                if (!warp_wait_bar(bar(B_BHALF, sb), (uint32_t)(j / NB) & 1u, abort_flag, hdr, 20)) break;
+                if (sender) {
+                    uint8_t *src = smem + OFF_B + sb * kBTile + half_off;
+                    bulk_copy_to_cluster(mapa_shared(smem_u32(src), peer), src, 2 * kBBlock, peer_bar(B_BCONV, sb));
+                }
+            }
+            if (lane == 0 && warp == kConvWarp0) RGLRU_TR(TR_CONV_DONE, j, globaltimer());
         }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            // this half's 128 rows of W_a and W_x: 4 K-blocks of 64 channels each
+            mbar_arrive_expect_tx(bar(B_W_FULL, 0), 2 * kWGate);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+                tma_load_2d(smem + OFF_W + kb * kWBlock, &tmap_wa, bar(B_W_FULL, 0), kb * 64, ch0);
+                tma_load_2d(smem + OFF_W + kWGate + kb * kWBlock, &tmap_wx, bar(B_W_FULL, 0), kb * 64, ch0);
+            }
+        }
+        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
+        const uint32_t wa = smem_u32(smem + OFF_W), wx = wa + kWGate;
+        bool w_ready = false;
+        int issued = 0;
+#pragma unroll 1
+        for (int j = 0;; ++j) {
+            const int ir = j % INFO_RING, sb = j % NB, sa = j % NA;
+            if (!warp_wait_bar(bar(B_INFO_FULL, ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 8)) break;
+            if (info[ir].u < 0) break;
+            if (j >= NA && !warp_wait_bar(bar(B_ACC_FREE, sa), (uint32_t)((j / NA) - 1) & 1u, abort_flag, hdr, 9)) break;
+            if (lane == 0) RGLRU_TR(TR_MMA_TFREE, j, globaltimer());
+            if (!warp_wait_bar(bar(B_BCONV, sb), (uint32_t)(j / NB) & 1u, abort_flag, hdr, 10)) break;
+            if (lane == 0) RGLRU_TR(TR_MMA_CONV, j, globaltimer());
+            if (!w_ready) {
+                if (!warp_wait_bar(bar(B_W_FULL, 0), 0u, abort_flag, hdr, 11)) break;
+                w_ready = true;
+            }
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t bt = smem_u32(smem + OFF_B + sb * kBTile);
+                const uint32_t d_r = tmem + kColAcc + sa * kColsAcc, d_i = d_r + NT;
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kWBlock + (kk & 3) * 32;
+                    const uint64_t bd = umma_desc_sw128(bt + (kk >> 2) * kBBlock + (kk & 3) * 32);
+                    umma_ss(d_r, umma_desc_sw128(wa + ko), bd, idesc, kk > 0);
+                    umma_ss(d_i, umma_desc_sw128(wx + ko), bd, idesc, kk > 0);
+                }
+                umma_commit(bar(B_MMA, sa));
+                umma_commit_cluster(bar(B_BFREE, sb), 0x3);  // this B slot is free in both CTAs' view
+                RGLRU_TR(TR_MMA_ISSUED, j, globaltimer());
+            }
+            __syncwarp();
+            ++issued;
+        }
+        // Before the final cluster barrier: the commits of both CTAs for the
+        // last tiles have landed on this CTA's B-slot barriers (so no arrival
+        // reaches a CTA that has exited), and the weight load is complete.
+        if (lane == 0) {
+            for (int k = max(0, issued - NB); k < issued; ++k) {
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait_cl(bar(B_BFREE, k % NB), (uint32_t)(k / NB) & 1u) && globaltimer() - t0 < kTimeoutNs) {
+                }
+            }
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(bar(B_W_FULL, 0), 0u) && globaltimer() - t0 < kTimeoutNs) {
+            }
+        }
+        __syncwarp();
     } else if (warp < kScanWarps) {
         // ------------------------------------------------------------ scan warps
-        const int sg = warp / 4;                 // scan group: tiles j with j % kScanGroups == sg
+        const int sg = warp / 4;  // scan group: tiles j with j % kScanGroups == sg
         const int c = threadIdx.x % kGroupThreads;
-        const int d = head * 256 + half * kHalf + c;
+        const int d = ch0 + c;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float hba = 0.5f * p.b_a[d], hbx = 0.5f * p.b_x[d];
         const float lam = p.lambda[d];
@@ -663,37 +703,58 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const f2_t hba2 = f2_splat(hba), hbx2 = f2_splat(hbx), hkl_2 = f2_splat(hkl), hkl2_2 = f2_splat(hkl2);
         const f2_t c13_2 = f2_splat(1.f / 3.f), c23_2 = f2_splat(2.f / 3.f), one_2 = f2_splat(1.f),
                    mtwo_2 = f2_splat(-2.f);
+        // GELU branch of the group's next tile into its shared-memory buffer
+        // (the tile was prefetched into L2 with its x): each thread copies the
+        // 4-byte words holding its own channel, so it reads only its own copies
+        __nv_bfloat16 *gbuf = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_G + sg * kGTile);
+        auto copy_g = [&](const TileInfo &ti) {
+            const int c2 = c & ~1;
+            const __nv_bfloat16 *gp = p.g + ((size_t)ti.b * p.T + ti.t0) * p.D + ch0 + c2;
+#pragma unroll 4
+            for (int t = 0; t < ti.valid; ++t) cp_async4(gbuf + t * kHalf + c2, gp + (size_t)t * p.D);
+        };
+        auto pack_h2 = [](float lo, float hi) -> uint32_t {
+            __half2 v = __floats2half2_rn(lo, hi);
+            return *reinterpret_cast<uint32_t *>(&v);
+        };
 
-        auto pass1 = [&](int j) -> bool {
-            const int s = j % SLOTS;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            const TileInfo ti = info[j % INFO_RING];
-            if (!warp_wait_bar(bar(BAR_MMA, s), ph, abort_flag, hdr, 7)) return false;
+        auto pass1 = [&](int j, const TileInfo &ti) -> bool {
+            const int sa = j % NA, ss = j % NS, sx = j % NX;
+            if (!warp_wait_bar(bar(B_MMA, sa), (uint32_t)(j / NA) & 1u, abort_flag, hdr, 12)) return false;
+            if (j >= NS) {
+                if (!warp_wait_bar(bar(B_STASH_FREE, ss), (uint32_t)((j / NS) - 1) & 1u, abort_flag, hdr, 13)) return false;
+                if (!warp_wait_bar(bar(B_PUB, ss), (uint32_t)((j / NS) - 1) & 1u, abort_flag, hdr, 14)) return false;
+            }
             if (c == 0) RGLRU_TR(TR_P1_START, j, globaltimer());
             tc_fence_after();
-            const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
-            // xh of tokens (2m, 2m + 1) of this channel: one 8-byte load
-            const float2 *xcs2 = reinterpret_cast<const float2 *>(smem + OFF_XCS + s * kXcsTile) + c;
-            float hl = 0.f, P = 1.f;
-            f2_t lsum = 0ull;  // clean chunks: sum of log2 a (P = 2^sum at the end)
+            const uint32_t acc = tmem + lane_off + kColAcc + sa * kColsAcc;
+            const uint32_t xhc = tmem + lane_off + kColXh + sx * kColsXh;
+            const uint32_t stc = tmem + lane_off + kColStash + ss * kColsStash;
+            float hl = 0.f, P = 1.f;  // local scan state from h = 0, running prod a
+            cp_async_wait_all();      // this tile's GELU branch
+            const uint16_t *gs = reinterpret_cast<const uint16_t *>(gbuf) + c;
 #pragma unroll 1
             for (int t8 = 0; t8 < NT; t8 += 8) {
-                uint32_t ar[8], ai[8];
-                tmem_ld8(col + t8, ar);
-                tmem_ld8(col + NT + t8, ai);
+                uint32_t ar[8], ai[8], xq[4];
+                tmem_ld8(acc + t8, ar);
+                tmem_ld8(acc + NT + t8, ai);
+                tmem_ld4(xhc + (t8 >> 1), xq);
                 tmem_wait_ld();
+                uint16_t gcur[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) gcur[k] = gs[(t8 + k) * kHalf];
+                uint32_t st[8];
                 const bool clean = ((ti.reset_mask >> t8) & 0xffu) == 0u && t8 + 8 <= ti.valid && series_ok;
                 if (clean) {
 #pragma unroll
                     for (int k = 0; k < 8; k += 2) {
-                        const float2 xh = xcs2[((t8 + k) >> 1) * kHalf];
+                        const float2 xh = __half22float2(*reinterpret_cast<const __half2 *>(&xq[k >> 1]));
                         const f2_t zr = f2_add(f2_make(__uint_as_float(ar[k]), __uint_as_float(ar[k + 1])), hba2);
                         const f2_t zi = f2_add(f2_make(__uint_as_float(ai[k]), __uint_as_float(ai[k + 1])), hbx2);
                         const f2_t tr = f2_make(tanh_approx(f2_lo(zr)), tanh_approx(f2_hi(zr)));
                         const f2_t tg = f2_make(tanh_approx(f2_lo(zi)), tanh_approx(f2_hi(zi)));
                         const f2_t ell = f2_fma(tr, hkl_2, hkl_2);    // log a
                         const f2_t la = f2_fma(tr, hkl2_2, hkl2_2);  // log2 a
-                        lsum = f2_add(lsum, la);
                         const float a0 = ex2_approx(f2_lo(la)), a1 = ex2_approx(f2_hi(la));
                         // 1 - exp(2 ell) by its series (see one_minus_exp2l_small)
                         f2_t sr = f2_fma(ell, c13_2, c23_2);
@@ -703,18 +764,23 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const f2_t nrm = f2_make(sqrt_approx(f2_lo(om)), sqrt_approx(f2_hi(om)));
                         const f2_t xh2 = f2_make(xh.x, xh.y);
                         const f2_t v = f2_mul(nrm, f2_fma(tg, xh2, xh2));  // sqrt(1-a^2) * i * xc
-                        hl = fmaf(a0, hl, f2_lo(v));
-                        hl = fmaf(a1, hl, f2_hi(v));
-                        ar[k] = __float_as_uint(a0);
-                        ar[k + 1] = __float_as_uint(a1);
-                        ai[k] = __float_as_uint(f2_lo(v));
-                        ai[k + 1] = __float_as_uint(f2_hi(v));
+                        const float h0 = fmaf(a0, hl, f2_lo(v));
+                        const float P0 = P * a0;
+                        hl = fmaf(a1, h0, f2_hi(v));
+                        P = P0 * a1;
+                        const f2_t G = gelu2(f2_make(__uint_as_float((uint32_t)gcur[k] << 16),
+                                                     __uint_as_float((uint32_t)gcur[k + 1] << 16)));
+                        const f2_t yl = f2_mul(G, f2_make(h0, hl));
+                        const f2_t qq = f2_mul(G, f2_make(P0, P));
+                        st[k] = pack_h2(f2_lo(yl), f2_lo(qq));
+                        st[k + 1] = pack_h2(f2_hi(yl), f2_hi(qq));
                     }
                 } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int t = t8 + k;
-                        const float xh = reinterpret_cast<const float *>(xcs2 + (t >> 1) * kHalf)[t & 1];
+                        const __half2 xq2 = *reinterpret_cast<const __half2 *>(&xq[k >> 1]);
+                        const float xh = (k & 1) ? __high2float(xq2) : __low2float(xq2);
                         const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
                         const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
                         const float ell = fmaf(tr, hkl, hkl);
@@ -732,77 +798,74 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         }
                         hl = fmaf(a, hl, v);
                         P *= a;
-                        ar[k] = __float_as_uint(a);
-                        ai[k] = __float_as_uint(v);
+                        const float G = gelu_tanh_fast(__uint_as_float((uint32_t)gcur[k] << 16));
+                        st[k] = pack_h2(G * hl, G * P);
                     }
                 }
-                tmem_st8(col + t8, ar);
-                tmem_st8(col + NT + t8, ai);
+                tmem_st8(stc + t8, st);
             }
-            P *= ex2_approx(f2_lo(lsum) + f2_hi(lsum));
-            mbar_arrive(bar(BAR_SMEM_FREE, s));  // xcs (and, via the MMA wait, the B tile) consumed
             tmem_wait_st();
-            // the look-back warp must have copied out this slot's previous aggregate
-            if (j >= SLOTS && !warp_wait_bar(bar(BAR_PUB, s), ph ^ 1u, abort_flag, hdr, 17)) return false;
-            reinterpret_cast<float2 *>(smem + OFF_AGG + s * kHalf * 8)[c] = make_float2(P, hl);
-            mbar_arrive(bar(BAR_PASS1, s));
+            tc_fence_before();
+            mbar_arrive(bar(B_ACC_FREE, sa));
+            mbar_arrive(bar(B_XH_FREE, sx));
+            reinterpret_cast<float2 *>(smem + OFF_AGG + ss * kHalf * 8)[c] = make_float2(P, hl);
+            mbar_arrive(bar(B_PASS1, ss));
             if (c == 0) RGLRU_TR(TR_P1_END, j, globaltimer());
             return true;
         };
 
+        // y leaves through the group's shared-memory tile and one tensor store
+        __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_Y + sg * kGTile);
+        const bool ystorer = c == 0;  // issues the group's tensor stores
+        int ystores = 0;               // tensor stores issued by this group
+
         auto pass2 = [&](int j) -> bool {
-            const int s = j % SLOTS, ir = j % INFO_RING;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
+            const int ss = j % NS, ir = j % INFO_RING;
             const TileInfo ti = info[ir];
-            if (!warp_wait_bar(bar(BAR_LB, s), ph, abort_flag, hdr, 8)) return false;
-            float h = reinterpret_cast<const float *>(smem + OFF_HIN + s * kHalf * 4)[c];
-            if (!warp_wait_bar(bar(BAR_G, s), ph, abort_flag, hdr, 9)) return false;
+            if (!warp_wait_bar(bar(B_LB, ss), (uint32_t)(j / NS) & 1u, abort_flag, hdr, 15)) return false;
             if (c == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
+            if (ystores > 0) {
+                // the previous tensor store must have read the y tile
+                if (ystorer) {
+                    bulk_wait_read_all();
+                    mbar_arrive(bar(B_YFREE, sg));
+                }
+                if (!warp_wait_bar(bar(B_YFREE, sg), (uint32_t)(ystores - 1) & 1u, abort_flag, hdr, 21)) return false;
+            }
+            const float h_in = reinterpret_cast<const float *>(smem + OFF_HIN + ss * kHalf * 4)[c];
             tc_fence_after();
-            const uint32_t col = tmem + lane_off + kColSlot0 + s * kColPerSlot;
-            const __nv_bfloat16 *gs = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_G + s * kGTile) + c;
-            __nv_bfloat16 *yp = p.y + ((size_t)ti.b * p.T + ti.t0) * p.D + d;
-            const size_t ystep = p.D;
+            const uint32_t stc = tmem + lane_off + kColStash + ss * kColsStash;
 #pragma unroll 1
-            for (int t8 = 0; t8 < NT; t8 += 8) {
-                uint32_t aa[8], vv[8];
-                tmem_ld8(col + t8, aa);
-                tmem_ld8(col + NT + t8, vv);
+            for (int t16 = 0; t16 < NT; t16 += 16) {
+                uint32_t r[16];
+                tmem_ld16(stc + t16, r);
                 tmem_wait_ld();
-                if (t8 + 8 <= ti.valid) {
+                if (c == 0 && t16 == 0) RGLRU_TR(TR_P2_LD, j, globaltimer());
 #pragma unroll
-                    for (int k = 0; k < 8; k += 2) {
-                        h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
-                        const float h0 = h;
-                        h = fmaf(__uint_as_float(aa[k + 1]), h, __uint_as_float(vv[k + 1]));
-                        const f2_t gv = f2_make(__bfloat162float(gs[(t8 + k) * kHalf]), __bfloat162float(gs[(t8 + k + 1) * kHalf]));
-                        const uint32_t yy = f2_to_bf16x2(f2_mul(gelu2(gv), f2_make(h0, h)));
-                        const __nv_bfloat162 y2 = *reinterpret_cast<const __nv_bfloat162 *>(&yy);
-                        yp[(size_t)(t8 + k) * ystep] = y2.x;
-                        yp[(size_t)(t8 + k + 1) * ystep] = y2.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int t = t8 + k;
-                        h = fmaf(__uint_as_float(aa[k]), h, __uint_as_float(vv[k]));
-                        if (t < ti.valid) {
-                            const float gv = __bfloat162float(gs[t * kHalf]);
-                            yp[(size_t)t * ystep] = __float2bfloat16_rn(gelu_tanh_fast(gv) * h);
-                        }
-                    }
+                for (int k = 0; k < 16; ++k) {
+                    // rows past the sequence end are clipped by the tensor store
+                    const float2 yq = __half22float2(*reinterpret_cast<const __half2 *>(&r[k]));
+                    ybuf[(t16 + k) * kHalf + c] = __float2bfloat16_rn(fmaf(yq.y, h_in, yq.x));
                 }
             }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(B_YFULL, sg));
+            if (warp == 4 * sg) {
+                if (!warp_wait_bar(bar(B_YFULL, sg), (uint32_t)ystores & 1u, abort_flag, hdr, 22)) return false;
+                if (ystorer) {
+                    tma_store_3d(&tmap_y, ybuf, ch0, ti.t0, ti.b);
+                    bulk_commit();
+                }
+            }
+            ++ystores;
+            if (c == 0) RGLRU_TR(TR_P2_ST, j, globaltimer());
             if (ti.first_last & 2) {
                 // The old states are read by the first tile of this sequence (its
-                // conv in both halves of the head, its look-back for h): wait until
-                // those reads are published before overwriting the states.
-                const size_t u0 = (size_t)ti.b * p.C;
-                const uint32_t *f_own = p.flags + (size_t)group * p.tiles_per_group + u0;
-                const uint32_t *f_oth = p.flags + (size_t)(group ^ 1) * p.tiles_per_group + u0;
-                if (warp_wait_flag(f_own, F_PREFIX, abort_flag, hdr, 10) == 0) return false;
-                if (warp_wait_flag(f_oth, F_AGG, abort_flag, hdr, 11) == 0) return false;
-                p.h_state[(size_t)ti.b * p.D + d] = h;
+                // conv and its look-back, in this CTA's half of the channels):
+                // wait until that tile's prefix is published before overwriting.
+                const uint32_t *f_first = p.flags + (size_t)group * p.tiles_per_head + (size_t)ti.b * p.C;
+                if (warp_wait_flag(f_first, F_PREFIX, abort_flag, hdr, 16) == 0) return false;
+                p.h_state[(size_t)ti.b * p.D + d] = reinterpret_cast<const float *>(smem + OFF_AGG + ss * kHalf * 8)[c];
                 __nv_bfloat16 ncs[3];
 #pragma unroll
                 for (int k = 0; k < 3; ++k) {
@@ -814,49 +877,78 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 for (int k = 0; k < 3; ++k) p.conv_state[((size_t)ti.b * 3 + k) * p.D + d] = ncs[k];
             }
             tc_fence_before();
-            mbar_arrive(bar(BAR_TMEM_FREE, s));
-            mbar_arrive(info_empty(ir));
+            mbar_arrive(bar(B_STASH_FREE, ss));
+            // the descriptor may be reused once both CTAs' pass-2 warps are done with it
+            __syncwarp();
+            if (lane == 0) {
+                // relaxed: the reuse needs no ordering of this warp's y stores
+                if (half == 0)
+                    mbar_arrive(bar(B_INFO_EMPTY, ir));
+                else
+                    mbar_arrive_cluster_relaxed(peer_bar(B_INFO_EMPTY, ir));
+            }
             if (c == 0) RGLRU_TR(TR_P2_END, j, globaltimer());
             return true;
         };
 
         // this group's tiles: j = sg, sg + kScanGroups, ...; pass 2 of a tile runs
-        // after pass 1 of the group's next tile (the look-back has that long)
-#pragma unroll 1
-        for (int j = sg;; j += kScanGroups) {
-            const int ir = j % INFO_RING;
-            bool end = !warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 12);
-            if (!end) end = info[ir].u < 0;
-            bool ok = true;
-            if (!end) ok = pass1(j);
-            if (ok && j >= kScanGroups) ok = pass2(j - kScanGroups);
-            if (!ok || end) break;
+        // kP2Lag of the group's tiles later (the look-back has that long)
+        int j = sg;
+        bool ok = warp_wait_bar(bar(B_INFO_FULL, j % INFO_RING), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 17);
+        TileInfo cur{};
+        if (ok) {
+            cur = info[j % INFO_RING];
+            if (cur.u >= 0) copy_g(cur);
         }
+#pragma unroll 1
+        for (;; j += kScanGroups) {
+            const bool end = !ok || cur.u < 0;
+            if (!end) ok = pass1(j, cur);
+            TileInfo nxt{};
+            if (ok && !end) {
+                const int jn = j + kScanGroups;
+                ok = warp_wait_bar(bar(B_INFO_FULL, jn % INFO_RING), (uint32_t)(jn / INFO_RING) & 1u, abort_flag, hdr,
+                                   17);
+                if (ok) {
+                    nxt = info[jn % INFO_RING];
+                    if (nxt.u >= 0) copy_g(nxt);  // lands while pass 2 below runs
+                }
+            }
+            const int jp = j - kScanGroups * kP2Lag;
+            if (ok && jp >= 0) ok = pass2(jp);
+            if (end || !ok) {
+                // the group's tiles still waiting for pass 2
+                for (int q = jp + kScanGroups; ok && q < j; q += kScanGroups)
+                    if (q >= 0) ok = pass2(q);
+                break;
+            }
+            cur = nxt;
+        }
+        if (ystorer && ystores > 0) bulk_wait_all();  // the group's y stores are complete
     } else if (warp >= kLbWarp0) {
         // ------------------------------------------------------------ look-back warps
-        // Warp s serves the tiles of slot s (j = s, s + SLOTS, ...), so it waits on
-        // its slot's barriers one phase at a time.  Per tile: publish the
-        // aggregate (later tiles of the sequence may combine it before this
-        // tile's own look-back has finished), find the anchor, fold, hand the
-        // carried-in state to pass 2, publish the inclusive prefix.  These warps
-        // are the only ones that fence for the aggregates and prefixes.
-        const int s = warp - kLbWarp0;
+        // Warp w serves the tiles j = w, w + kLbWarps, ...; their stash slots
+        // recur every NS tiles, so each barrier is waited on one phase at a
+        // time.  Per tile: publish the aggregate (later tiles of the sequence
+        // may combine it before this tile's own look-back has finished), find
+        // the anchor, fold, hand h_in (and the prefix) to pass 2, publish the
+        // inclusive prefix.  These warps are the only ones that fence for the
+        // aggregates and prefixes.
         const int ch = lane * 4;  // 4 channels per lane
-        const size_t dch = (size_t)head * 256 + half * kHalf + ch;
-        const size_t gbase = (size_t)group * p.tiles_per_group;
+        const size_t dch = (size_t)ch0 + ch;
+        const size_t gbase = (size_t)group * p.tiles_per_head;
         constexpr int kFoldBatch = 4;  // aggregates loaded per round trip
 #pragma unroll 1
-        for (int j = s;; j += SLOTS) {
-            const int ir = j % INFO_RING;
-            const uint32_t ph = (uint32_t)(j / SLOTS) & 1u;
-            if (!warp_wait_bar(info_full(ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 13)) break;
+        for (int j = warp - kLbWarp0;; j += kLbWarps) {
+            const int ss = j % NS, ir = j % INFO_RING;
+            if (!warp_wait_bar(bar(B_INFO_FULL, ir), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 18)) break;
             const TileInfo ti = info[ir];
             if (ti.u < 0) break;
-            if (!warp_wait_bar(bar(BAR_PASS1, s), ph, abort_flag, hdr, 14)) break;
+            if (!warp_wait_bar(bar(B_PASS1, ss), (uint32_t)(j / NS) & 1u, abort_flag, hdr, 19)) break;
             if (lane == 0) RGLRU_TR(TR_LB_START, j, globaltimer());
-            const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + s * kHalf * 8);
+            const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + ss * kHalf * 8);
             const float4 g01 = sagg[lane * 2], g23 = sagg[lane * 2 + 1];  // (A,H) of 4 channels
-            mbar_arrive(bar(BAR_PUB, s));  // the slot's aggregate buffer is free again
+            mbar_arrive(bar(B_PUB, ss));  // the aggregate slot is free again
             const float A[4] = {g01.x, g01.z, g23.x, g23.z};
             const float Hh[4] = {g01.y, g01.w, g23.y, g23.w};
             const size_t gu = gbase + ti.u;
@@ -916,14 +1008,19 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             if (!ok) break;
             if (lane == 0) RGLRU_TR(TR_LB_HIN, j, globaltimer());
-            // pass 2 needs only the carried-in state: hand it over before publishing
-            *reinterpret_cast<float4 *>(smem + OFF_HIN + s * kHalf * 4 + ch * 4) =
-                make_float4(hin[0], hin[1], hin[2], hin[3]);
-            mbar_arrive(bar(BAR_LB, s));
-            if (!suppress) {
-                float pre[4];
+            float pre[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
+            for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
+            // pass 2 needs only the carried-in state (and, at the sequence end,
+            // the state after the tile): hand them over before publishing
+            *reinterpret_cast<float4 *>(smem + OFF_HIN + ss * kHalf * 4 + ch * 4) =
+                make_float4(hin[0], hin[1], hin[2], hin[3]);
+            // (the aggregate slot was read above and stays untouched until this
+            // tile's pass 2 has run: pass 1 of the slot's next tile waits for both)
+            *reinterpret_cast<float4 *>(smem + OFF_AGG + ss * kHalf * 8 + ch * 4) =
+                make_float4(pre[0], pre[1], pre[2], pre[3]);
+            mbar_arrive(bar(B_LB, ss));
+            if (!suppress) {
                 *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
                 __threadfence();
                 __syncwarp();
@@ -934,8 +1031,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     }
 
     // ------------------------------------------------------------------ teardown
+    // No thread of either CTA writes into or arrives on the other after this.
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
@@ -989,24 +1087,45 @@ size_t fused_workspace_bytes(int B, int T, int D) { return layout_of(B, T, D).to
 rglru_status fused_prefill(const PrefillArgs &a)
 {
     const Layout L = layout_of(a.B, a.T, a.D);
-    if ((size_t)L.tpg > 0x7fffffffu / 2 || L.G > (int)(sizeof(WsHeader::ticket) / sizeof(unsigned int)))
+    const int H = a.D / kHead;
+    if ((size_t)L.tpg > 0x7fffffffu / 2 || H > (int)(sizeof(WsHeader::ticket) / sizeof(unsigned int)))
         return RGLRU_ERR_UNSUPPORTED;
     auto encode = encode_fn();
     if (!encode) return RGLRU_ERR_CUDA;
 
-    CUtensorMap tmap;
-    const cuuint64_t gdim[3] = {(cuuint64_t)a.D, (cuuint64_t)a.T, (cuuint64_t)a.B};
-    const cuuint64_t gstride[2] = {(cuuint64_t)a.D * 2, (cuuint64_t)a.T * a.D * 2};
-    const cuuint32_t box[3] = {kHalf, NT, 1};
     const cuuint32_t estride[3] = {1, 1, 1};
-    if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.g), gdim, gstride, box, estride,
+    // x [B, T, D]: this half's 128 channels x (32 + 3) tokens of one sequence
+    CUtensorMap tmap_x;
+    const cuuint64_t xdim[3] = {(cuuint64_t)a.D, (cuuint64_t)a.T, (cuuint64_t)a.B};
+    const cuuint64_t xstride[2] = {(cuuint64_t)a.D * 2, (cuuint64_t)a.T * a.D * 2};
+    const cuuint32_t xbox[3] = {(cuuint32_t)kHalf, (cuuint32_t)kXRows, 1};
+    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.x), xdim, xstride, xbox, estride,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RGLRU_ERR_CUDA;
-    CUtensorMap tmap_x;
-    const cuuint32_t xbox[3] = {256, kXRows, 1};
-    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.x), gdim, gstride, xbox, estride,
+    // GELU branch [B, T, D]: this half's 128 channels x 32 tokens (L2 prefetch boxes)
+    CUtensorMap tmap_g;
+    const cuuint32_t gbox[3] = {(cuuint32_t)kHalf, (cuuint32_t)NT, 1};
+    if (encode(&tmap_g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.g), xdim, xstride, gbox, estride,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RGLRU_ERR_CUDA;
+    // y [B, T, D]: tensor stores of this half's 128 channels x 32 tokens
+    CUtensorMap tmap_y;
+    if (encode(&tmap_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.y, xdim, xstride, gbox, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return RGLRU_ERR_CUDA;
+    // gate matrices [D rows, 256]: 128-row x 64-channel boxes in the 128-byte
+    // swizzle of the tensor core's K-major operand
+    CUtensorMap tmap_wa, tmap_wx;
+    const cuuint64_t wdim[2] = {256, (cuuint64_t)a.D}, wstride[1] = {256 * 2};
+    const cuuint32_t wbox[2] = {64, (cuuint32_t)kHalf};
+    if (encode(&tmap_wa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.W_a), wdim, wstride, wbox,
+               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        encode(&tmap_wx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.W_x), wdim, wstride, wbox,
+               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RGLRU_ERR_CUDA;
 
@@ -1028,11 +1147,11 @@ rglru_status fused_prefill(const PrefillArgs &a)
         return RGLRU_ERR_CUDA;
 
     FusedParams p;
-    p.B = a.B; p.T = a.T; p.D = a.D; p.C = L.C; p.G = L.G; p.tiles_per_group = L.tpg;
+    p.B = a.B; p.T = a.T; p.D = a.D; p.C = L.C; p.tiles_per_head = L.tpg;
     p.x = static_cast<const __nv_bfloat16 *>(a.x);
+    p.g = static_cast<const __nv_bfloat16 *>(a.g);
     p.conv_w = a.conv_w; p.conv_b = a.conv_b;
-    p.W_a = static_cast<const __nv_bfloat16 *>(a.W_a); p.b_a = a.b_a;
-    p.W_x = static_cast<const __nv_bfloat16 *>(a.W_x); p.b_x = a.b_x;
+    p.b_a = a.b_a; p.b_x = a.b_x;
     p.lambda = a.lambda; p.segpos = a.segpos;
     p.conv_state = static_cast<__nv_bfloat16 *>(a.conv_state);
     p.h_state = a.h_state;
@@ -1043,9 +1162,12 @@ rglru_status fused_prefill(const PrefillArgs &a)
     p.prefix = reinterpret_cast<float *>(ws + L.prefix_off);
     p.trace = L.trace_off ? reinterpret_cast<unsigned long long *>(ws + L.trace_off) : nullptr;
 
-    const int per_group = max(1, sms / L.G);
-    const int grid = per_group * L.G;
-    rglru_prefill_fused_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(p, tmap, tmap_x);
+    // one cluster of two CTAs (the two halves of a head) per SM pair; the same
+    // number of clusters per head, which claim that head's tiles in order
+    const int per_head = max(1, (sms / 2) / H);
+    const long long grid = 2LL * per_head * H;
+    if (grid > 0x7fffffffLL) return RGLRU_ERR_UNSUPPORTED;
+    rglru_prefill_fused_kernel<<<(unsigned)grid, kThreads, kSmemBytes, a.stream>>>(p, tmap_x, tmap_g, tmap_y, tmap_wa, tmap_wx);
     return cuda_status(cudaGetLastError());
 }
 
