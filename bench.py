@@ -42,6 +42,24 @@ def _env_rank():
         int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(value: float, device="cpu") -> float:
+    """The maximum of ``value`` over all ranks of the default process group
+    (the value itself without one).  Time-like values are reduced this way, so
+    the slowest rank sets the job's time."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the units every rank processed in one step, divided
+    by the (max-over-ranks) step time."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -286,13 +304,9 @@ def run_cuda(args, w):
     st = api.device_status(ws)
     if st != api.OK:
         raise RuntimeError(f"prefill reported device status {api.status_string(st)}: no valid timing")
-    ms_t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if distributed:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    per_step_ms = ms_max / args.steps
+    per_step_ms = max_over_ranks(ms, dev) / args.steps
     tokens = w.tokens * world
-    value = tokens / (per_step_ms * 1e-3)
+    value = job_throughput(w.tokens, world, per_step_ms)
 
     # ---- end to end through the public API: pinned host inputs in, y back to host
     hx = torch.from_numpy(inp["x"]).to(bf).pin_memory()
@@ -318,10 +332,7 @@ def run_cuda(args, w):
         e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    e_ms = torch.tensor([ev0.elapsed_time(ev1)], device=dev, dtype=torch.float64)
-    if distributed:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e_value = tokens / (float(e_ms.item()) / e_steps * 1e-3)
+    e_value = job_throughput(w.tokens, world, max_over_ranks(ev0.elapsed_time(ev1), dev) / e_steps)
     st = api.device_status(ws)
     if st != api.OK:
         raise RuntimeError(f"prefill reported device status {api.status_string(st)} in the e2e loop")
@@ -466,15 +477,12 @@ def run_decode(d, launch_count, stream, distributed):
     del graph
     if st != 0:
         raise RuntimeError(f"decode reported device status {st}: no valid timing")
-    ms = torch.tensor([ev0.elapsed_time(ev1)], device=stream.device, dtype=torch.float64)
-    if distributed:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    ms = float(ms.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), stream.device)
     world = dist.get_world_size() if distributed else 1
     per_step_us = 1e3 * ms / steps
     step_bytes = W.decode_step_bytes(w)
     n_launch, names = launch_count
-    return {"workload": w.scaled(T=steps).describe(), "value": world * w.B * steps / (ms * 1e-3),
+    return {"workload": w.scaled(T=steps).describe(), "value": job_throughput(w.B, world, ms / steps),
             "unit": "tokens/s", "us_per_step": per_step_us, "steps": steps,
             "algorithmic_gbs": step_bytes / (per_step_us * 1e-6) / 1e9,
             "algorithmic_bytes_per_step": step_bytes, "gpu_launches": n_launch * steps,

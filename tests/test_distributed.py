@@ -1,0 +1,75 @@
+"""The N > 1 path of bench.py on CPU: world-size-2 process groups over gloo.
+
+bench.py runs one replica of the workload per GPU (no data-path collective);
+the only cross-rank steps are the max-over-ranks reduction of the timed
+region and the whole-job throughput derived from it.  These tests run those
+steps on two gloo ranks, and check that the reference arm does its work on
+rank 0 only.
+"""
+import json
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out_dir: str):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # each rank's own step time; the slowest sets the job's time
+        own_ms = 1.5 * (rank + 1)
+        ms = bench.max_over_ranks(own_ms)
+        value = bench.job_throughput(32768, world, ms)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"ms": ms, "value": value}, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_job_throughput_gloo(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    got = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    for g in got:
+        assert g["ms"] == pytest.approx(3.0)                       # the slower rank's time
+        assert g["value"] == pytest.approx(32768 * 2 / 3.0e-3)     # all ranks' units / that time
+
+
+def test_single_process_reduction_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(2.25) == 2.25
+    assert bench.job_throughput(10, 1, 2.0) == pytest.approx(5000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+    from lm_causal_depthwise_b200 import workloads as W
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = argparse.Namespace(steps=1, warmup=0)
+    assert bench.run_reference(args, W.TINY_F32) == 0
+    assert capsys.readouterr().out == ""
