@@ -66,7 +66,7 @@ constexpr int kP2Lag = 2;       // a group runs pass 2 of its tile kP2Lag tiles 
 constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
 constexpr int kConvWarp0 = kScanWarps;
 constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kSchedWarp = kMmaWarp + 1;
-constexpr int kLbWarp0 = kMmaWarp + 2, kLbWarps = 3;
+constexpr int kLbWarp0 = kMmaWarp + 2, kLbWarps = 6;
 constexpr int kThreads = 32 * (kLbWarp0 + kLbWarps);
 constexpr int kGroupThreads = 128;  // threads of one scan group or of the conv warps (one per channel)
 constexpr int kEndMarkers = kLbWarps > kScanGroups ? kLbWarps : kScanGroups;
@@ -352,6 +352,20 @@ __device__ __forceinline__ f2_t gelu2(f2_t g)
     return f2_fma(hg, f2_make(t0, t1), hg);
 }
 
+// two fp32 rounded to nearest-even as a bf16 pair / an f16 pair (element 0 low)
+__device__ __forceinline__ uint32_t pack_bf16_pair(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_f16_pair(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 __device__ __forceinline__ float gelu_tanh_fast(float g)
 {
     const float k0 = 0.7978845608028654f, k1 = 0.7978845608028654f * 0.044715f;
@@ -564,36 +578,41 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const bool clean = (ti.reset_mask | ti.m2 | ti.m3) == 0u && ti.valid == NT;
             auto run = [&](auto clean_tag) {
                 constexpr bool kClean = decltype(clean_tag)::value;
+                // one token: the four taps (lag k dropped when segment_pos < k)
+                auto conv1 = [&](int t, float m3, float m2, float m1, float x0) -> float {
+                    if constexpr (kClean) {
+                        return fmaf(w3, x0, fmaf(w2, m1, fmaf(w1, m2, fmaf(w0, m3, cb))));
+                    } else {
+                        float v = cb;
+                        if (!((ti.m3 >> t) & 1u)) v = fmaf(w0, m3, v);
+                        if (!((ti.m2 >> t) & 1u)) v = fmaf(w1, m2, v);
+                        if (!((ti.reset_mask >> t) & 1u)) v = fmaf(w2, m1, v);
+                        v = fmaf(w3, x0, v);
+                        return t < ti.valid ? v : 0.f;
+                    }
+                };
 #pragma unroll 1
                 for (int t8 = 0; t8 < NT; t8 += 8) {
                     uint32_t xq[4];
+                    const uint32_t brow = bl + (uint32_t)t8 * 128;  // t8 is a multiple of 8: row t8 + k swizzles by k
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
+                    for (int k = 0; k < 8; k += 2) {
                         const int t = t8 + k;
                         const float x0 = __bfloat162float(xs[(t + 3) * kHalf]);
-                        float v;
-                        if constexpr (kClean) {
-                            v = fmaf(w3, x0, fmaf(w2, xm1, fmaf(w1, xm2, fmaf(w0, xm3, cb))));
-                        } else {
-                            // tap of lag k dropped when segment_pos < k (document start)
-                            v = cb;
-                            if (!((ti.m3 >> t) & 1u)) v = fmaf(w0, xm3, v);
-                            if (!((ti.m2 >> t) & 1u)) v = fmaf(w1, xm2, v);
-                            if (!((ti.reset_mask >> t) & 1u)) v = fmaf(w2, xm1, v);
-                            v = fmaf(w3, x0, v);
-                            if (t >= ti.valid) v = 0.f;
-                        }
-                        const uint32_t off = (uint32_t)t * 128 + ((chunk ^ (uint32_t)(t & 7)) << 4) + sub;
-                        const uint16_t bv = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(bl + off), "h"(bv) : "memory");
-                        const __half hv = __float2half_rn(v);
-                        if (k & 1)
-                            xq[k >> 1] |= (uint32_t)__half_as_ushort(hv) << 16;
-                        else
-                            xq[k >> 1] = (uint32_t)__half_as_ushort(hv);
-                        xm3 = xm2;
-                        xm2 = xm1;
-                        xm1 = x0;
+                        const float x1 = __bfloat162float(xs[(t + 4) * kHalf]);
+                        const float v0 = conv1(t, xm3, xm2, xm1, x0);
+                        const float v1 = conv1(t + 1, xm2, xm1, x0, x1);
+                        const uint32_t bw = pack_bf16_pair(v0, v1);
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(brow + k * 128 + ((chunk ^ (uint32_t)k) << 4) + sub),
+                                     "h"((uint16_t)bw)
+                                     : "memory");
+                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(brow + (k + 1) * 128 + ((chunk ^ (uint32_t)(k + 1)) << 4) + sub),
+                                     "h"((uint16_t)(bw >> 16))
+                                     : "memory");
+                        xq[k >> 1] = pack_f16_pair(v0, v1);
+                        xm3 = xm1;
+                        xm2 = x0;
+                        xm1 = x1;
                     }
                     tmem_st4(xh_col + (uint32_t)(t8 >> 1), xq);
                 }
@@ -697,12 +716,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // r = (1 + tr) / 2 with tr = tanh(half pre-activation): log a = tr * hkl + hkl
         const float hkl = 0.5f * kl;
         const float hkl2 = hkl * 1.4426950408889634f;  // same in log2
-        // every log a of this channel lies in [kl, 0]: the short series for
-        // 1 - a^2 applies to all of them when kl > -1/8
-        const bool series_ok = kl > -0.125f;
         const f2_t hba2 = f2_splat(hba), hbx2 = f2_splat(hbx), hkl_2 = f2_splat(hkl), hkl2_2 = f2_splat(hkl2);
-        const f2_t c13_2 = f2_splat(1.f / 3.f), c23_2 = f2_splat(2.f / 3.f), one_2 = f2_splat(1.f),
-                   mtwo_2 = f2_splat(-2.f);
+        const f2_t one_2 = f2_splat(1.f);
         // GELU branch of the group's next tile into its shared-memory buffer
         // (the tile was prefetched into L2 with its x): each thread copies the
         // 4-byte words holding its own channel, so it reads only its own copies
@@ -744,7 +759,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 #pragma unroll
                 for (int k = 0; k < 8; ++k) gcur[k] = gs[(t8 + k) * kHalf];
                 uint32_t st[8];
-                const bool clean = ((ti.reset_mask >> t8) & 0xffu) == 0u && t8 + 8 <= ti.valid && series_ok;
+                const bool clean = ((ti.reset_mask >> t8) & 0xffu) == 0u && t8 + 8 <= ti.valid;
                 if (clean) {
 #pragma unroll
                     for (int k = 0; k < 8; k += 2) {
@@ -753,14 +768,14 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const f2_t zi = f2_add(f2_make(__uint_as_float(ai[k]), __uint_as_float(ai[k + 1])), hbx2);
                         const f2_t tr = f2_make(tanh_approx(f2_lo(zr)), tanh_approx(f2_hi(zr)));
                         const f2_t tg = f2_make(tanh_approx(f2_lo(zi)), tanh_approx(f2_hi(zi)));
-                        const f2_t ell = f2_fma(tr, hkl_2, hkl_2);    // log a
                         const f2_t la = f2_fma(tr, hkl2_2, hkl2_2);  // log2 a
                         const float a0 = ex2_approx(f2_lo(la)), a1 = ex2_approx(f2_hi(la));
-                        // 1 - exp(2 ell) by its series (see one_minus_exp2l_small)
-                        f2_t sr = f2_fma(ell, c13_2, c23_2);
-                        sr = f2_fma(ell, sr, one_2);
-                        sr = f2_fma(ell, sr, one_2);
-                        const f2_t om = f2_mul(f2_mul(ell, mtwo_2), sr);
+                        // 1 - a^2 directly: with a good to ~2^-22 relative, its
+                        // absolute error is under 5e-7, so sqrt(1 - a^2) errs by at
+                        // most ~6e-5 absolute even as a -> 1 (small r), where the
+                        // term it scales is itself that small
+                        const f2_t a2 = f2_make(a0, a1);
+                        const f2_t om = f2_fma(f2_mul(a2, f2_splat(-1.f)), a2, one_2);
                         const f2_t nrm = f2_make(sqrt_approx(f2_lo(om)), sqrt_approx(f2_hi(om)));
                         const f2_t xh2 = f2_make(xh.x, xh.y);
                         const f2_t v = f2_mul(nrm, f2_fma(tg, xh2, xh2));  // sqrt(1-a^2) * i * xc
