@@ -22,6 +22,9 @@
 //   4. the epilogue applies the gates, a = sigmoid(Lambda)^(8 r), the
 //      normalised one-step update (a reset when segment_pos == 0) and the GELU
 //      product; y goes out through shared memory and a TMA store, h directly.
+// The launch allows programmatic dependent launch: barrier and TMEM set-up
+// may overlap the previous kernel's tail; every global access follows
+// griddepcontrol.wait.
 // Each CTA reads and writes only its own channels of the states, so the two
 // CTAs never race.  Waits on mbarriers are bounded (RGLRU_ERR_TIMEOUT in the
 // workspace header); the two cluster barriers are reached exactly once by every
@@ -145,12 +148,20 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const int d = ch0 + c;
     const int n0 = (warp >> 2) * kRows;
 
-    // ---- 1. loads
+    // ---- 0. set-up that touches no global memory, which may overlap the tail
+    // of the previous kernel on the stream (programmatic dependent launch)
     if (tid == 32) {
         mbar_init(bar_in, 1);
         mbar_init(bar_w, 1);
         mbar_init(bar_mma, 1);
         mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
+    griddep_launch_dependents();
+    griddep_wait();  // every global read below sees the previous kernel's writes
+
+    // ---- 1. loads
+    if (tid == 32) {
         mbar_arrive_expect_tx(bar_in, kXTile + kCsTile);  // whole boxes: rows past B arrive zero-filled
         tma_load_2d(smem + OFF_X, &tm_x, bar_in, ch0, b0);
         tma_load_3d(smem + OFF_CS, &tm_cs, bar_in, ch0, 0, b0);
@@ -162,7 +173,6 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         }
     }
     if (tid < kTok) sp_s[tid] = tid < nb ? p.segpos[b0 + tid] : 3;
-    if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
     float hprev[kRows];
     uint32_t graw[kRows / 2];  // bf16 pairs of consecutive rows
 #pragma unroll
@@ -371,9 +381,20 @@ rglru_status decode_step(const PrefillArgs &a)
     p.hdr = reinterpret_cast<WsHeader *>(a.ws);
     const long long clusters = (long long)(a.D / kHead) * p.nblk;
     if (clusters * 2 > 0x7fffffffLL) return RGLRU_ERR_UNSUPPORTED;
-    rglru_decode_kernel<<<(unsigned)(clusters * 2), kThreads, kSmemBytes, a.stream>>>(p, tm_wa, tm_wx, tm_x, tm_y,
-                                                                                     tm_cs);
-    return cuda_status(cudaGetLastError());
+    // programmatic stream serialization: the kernel may be scheduled while the
+    // previous one on the stream finishes; it waits (griddepcontrol.wait)
+    // before its first global memory access
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(clusters * 2));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, rglru_decode_kernel, p, tm_wa, tm_wx, tm_x, tm_y, tm_cs));
 }
 
 }  // namespace rglru

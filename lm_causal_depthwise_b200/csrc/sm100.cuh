@@ -338,6 +338,17 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src)
 // this thread's cp.async copies have landed
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// this grid's dependents (launched with programmatic stream serialization) may
+// be scheduled now; they still wait for this grid's completion in griddep_wait
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// the grids this one depends on have completed and their memory is visible
+// (returns at once when there are none)
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- thread-block clusters
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
