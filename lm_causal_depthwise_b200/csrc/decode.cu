@@ -69,6 +69,25 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kTmemCols = 2 * kTok;        // D_r then D_i
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
+// Tracing (compiled in with -DRGLRU_TRACE only): CTAs below kTraceCtas record
+// %globaltimer at each phase into trace[cta * kTraceEvents + event].
+enum DecTraceEvent {
+    DT_START, DT_WAITED, DT_INPUTS, DT_CONV, DT_CLUSTER, DT_WEIGHTS, DT_MMA, DT_EPI0, DT_EPI1, DT_END, kTraceEvents
+};
+#ifdef RGLRU_TRACE
+constexpr int kTraceCtas = 8;
+#define DEC_TR(ev)                                                                                     \
+    do {                                                                                              \
+        if (blockIdx.x < kTraceCtas)                                                                  \
+            reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(p.hdr) + kWsHeaderBytes)  \
+                [blockIdx.x * kTraceEvents + (ev)] = globaltimer();                                   \
+    } while (0)
+#else
+#define DEC_TR(ev) \
+    do {           \
+    } while (0)
+#endif
+
 struct DecodeParams {
     int B, D, nblk;
     const __nv_bfloat16 *g;
@@ -148,6 +167,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const int d = ch0 + c;
     const int n0 = (warp >> 2) * kRows;
 
+    if (tid == 0) DEC_TR(DT_START);
     // ---- 0. set-up that touches no global memory, which may overlap the tail
     // of the previous kernel on the stream (programmatic dependent launch)
     if (tid == 32) {
@@ -159,6 +179,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
     griddep_launch_dependents();
     griddep_wait();  // every global read below sees the previous kernel's writes
+    if (tid == 0) DEC_TR(DT_WAITED);
 
     // ---- 1. loads
     if (tid == 32) {
@@ -173,17 +194,16 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         }
     }
     if (tid < kTok) sp_s[tid] = tid < nb ? p.segpos[b0 + tid] : 3;
+    // (kept as loaded, one register each, so that nothing waits for them
+    // before the epilogue uses them)
     float hprev[kRows];
-    uint32_t graw[kRows / 2];  // bf16 pairs of consecutive rows
+    uint16_t graw[kRows];
 #pragma unroll
-    for (int k = 0; k < kRows; k += 2) {
+    for (int k = 0; k < kRows; ++k) {
         const int n = n0 + k;
-        const size_t e0 = (size_t)(b0 + n) * p.D + d, e1 = e0 + p.D;
-        const uint32_t g0 = n < nb ? (uint32_t)__bfloat16_as_ushort(p.g[e0]) : 0u;
-        const uint32_t g1 = n + 1 < nb ? (uint32_t)__bfloat16_as_ushort(p.g[e1]) : 0u;
-        graw[k / 2] = g0 | (g1 << 16);
-        hprev[k] = n < nb ? p.h_state[e0] : 0.f;
-        hprev[k + 1] = n + 1 < nb ? p.h_state[e1] : 0.f;
+        const size_t e = (size_t)(b0 + n) * p.D + d;
+        graw[k] = n < nb ? __bfloat16_as_ushort(p.g[e]) : (uint16_t)0;
+        hprev[k] = n < nb ? p.h_state[e] : 0.f;
     }
     const float w0 = 0.5f * p.conv_w[d], w1 = 0.5f * p.conv_w[(size_t)p.D + d],
                 w2 = 0.5f * p.conv_w[2 * (size_t)p.D + d], w3 = 0.5f * p.conv_w[3 * (size_t)p.D + d];
@@ -197,6 +217,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     // ---- 2. conv: xh = xc / 2 (halving is exact: the MMA then gives half
     // pre-activations for sigmoid(z) = (1 + tanh(z / 2)) / 2)
     bool ok = dec_wait(bar_in, 0, p.hdr, 0);
+    if (tid == 0) DEC_TR(DT_INPUTS);
     float xh[kRows];
     {
         const int k = (int)half * kHalfCh + c;  // channel within the head = K index of the B tile
@@ -226,10 +247,12 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(b_peer + off), "h"(bv) : "memory");
         }
     }
+    if (tid == 0) DEC_TR(DT_CONV);
     fence_proxy_async_cluster();  // B tiles (both CTAs) and the conv_state tile, for the async proxy
     tc_fence_before();
     cluster_sync();               // both halves of both B tiles written
     tc_fence_after();
+    if (tid == 0) DEC_TR(DT_CLUSTER);
 
     // ---- 3. conv_state write-back and the gate projections
     if (warp == 1) {
@@ -238,6 +261,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             bulk_commit();
         }
         ok = dec_wait(bar_w, 0, p.hdr, 1) && ok;
+        if (lane == 0) DEC_TR(DT_WEIGHTS);
         if (ok && lane == 0) {
             tc_fence_after();
             const uint32_t idesc = umma_idesc_bf16(kHalfCh, kTok);
@@ -250,12 +274,14 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 umma_ss(tmem + kTok, umma_desc_sw128(wx + ko), bd, idesc, kk > 0);
             }
             umma_commit(bar_mma);
+            DEC_TR(DT_MMA);
         }
         __syncwarp();
     }
 
     // ---- 4. epilogue
     ok = dec_wait(bar_mma, 0, p.hdr, 2) && ok;
+    if (tid == 0) DEC_TR(DT_EPI0);
     tc_fence_after();
     __nv_bfloat16 *y_s = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_X);  // the x tile is dead
     if (ok) {
@@ -281,13 +307,13 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 const float om = ell > -0.125f ? one_minus_exp2l(ell) : fmaf(-a, a, 1.f);
                 const float uu = fmaf(tg, xh[i], xh[i]);  // i * xc
                 const float h = sp_s[n] == 0 ? uu : fmaf(a, hprev[i], sqrt_approx(om) * uu);
-                const uint32_t gw = graw[i / 2];
-                const float gv = __uint_as_float((i & 1) ? (gw & 0xffff0000u) : (gw << 16));
+                const float gv = __uint_as_float((uint32_t)graw[i] << 16);
                 y_s[n * kHalfCh + c] = __float2bfloat16_rn(gelu_tanh(gv) * h);
                 if (n < nb) p.h_state[(size_t)(b0 + n) * p.D + d] = h;
             }
         }
     }
+    if (tid == 0) DEC_TR(DT_EPI1);
     fence_proxy_async_smem();  // y tile, for the async proxy
     tc_fence_before();
     __syncthreads();
@@ -298,6 +324,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             bulk_commit();
         }
         bulk_wait_read_all();  // shared memory stays valid until the stores have read it
+        DEC_TR(DT_END);
     }
     if (warp == 0) {
         if (!ok) {
@@ -335,7 +362,11 @@ bool encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *m, const
 
 }  // namespace
 
+#ifdef RGLRU_TRACE
+size_t decode_workspace_bytes(int, int) { return kWsHeaderBytes + kTraceCtas * kTraceEvents * 8; }
+#else
 size_t decode_workspace_bytes(int, int) { return kWsHeaderBytes; }
+#endif
 
 rglru_status decode_step(const PrefillArgs &a)
 {
