@@ -11,24 +11,25 @@
 //                CTAs (the two halves of the head's 256 input channels meet in
 //                each CTA's shared memory through the cluster).
 //   MMA thread   both block-diagonal gate projections on the tensor cores:
-//                D[128 out x 32 tok] = W[128 x 256] * xc^T, A (this half's rows
-//                of W_a or W_x, TMA-loaded once, 128-byte swizzled) and B in
-//                shared memory, fp32 accumulators in TMEM.
+//                D[128 out x 32 tok] = W[128 x 256] * xc^T with A (this half's
+//                rows of W_a or W_x) resident in TMEM, written once by the scan
+//                warps, and B in shared memory; fp32 accumulators in TMEM.
 //   scan warps   thread = channel, two groups taking alternate tiles.  Pass 1:
 //                sigmoid gates, a = sigmoid(Lambda)^(8 r), sqrt(1-a^2)
-//                normaliser, resets, GELU_tanh(g); the local scan from h = 0
-//                gives the tile aggregate (prod a, h_end) and, per token, the
-//                output without the carried-in state, y_loc = G h_loc, and its
-//                coefficient q = G prod a, kept in TMEM as f16 pairs (the
-//                accumulators are free again at once).  Pass 2 (two tiles
-//                later): y = y_loc + q h_in.
+//                normaliser, resets, GELU_tanh(g) (the g tile arrives by one
+//                tensor load); the local scan from h = 0 gives the tile
+//                aggregate (prod a, h_end) and, per token, the output without
+//                the carried-in state, y_loc = G h_loc, and its coefficient
+//                q = G prod a, stashed in shared memory as f16 pairs (the
+//                accumulators and xc are free again at once).
 //   look-back    publish each tile aggregate as soon as pass 1 ends, walk back
 //   warps        over predecessor tiles of the sequence to the nearest anchor
 //                (a published inclusive prefix, or a tile holding a reset: A =
 //                0), fold h <- A h + H forward from it in sequence order
 //                (decoupled look-back with a fixed combination order, so
-//                results are bit-reproducible), hand h_in to pass 2, publish
-//                the inclusive prefix.
+//                results are bit-reproducible), publish the inclusive prefix,
+//                then pass 2 of the tile: y = y_loc + q h_in from the stash,
+//                4 channels per lane, stored straight to global memory.
 //   scheduler    rank 0 claims tiles and fills both CTAs' descriptor rings;
 //                each CTA TMA-loads its own channels of x (tile + 3 halo rows).
 // Every wait is bounded: a wait that runs out records RGLRU_ERR_TIMEOUT in the
@@ -56,13 +57,12 @@ using namespace sm100;
 constexpr int NT = 32;          // tokens per tile (MMA N)
 constexpr int kHalf = 128;      // channels per CTA (MMA M, TMEM lanes)
 constexpr int NX = 4;           // xc/2 slots in TMEM (conv -> pass 1)
-constexpr int NA = 4;           // accumulator slots in TMEM (MMA -> pass 1)
-constexpr int NS = 6;           // stash slots in TMEM (pass 1 -> pass 2)
+constexpr int NA = 2;           // accumulator slots in TMEM (MMA -> pass 1), one per scan group
+constexpr int NS = 6;           // stash slots in shared memory (pass 1 -> look-back and pass 2)
 constexpr int NB = 2;           // B tiles in shared memory (conv -> MMA, both CTAs)
 constexpr int XRING = 2;        // x tiles in shared memory (TMA -> conv)
 constexpr int INFO_RING = 16;   // tile descriptors in flight
 constexpr int kScanGroups = 2;  // scan warp groups, alternate tiles
-constexpr int kP2Lag = 2;       // a group runs pass 2 of its tile kP2Lag tiles back
 constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
 constexpr int kConvWarp0 = kScanWarps;
 constexpr int kMmaWarp = kConvWarp0 + kConvWarps, kSchedWarp = kMmaWarp + 1;
@@ -74,33 +74,32 @@ constexpr int kEndMarkers = kLbWarps > kScanGroups ? kLbWarps : kScanGroups;
 // group's tiles use only its own accumulator and stash slots, a look-back
 // warp's tiles revisit a stash slot every lcm(kLbWarps, NS) = NS tiles
 static_assert(NA % kScanGroups == 0 && NS % kScanGroups == 0 && NS % kLbWarps == 0, "slot residues");
-static_assert(NS == kScanGroups * (kP2Lag + 1), "stash slots cover the pass-2 lag");
 static_assert(kEndMarkers <= INFO_RING, "end markers fit the ring");
 
-// TMEM columns (512): xc/2 f16 pairs, accumulators [pre_r | pre_i], stash f16 pairs
-constexpr uint32_t kColXh = 0, kColsXh = NT / 2;
-constexpr uint32_t kColAcc = kColXh + NX * kColsXh, kColsAcc = 2 * NT;
-constexpr uint32_t kColStash = kColAcc + NA * kColsAcc, kColsStash = NT;
-static_assert(kColStash + NS * kColsStash <= 512, "TMEM budget");
+// TMEM columns (512): this half's rows of W_a then W_x (the MMA's A operand,
+// bf16 pairs: K-step kk of a gate at column 8 kk), accumulators
+// [pre_r | pre_i], xc/2 f16 pairs
+constexpr uint32_t kColW = 0, kColsWGate = 128;
+constexpr uint32_t kColAcc = kColW + 2 * kColsWGate, kColsAcc = 2 * NT;
+constexpr uint32_t kColXh = kColAcc + NA * kColsAcc, kColsXh = NT / 2;
+static_assert(kColXh + NX * kColsXh <= 512, "TMEM budget");
 
 // Shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kWBlock = kHalf * 128;            // 128 weight rows x 64 channels (bf16)
-constexpr int kWGate = 4 * kWBlock;             // one gate, K = 256
 constexpr int kBBlock = NT * 128;               // one K-block of the B tile: NT rows x 128 B
 constexpr int kBTile = 4 * kBBlock;             // bf16 xc of all 256 channels of the head
 constexpr int kXRows = NT + 3;
 constexpr int kXTile = kXRows * kHalf * 2;      // bf16 x of this half, 3 halo rows first
-constexpr int OFF_W = 0;                        // W_a rows, then W_x rows of this half
-constexpr int OFF_B = OFF_W + 2 * kWGate;
+constexpr int OFF_B = 0;
 constexpr int OFF_X = OFF_B + NB * kBTile;
 constexpr int kGTile = NT * kHalf * 2;          // bf16 GELU branch of this half: [token][channel]
 constexpr int OFF_G = OFF_X + XRING * kXTile;   // one per scan group
-constexpr int OFF_Y = OFF_G + kScanGroups * kGTile;  // bf16 y of a tile, one per scan group
-// per stash slot: (prod a, h_end) per channel from pass 1; the look-back then
-// leaves the state after the tile (per channel) in the first half
-constexpr int OFF_AGG = OFF_Y + kScanGroups * kGTile;
-constexpr int OFF_HIN = OFF_AGG + NS * kHalf * 8;         // per stash slot: carried-in h per channel
-constexpr int OFF_INFO = OFF_HIN + NS * kHalf * 4;
+// stash slots: per token t and channel c, (y_loc, q) as an f16 pair at
+// (t * 128 + c) * 4 (a look-back lane reads its 4 channels of a token at once)
+constexpr int kStash = NT * kHalf * 4;
+constexpr int OFF_ST = OFF_G + kScanGroups * kGTile;
+// per stash slot: (prod a, h_end) per channel from pass 1
+constexpr int OFF_AGG = OFF_ST + NS * kStash;
+constexpr int OFF_INFO = OFF_AGG + NS * kHalf * 8;
 constexpr int OFF_BAR = OFF_INFO + INFO_RING * 32;
 // barrier arrays: [first index, count]
 enum {
@@ -114,14 +113,12 @@ enum {
     B_MMA = B_BFREE + NB,
     B_ACC_FREE = B_MMA + NA,
     B_PASS1 = B_ACC_FREE + NA,
-    B_PUB = B_PASS1 + NS,
-    B_LB = B_PUB + NS,
-    B_STASH_FREE = B_LB + NS,
+    B_STASH_FREE = B_PASS1 + NS,   // the look-back warp is done with the stash slot (and its aggregate)
     B_BHALF = B_STASH_FREE + NS,   // this CTA's half of a B tile written (before the copy to the peer)
-    B_YFULL = B_BHALF + NB,        // per scan group: its y tile written (before the tensor store)
-    B_YFREE = B_YFULL + kScanGroups,  // per scan group: the previous tensor store has read its y tile
-    B_W_FULL = B_YFREE + kScanGroups,
-    B_COUNT
+    B_W_FULL = B_BHALF + NB,
+    B_GFULL = B_W_FULL + 1,           // per scan group: the GELU-branch tile of its next tile has landed
+    B_GFREE = B_GFULL + kScanGroups,  // per scan group: pass 1 has read the GELU-branch tile
+    B_COUNT = B_GFREE + kScanGroups
 };
 constexpr int OFF_MISC = OFF_BAR + B_COUNT * 8;
 constexpr int kSmemUsed = OFF_MISC + 16;
@@ -145,6 +142,7 @@ struct FusedParams {
     const __nv_bfloat16 *x, *g;
     const float *conv_w, *conv_b;
     const float *b_a, *b_x, *lambda;
+    const __nv_bfloat16 *w_a, *w_x;  // [D rows][256] (row = output channel)
     const int32_t *segpos;
     __nv_bfloat16 *conv_state;
     float *h_state;
@@ -162,10 +160,10 @@ struct FusedParams {
 enum TraceEvent {
     TR_SCHED_INFO, TR_CONV_START, TR_CONV_DONE, TR_MMA_ISSUED, TR_P1_START, TR_P1_END, TR_LB_START,
     TR_LB_HIN, TR_LB_DONE, TR_P2_START, TR_P2_END, TR_TILE_U, TR_MMA_TFREE, TR_MMA_TMA, TR_MMA_CONV,
-    TR_CONV_GO, TR_P2_LD, TR_P2_ST, TR_CONV_LOOP, kTraceEvents
+    TR_CONV_GO, TR_CONV_LOOP, TR_P1_G, TR_P1_LD, TR_LB_ANC, TR_LB_K, kTraceEvents
 };
 #ifdef RGLRU_TRACE
-constexpr int kTraceCtas = 4, kTraceTiles = 128;
+constexpr int kTraceCtas = 4, kTraceTiles = 192;
 #define RGLRU_TR(ev, j, val)                                                                                   \
     do {                                                                                                      \
         if (p.trace != nullptr && blockIdx.x < kTraceCtas && (j) < kTraceTiles)                               \
@@ -193,9 +191,10 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile i
     if (mbar_try_wait_cl(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        // suspended in hardware until the phase completes (or 20 us pass)
+        // suspended in hardware until the phase completes (or a time limit
+        // passes); the abort and timeout checks run every 16th round
         if (mbar_try_wait_sleep_cl(bar, parity, 20000u)) return true;
-        {
+        if ((it & 15u) == 0) {
             if (*abort_flag) return false;
             if (*(volatile int *)&hdr->status != 0) {
                 *abort_flag = 1;
@@ -376,8 +375,7 @@ __device__ __forceinline__ float gelu_tanh_fast(float g)
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap tmap_x,
-                           const __grid_constant__ CUtensorMap tmap_g, const __grid_constant__ CUtensorMap tmap_y,
-                           const __grid_constant__ CUtensorMap tmap_wa, const __grid_constant__ CUtensorMap tmap_wx)
+                           const __grid_constant__ CUtensorMap tmap_g)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -402,7 +400,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         if (lane == 0) {
             for (int i = 0; i < INFO_RING; ++i) {
                 mbar_init(bar(B_INFO_FULL, i), 1);
-                mbar_init(bar(B_INFO_EMPTY, i), 2 * 4);  // pass-2 warps of both CTAs (rank 0's ring only)
+                mbar_init(bar(B_INFO_EMPTY, i), 2);  // the tile's look-back warps of both CTAs (rank 0's ring only)
             }
             for (int i = 0; i < XRING; ++i) {
                 mbar_init(bar(B_X_FULL, i), 1);
@@ -422,15 +420,13 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             }
             for (int i = 0; i < NS; ++i) {
                 mbar_init(bar(B_PASS1, i), kGroupThreads);
-                mbar_init(bar(B_PUB, i), 32);
-                mbar_init(bar(B_LB, i), 32);
-                mbar_init(bar(B_STASH_FREE, i), kGroupThreads);
+                mbar_init(bar(B_STASH_FREE, i), 32);
             }
             for (int i = 0; i < kScanGroups; ++i) {
-                mbar_init(bar(B_YFULL, i), kGroupThreads);
-                mbar_init(bar(B_YFREE, i), 1);
+                mbar_init(bar(B_GFULL, i), 1);
+                mbar_init(bar(B_GFREE, i), kGroupThreads);
             }
-            mbar_init(bar(B_W_FULL, 0), 1);
+            mbar_init(bar(B_W_FULL, 0), 2 * kGroupThreads);  // both scan groups' weight rows in TMEM
             *abort_flag = 0;
             mbar_fence_init();
         }
@@ -439,6 +435,13 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     cluster_sync();  // both CTAs' barriers initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+#ifdef RGLRU_TRACE
+    if (threadIdx.x == 0) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        RGLRU_TR(0, kTraceTiles - 1, (unsigned long long)smid);
+    }
+#endif
     const int debug_unit = *(volatile int *)&hdr->debug_unit_plus1 - 1;
 
     if (warp == kSchedWarp) {
@@ -645,17 +648,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            // this half's 128 rows of W_a and W_x: 4 K-blocks of 64 channels each
-            mbar_arrive_expect_tx(bar(B_W_FULL, 0), 2 * kWGate);
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-                tma_load_2d(smem + OFF_W + kb * kWBlock, &tmap_wa, bar(B_W_FULL, 0), kb * 64, ch0);
-                tma_load_2d(smem + OFF_W + kWGate + kb * kWBlock, &tmap_wx, bar(B_W_FULL, 0), kb * 64, ch0);
-            }
-        }
         const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
-        const uint32_t wa = smem_u32(smem + OFF_W), wx = wa + kWGate;
         bool w_ready = false;
         int issued = 0;
 #pragma unroll 1
@@ -677,10 +670,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 const uint32_t d_r = tmem + kColAcc + sa * kColsAcc, d_i = d_r + NT;
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk) {
-                    const uint32_t ko = (kk >> 2) * kWBlock + (kk & 3) * 32;
+                    // A (16 input channels of this half's weight rows) from TMEM
                     const uint64_t bd = umma_desc_sw128(bt + (kk >> 2) * kBBlock + (kk & 3) * 32);
-                    umma_ss(d_r, umma_desc_sw128(wa + ko), bd, idesc, kk > 0);
-                    umma_ss(d_i, umma_desc_sw128(wx + ko), bd, idesc, kk > 0);
+                    umma_ts(d_r, tmem + kColW + kk * 8, bd, idesc, kk > 0);
+                    umma_ts(d_i, tmem + kColW + kColsWGate + kk * 8, bd, idesc, kk > 0);
                 }
                 umma_commit(bar(B_MMA, sa));
                 umma_commit_cluster(bar(B_BFREE, sb), 0x3);  // this B slot is free in both CTAs' view
@@ -691,15 +684,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         }
         // Before the final cluster barrier: the commits of both CTAs for the
         // last tiles have landed on this CTA's B-slot barriers (so no arrival
-        // reaches a CTA that has exited), and the weight load is complete.
+        // reaches a CTA that has exited).
         if (lane == 0) {
             for (int k = max(0, issued - NB); k < issued; ++k) {
                 const uint64_t t0 = globaltimer();
                 while (!mbar_try_wait_cl(bar(B_BFREE, k % NB), (uint32_t)(k / NB) & 1u) && globaltimer() - t0 < kTimeoutNs) {
                 }
-            }
-            const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(bar(B_W_FULL, 0), 0u) && globaltimer() - t0 < kTimeoutNs) {
             }
         }
         __syncwarp();
@@ -709,6 +699,27 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const int c = threadIdx.x % kGroupThreads;
         const int d = ch0 + c;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        {
+            // this channel's row of W_a (group 0) or W_x (group 1) into its TMEM
+            // lane: 256 bf16 = 128 columns, read once from global memory
+            const uint4 *src = reinterpret_cast<const uint4 *>((sg == 0 ? p.w_a : p.w_x) + (size_t)d * 256);
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 v = __ldg(src + q * 8 + k);
+                    r[4 * k] = v.x;
+                    r[4 * k + 1] = v.y;
+                    r[4 * k + 2] = v.z;
+                    r[4 * k + 3] = v.w;
+                }
+                tmem_st32(tmem + lane_off + kColW + sg * kColsWGate + q * 32, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_W_FULL, 0));
+        }
         const float hba = 0.5f * p.b_a[d], hbx = 0.5f * p.b_x[d];
         const float lam = p.lambda[d];
         const float ls = lam >= 0.f ? -log1pf(expf(-lam)) : lam - log1pf(expf(lam));  // log sigmoid(Lambda)
@@ -719,14 +730,20 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const f2_t hba2 = f2_splat(hba), hbx2 = f2_splat(hbx), hkl_2 = f2_splat(hkl), hkl2_2 = f2_splat(hkl2);
         const f2_t one_2 = f2_splat(1.f);
         // GELU branch of the group's next tile into its shared-memory buffer
-        // (the tile was prefetched into L2 with its x): each thread copies the
-        // 4-byte words holding its own channel, so it reads only its own copies
+        // [token][channel] by one tensor load (the tile was prefetched into L2
+        // with its x; rows past the sequence end arrive zero-filled), issued
+        // once pass 1 of the group's previous tile has read the buffer.
         __nv_bfloat16 *gbuf = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_G + sg * kGTile);
-        auto copy_g = [&](const TileInfo &ti) {
-            const int c2 = c & ~1;
-            const __nv_bfloat16 *gp = p.g + ((size_t)ti.b * p.T + ti.t0) * p.D + ch0 + c2;
-#pragma unroll 4
-            for (int t = 0; t < ti.valid; ++t) cp_async4(gbuf + t * kHalf + c2, gp + (size_t)t * p.D);
+        int g_loads = 0;  // tensor loads issued into gbuf (the k-th completes phase k of B_GFULL)
+        auto load_g = [&](const TileInfo &ti) {
+            if (c == 0) {
+                if (g_loads == 0 || wait_bar(bar(B_GFREE, sg), (uint32_t)(g_loads - 1) & 1u, abort_flag, hdr, 24)) {
+                    mbar_arrive_expect_tx(bar(B_GFULL, sg), kGTile);
+                    tma_load_3d(gbuf, &tmap_g, bar(B_GFULL, sg), ch0, ti.t0, ti.b);
+                    ++g_loads;
+                }
+            }
+            __syncwarp();
         };
         auto pack_h2 = [](float lo, float hi) -> uint32_t {
             __half2 v = __floats2half2_rn(lo, hi);
@@ -736,17 +753,18 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         auto pass1 = [&](int j, const TileInfo &ti) -> bool {
             const int sa = j % NA, ss = j % NS, sx = j % NX;
             if (!warp_wait_bar(bar(B_MMA, sa), (uint32_t)(j / NA) & 1u, abort_flag, hdr, 12)) return false;
-            if (j >= NS) {
-                if (!warp_wait_bar(bar(B_STASH_FREE, ss), (uint32_t)((j / NS) - 1) & 1u, abort_flag, hdr, 13)) return false;
-                if (!warp_wait_bar(bar(B_PUB, ss), (uint32_t)((j / NS) - 1) & 1u, abort_flag, hdr, 14)) return false;
-            }
+            // the look-back warp of the slot's previous tile is done with it
+            if (j >= NS && !warp_wait_bar(bar(B_STASH_FREE, ss), (uint32_t)((j / NS) - 1) & 1u, abort_flag, hdr, 14))
+                return false;
             if (c == 0) RGLRU_TR(TR_P1_START, j, globaltimer());
             tc_fence_after();
             const uint32_t acc = tmem + lane_off + kColAcc + sa * kColsAcc;
             const uint32_t xhc = tmem + lane_off + kColXh + sx * kColsXh;
-            const uint32_t stc = tmem + lane_off + kColStash + ss * kColsStash;
+            const uint32_t stc = smem_u32(smem + OFF_ST + ss * kStash) + (uint32_t)c * 4;
             float hl = 0.f, P = 1.f;  // local scan state from h = 0, running prod a
-            cp_async_wait_all();      // this tile's GELU branch
+            // this tile's GELU branch (the group's (j / kScanGroups)-th load)
+            if (!warp_wait_bar(bar(B_GFULL, sg), (uint32_t)(j / kScanGroups) & 1u, abort_flag, hdr, 23)) return false;
+            if (c == 0) RGLRU_TR(TR_P1_G, j, globaltimer());
             const uint16_t *gs = reinterpret_cast<const uint16_t *>(gbuf) + c;
 #pragma unroll 1
             for (int t8 = 0; t8 < NT; t8 += 8) {
@@ -755,6 +773,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 tmem_ld8(acc + NT + t8, ai);
                 tmem_ld4(xhc + (t8 >> 1), xq);
                 tmem_wait_ld();
+                if (c == 0 && t8 == 0) RGLRU_TR(TR_P1_LD, j, globaltimer());
                 uint16_t gcur[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) gcur[k] = gs[(t8 + k) * kHalf];
@@ -817,10 +836,11 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         st[k] = pack_h2(G * hl, G * P);
                     }
                 }
-                tmem_st8(stc + t8, st);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) st_shared_u32(stc + (uint32_t)(t8 + k) * (kHalf * 4), st[k]);
             }
-            tmem_wait_st();
-            tc_fence_before();
+            tc_fence_before();  // the accumulator and xc loads above, before the slots are handed back
+            mbar_arrive(bar(B_GFREE, sg));
             mbar_arrive(bar(B_ACC_FREE, sa));
             mbar_arrive(bar(B_XH_FREE, sx));
             reinterpret_cast<float2 *>(smem + OFF_AGG + ss * kHalf * 8)[c] = make_float2(P, hl);
@@ -829,126 +849,40 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             return true;
         };
 
-        // y leaves through the group's shared-memory tile and one tensor store
-        __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_Y + sg * kGTile);
-        const bool ystorer = c == 0;  // issues the group's tensor stores
-        int ystores = 0;               // tensor stores issued by this group
-
-        auto pass2 = [&](int j) -> bool {
-            const int ss = j % NS, ir = j % INFO_RING;
-            const TileInfo ti = info[ir];
-            if (!warp_wait_bar(bar(B_LB, ss), (uint32_t)(j / NS) & 1u, abort_flag, hdr, 15)) return false;
-            if (c == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
-            if (ystores > 0) {
-                // the previous tensor store must have read the y tile
-                if (ystorer) {
-                    bulk_wait_read_all();
-                    mbar_arrive(bar(B_YFREE, sg));
-                }
-                if (!warp_wait_bar(bar(B_YFREE, sg), (uint32_t)(ystores - 1) & 1u, abort_flag, hdr, 21)) return false;
-            }
-            const float h_in = reinterpret_cast<const float *>(smem + OFF_HIN + ss * kHalf * 4)[c];
-            tc_fence_after();
-            const uint32_t stc = tmem + lane_off + kColStash + ss * kColsStash;
-#pragma unroll 1
-            for (int t16 = 0; t16 < NT; t16 += 16) {
-                uint32_t r[16];
-                tmem_ld16(stc + t16, r);
-                tmem_wait_ld();
-                if (c == 0 && t16 == 0) RGLRU_TR(TR_P2_LD, j, globaltimer());
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    // rows past the sequence end are clipped by the tensor store
-                    const float2 yq = __half22float2(*reinterpret_cast<const __half2 *>(&r[k]));
-                    ybuf[(t16 + k) * kHalf + c] = __float2bfloat16_rn(fmaf(yq.y, h_in, yq.x));
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(bar(B_YFULL, sg));
-            if (warp == 4 * sg) {
-                if (!warp_wait_bar(bar(B_YFULL, sg), (uint32_t)ystores & 1u, abort_flag, hdr, 22)) return false;
-                if (ystorer) {
-                    tma_store_3d(&tmap_y, ybuf, ch0, ti.t0, ti.b);
-                    bulk_commit();
-                }
-            }
-            ++ystores;
-            if (c == 0) RGLRU_TR(TR_P2_ST, j, globaltimer());
-            if (ti.first_last & 2) {
-                // The old states are read by the first tile of this sequence (its
-                // conv and its look-back, in this CTA's half of the channels):
-                // wait until that tile's prefix is published before overwriting.
-                const uint32_t *f_first = p.flags + (size_t)group * p.tiles_per_head + (size_t)ti.b * p.C;
-                if (warp_wait_flag(f_first, F_PREFIX, abort_flag, hdr, 16) == 0) return false;
-                p.h_state[(size_t)ti.b * p.D + d] = reinterpret_cast<const float *>(smem + OFF_AGG + ss * kHalf * 8)[c];
-                __nv_bfloat16 ncs[3];
-#pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    const int ts = p.T - 3 + k;
-                    ncs[k] = ts >= 0 ? p.x[((size_t)ti.b * p.T + ts) * p.D + d]
-                                     : p.conv_state[((size_t)ti.b * 3 + 3 + ts) * p.D + d];
-                }
-#pragma unroll
-                for (int k = 0; k < 3; ++k) p.conv_state[((size_t)ti.b * 3 + k) * p.D + d] = ncs[k];
-            }
-            tc_fence_before();
-            mbar_arrive(bar(B_STASH_FREE, ss));
-            // the descriptor may be reused once both CTAs' pass-2 warps are done with it
-            __syncwarp();
-            if (lane == 0) {
-                // relaxed: the reuse needs no ordering of this warp's y stores
-                if (half == 0)
-                    mbar_arrive(bar(B_INFO_EMPTY, ir));
-                else
-                    mbar_arrive_cluster_relaxed(peer_bar(B_INFO_EMPTY, ir));
-            }
-            if (c == 0) RGLRU_TR(TR_P2_END, j, globaltimer());
-            return true;
-        };
-
-        // this group's tiles: j = sg, sg + kScanGroups, ...; pass 2 of a tile runs
-        // kP2Lag of the group's tiles later (the look-back has that long)
+        // this group's tiles: j = sg, sg + kScanGroups, ...
         int j = sg;
         bool ok = warp_wait_bar(bar(B_INFO_FULL, j % INFO_RING), (uint32_t)(j / INFO_RING) & 1u, abort_flag, hdr, 17);
         TileInfo cur{};
         if (ok) {
             cur = info[j % INFO_RING];
-            if (cur.u >= 0) copy_g(cur);
+            if (cur.u >= 0) load_g(cur);
         }
 #pragma unroll 1
-        for (;; j += kScanGroups) {
-            const bool end = !ok || cur.u < 0;
-            if (!end) ok = pass1(j, cur);
-            TileInfo nxt{};
-            if (ok && !end) {
-                const int jn = j + kScanGroups;
-                ok = warp_wait_bar(bar(B_INFO_FULL, jn % INFO_RING), (uint32_t)(jn / INFO_RING) & 1u, abort_flag, hdr,
-                                   17);
-                if (ok) {
-                    nxt = info[jn % INFO_RING];
-                    if (nxt.u >= 0) copy_g(nxt);  // lands while pass 2 below runs
-                }
-            }
-            const int jp = j - kScanGroups * kP2Lag;
-            if (ok && jp >= 0) ok = pass2(jp);
-            if (end || !ok) {
-                // the group's tiles still waiting for pass 2
-                for (int q = jp + kScanGroups; ok && q < j; q += kScanGroups)
-                    if (q >= 0) ok = pass2(q);
-                break;
-            }
-            cur = nxt;
+        for (; ok && cur.u >= 0; j += kScanGroups) {
+            ok = pass1(j, cur);
+            if (!ok) break;
+            const int jn = j + kScanGroups;
+            ok = warp_wait_bar(bar(B_INFO_FULL, jn % INFO_RING), (uint32_t)(jn / INFO_RING) & 1u, abort_flag, hdr, 17);
+            if (!ok) break;
+            cur = info[jn % INFO_RING];
+            if (cur.u >= 0) load_g(cur);  // lands while the group waits for the tile's MMA
         }
-        if (ystorer && ystores > 0) bulk_wait_all();  // the group's y stores are complete
+        if (c == 0 && g_loads > 0) {
+            // a GELU-branch load still in flight (after an abort) lands before the CTA exits
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(bar(B_GFULL, sg), (uint32_t)(g_loads - 1) & 1u) && globaltimer() - t0 < kTimeoutNs) {
+            }
+        }
     } else if (warp >= kLbWarp0) {
         // ------------------------------------------------------------ look-back warps
         // Warp w serves the tiles j = w, w + kLbWarps, ...; their stash slots
         // recur every NS tiles, so each barrier is waited on one phase at a
         // time.  Per tile: publish the aggregate (later tiles of the sequence
         // may combine it before this tile's own look-back has finished), find
-        // the anchor, fold, hand h_in (and the prefix) to pass 2, publish the
-        // inclusive prefix.  These warps are the only ones that fence for the
-        // aggregates and prefixes.
+        // the anchor, fold, publish the inclusive prefix, then pass 2 of the
+        // tile: y = y_loc + q h_in from the stash, 4 channels per lane, and at
+        // a sequence end the new states.  These warps are the only ones that
+        // fence for the aggregates and prefixes.
         const int ch = lane * 4;  // 4 channels per lane
         const size_t dch = (size_t)ch0 + ch;
         const size_t gbase = (size_t)group * p.tiles_per_head;
@@ -963,7 +897,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             if (lane == 0) RGLRU_TR(TR_LB_START, j, globaltimer());
             const float4 *sagg = reinterpret_cast<const float4 *>(smem + OFF_AGG + ss * kHalf * 8);
             const float4 g01 = sagg[lane * 2], g23 = sagg[lane * 2 + 1];  // (A,H) of 4 channels
-            mbar_arrive(bar(B_PUB, ss));  // the aggregate slot is free again
             const float A[4] = {g01.x, g01.z, g23.x, g23.z};
             const float Hh[4] = {g01.y, g01.w, g23.y, g23.w};
             const size_t gu = gbase + ti.u;
@@ -986,6 +919,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 int anchor = -1;
                 uint32_t aflag = 0;
                 ok = find_anchor(p.flags + gbase, ti.u - 1, ti.b * p.C, anchor, aflag, abort_flag, hdr);
+                if (lane == 0) {
+                    RGLRU_TR(TR_LB_ANC, j, globaltimer());
+                    RGLRU_TR(TR_LB_K, j, (unsigned long long)(ti.u - anchor) | ((unsigned long long)aflag << 32));
+                }
                 if (ok) {
                     // carried-in state = the chain h <- A h + H folded forward in
                     // sequence order from the anchor, the same order whichever
@@ -1026,20 +963,60 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             float pre[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
-            // pass 2 needs only the carried-in state (and, at the sequence end,
-            // the state after the tile): hand them over before publishing
-            *reinterpret_cast<float4 *>(smem + OFF_HIN + ss * kHalf * 4 + ch * 4) =
-                make_float4(hin[0], hin[1], hin[2], hin[3]);
-            // (the aggregate slot was read above and stays untouched until this
-            // tile's pass 2 has run: pass 1 of the slot's next tile waits for both)
-            *reinterpret_cast<float4 *>(smem + OFF_AGG + ss * kHalf * 8 + ch * 4) =
-                make_float4(pre[0], pre[1], pre[2], pre[3]);
-            mbar_arrive(bar(B_LB, ss));
             if (!suppress) {
                 *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
                 __threadfence();
                 __syncwarp();
                 if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
+            }
+            if (lane == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
+            // pass 2: token t of this lane's 4 channels is one 16-byte stash word;
+            // y goes out as 8 bytes per lane (256 contiguous bytes per warp)
+            {
+                const uint32_t stw = smem_u32(smem + OFF_ST + ss * kStash) + (uint32_t)ch * 4;
+                __nv_bfloat16 *yrow = p.y + ((size_t)ti.b * p.T + ti.t0) * p.D + dch;
+#pragma unroll 4
+                for (int t = 0; t < ti.valid; ++t) {
+                    uint32_t w0, w1, w2, w3;
+                    ld_shared_v4(stw + (uint32_t)t * (kHalf * 4), w0, w1, w2, w3);
+                    const float2 q0 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
+                    const float2 q1 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
+                    const float2 q2 = __half22float2(*reinterpret_cast<const __half2 *>(&w2));
+                    const float2 q3 = __half22float2(*reinterpret_cast<const __half2 *>(&w3));
+                    uint2 yv;
+                    yv.x = pack_bf16_pair(fmaf(q0.y, hin[0], q0.x), fmaf(q1.y, hin[1], q1.x));
+                    yv.y = pack_bf16_pair(fmaf(q2.y, hin[2], q2.x), fmaf(q3.y, hin[3], q3.x));
+                    *reinterpret_cast<uint2 *>(yrow + (size_t)t * p.D) = yv;
+                }
+            }
+            if (ti.first_last & 2) {
+                // The old states are read by the first tile of this sequence (its
+                // conv and its look-back, in this CTA's half of the channels):
+                // wait until that tile's prefix is published before overwriting.
+                const uint32_t *f_first = p.flags + gbase + (size_t)ti.b * p.C;
+                if (warp_wait_flag(f_first, F_PREFIX, abort_flag, hdr, 16) == 0) break;
+                *reinterpret_cast<float4 *>(p.h_state + (size_t)ti.b * p.D + dch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
+                uint2 ncs[3];
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int ts = p.T - 3 + k;
+                    ncs[k] = ts >= 0 ? *reinterpret_cast<const uint2 *>(p.x + ((size_t)ti.b * p.T + ts) * p.D + dch)
+                                     : *reinterpret_cast<const uint2 *>(p.conv_state + ((size_t)ti.b * 3 + 3 + ts) * p.D + dch);
+                }
+#pragma unroll
+                for (int k = 0; k < 3; ++k) *reinterpret_cast<uint2 *>(p.conv_state + ((size_t)ti.b * 3 + k) * p.D + dch) = ncs[k];
+            }
+            // the stash slot (and its aggregate) may be reused, and the descriptor
+            // once both CTAs' look-back warps are done with it
+            mbar_arrive(bar(B_STASH_FREE, ss));
+            __syncwarp();
+            if (lane == 0) {
+                // relaxed: the reuse needs no ordering of this warp's y stores
+                if (half == 0)
+                    mbar_arrive(bar(B_INFO_EMPTY, ir));
+                else
+                    mbar_arrive_cluster_relaxed(peer_bar(B_INFO_EMPTY, ir));
+                RGLRU_TR(TR_P2_END, j, globaltimer());
             }
             if (lane == 0) RGLRU_TR(TR_LB_DONE, j, globaltimer());
         }
@@ -1125,24 +1102,6 @@ rglru_status fused_prefill(const PrefillArgs &a)
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return RGLRU_ERR_CUDA;
-    // y [B, T, D]: tensor stores of this half's 128 channels x 32 tokens
-    CUtensorMap tmap_y;
-    if (encode(&tmap_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.y, xdim, xstride, gbox, estride,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return RGLRU_ERR_CUDA;
-    // gate matrices [D rows, 256]: 128-row x 64-channel boxes in the 128-byte
-    // swizzle of the tensor core's K-major operand
-    CUtensorMap tmap_wa, tmap_wx;
-    const cuuint64_t wdim[2] = {256, (cuuint64_t)a.D}, wstride[1] = {256 * 2};
-    const cuuint32_t wbox[2] = {64, (cuuint32_t)kHalf};
-    if (encode(&tmap_wa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.W_a), wdim, wstride, wbox,
-               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
-        encode(&tmap_wx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.W_x), wdim, wstride, wbox,
-               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return RGLRU_ERR_CUDA;
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
@@ -1168,6 +1127,8 @@ rglru_status fused_prefill(const PrefillArgs &a)
     p.conv_w = a.conv_w; p.conv_b = a.conv_b;
     p.b_a = a.b_a; p.b_x = a.b_x;
     p.lambda = a.lambda; p.segpos = a.segpos;
+    p.w_a = static_cast<const __nv_bfloat16 *>(a.W_a);
+    p.w_x = static_cast<const __nv_bfloat16 *>(a.W_x);
     p.conv_state = static_cast<__nv_bfloat16 *>(a.conv_state);
     p.h_state = a.h_state;
     p.y = static_cast<__nv_bfloat16 *>(a.y);
@@ -1182,7 +1143,7 @@ rglru_status fused_prefill(const PrefillArgs &a)
     const int per_head = max(1, (sms / 2) / H);
     const long long grid = 2LL * per_head * H;
     if (grid > 0x7fffffffLL) return RGLRU_ERR_UNSUPPORTED;
-    rglru_prefill_fused_kernel<<<(unsigned)grid, kThreads, kSmemBytes, a.stream>>>(p, tmap_x, tmap_g, tmap_y, tmap_wa, tmap_wx);
+    rglru_prefill_fused_kernel<<<(unsigned)grid, kThreads, kSmemBytes, a.stream>>>(p, tmap_x, tmap_g);
     return cuda_status(cudaGetLastError());
 }
 

@@ -330,14 +330,6 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const
                  : "memory");
 }
 
-// 4-byte global -> shared copy, asynchronous to the issuing thread (cp.async)
-__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-// this thread's cp.async copies have landed
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
 // ---------------------------------------------------------------- programmatic dependent launch
 // this grid's dependents (launched with programmatic stream serialization) may
 // be scheduled now; they still wait for this grid's completion in griddep_wait
@@ -366,6 +358,15 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t ran
 __device__ __forceinline__ void st_cluster_u16(uint32_t cluster_addr, uint16_t v)
 {
     asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(cluster_addr), "h"(v) : "memory");
+}
+// 4-byte shared-memory store, 16-byte load, at a shared-window address.
+__device__ __forceinline__ void st_shared_u32(uint32_t saddr, uint32_t v)
+{
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t saddr, uint32_t &a, uint32_t &b, uint32_t &c, uint32_t &d)
+{
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(saddr) : "memory");
 }
 __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v)
 {
