@@ -22,9 +22,10 @@
 //   4. the epilogue applies the gates, a = sigmoid(Lambda)^(8 r), the
 //      normalised one-step update (a reset when segment_pos == 0) and the GELU
 //      product; y goes out through shared memory and a TMA store, h directly.
-// The launch allows programmatic dependent launch: barrier and TMEM set-up
-// may overlap the previous kernel's tail; every global access follows
-// griddepcontrol.wait.
+// The launch allows programmatic dependent launch: barrier and TMEM set-up,
+// and the loads of the parameters (gate weights and conv taps, which no
+// kernel of this library writes), may overlap the previous kernel's tail;
+// every other global access follows griddepcontrol.wait.
 // Each CTA reads and writes only its own channels of the states, so the two
 // CTAs never race.  Waits on mbarriers are bounded (RGLRU_ERR_TIMEOUT in the
 // workspace header); the two cluster barriers are reached exactly once by every
@@ -175,8 +176,18 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         mbar_init(bar_w, 1);
         mbar_init(bar_mma, 1);
         mbar_fence_init();
+        // this half's rows of W_a and W_x (parameters: read before the wait)
+        mbar_arrive_expect_tx(bar_w, 2 * kWGate);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+            tma_load_2d(smem + OFF_W + kb * kWBlock, &tm_wa, bar_w, kb * 64, ch0);
+            tma_load_2d(smem + OFF_W + kWGate + kb * kWBlock, &tm_wx, bar_w, kb * 64, ch0);
+        }
     }
     if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
+    const float w0 = 0.5f * p.conv_w[d], w1 = 0.5f * p.conv_w[(size_t)p.D + d],
+                w2 = 0.5f * p.conv_w[2 * (size_t)p.D + d], w3 = 0.5f * p.conv_w[3 * (size_t)p.D + d];
+    const float cb = 0.5f * p.conv_b[d];
     griddep_launch_dependents();
     griddep_wait();  // every global read below sees the previous kernel's writes
     if (tid == 0) DEC_TR(DT_WAITED);
@@ -186,12 +197,6 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         mbar_arrive_expect_tx(bar_in, kXTile + kCsTile);  // whole boxes: rows past B arrive zero-filled
         tma_load_2d(smem + OFF_X, &tm_x, bar_in, ch0, b0);
         tma_load_3d(smem + OFF_CS, &tm_cs, bar_in, ch0, 0, b0);
-        mbar_arrive_expect_tx(bar_w, 2 * kWGate);
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-            tma_load_2d(smem + OFF_W + kb * kWBlock, &tm_wa, bar_w, kb * 64, ch0);
-            tma_load_2d(smem + OFF_W + kWGate + kb * kWBlock, &tm_wx, bar_w, kb * 64, ch0);
-        }
     }
     if (tid < kTok) sp_s[tid] = tid < nb ? p.segpos[b0 + tid] : 3;
     // (kept as loaded, one register each, so that nothing waits for them
@@ -205,9 +210,6 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         graw[k] = n < nb ? __bfloat16_as_ushort(p.g[e]) : (uint16_t)0;
         hprev[k] = n < nb ? p.h_state[e] : 0.f;
     }
-    const float w0 = 0.5f * p.conv_w[d], w1 = 0.5f * p.conv_w[(size_t)p.D + d],
-                w2 = 0.5f * p.conv_w[2 * (size_t)p.D + d], w3 = 0.5f * p.conv_w[3 * (size_t)p.D + d];
-    const float cb = 0.5f * p.conv_b[d];
     // the peer CTA must be running before its shared memory is written
     tc_fence_before();
     cluster_sync();
