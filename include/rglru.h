@@ -140,6 +140,12 @@ RGLRU_API size_t rglru_decode_workspace_size(int B, int D, rglru_io_dtype dt);
  * Decode: one token for each of B sequences (the prefill recurrence with
  * T = 1).  x, gate_branch, y are [B, D]; segment_pos is [B]; conv_state and
  * h_state are updated in place.  Other arguments as rglru_prefill.
+ * The bf16 kernel is launched with programmatic dependent launch: it may
+ * start while the previous kernel on the stream finishes, and it reads
+ * W_a, W_x and conv_w / conv_b before waiting for that kernel.  So these
+ * parameters must not be written by a kernel that directly precedes the
+ * call on the stream and releases its dependents early; every other input
+ * is read only after the previous kernel has completed.
  */
 RGLRU_API rglru_status rglru_decode_step(int B, int D, rglru_io_dtype dt,
                                const void *x, const void *gate_branch,

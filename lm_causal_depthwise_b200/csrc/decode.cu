@@ -415,8 +415,8 @@ rglru_status decode_step(const PrefillArgs &a)
     const long long clusters = (long long)(a.D / kHead) * p.nblk;
     if (clusters * 2 > 0x7fffffffLL) return RGLRU_ERR_UNSUPPORTED;
     // programmatic stream serialization: the kernel may be scheduled while the
-    // previous one on the stream finishes; it waits (griddepcontrol.wait)
-    // before its first global memory access
+    // previous one on the stream finishes; it reads only the parameters (gate
+    // weights, conv taps) before griddepcontrol.wait
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(clusters * 2));
     cfg.blockDim = dim3(kThreads);
