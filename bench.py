@@ -70,11 +70,17 @@ def measured_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# sources the fused prefill kernel is compiled from: its own file and the
+# shared headers (the decode and SIMT kernels live in files of their own)
+PREFILL_SOURCES = ("prefill_fused.cu", ".h", ".cuh")
+
+
 def source_digest() -> str:
+    """Digest of the fused prefill kernel's sources, which a traffic record is tied to."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "lm_causal_depthwise_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".h", ".cuh")):
+        if name == PREFILL_SOURCES[0] or name.endswith(PREFILL_SOURCES[1:]):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())
