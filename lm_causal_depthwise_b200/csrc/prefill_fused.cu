@@ -85,8 +85,11 @@ constexpr uint32_t kColXh = kColAcc + NA * kColsAcc, kColsXh = NT / 2;
 static_assert(kColXh + NX * kColsXh <= 512, "TMEM budget");
 
 // Shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kBBlock = NT * 128;               // one K-block of the B tile: NT rows x 128 B
-constexpr int kBTile = 4 * kBBlock;             // bf16 xc of all 256 channels of the head
+// B tile (bf16 xc/2 of all 256 channels of the head), N-major: 8 channels x
+// NT tokens per group of core matrices
+constexpr int kBGroup = 8 * NT * 2;             // 512 bytes
+constexpr int kBTile = 32 * kBGroup;            // 16 KB
+constexpr int kBHalf = 16 * kBGroup;            // one CTA's 128 channels: 8 KB, contiguous
 constexpr int kXRows = NT + 3;
 constexpr int kXTile = kXRows * kHalf * 2;      // bf16 x of this half, 3 halo rows first
 constexpr int OFF_B = 0;
@@ -544,13 +547,13 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         const float w2 = 0.5f * p.conv_w[2 * (size_t)p.D + d], w3 = 0.5f * p.conv_w[3 * (size_t)p.D + d];
         const float cb = 0.5f * p.conv_b[d];
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        // B tile: row n = token, K index = channel within the head (K-major,
-        // 128-byte swizzle: 16-byte chunk (k & 63) >> 3 of row n sits at chunk ^ (n & 7))
+        // B tile, N-major without swizzle: the thread's channel k of the head
+        // holds 8 tokens per 16-byte row of a core matrix at
+        // (k / 8) * kBGroup + (k % 8) * 16 + (t / 8) * 128
         const int kidx = (int)half * kHalf + c;
-        const uint32_t b_local = smem_u32(smem + OFF_B + (kidx >> 6) * kBBlock);
-        const uint32_t chunk = (uint32_t)((kidx & 63) >> 3), sub = (uint32_t)(kidx & 7) * 2;
-        // this half's two K-blocks of a B tile: 8 KB, contiguous, sent to the peer in one copy
-        const int half_off = (int)half * 2 * kBBlock;
+        const uint32_t b_local = smem_u32(smem + OFF_B) + (uint32_t)(kidx >> 3) * kBGroup + (uint32_t)(kidx & 7) * 16;
+        // this half's 128 channels of a B tile: 8 KB, contiguous, sent to the peer in one copy
+        const int half_off = (int)half * kBHalf;
         const bool sender = warp == kConvWarp0 && lane == 0;
 #pragma unroll 1
         for (int j = 0;; ++j) {
@@ -596,8 +599,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 };
 #pragma unroll 1
                 for (int t8 = 0; t8 < NT; t8 += 8) {
-                    uint32_t xq[4];
-                    const uint32_t brow = bl + (uint32_t)t8 * 128;  // t8 is a multiple of 8: row t8 + k swizzles by k
+                    uint32_t xq[4], bq[4];
 #pragma unroll
                     for (int k = 0; k < 8; k += 2) {
                         const int t = t8 + k;
@@ -605,18 +607,15 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const float x1 = __bfloat162float(xs[(t + 4) * kHalf]);
                         const float v0 = conv1(t, xm3, xm2, xm1, x0);
                         const float v1 = conv1(t + 1, xm2, xm1, x0, x1);
-                        const uint32_t bw = pack_bf16_pair(v0, v1);
-                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(brow + k * 128 + ((chunk ^ (uint32_t)k) << 4) + sub),
-                                     "h"((uint16_t)bw)
-                                     : "memory");
-                        asm volatile("st.shared.b16 [%0], %1;" ::"r"(brow + (k + 1) * 128 + ((chunk ^ (uint32_t)(k + 1)) << 4) + sub),
-                                     "h"((uint16_t)(bw >> 16))
-                                     : "memory");
+                        bq[k >> 1] = pack_bf16_pair(v0, v1);
                         xq[k >> 1] = pack_f16_pair(v0, v1);
                         xm3 = xm1;
                         xm2 = x0;
                         xm1 = x1;
                     }
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(bl + (uint32_t)(t8 >> 3) * 128), "r"(bq[0]),
+                                 "r"(bq[1]), "r"(bq[2]), "r"(bq[3])
+                                 : "memory");
                     tmem_st4(xh_col + (uint32_t)(t8 >> 1), xq);
                 }
             };
@@ -632,7 +631,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             fence_proxy_async_smem();
             mbar_arrive(bar(B_X_EMPTY, xr));
             if (sender)
-                mbar_arrive_expect_tx(bar(B_BCONV, sb), 2 * kBBlock);  // the peer's half, arriving by copy
+                mbar_arrive_expect_tx(bar(B_BCONV, sb), kBHalf);  // the peer's half, arriving by copy
             else
                 mbar_arrive(bar(B_BCONV, sb));
             mbar_arrive(bar(B_BHALF, sb));
@@ -641,14 +640,14 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 if (!warp_wait_bar(bar(B_BHALF, sb), (uint32_t)(j / NB) & 1u, abort_flag, hdr, 20)) break;
                 if (sender) {
                     uint8_t *src = smem + OFF_B + sb * kBTile + half_off;
-                    bulk_copy_to_cluster(mapa_shared(smem_u32(src), peer), src, 2 * kBBlock, peer_bar(B_BCONV, sb));
+                    bulk_copy_to_cluster(mapa_shared(smem_u32(src), peer), src, kBHalf, peer_bar(B_BCONV, sb));
                 }
             }
             if (lane == 0 && warp == kConvWarp0) RGLRU_TR(TR_CONV_DONE, j, globaltimer());
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        const uint32_t idesc = umma_idesc_bf16(kHalf, NT);
+        const uint32_t idesc = umma_idesc_bf16_bn(kHalf, NT);
         bool w_ready = false;
         int issued = 0;
 #pragma unroll 1
@@ -671,7 +670,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk) {
                     // A (16 input channels of this half's weight rows) from TMEM
-                    const uint64_t bd = umma_desc_sw128(bt + (kk >> 2) * kBBlock + (kk & 3) * 32);
+                    // 16 input channels = two 8-channel groups of the N-major B tile
+                    const uint64_t bd = umma_desc_mn_noswizzle(bt + kk * 2 * kBGroup, kBGroup, 128);
                     umma_ts(d_r, tmem + kColW + kk * 8, bd, idesc, kk > 0);
                     umma_ts(d_i, tmem + kColW + kColsWGate + kk * 8, bd, idesc, kk > 0);
                 }

@@ -236,6 +236,16 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Same, with B N-major (its N index contiguous in memory).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_bn(int M, int N) { return umma_idesc_bf16(M, N) | (1u << 16); }
+// Shared-memory matrix descriptor of an MN-major operand without swizzle: core
+// matrices of 8 K rows x 16 bytes (8 MN elements); lbo = byte distance of the
+// next 8 K rows, sbo = byte distance of the next 8 MN elements.
+__device__ __forceinline__ uint64_t umma_desc_mn_noswizzle(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
 // D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate)
