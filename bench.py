@@ -35,6 +35,7 @@ from lm_causal_depthwise_b200 import workloads as W  # noqa: E402
 
 METRIC = "RG-LRU block prefill tokens/s & HBM GB/s vs peak; decode tok/s at B=256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+E2E_ROWS = 1  # sequences per chunk of the end-to-end (host-buffer) call
 
 
 def _env_rank():
@@ -314,19 +315,20 @@ def run_cuda(args, w):
     tokens = w.tokens * world
     value = job_throughput(w.tokens, world, per_step_ms)
 
-    # ---- end to end through the public API: pinned host inputs in, y back to host
+    # ---- end to end through the public API: rglru_prefill_host reads the
+    # pinned host inputs and writes y back to host memory, its copies
+    # overlapped with the kernels chunk by chunk (E2E_ROWS sequences each)
     hx = torch.from_numpy(inp["x"]).to(bf).pin_memory()
     hg = torch.from_numpy(inp["g"]).to(bf).pin_memory()
     hsp = torch.from_numpy(inp["segpos"]).pin_memory()
     hy = torch.empty(tuple(y.shape), dtype=bf).pin_memory()
     e_steps = max(3, min(args.steps, 20))
+    e_rows = min(w.B, E2E_ROWS)
+    staging = torch.empty(api.prefill_host_staging_size(w.B, w.T, w.D, bf, e_rows), dtype=torch.uint8, device=dev)
+    ws_host = api.new_workspace(api.workspace_size(e_rows, w.T, w.D, bf), dev)
 
     def e2e_step():
-        x.copy_(hx, non_blocking=True)
-        g.copy_(hg, non_blocking=True)
-        sp.copy_(hsp, non_blocking=True)
-        api.prefill(x, g, p, sp, cs, hs, workspace=ws, y=y)
-        hy.copy_(y, non_blocking=True)
+        api.prefill_host(hx, hg, p, hsp, cs, hs, hy, rows_per_chunk=e_rows, staging=staging, workspace=ws_host)
 
     for _ in range(2):
         e2e_step()
@@ -339,7 +341,7 @@ def run_cuda(args, w):
     ev1.record(stream)
     torch.cuda.synchronize()
     e_value = job_throughput(w.tokens, world, max_over_ranks(ev0.elapsed_time(ev1), dev) / e_steps)
-    st = api.device_status(ws)
+    st = api.device_status(ws_host)
     if st != api.OK:
         raise RuntimeError(f"prefill reported device status {api.status_string(st)} in the e2e loop")
     h2d = hx.numel() * hx.element_size() + hg.numel() * hg.element_size() + hsp.numel() * 4
@@ -377,7 +379,8 @@ def run_cuda(args, w):
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel": kernel_names},
         "e2e": {"value": e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e_steps,
+                "api": f"rglru_prefill_host, {e_rows} sequence(s) per chunk"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "source_digest": source_digest(),

@@ -21,6 +21,7 @@
  *
  * Conventions for every call below
  *   - All tensor pointers are DEVICE pointers (cudaMalloc'd, or managed),
+ *     except the *_host arguments of rglru_prefill_host,
  *     owned by the caller, 16-byte aligned.  The library allocates nothing,
  *     keeps no global state and never synchronises the stream (except
  *     rglru_get_device_status).  Work is enqueued on `stream`.
@@ -109,6 +110,51 @@ RGLRU_API rglru_status rglru_prefill(int B, int T, int D, rglru_io_dtype dt,
                            void *conv_state, float *h_state, void *y,
                            void *workspace, size_t workspace_bytes,
                            cudaStream_t stream);
+
+/*
+ * Staging bytes rglru_prefill_host needs (0 on bad arguments): two slots,
+ * each holding x, gate_branch and y for rows_per_chunk sequences
+ * ([rows, T, D] io dtype) and their segment_pos ([rows, T] int32), every
+ * piece 256-byte aligned.
+ */
+RGLRU_API size_t rglru_prefill_host_staging_size(int B, int T, int D, rglru_io_dtype dt,
+                                                 int rows_per_chunk);
+
+/*
+ * rglru_prefill with the activations in HOST memory: x_host,
+ * gate_branch_host ([B,T,D] io dtype) and segment_pos_host ([B,T] int32)
+ * are read from host memory and y_host ([B,T,D]) is written there.
+ * Page-locked host memory lets the copies run asynchronously; pageable
+ * memory gives the same result without the overlap.  The parameters,
+ * conv_state, h_state, the workspace and `staging` are device memory as for
+ * rglru_prefill.
+ *   rows_per_chunk  sequences per chunk (>= 1; values above B mean B).  The
+ *                   batch is processed chunk by chunk: the upload of chunk
+ *                   k + 1, the kernels of chunk k and the download of chunk
+ *                   k - 1 run at once.
+ *   staging         device memory of rglru_prefill_host_staging_size bytes,
+ *                   256-byte aligned, not in use by other work.
+ *   workspace       at least rglru_workspace_size(min(B, rows_per_chunk),
+ *                   T, D, dt) bytes.
+ * The result equals copying the inputs to the device, calling
+ * rglru_prefill and copying y back (bit for bit in bf16 mode: the fused
+ * kernel's results do not depend on how the batch is split).  Everything is
+ * enqueued asynchronously: y_host, conv_state and h_state are complete for
+ * work enqueued on `stream` after the call, and the host buffers must stay
+ * valid until then.  The call creates two CUDA streams and a few events for
+ * the copies and releases them before it returns (their work may still be
+ * pending).  It synchronises nothing.
+ */
+RGLRU_API rglru_status rglru_prefill_host(int B, int T, int D, rglru_io_dtype dt,
+                                const void *x_host, const void *gate_branch_host,
+                                const float *conv_w, const float *conv_b,
+                                const void *W_a, const float *b_a,
+                                const void *W_x, const float *b_x,
+                                const float *lambda, const int32_t *segment_pos_host,
+                                void *conv_state, float *h_state, void *y_host,
+                                int rows_per_chunk, void *staging, size_t staging_bytes,
+                                void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
 
 /*
  * Workspace bytes rglru_prefill_simt needs (0 on bad sizes): the device

@@ -24,7 +24,7 @@ IO_F32, IO_BF16 = 0, 1
 SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglru_prefill",
            "rglru_simt_workspace_size", "rglru_prefill_simt", "rglru_decode_workspace_size",
            "rglru_decode_step", "rglru_get_device_status", "rglru_debug_suppress_publish",
-           "rglru_prefill_noalloc")
+           "rglru_prefill_noalloc", "rglru_prefill_host_staging_size", "rglru_prefill_host")
 
 _lib = None
 
@@ -67,6 +67,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_debug_suppress_publish.argtypes = [vp, i, vp]
     lib.rglru_prefill_noalloc.restype = i
     lib.rglru_prefill_noalloc.argtypes = [i, i, i, i] + [vp] * 13 + [vp]
+    lib.rglru_prefill_host_staging_size.restype = sz
+    lib.rglru_prefill_host_staging_size.argtypes = [i, i, i, i, i]
+    lib.rglru_prefill_host.restype = i
+    lib.rglru_prefill_host.argtypes = [i, i, i, i] + [vp] * 13 + [i, vp, sz, vp, sz, vp]
     _lib = lib
     return lib
 
@@ -243,3 +247,55 @@ def debug_suppress_publish(workspace: torch.Tensor, unit: int) -> None:
     st = load().rglru_debug_suppress_publish(_ptr(workspace), int(unit), _stream(workspace.device))
     if st != OK:
         raise RGLRUError(st, "rglru_debug_suppress_publish")
+
+
+def prefill_host_staging_size(B: int, T: int, D: int, io_dtype: torch.dtype, rows_per_chunk: int) -> int:
+    dt = IO_BF16 if io_dtype == torch.bfloat16 else IO_F32
+    n = int(load().rglru_prefill_host_staging_size(B, T, D, dt, rows_per_chunk))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "prefill_host_staging_size")
+    return n
+
+
+def prefill_host(x_host, gate_branch_host, p: Params, segment_pos_host, conv_state, h_state, y_host=None,
+                 rows_per_chunk: int = 1, staging=None, workspace=None) -> torch.Tensor:
+    """rglru_prefill_host: x_host, gate_branch_host [B,T,D], segment_pos_host
+    [B,T] and y_host are CPU tensors (page-locked for overlapped copies);
+    the parameters, conv_state, h_state, staging and workspace are on the
+    device.  Enqueued on the current stream of the states' device: y_host is
+    complete once that stream has finished the call (synchronise before
+    reading it)."""
+    if x_host.dim() != 3:
+        raise ValueError("x_host must be [B,T,D]")
+    B, T, D = x_host.shape
+    dev = conv_state.device
+    for t, n, shape in ((x_host, "x_host", (B, T, D)), (gate_branch_host, "gate_branch_host", (B, T, D)),
+                        (segment_pos_host, "segment_pos_host", (B, T))):
+        _check(t, n, shape, torch.int32 if n == "segment_pos_host" else x_host.dtype, torch.device("cpu"))
+    if y_host is None:
+        y_host = torch.empty(tuple(x_host.shape), dtype=x_host.dtype, pin_memory=x_host.is_pinned())
+    _check(y_host, "y_host", (B, T, D), x_host.dtype, torch.device("cpu"))
+    dt = _dt(x_host)
+    H = D // 256
+    _check(p.conv_w, "conv_w", (4, D), torch.float32, dev)
+    for n in ("conv_b", "b_a", "b_x", "lam"):
+        _check(getattr(p, n), n, (D,), torch.float32, dev)
+    _check(p.W_a, "W_a", (H, 256, 256), x_host.dtype, dev)
+    _check(p.W_x, "W_x", (H, 256, 256), x_host.dtype, dev)
+    _check(conv_state, "conv_state", (B, 3, D), x_host.dtype, dev)
+    _check(h_state, "h_state", (B, D), torch.float32, dev)
+    need_st = prefill_host_staging_size(B, T, D, x_host.dtype, rows_per_chunk)
+    if staging is None:
+        staging = torch.empty(need_st, dtype=torch.uint8, device=dev)
+    need_ws = workspace_size(min(B, rows_per_chunk), T, D, x_host.dtype)
+    if workspace is None:
+        workspace = new_workspace(need_ws, dev)
+    st = load().rglru_prefill_host(B, T, D, dt, _ptr(x_host), _ptr(gate_branch_host), _ptr(p.conv_w), _ptr(p.conv_b),
+                                   _ptr(p.W_a), _ptr(p.b_a), _ptr(p.W_x), _ptr(p.b_x), _ptr(p.lam),
+                                   _ptr(segment_pos_host), _ptr(conv_state), _ptr(h_state), _ptr(y_host),
+                                   int(rows_per_chunk), _ptr(staging),
+                                   ctypes.c_size_t(staging.numel() * staging.element_size()), _ptr(workspace),
+                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_prefill_host")
+    return y_host

@@ -115,3 +115,41 @@ def test_status_calls_reject_null_workspace(lib):
     assert lib.rglru_get_device_status(None, None) == api.ERR_WORKSPACE
     assert lib.rglru_debug_suppress_publish(None, 0, None) == api.ERR_WORKSPACE
     assert lib.rglru_debug_suppress_publish(ctypes.c_void_p(1 << 20), -2, None) == api.ERR_INVALID_ARG
+
+
+def _al(n):
+    return (n + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,T,D,dt,rows", [(8, 4096, 2560, 1, 1), (5, 300, 512, 0, 2), (3, 7, 256, 1, 9)])
+def test_host_prefill_staging_size(lib, B, T, D, dt, rows):
+    r = min(B, rows)
+    e = 2 if dt == 1 else 4
+    want = 2 * (3 * _al(r * T * D * e) + _al(r * T * 4))
+    assert lib.rglru_prefill_host_staging_size(B, T, D, dt, rows) == want
+
+
+@pytest.mark.parametrize("args", [(0, 4, 256, 1, 1), (2, 4, 255, 1, 1), (2, 4, 256, 1, 0), (2, 4, 256, 7, 1)])
+def test_host_prefill_staging_size_rejects(lib, args):
+    assert lib.rglru_prefill_host_staging_size(*args) == 0
+
+
+def test_host_prefill_rejects_before_any_cuda_call(lib):
+    """Null host buffers, missing or small staging and a small workspace are
+    refused before a stream or event is created."""
+    host = ctypes.create_string_buffer(1 << 16)
+    fake_dev = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+    B, T, D, dt, rows = 2, 8, 256, 1, 1
+    st_need = lib.rglru_prefill_host_staging_size(B, T, D, dt, rows)
+    ws_need = lib.rglru_workspace_size(rows, T, D, dt)
+    hp = ctypes.cast(host, ctypes.c_void_p)
+
+    def call(xh, yh, staging, st_bytes, ws_bytes):
+        return lib.rglru_prefill_host(B, T, D, dt, xh, hp, fake_dev, fake_dev, fake_dev, fake_dev, fake_dev,
+                                      fake_dev, fake_dev, hp, fake_dev, fake_dev, yh, rows, staging, st_bytes,
+                                      fake_dev, ws_bytes, None)
+    assert call(None, hp, fake_dev, st_need, ws_need) == api.ERR_INVALID_ARG
+    assert call(hp, None, fake_dev, st_need, ws_need) == api.ERR_INVALID_ARG
+    assert call(hp, hp, None, st_need, ws_need) == api.ERR_WORKSPACE
+    assert call(hp, hp, fake_dev, st_need - 1, ws_need) == api.ERR_WORKSPACE
+    assert call(hp, hp, fake_dev, st_need, ws_need - 1) == api.ERR_WORKSPACE

@@ -248,3 +248,28 @@ def test_fused_prefill_is_bit_reproducible():
         b = run_gpu(to_device(inp, "bf16"))
         np.testing.assert_array_equal(a["y"], b["y"])
         np.testing.assert_array_equal(a["h_state"], b["h_state"])
+
+
+@pytest.mark.parametrize("io,rows", [("bf16", 1), ("bf16", 3), ("bf16", 9), ("f32", 2)])
+def test_prefill_from_host_buffers_equals_device_call(io, rows):
+    """rglru_prefill_host (host activations, chunks of `rows` sequences, copies
+    overlapped with the kernels) gives the device call's bits: sequences are
+    independent and the kernels' results do not depend on how the batch is
+    split.  Also checked against the oracle."""
+    _, inp = _case(5, 300, 512, io=io, doc_len=120)
+    ref_dev = to_device(inp, io)
+    want = run_gpu(ref_dev)
+    dev = to_device(inp, io)
+    hx = dev["x"].cpu().pin_memory()
+    hg = dev["g"].cpu().pin_memory()
+    hsp = dev["segpos"].cpu().pin_memory()
+    ws = api.new_workspace(api.workspace_size(min(5, rows), 300, 512, dev["x"].dtype))
+    hy = api.prefill_host(hx, hg, dev["params"], hsp, dev["conv_state"], dev["h_state"],
+                          rows_per_chunk=rows, workspace=ws)
+    torch.cuda.synchronize()
+    assert api.device_status(ws) == api.OK
+    np.testing.assert_array_equal(hy.float().numpy(), want["y"])
+    np.testing.assert_array_equal(dev["conv_state"].float().cpu().numpy(), want["conv_state"])
+    np.testing.assert_array_equal(dev["h_state"].cpu().numpy(), want["h_state"])
+    ref = run_oracle(inp)
+    check(io, hy.float().numpy(), ref["y"], "y")
