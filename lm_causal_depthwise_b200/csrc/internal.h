@@ -45,6 +45,11 @@ struct PrefillArgs {
     cudaStream_t stream;
 };
 
+// Synchronous argument checks of a prefill or decode call (rglru_api.cu): io
+// dtype, sizes, non-null 16-byte aligned pointers, no overlap between y, the
+// inputs, the states and the workspace, and a workspace of `need` bytes.
+rglru_status validate_prefill(const PrefillArgs &a, size_t need);
+
 // SIMT path (simt_path.cu)
 size_t simt_workspace_bytes(int B, int T, int D);
 rglru_status simt_prefill(const PrefillArgs &a);

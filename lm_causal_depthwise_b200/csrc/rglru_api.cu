@@ -33,7 +33,9 @@ bool sizes_ok(int B, int T, int D)
     return (int64_t)B * T * D <= kMaxElems;
 }
 
-rglru_status validate(const PrefillArgs &a, size_t need)
+}  // namespace
+
+rglru_status rglru::validate_prefill(const PrefillArgs &a, size_t need)
 {
     if (a.dt != RGLRU_IO_F32 && a.dt != RGLRU_IO_BF16) return RGLRU_ERR_INVALID_ARG;
     if (!sizes_ok(a.B, a.T, a.D)) return RGLRU_ERR_INVALID_ARG;
@@ -56,6 +58,8 @@ rglru_status validate(const PrefillArgs &a, size_t need)
         return RGLRU_ERR_INVALID_ARG;
     return RGLRU_OK;
 }
+
+namespace {
 
 PrefillArgs pack(int B, int T, int D, rglru_io_dtype dt, const void *x, const void *g,
                  const float *conv_w, const float *conv_b, const void *W_a, const float *b_a,
@@ -121,7 +125,7 @@ RGLRU_API rglru_status rglru_prefill_simt(int B, int T, int D, rglru_io_dtype dt
                                workspace_bytes, stream);
     const size_t need = rglru_simt_workspace_size(B, T, D, dt);
     if (need == 0) return RGLRU_ERR_INVALID_ARG;
-    const rglru_status v = validate(a, need);
+    const rglru_status v = validate_prefill(a, need);
     if (v != RGLRU_OK) return v;
     return simt_prefill(a);
 }
@@ -138,7 +142,7 @@ RGLRU_API rglru_status rglru_prefill(int B, int T, int D, rglru_io_dtype dt, con
                                workspace_bytes, stream);
     const size_t need = rglru_workspace_size(B, T, D, dt);
     if (need == 0) return RGLRU_ERR_INVALID_ARG;
-    const rglru_status v = validate(a, need);
+    const rglru_status v = validate_prefill(a, need);
     if (v != RGLRU_OK) return v;
     return dt == RGLRU_IO_BF16 ? fused_prefill(a) : simt_prefill(a);
 }
@@ -155,7 +159,7 @@ RGLRU_API rglru_status rglru_decode_step(int B, int D, rglru_io_dtype dt, const 
                                workspace_bytes, stream);
     const size_t need = rglru_decode_workspace_size(B, D, dt);
     if (need == 0) return RGLRU_ERR_INVALID_ARG;
-    const rglru_status v = validate(a, need);
+    const rglru_status v = validate_prefill(a, need);
     if (v != RGLRU_OK) return v;
     return dt == RGLRU_IO_BF16 ? decode_step(a) : simt_prefill(a);
 }

@@ -153,3 +153,42 @@ def test_host_prefill_rejects_before_any_cuda_call(lib):
     assert call(hp, hp, None, st_need, ws_need) == api.ERR_WORKSPACE
     assert call(hp, hp, fake_dev, st_need - 1, ws_need) == api.ERR_WORKSPACE
     assert call(hp, hp, fake_dev, st_need, ws_need - 1) == api.ERR_WORKSPACE
+
+
+def test_host_prefill_rejects_overlaps_before_any_cuda_call(lib):
+    """Overlapping host buffers, a missing state, and a chunk whose staging
+    overlaps the states or the workspace are all refused before a stream is
+    created (every chunk's arguments are checked up front)."""
+    B, T, D, dt, rows = 3, 8, 256, 1, 1
+    act = T * D * 2
+    host = ctypes.create_string_buffer(4 * B * act + (1 << 12))
+    base = ctypes.addressof(host)
+    hx, hg, hsp, hy = (ctypes.c_void_p(base + i * B * act) for i in range(4))
+    st_need = lib.rglru_prefill_host_staging_size(B, T, D, dt, rows)
+    ws_need = lib.rglru_workspace_size(rows, T, D, dt)
+    staging = 0x100000  # fake device addresses: never dereferenced, validation fails first
+    par = [ctypes.c_void_p(0x40000000 + i * 0x100000) for i in range(7)]
+    ws = ctypes.c_void_p(0x50000000)
+
+    def call(x, y, cs, hs, wsp):
+        return lib.rglru_prefill_host(B, T, D, dt, x, hg, *par, hsp, cs, hs, y, rows,
+                                      ctypes.c_void_p(staging), st_need, wsp, ws_need, None)
+    cs_ok, hs_ok = ctypes.c_void_p(0x60000000), ctypes.c_void_p(0x70000000)
+    # y_host overlapping x_host
+    assert call(hx, ctypes.c_void_p(base + act), cs_ok, hs_ok, ws) == api.ERR_INVALID_ARG
+    # missing conv_state / h_state
+    assert call(hx, hy, None, hs_ok, ws) == api.ERR_INVALID_ARG
+    assert call(hx, hy, cs_ok, None, ws) == api.ERR_INVALID_ARG
+    # conv_state inside the second staging slot (only chunk 1 uses that slot)
+    slot = st_need // 2
+    act_al = (rows * act + 255) // 256 * 256
+    assert call(hx, hy, ctypes.c_void_p(staging + slot), hs_ok, ws) == api.ERR_INVALID_ARG
+    # h_state overlapping the end of the staging buffer
+    assert call(hx, hy, cs_ok, ctypes.c_void_p(staging + st_need - 16), ws) == api.ERR_INVALID_ARG
+    # workspace inside the first slot's y tile
+    assert call(hx, hy, cs_ok, hs_ok, ctypes.c_void_p(staging + 2 * act_al + 16)) == api.ERR_INVALID_ARG
+    # a weight matrix inside the staging buffer
+    par_bad = list(par)
+    par_bad[4] = ctypes.c_void_p(staging + 64)  # W_x
+    assert lib.rglru_prefill_host(B, T, D, dt, hx, hg, *par_bad, hsp, cs_ok, hs_ok, hy, rows,
+                                  ctypes.c_void_p(staging), st_need, ws, ws_need, None) == api.ERR_INVALID_ARG
