@@ -18,10 +18,16 @@ Recipe (fixed draw order from ``numpy.random.default_rng(seed)``):
   b_a, b_x [D]     ~ N(0, 0.1)  (std 0.316)          fp32
   Lambda [D]       : u ~ U[0.9, 0.999], s = u^(1/8), Lambda = log(s/(1-s)),
                      so that sigmoid(Lambda)^8 = u                     fp32
+                     (decay="wide": the same draws mapped linearly onto
+                     Lambda in [-10, 10], so that sigmoid(Lambda)^8 spans
+                     about 1e-35 .. 1 and fast-decay channels occur)
   resets           : a reset at t=0 plus (T/L - 1) distinct positions drawn
                      uniformly from [1, T) per sequence (L = mean document
                      length); segment_pos counts up from each reset.
   initial state    : zero, or h ~ N(0, 0.1), conv ~ N(0, 1) (io dtype).
+  x_scale          : x (and the random conv state) multiplied by this factor
+                     before rounding (1 in every benchmark workload; parity
+                     cases use it for large-magnitude inputs).
 Values in bf16 mode are produced in fp32 and rounded to nearest-even bf16
 once; they are kept as fp32 arrays that hold exactly bf16-representable values.
 """
@@ -49,6 +55,8 @@ class Workload:
     continue_doc: bool = False     # no reset at all: segment_pos = t + 3
     init_state: str = "zero"       # "zero" or "random"
     decode_steps: int = 0          # >0: a batched decode workload of this many steps
+    decay: str = "init"            # "init": sigmoid(Lambda)^8 ~ U[0.9, 0.999]; "wide": Lambda in [-10, 10]
+    x_scale: float = 1.0           # x and the conv state drawn as x_scale * N(0, 1)
 
     @property
     def H(self) -> int:
@@ -130,11 +138,12 @@ def generate(w: Workload) -> dict:
         raise ValueError("D must be a multiple of 256")
     rng = np.random.default_rng(w.seed)
     B, T, D, H = w.B, w.T, w.D, w.H
+    xs = np.float32(w.x_scale)
     if w.io == "f32":
-        x = rng.standard_normal((B, T, D)).astype(np.float32)
+        x = (xs * rng.standard_normal((B, T, D))).astype(np.float32)
         g = rng.standard_normal((B, T, D)).astype(np.float32)
     else:
-        x = round_bf16(rng.standard_normal((B, T, D), dtype=np.float32))
+        x = round_bf16(xs * rng.standard_normal((B, T, D), dtype=np.float32))
         g = round_bf16(rng.standard_normal((B, T, D), dtype=np.float32))
     conv_w = (0.5 * rng.standard_normal((4, D))).astype(np.float32)
     conv_b = np.zeros((D,), dtype=np.float32)
@@ -143,12 +152,17 @@ def generate(w: Workload) -> dict:
     W_x = _io(rng.standard_normal((H, HEAD, HEAD)) / 16.0, w.io)
     b_x = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
     u = rng.uniform(0.9, 0.999, size=D)
-    s = u ** (1.0 / 8.0)
-    lam = np.log(s / (1.0 - s)).astype(np.float32)
+    if w.decay == "wide":
+        lam = (-10.0 + 20.0 * (u - 0.9) / 0.099).astype(np.float32)
+    elif w.decay == "init":
+        s = u ** (1.0 / 8.0)
+        lam = np.log(s / (1.0 - s)).astype(np.float32)
+    else:
+        raise ValueError(f"unknown decay recipe {w.decay!r}")
     segpos = segment_positions(rng, w)
     if w.init_state == "random":
         h_state = (np.sqrt(0.1) * rng.standard_normal((B, D))).astype(np.float32)
-        conv_state = _io(rng.standard_normal((B, 3, D)), w.io)
+        conv_state = _io(w.x_scale * rng.standard_normal((B, 3, D)), w.io)
     else:
         h_state = np.zeros((B, D), dtype=np.float32)
         conv_state = np.zeros((B, 3, D), dtype=np.float32)

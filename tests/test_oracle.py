@@ -20,9 +20,10 @@ HEAD = 256
 
 
 def _inputs(B=2, T=24, D=512, seed=7, io="f32", doc_len=None, reset_at=(0,),
-            continue_doc=False, init_state="random"):
+            continue_doc=False, init_state="random", decay="init"):
     w = W.Workload("pin", B=B, T=T, D=D, io=io, seed=seed, doc_len=doc_len,
-                   reset_at=reset_at, continue_doc=continue_doc, init_state=init_state)
+                   reset_at=reset_at, continue_doc=continue_doc, init_state=init_state,
+                   decay=decay)
     inp = W.generate(w)
     return {k: (v.astype(np.float64) if v.dtype != np.int32 else v) for k, v in inp.items()}
 
@@ -51,11 +52,16 @@ def _conv_np(inp, b, d, masked_state):
 
 # ---------------------------------------------------------------- closed forms
 
-def test_geometric_closed_form():
+@pytest.mark.parametrize("decay", ["init", "wide"])
+def test_geometric_closed_form(decay):
     """W=0 gives constant gates; identity conv and a per-document constant
-    input give h_{s+n} = i u (a^n + sqrt(1-a^2) (1-a^n)/(1-a)) after a reset at s."""
+    input give h_{s+n} = i u (a^n + sqrt(1-a^2) (1-a^n)/(1-a)) after a reset at s.
+    "wide" draws Lambda in [-10, 10], so both branches of log sigmoid(Lambda)
+    and fast-decay channels (sigmoid(Lambda)^8 down to ~1e-35) are covered."""
     T, D = 40, 256
-    inp = _inputs(B=1, T=T, D=D, reset_at=(0, 17), init_state="random")
+    inp = _inputs(B=1, T=T, D=D, reset_at=(0, 17), init_state="random", decay=decay)
+    if decay == "wide":
+        assert (inp["lam"] < -5).any() and (inp["lam"] > 5).any()
     inp["W_a"][:] = 0.0
     inp["W_x"][:] = 0.0
     inp["conv_w"][:] = 0.0
@@ -131,11 +137,41 @@ def test_gates_match_dense_block_diagonal_matmul():
                                scipy.special.expit(xc @ Wx.T + inp["b_x"]), rtol=1e-12)
 
 
-def test_decay_matches_power_form():
-    inp = _inputs(B=1, T=10, D=256)
+@pytest.mark.parametrize("decay", ["init", "wide"])
+def test_decay_matches_power_form(decay):
+    """a = sigmoid(Lambda)^(8 r) against scipy's logistic and numpy's power; the
+    wide recipe puts half of the channels at Lambda < 0."""
+    inp = _inputs(B=1, T=10, D=256, decay=decay)
     out = _run(inp, trace=True)
     want = np.power(scipy.special.expit(inp["lam"])[None, None, :], 8.0 * out["r"])
     np.testing.assert_allclose(out["a"], want, rtol=1e-13)
+
+
+def test_decay_at_fixed_negative_lambda():
+    """Lambda = -2 and -7 with constant gates (W = 0, b_a = 0 so r = 1/2):
+    a = sigmoid(Lambda)^4 exactly, h after a reset is the geometric sum of the
+    closed form, and the normaliser sqrt(1 - a^2) is evaluated at a ~ 1e-3
+    and ~ 1e-12."""
+    T, D = 12, 256
+    inp = _inputs(B=1, T=T, D=D, reset_at=(0,), init_state="zero")
+    inp["W_a"][:] = 0.0
+    inp["W_x"][:] = 0.0
+    inp["b_a"][:] = 0.0
+    inp["conv_w"][:] = 0.0
+    inp["conv_w"][3] = 1.0
+    inp["conv_b"][:] = 0.0
+    inp["lam"][:128] = -2.0
+    inp["lam"][128:] = -7.0
+    u = np.random.default_rng(5).standard_normal(D)
+    inp["x"][0, :] = u
+    out = _run(inp, trace=True)
+    a = np.where(np.arange(D) < 128, (1.0 / (1.0 + np.exp(2.0))) ** 4, (1.0 / (1.0 + np.exp(7.0))) ** 4)
+    np.testing.assert_allclose(out["a"][0], np.broadcast_to(a, (T, D)), rtol=1e-13)
+    i = 1.0 / (1.0 + np.exp(-inp["b_x"]))
+    n = np.arange(T)[:, None]
+    an = a[None, :] ** n
+    want = i * u * (an + np.sqrt(1 - a * a) * (1 - an) / (1 - a))
+    np.testing.assert_allclose(out["h"][0], want, rtol=1e-12, atol=1e-15)
 
 
 def test_gelu_is_torch_tanh_gelu():
