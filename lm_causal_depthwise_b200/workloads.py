@@ -19,8 +19,9 @@ Recipe (fixed draw order from ``numpy.random.default_rng(seed)``):
   Lambda [D]       : u ~ U[0.9, 0.999], s = u^(1/8), Lambda = log(s/(1-s)),
                      so that sigmoid(Lambda)^8 = u                     fp32
                      (decay="wide": the same draws mapped linearly onto
-                     Lambda in [-10, 10], so that sigmoid(Lambda)^8 spans
-                     about 1e-35 .. 1 and fast-decay channels occur)
+                     Lambda in [-10, 6.9], so that sigmoid(Lambda)^8 spans
+                     about 1e-35 .. 0.999: fast-decay channels, Lambda < 0,
+                     up to the slowest decay of the default recipe)
   resets           : a reset at t=0 plus (T/L - 1) distinct positions drawn
                      uniformly from [1, T) per sequence (L = mean document
                      length); segment_pos counts up from each reset.
@@ -55,7 +56,7 @@ class Workload:
     continue_doc: bool = False     # no reset at all: segment_pos = t + 3
     init_state: str = "zero"       # "zero" or "random"
     decode_steps: int = 0          # >0: a batched decode workload of this many steps
-    decay: str = "init"            # "init": sigmoid(Lambda)^8 ~ U[0.9, 0.999]; "wide": Lambda in [-10, 10]
+    decay: str = "init"            # "init": sigmoid(Lambda)^8 ~ U[0.9, 0.999]; "wide": Lambda in [-10, 6.9]
     x_scale: float = 1.0           # x and the conv state drawn as x_scale * N(0, 1)
 
     @property
@@ -153,7 +154,7 @@ def generate(w: Workload) -> dict:
     b_x = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
     u = rng.uniform(0.9, 0.999, size=D)
     if w.decay == "wide":
-        lam = (-10.0 + 20.0 * (u - 0.9) / 0.099).astype(np.float32)
+        lam = (-10.0 + 16.9 * (u - 0.9) / 0.099).astype(np.float32)
     elif w.decay == "init":
         s = u ** (1.0 / 8.0)
         lam = np.log(s / (1.0 - s)).astype(np.float32)
@@ -197,3 +198,27 @@ def gate_flops(w: Workload, tokens: Optional[int] = None) -> int:
     """Dense-contraction flops of the two block-diagonal gate projections."""
     n = w.tokens if tokens is None else tokens
     return 2 * 2 * n * w.D * HEAD
+
+
+def generate_block(w: Workload) -> dict:
+    """Inputs of the whole recurrent block for workload ``w``: everything
+    ``generate(w)`` draws (the core's parameters, segment positions and initial
+    states; its x and g are not block inputs), plus, from
+    ``default_rng((seed, 1))`` in this order:
+      u [B,T,D]                   ~ N(0, 1)          bf16 (the block input)
+      W_lin_x, W_lin_y, W_out [D,D] ~ N(0, 1/D)      bf16 (torch Linear init scale)
+      b_lin_x, b_lin_y, b_out [D]   ~ N(0, 0.1)      fp32
+    """
+    inp = generate(w)
+    rng = np.random.default_rng((w.seed, 1))
+    B, T, D = w.B, w.T, w.D
+    inp["u"] = round_bf16(rng.standard_normal((B, T, D), dtype=np.float32))
+    for name in ("lin_x", "lin_y", "out"):
+        inp[f"W_{name}"] = round_bf16((rng.standard_normal((D, D)) / np.sqrt(D)).astype(np.float32))
+        inp[f"b_{name}"] = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
+    return inp
+
+
+def block_gemm_flops(w: Workload) -> int:
+    """Dense flops of the block's three D x D projections over its tokens."""
+    return 3 * 2 * w.tokens * w.D * w.D
