@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -242,6 +243,129 @@ def count_launches(fns, prefix=("rglru",)):
     return [(len(g), sorted(set(g))) for g in groups[:len(fns)]]
 
 
+OTHER_PREFILL = ("prefill-long", "prefill-long-carry", "prefill-9b")
+SUSTAINED_S = 1.0  # the sustained run of the headline workload lasts at least this long
+
+
+def roofline(alg_bytes: int, ms_per_launch: float, peaks: dict, peak_kind: str, traffic, kernels):
+    achieved = alg_bytes / (ms_per_launch * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": f"{peak_kind} copy bandwidth",
+            "frac_of_nominal_8tbs": achieved / 8000.0,
+            "algorithmic_bytes_per_launch": alg_bytes, "kernel": kernels}
+
+
+class PrefillCase:
+    """Device buffers of one prefill workload and its timed step."""
+
+    def __init__(self, w, dev):
+        import torch
+        from lm_causal_depthwise_b200 import api
+        self.w, self.dev = w, dev
+        bf = torch.bfloat16 if w.io == "bf16" else torch.float32
+        self.bf = bf
+        self.inp = W.generate(w)
+        inp = self.inp
+        self.x = torch.from_numpy(inp["x"]).to(dev).to(bf)
+        self.g = torch.from_numpy(inp["g"]).to(dev).to(bf)
+        self.sp = torch.from_numpy(inp["segpos"]).to(dev)
+        self.cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
+        self.hs = torch.from_numpy(inp["h_state"]).to(dev)
+        self.p = api.Params.from_arrays(inp, bf, dev)
+        self.y = torch.empty_like(self.x)
+        self.ws = api.new_workspace(api.workspace_size(w.B, w.T, w.D, bf), dev)
+
+    def step(self):
+        from lm_causal_depthwise_b200 import api
+        api.prefill(self.x, self.g, self.p, self.sp, self.cs, self.hs, workspace=self.ws, y=self.y)
+
+    def status(self):
+        from lm_causal_depthwise_b200 import api
+        return api.device_status(self.ws)
+
+    def timed(self, steps: int, stream, distributed: bool, sampler_index=None):
+        """Time exactly ``steps`` launches on ``stream`` with CUDA events,
+        bracketed by a barrier and a device synchronize; max over ranks."""
+        import torch
+        import torch.distributed as dist
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if distributed:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(sampler_index if sampler_index is not None else 0) as clk:
+            ev0.record(stream)
+            for _ in range(steps):
+                self.step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        if distributed:
+            dist.barrier()
+        ms = max_over_ranks(ev0.elapsed_time(ev1), stream.device)
+        st = self.status()
+        if st != 0:
+            from lm_causal_depthwise_b200 import api
+            raise RuntimeError(f"{self.w.name}: device status {api.status_string(st)}: no valid timing")
+        return ms / steps, clk.summary()
+
+
+def cpu_sample_tokens(w: W.Workload, budget_s: float):
+    """The oracle on a bounded sample of ``w``: whole rows while they fit the
+    budget, else the first tokens of one row (all heads)."""
+    from oracle import oracle
+    probe = min(w.T, 1024)
+    inp = W.generate(w.scaled(B=1, T=probe))
+    t0 = time.perf_counter()
+    oracle.prefill(**inp)
+    per_tok = (time.perf_counter() - t0) / probe
+    tokens = int(max(probe, min(w.B * w.T, budget_s / max(per_tok, 1e-9))))
+    if tokens >= w.T:
+        rows, T = min(w.B, tokens // w.T), w.T
+    else:
+        rows, T = 1, tokens
+    inp = W.generate(w.scaled(B=rows, T=T))
+    t0 = time.perf_counter()
+    oracle.prefill(**inp)
+    dt = time.perf_counter() - t0
+    return rows * T / dt, oracle.threads(), \
+        f"{rows} of {w.B} sequences x first {T} of {w.T} tokens x D={w.D} (all heads), " \
+        f"float64 C oracle, {dt:.1f} s"
+
+
+def copy_only_rates(hx, hg, hsp, hy, stream):
+    """Host<->device copy rates of the same pinned buffers the end-to-end call
+    uses, measured alone: H2D of x, g and segment_pos, D2H of y, each as one
+    cudaMemcpyAsync per tensor on ``stream``."""
+    import torch
+    dx, dg, dsp = (torch.empty_like(t, device=stream.device) for t in (hx, hg, hsp))
+    dy = torch.empty_like(hy, device=stream.device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def h2d():
+        dx.copy_(hx, non_blocking=True)
+        dg.copy_(hg, non_blocking=True)
+        dsp.copy_(hsp, non_blocking=True)
+
+    def d2h():
+        hy.copy_(dy, non_blocking=True)
+
+    out = {}
+    for name, fn, nbytes in (("h2d", h2d, hx.nbytes + hg.nbytes + hsp.nbytes), ("d2h", d2h, hy.nbytes)):
+        fn()
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(3):
+            ev0.record(stream)
+            fn()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            ms = ev0.elapsed_time(ev1)
+            best = ms if best is None else min(best, ms)
+        out[name] = nbytes / (best * 1e-3) / 1e9
+    del dx, dg, dsp, dy
+    return out
+
+
 def run_cuda(args, w):
     import torch
     import torch.distributed as dist
@@ -259,31 +383,18 @@ def run_cuda(args, w):
 
     if args.profile_run and w.decode_steps:
         return profile_decode(args, w, dev, rank, distributed)
-    bf = torch.bfloat16 if w.io == "bf16" else torch.float32
-    inp = W.generate(w)
-    x = torch.from_numpy(inp["x"]).to(dev).to(bf)
-    g = torch.from_numpy(inp["g"]).to(dev).to(bf)
-    sp = torch.from_numpy(inp["segpos"]).to(dev)
-    cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
-    hs = torch.from_numpy(inp["h_state"]).to(dev)
-    p = api.Params.from_arrays(inp, bf, dev)
-    y = torch.empty_like(x)
-    ws = api.new_workspace(api.workspace_size(w.B, w.T, w.D, bf), dev)
-
-    def step():
-        api.prefill(x, g, p, sp, cs, hs, workspace=ws, y=y)
-
+    case = PrefillCase(w, dev)
     for _ in range(args.warmup):
-        step()
+        case.step()
     torch.cuda.synchronize()
     if args.profile_run:
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
         for _ in range(args.steps):
-            step()
+            case.step()
         ev1.record(stream)
         torch.cuda.synchronize()
-        st = api.device_status(ws)
+        st = case.status()
         if rank == 0:
             print(json.dumps({"profile_run": w.describe(), "steps": args.steps,
                               "ms_per_step": ev0.elapsed_time(ev1) / args.steps, "device_status": st}))
@@ -291,68 +402,79 @@ def run_cuda(args, w):
             dist.destroy_process_group()
         return 0 if st == 0 else 1
     dec_setup = None if args.no_decode else setup_decode(args, dev)
-    fns = [step] + ([dec_setup["one"]] if dec_setup else [])
+    fns = [case.step] + ([dec_setup["one"]] if dec_setup else [])
     counts = count_launches(fns)
     launches_per_step, kernel_names = counts[0]
 
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if distributed:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    if distributed:
-        dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    st = api.device_status(ws)
-    if st != api.OK:
-        raise RuntimeError(f"prefill reported device status {api.status_string(st)}: no valid timing")
-    per_step_ms = max_over_ranks(ms, dev) / args.steps
-    tokens = w.tokens * world
+    # ---- the contract's timed region: exactly K steps
+    per_step_ms, clocks = case.timed(args.steps, stream, distributed, local)
     value = job_throughput(w.tokens, world, per_step_ms)
+    # ---- the same workload sustained for >= SUSTAINED_S (a stable clock record)
+    n_sus = int(max(args.steps, math.ceil(SUSTAINED_S / (per_step_ms * 1e-3))))
+    if distributed:
+        n_sus = int(max_over_ranks(n_sus, dev))
+    sus_ms, sus_clocks = case.timed(n_sus, stream, distributed, local)
 
     # ---- end to end through the public API: rglru_prefill_host reads the
     # pinned host inputs and writes y back to host memory, its copies
     # overlapped with the kernels chunk by chunk (E2E_ROWS sequences each)
-    hx = torch.from_numpy(inp["x"]).to(bf).pin_memory()
-    hg = torch.from_numpy(inp["g"]).to(bf).pin_memory()
-    hsp = torch.from_numpy(inp["segpos"]).pin_memory()
-    hy = torch.empty(tuple(y.shape), dtype=bf).pin_memory()
+    bf = case.bf
+    hx = torch.from_numpy(case.inp["x"]).to(bf).pin_memory()
+    hg = torch.from_numpy(case.inp["g"]).to(bf).pin_memory()
+    hsp = torch.from_numpy(case.inp["segpos"]).pin_memory()
+    hy = torch.empty(tuple(case.y.shape), dtype=bf).pin_memory()
     e_steps = max(3, min(args.steps, 20))
     e_rows = min(w.B, E2E_ROWS)
-    staging = torch.empty(api.prefill_host_staging_size(w.B, w.T, w.D, bf, e_rows), dtype=torch.uint8, device=dev)
+    staging = torch.empty(api.prefill_host_staging_size(w.B, w.T, w.D, bf, e_rows), dtype=torch.uint8,
+                          device=dev)
     ws_host = api.new_workspace(api.workspace_size(e_rows, w.T, w.D, bf), dev)
 
     def e2e_step():
-        api.prefill_host(hx, hg, p, hsp, cs, hs, hy, rows_per_chunk=e_rows, staging=staging, workspace=ws_host)
+        api.prefill_host(hx, hg, case.p, hsp, case.cs, case.hs, hy, rows_per_chunk=e_rows, staging=staging,
+                         workspace=ws_host)
 
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
     if distributed:
         dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(e_steps):
         e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    e_value = job_throughput(w.tokens, world, max_over_ranks(ev0.elapsed_time(ev1), dev) / e_steps)
+    e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev) / e_steps
+    e_value = job_throughput(w.tokens, world, e_ms)
     st = api.device_status(ws_host)
     if st != api.OK:
         raise RuntimeError(f"prefill reported device status {api.status_string(st)} in the e2e loop")
-    h2d = hx.numel() * hx.element_size() + hg.numel() * hg.element_size() + hsp.numel() * 4
-    d2h = hy.numel() * hy.element_size()
+    h2d = hx.nbytes + hg.nbytes + hsp.nbytes
+    d2h = hy.nbytes
+    copy_rates = copy_only_rates(hx, hg, hsp, hy, stream)
+    del hx, hg, hy, hsp, staging, ws_host
+    del case
+    torch.cuda.empty_cache()
+
+    # ---- the other prefill workloads, each timed the same way (K steps)
+    others = []
+    if not args.headline_only:
+        for name in OTHER_PREFILL:
+            ow = W.ALL[name]
+            oc = PrefillCase(ow, dev)
+            for _ in range(args.warmup):
+                oc.step()
+            torch.cuda.synchronize()
+            o_ms, o_clk = oc.timed(max(3, min(args.steps, 20)), stream, distributed, local)
+            others.append((ow, o_ms, o_clk, max(3, min(args.steps, 20))))
+            del oc
+            torch.cuda.empty_cache()
 
     # ---- batched decode at B=256 (a separate timed loop of single-token steps)
     dec = None
     if dec_setup is not None:
         dec = run_decode(dec_setup, counts[1], stream, distributed)
 
-    del hx, hg, hy, hsp
     if distributed:
         dist.barrier()
         dist.destroy_process_group()
@@ -360,9 +482,6 @@ def run_cuda(args, w):
         return 0
 
     peaks, peak_kind = measured_peaks()
-    alg_bytes = W.algorithmic_bytes(w)
-    achieved = alg_bytes / (per_step_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
@@ -371,23 +490,44 @@ def run_cuda(args, w):
         "config": {"workload": w.describe(), "B": w.B, "T": w.T, "D": w.D,
                    "tokens_per_gpu": w.tokens, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "l2": "no flush: x, g, y are each larger than L2 (126 MB)"},
-        "hbm_gbs": achieved,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "peak_source": f"{peak_kind} copy bandwidth",
-                     "frac_of_nominal_8tbs": achieved / 8000.0,
-                     "algorithmic_bytes_per_launch": alg_bytes,
-                     "kernel": kernel_names},
+        "hbm_gbs": W.algorithmic_bytes(w) / (per_step_ms * 1e-3) / 1e9,
+        "roofline": roofline(W.algorithmic_bytes(w), per_step_ms, peaks, peak_kind, recorded_traffic(w.name),
+                             kernel_names),
         "e2e": {"value": e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e_steps,
-                "api": f"rglru_prefill_host, {e_rows} sequence(s) per chunk"},
+                "api": f"rglru_prefill_host, {e_rows} sequence(s) per chunk",
+                "ms_per_step": e_ms,
+                "h2d_gbs": h2d / (e_ms * 1e-3) / 1e9, "d2h_gbs": d2h / (e_ms * 1e-3) / 1e9,
+                "copy_only_h2d_gbs": copy_rates["h2d"], "copy_only_d2h_gbs": copy_rates["d2h"],
+                "h2d_frac_of_copy_only": h2d / (e_ms * 1e-3) / 1e9 / copy_rates["h2d"]},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
+        "sustained": {"steps": n_sus, "seconds": n_sus * sus_ms * 1e-3, "ms_per_step": sus_ms,
+                      "value": job_throughput(w.tokens, world, sus_ms), "unit": "tokens/s",
+                      "roofline_frac": W.algorithmic_bytes(w) / (sus_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "clocks": sus_clocks},
         "source_digest": source_digest(),
     }
+    cpu_on = world == 1 and not args.no_cpu_baseline
+    if others:
+        rows = []
+        for ow, o_ms, o_clk, o_steps in others:
+            r = {"workload": ow.describe(), "value": job_throughput(ow.tokens, world, o_ms), "unit": "tokens/s",
+                 "ms_per_step": o_ms, "steps": o_steps, "tokens_per_gpu": ow.tokens,
+                 "hbm_gbs": W.algorithmic_bytes(ow) / (o_ms * 1e-3) / 1e9,
+                 "roofline": roofline(W.algorithmic_bytes(ow), o_ms, peaks, peak_kind,
+                                      recorded_traffic(ow.name), kernel_names),
+                 "tensor_tflops": W.gate_flops(ow) / (o_ms * 1e-3) / 1e12,
+                 "clocks": o_clk}
+            if cpu_on:
+                v, cores, sample = cpu_sample_tokens(ow, 4.0)
+                r["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                     "sample": sample}
+            rows.append(r)
+        line["prefill_workloads"] = rows
     if dec is not None:
         line["decode"] = dec
-    if world == 1 and not args.no_cpu_baseline:
+    if cpu_on:
         v, cores, sample = cpu_sample_run(w)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
@@ -508,6 +648,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline prefill workload (not the other prefill workloads)")
     ap.add_argument("--profile-run", action="store_true",
                     help="only the warm-up and timed prefill steps (no profiler, e2e, decode or "
                          "CPU legs): the command an ncu capture wraps")

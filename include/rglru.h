@@ -232,6 +232,9 @@ RGLRU_API rglru_status rglru_debug_suppress_publish(void *workspace, int unit, c
  *     RGLRU_ERR_WORKSPACE before anything is enqueued.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is cached per device index for the life of the process, so
+ *     a process that calls cudaDeviceReset on a device must not use this
+ *     entry point on that device afterwards.
  *   - Every call shares the array and zeroes what must start at zero; calls
  *     that can overlap on the GPU (other streams, other host threads) race
  *     on it, so the caller must serialise them.
@@ -247,6 +250,76 @@ RGLRU_API rglru_status rglru_prefill_noalloc(int B, int T, int D, rglru_io_dtype
                                              const float *lambda, const int32_t *segment_pos,
                                              void *conv_state, float *h_state, void *y,
                                              cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Dense projections around the core and the whole recurrent block.
+ *
+ * "Gemma explained: RecurrentGemma architecture", the
+ * RecurrentGemmaRecurrentBlock printout (linear_y, linear_x, linear_out:
+ * Linear(2560, 2560, bias=True)) and section "Residual block with recurrent
+ * block": the block input u feeds linear_x (then the conv and the RG-LRU)
+ * and linear_y (the GELU branch); their product feeds linear_out.  The
+ * RecurrentGemmaMlp printout gives gate_proj / up_proj (2560 -> 7680) with a
+ * tanh GELU on the gate, and down_proj (7680 -> 2560).
+ *
+ * All of them: bf16 operands and outputs, fp32 bias, fp32 accumulation on
+ * the tensor cores.  Weights use torch's Linear layout W [out, in] (row
+ * = output feature, the input dimension contiguous).  Activations are
+ * row-major [M, features] (M = B * T tokens).  Sizes: K (input features) a
+ * multiple of 64, N (output features) a multiple of 256 (128 for
+ * rglru_linear_geglu), M >= 1.  Pointers are device pointers, 16-byte
+ * aligned; outputs must not overlap inputs (except out == residual).  The
+ * workspace holds the device status word (rglru_linear_workspace_size bytes,
+ * zero-filled once before first use); a bounded device wait that gave up is
+ * read back with rglru_get_device_status.  Unsupported sizes return
+ * RGLRU_ERR_UNSUPPORTED before anything is enqueued.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes of the rglru_linear* calls (the device status header). */
+RGLRU_API size_t rglru_linear_workspace_size(void);
+
+/* out[M, N] = A[M, K] W[N, K]^T + bias[N]   (bias may be NULL) */
+RGLRU_API rglru_status rglru_linear(int M, int N, int K, const void *A, const void *W, const float *bias,
+                                    void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Two projections of the same input in one launch (linear_x and linear_y of
+ * the block): out0 = A W0^T + bias0, out1 = A W1^T + bias1, each [M, N]. */
+RGLRU_API rglru_status rglru_linear_pair(int M, int N, int K, const void *A, const void *W0, const float *bias0,
+                                         void *out0, const void *W1, const float *bias1, void *out1,
+                                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* out = A W^T + bias + residual  (residual [M, N]; out may equal residual) */
+RGLRU_API rglru_status rglru_linear_residual(int M, int N, int K, const void *A, const void *W, const float *bias,
+                                             const void *residual, void *out, void *workspace,
+                                             size_t workspace_bytes, cudaStream_t stream);
+
+/* MLP up-projection: out[M, N] = GELU_tanh(A W_gate^T + b_gate) * (A W_up^T + b_up),
+ * W_gate, W_up [N, K]; biases required. */
+RGLRU_API rglru_status rglru_linear_geglu(int M, int N, int K, const void *A, const void *W_gate,
+                                          const float *b_gate, const void *W_up, const float *b_up, void *out,
+                                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes of rglru_recurrent_block_prefill (0 on bad sizes): the
+ * core's workspace plus the bf16 intermediates x, gate branch and core output. */
+RGLRU_API size_t rglru_recurrent_block_workspace_size(int B, int T, int D);
+
+/*
+ * The recurrent block over T tokens of B sequences, bf16:
+ *   x = u W_lin_x^T + b_lin_x,  g = u W_lin_y^T + b_lin_y      (one launch)
+ *   y = rglru_prefill core (x, g, ...)                        (fused kernel)
+ *   out = y W_out^T + b_out
+ * u, out [B, T, D] bf16; W_lin_x, W_lin_y, W_out [D, D] bf16; their biases
+ * [D] fp32; the core's parameters, segment_pos and states as rglru_prefill
+ * (bf16 mode).  x, g and y are held in the workspace as bf16 [B, T, D], the
+ * dtype of the core's inputs and output.  The workspace (zero-filled once)
+ * carries one status word for all three launches.
+ */
+RGLRU_API rglru_status rglru_recurrent_block_prefill(
+    int B, int T, int D, const void *u, const void *W_lin_x, const float *b_lin_x, const void *W_lin_y,
+    const float *b_lin_y, const float *conv_w, const float *conv_b, const void *W_a, const float *b_a,
+    const void *W_x, const float *b_x, const float *lambda, const int32_t *segment_pos, void *conv_state,
+    float *h_state, const void *W_out, const float *b_out, void *out, void *workspace, size_t workspace_bytes,
+    cudaStream_t stream);
 
 #ifdef __cplusplus
 }

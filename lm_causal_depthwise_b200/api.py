@@ -24,7 +24,9 @@ IO_F32, IO_BF16 = 0, 1
 SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglru_prefill",
            "rglru_simt_workspace_size", "rglru_prefill_simt", "rglru_decode_workspace_size",
            "rglru_decode_step", "rglru_get_device_status", "rglru_debug_suppress_publish",
-           "rglru_prefill_noalloc", "rglru_prefill_host_staging_size", "rglru_prefill_host")
+           "rglru_prefill_noalloc", "rglru_prefill_host_staging_size", "rglru_prefill_host",
+           "rglru_linear_workspace_size", "rglru_linear", "rglru_linear_pair", "rglru_linear_residual",
+           "rglru_linear_geglu", "rglru_recurrent_block_workspace_size", "rglru_recurrent_block_prefill")
 
 _lib = None
 
@@ -71,6 +73,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_prefill_host_staging_size.argtypes = [i, i, i, i, i]
     lib.rglru_prefill_host.restype = i
     lib.rglru_prefill_host.argtypes = [i, i, i, i] + [vp] * 13 + [i, vp, sz, vp, sz, vp]
+    lib.rglru_linear_workspace_size.restype = sz
+    lib.rglru_linear_workspace_size.argtypes = []
+    lib.rglru_linear.restype = i
+    lib.rglru_linear.argtypes = [i, i, i] + [vp] * 5 + [sz, vp]
+    lib.rglru_linear_pair.restype = i
+    lib.rglru_linear_pair.argtypes = [i, i, i] + [vp] * 8 + [sz, vp]
+    lib.rglru_linear_residual.restype = i
+    lib.rglru_linear_residual.argtypes = [i, i, i] + [vp] * 6 + [sz, vp]
+    lib.rglru_linear_geglu.restype = i
+    lib.rglru_linear_geglu.argtypes = [i, i, i] + [vp] * 7 + [sz, vp]
+    lib.rglru_recurrent_block_workspace_size.restype = sz
+    lib.rglru_recurrent_block_workspace_size.argtypes = [i, i, i]
+    lib.rglru_recurrent_block_prefill.restype = i
+    lib.rglru_recurrent_block_prefill.argtypes = [i, i, i] + [vp] * 19 + [sz, vp]
     _lib = lib
     return lib
 
@@ -299,3 +315,166 @@ def prefill_host(x_host, gate_branch_host, p: Params, segment_pos_host, conv_sta
     if st != OK:
         raise RGLRUError(st, "rglru_prefill_host")
     return y_host
+
+
+# ----------------------------------------------------------------------------- projections and the block
+
+def linear_workspace(device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for the rglru_linear* calls (the device status header)."""
+    return new_workspace(int(load().rglru_linear_workspace_size()), device)
+
+
+def _lin_common(A, W, name):
+    if A.dim() != 2 or W.dim() != 2:
+        raise ValueError(f"{name}: A must be [M, K] and W [N, K]")
+    M, K = A.shape
+    N = W.shape[0]
+    _check(A, "A", (M, K), torch.bfloat16, A.device)
+    _check(W, "W", (N, K), torch.bfloat16, A.device)
+    return M, N, K
+
+
+def _bias(b, N, dev, name):
+    if b is None:
+        return ctypes.c_void_p(None)
+    _check(b, name, (N,), torch.float32, dev)
+    return _ptr(b)
+
+
+def _ws(workspace, dev):
+    if workspace is None:
+        workspace = linear_workspace(dev)
+    return workspace, ctypes.c_size_t(workspace.numel() * workspace.element_size())
+
+
+def linear(A, W, bias=None, out=None, workspace=None) -> torch.Tensor:
+    """out[M, N] = A[M, K] W[N, K]^T + bias (rglru_linear, bf16 on the tensor cores)."""
+    M, N, K = _lin_common(A, W, "linear")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check(out, "out", (M, N), torch.bfloat16, A.device)
+    workspace, nb = _ws(workspace, A.device)
+    st = load().rglru_linear(M, N, K, _ptr(A), _ptr(W), _bias(bias, N, A.device, "bias"), _ptr(out),
+                             _ptr(workspace), nb, _stream(A.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_linear")
+    return out
+
+
+def linear_pair(A, W0, b0, W1, b1, out0=None, out1=None, workspace=None):
+    """(A W0^T + b0, A W1^T + b1) in one launch (rglru_linear_pair)."""
+    M, N, K = _lin_common(A, W0, "linear_pair")
+    _check(W1, "W1", (N, K), torch.bfloat16, A.device)
+    outs = []
+    for o in (out0, out1):
+        if o is None:
+            o = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+        _check(o, "out", (M, N), torch.bfloat16, A.device)
+        outs.append(o)
+    workspace, nb = _ws(workspace, A.device)
+    st = load().rglru_linear_pair(M, N, K, _ptr(A), _ptr(W0), _bias(b0, N, A.device, "bias0"), _ptr(outs[0]),
+                                  _ptr(W1), _bias(b1, N, A.device, "bias1"), _ptr(outs[1]), _ptr(workspace), nb,
+                                  _stream(A.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_linear_pair")
+    return outs[0], outs[1]
+
+
+def linear_residual(A, W, bias, residual, out=None, workspace=None) -> torch.Tensor:
+    """out = A W^T + bias + residual (rglru_linear_residual); out may be residual."""
+    M, N, K = _lin_common(A, W, "linear_residual")
+    _check(residual, "residual", (M, N), torch.bfloat16, A.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check(out, "out", (M, N), torch.bfloat16, A.device)
+    workspace, nb = _ws(workspace, A.device)
+    st = load().rglru_linear_residual(M, N, K, _ptr(A), _ptr(W), _bias(bias, N, A.device, "bias"), _ptr(residual),
+                                      _ptr(out), _ptr(workspace), nb, _stream(A.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_linear_residual")
+    return out
+
+
+def linear_geglu(A, W_gate, b_gate, W_up, b_up, out=None, workspace=None) -> torch.Tensor:
+    """out = GELU_tanh(A W_gate^T + b_gate) * (A W_up^T + b_up) (rglru_linear_geglu)."""
+    M, N, K = _lin_common(A, W_gate, "linear_geglu")
+    _check(W_up, "W_up", (N, K), torch.bfloat16, A.device)
+    _check(b_gate, "b_gate", (N,), torch.float32, A.device)
+    _check(b_up, "b_up", (N,), torch.float32, A.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check(out, "out", (M, N), torch.bfloat16, A.device)
+    workspace, nb = _ws(workspace, A.device)
+    st = load().rglru_linear_geglu(M, N, K, _ptr(A), _ptr(W_gate), _ptr(b_gate), _ptr(W_up), _ptr(b_up), _ptr(out),
+                                   _ptr(workspace), nb, _stream(A.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_linear_geglu")
+    return out
+
+
+@dataclass
+class BlockParams:
+    """Projections around the core (bf16 [D, D] weights, fp32 [D] biases) and
+    the core's own parameters."""
+    W_lin_x: torch.Tensor
+    b_lin_x: torch.Tensor
+    W_lin_y: torch.Tensor
+    b_lin_y: torch.Tensor
+    W_out: torch.Tensor
+    b_out: torch.Tensor
+    core: Params
+
+    @staticmethod
+    def from_arrays(inp: dict, device="cuda") -> "BlockParams":
+        def w(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).to(torch.bfloat16).contiguous()
+
+        def f32(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).contiguous()
+        return BlockParams(w(inp["W_lin_x"]), f32(inp["b_lin_x"]), w(inp["W_lin_y"]), f32(inp["b_lin_y"]),
+                           w(inp["W_out"]), f32(inp["b_out"]), Params.from_arrays(inp, torch.bfloat16, device))
+
+
+def recurrent_block_workspace_size(B: int, T: int, D: int) -> int:
+    n = int(load().rglru_recurrent_block_workspace_size(B, T, D))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "recurrent_block_workspace_size")
+    return n
+
+
+def recurrent_block_prefill(u, bp: BlockParams, segment_pos, conv_state, h_state, out=None,
+                            workspace=None) -> torch.Tensor:
+    """out = linear_out(GELU(linear_y(u)) * RG-LRU(conv(linear_x(u)))) over u [B,T,D] bf16
+    (rglru_recurrent_block_prefill); conv_state and h_state are updated in place."""
+    if u.dim() != 3:
+        raise ValueError("u must be [B,T,D]")
+    B, T, D = u.shape
+    dev = u.device
+    _check(u, "u", (B, T, D), torch.bfloat16, dev)
+    for n in ("W_lin_x", "W_lin_y", "W_out"):
+        _check(getattr(bp, n), n, (D, D), torch.bfloat16, dev)
+    for n in ("b_lin_x", "b_lin_y", "b_out"):
+        _check(getattr(bp, n), n, (D,), torch.float32, dev)
+    p = bp.core
+    _check(p.conv_w, "conv_w", (4, D), torch.float32, dev)
+    for n in ("conv_b", "b_a", "b_x", "lam"):
+        _check(getattr(p, n), n, (D,), torch.float32, dev)
+    _check(p.W_a, "W_a", (D // 256, 256, 256), torch.bfloat16, dev)
+    _check(p.W_x, "W_x", (D // 256, 256, 256), torch.bfloat16, dev)
+    _check(segment_pos, "segment_pos", (B, T), torch.int32, dev)
+    _check(conv_state, "conv_state", (B, 3, D), torch.bfloat16, dev)
+    _check(h_state, "h_state", (B, D), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(u)
+    _check(out, "out", (B, T, D), torch.bfloat16, dev)
+    need = recurrent_block_workspace_size(B, T, D)
+    if workspace is None:
+        workspace = new_workspace(need, dev)
+    st = load().rglru_recurrent_block_prefill(
+        B, T, D, _ptr(u), _ptr(bp.W_lin_x), _ptr(bp.b_lin_x), _ptr(bp.W_lin_y), _ptr(bp.b_lin_y), _ptr(p.conv_w),
+        _ptr(p.conv_b), _ptr(p.W_a), _ptr(p.b_a), _ptr(p.W_x), _ptr(p.b_x), _ptr(p.lam), _ptr(segment_pos),
+        _ptr(conv_state), _ptr(h_state), _ptr(bp.W_out), _ptr(bp.b_out), _ptr(out), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_recurrent_block_prefill")
+    return out

@@ -339,29 +339,6 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-bool encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *m, const void *base, int rank,
-                 const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle sw)
-{
-    const cuuint32_t estride[3] = {1, 1, 1};
-    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 #ifdef RGLRU_TRACE
@@ -392,12 +369,9 @@ rglru_status decode_step(const PrefillArgs &a)
         !encode_bf16(encode, &tm_y, a.y, 2, rdim, rstride, rbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !encode_bf16(encode, &tm_cs, a.conv_state, 3, cdim, cstride, cbox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return RGLRU_ERR_CUDA;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(rglru_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    });
-    if (attr_err != cudaSuccess) return RGLRU_ERR_CUDA;
+    static PerDeviceFlag smem_set;
+    const rglru_status st = set_smem_limit_once((const void *)rglru_decode_kernel, kSmemBytes, smem_set);
+    if (st != RGLRU_OK) return st;
 
     DecodeParams p;
     p.B = a.B;

@@ -6,8 +6,8 @@
 // sequence, claimed in order from the head's ticket counter by rank 0, which
 // writes each tile descriptor into both CTAs).  Per tile:
 //   conv warps   thread = channel: causal depthwise conv (k=4, document mask)
-//                of its channel over the tile in fp32; xc / 2 goes to TMEM (f16
-//                pairs) for the scan, its bf16 copy into the MMA B tile of BOTH
+//                of its channel over the tile in fp32; xc / 2 goes to TMEM (fp32)
+//                for the scan, its bf16 copy into the MMA B tile of BOTH
 //                CTAs (the two halves of the head's 256 input channels meet in
 //                each CTA's shared memory through the cluster).
 //   MMA thread   both block-diagonal gate projections on the tensor cores:
@@ -56,7 +56,7 @@ using namespace sm100;
 
 constexpr int NT = 32;          // tokens per tile (MMA N)
 constexpr int kHalf = 128;      // channels per CTA (MMA M, TMEM lanes)
-constexpr int NX = 4;           // xc/2 slots in TMEM (conv -> pass 1)
+constexpr int NX = 4;           // xc/2 slots in TMEM (conv -> pass 1), fp32
 constexpr int NA = 2;           // accumulator slots in TMEM (MMA -> pass 1), one per scan group
 constexpr int NS = 6;           // stash slots in shared memory (pass 1 -> look-back and pass 2)
 constexpr int NB = 2;           // B tiles in shared memory (conv -> MMA, both CTAs)
@@ -78,10 +78,10 @@ static_assert(kEndMarkers <= INFO_RING, "end markers fit the ring");
 
 // TMEM columns (512): this half's rows of W_a then W_x (the MMA's A operand,
 // bf16 pairs: K-step kk of a gate at column 8 kk), accumulators
-// [pre_r | pre_i], xc/2 f16 pairs
+// [pre_r | pre_i], xc/2 in fp32 (one column per token)
 constexpr uint32_t kColW = 0, kColsWGate = 128;
 constexpr uint32_t kColAcc = kColW + 2 * kColsWGate, kColsAcc = 2 * NT;
-constexpr uint32_t kColXh = kColAcc + NA * kColsAcc, kColsXh = NT / 2;
+constexpr uint32_t kColXh = kColAcc + NA * kColsAcc, kColsXh = NT;
 static_assert(kColXh + NX * kColsXh <= 512, "TMEM budget");
 
 // Shared memory map (offsets from a 1024-byte aligned base)
@@ -361,12 +361,6 @@ __device__ __forceinline__ uint32_t pack_bf16_pair(float lo, float hi)
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-__device__ __forceinline__ uint32_t pack_f16_pair(float lo, float hi)
-{
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
 
 __device__ __forceinline__ float gelu_tanh_fast(float g)
 {
@@ -449,22 +443,28 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 
     if (warp == kSchedWarp) {
         // ------------------------------------------------------------ scheduler
-        // Rank 0 claims the head's tiles in order, one ahead of the ring, and
-        // writes each descriptor into both CTAs; each CTA then loads its own
+        // Rank 0 claims the head's tiles, one ahead of the ring, and writes
+        // each descriptor into both CTAs; each CTA then loads its own
         // channels of x: rows t0 - 3 .. t0 + 31 (rows before t = 0 arrive
-        // zero-filled; the conv reads conv_state there).
+        // zero-filled; the conv reads conv_state there).  Ticket k is tile
+        // k / B of sequence k % B: consecutive tickets go to different
+        // sequences, so a tile's predecessor in its sequence was claimed B
+        // tickets earlier and has usually published its aggregate (and its
+        // prefix) by the time the tile's own look-back starts.  The look-back
+        // indexes tiles by u = b C + c, their order inside the sequence.
         auto claim = [&]() -> TileInfo {
-            int u = -1;
+            int k = -1;
             if (lane == 0 && !*abort_flag) {
-                u = (int)atomicAdd(&hdr->ticket[head], 1u);
-                if (u >= p.tiles_per_head) u = -1;
+                k = (int)atomicAdd(&hdr->ticket[head], 1u);
+                if (k >= p.tiles_per_head) k = -1;
             }
-            u = __shfl_sync(0xffffffffu, u, 0);
+            k = __shfl_sync(0xffffffffu, k, 0);
             TileInfo ti{};
-            ti.u = u;
-            if (u >= 0) {
-                ti.b = u / p.C;
-                const int c = u % p.C;
+            ti.u = -1;
+            if (k >= 0) {
+                ti.b = k % p.B;
+                const int c = k / p.B;
+                ti.u = ti.b * p.C + c;
                 ti.t0 = c * NT;
                 ti.valid = min(NT, p.T - ti.t0);
                 ti.first_last = (c == 0 ? 1 : 0) | (c == p.C - 1 ? 2 : 0);
@@ -599,7 +599,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 };
 #pragma unroll 1
                 for (int t8 = 0; t8 < NT; t8 += 8) {
-                    uint32_t xq[4], bq[4];
+                    uint32_t xq[8], bq[4];
 #pragma unroll
                     for (int k = 0; k < 8; k += 2) {
                         const int t = t8 + k;
@@ -608,7 +608,8 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const float v0 = conv1(t, xm3, xm2, xm1, x0);
                         const float v1 = conv1(t + 1, xm2, xm1, x0, x1);
                         bq[k >> 1] = pack_bf16_pair(v0, v1);
-                        xq[k >> 1] = pack_f16_pair(v0, v1);
+                        xq[k] = __float_as_uint(v0);
+                        xq[k + 1] = __float_as_uint(v1);
                         xm3 = xm1;
                         xm2 = x0;
                         xm1 = x1;
@@ -616,7 +617,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(bl + (uint32_t)(t8 >> 3) * 128), "r"(bq[0]),
                                  "r"(bq[1]), "r"(bq[2]), "r"(bq[3])
                                  : "memory");
-                    tmem_st4(xh_col + (uint32_t)(t8 >> 1), xq);
+                    tmem_st8(xh_col + (uint32_t)t8, xq);
                 }
             };
             if (clean)
@@ -768,10 +769,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const uint16_t *gs = reinterpret_cast<const uint16_t *>(gbuf) + c;
 #pragma unroll 1
             for (int t8 = 0; t8 < NT; t8 += 8) {
-                uint32_t ar[8], ai[8], xq[4];
+                uint32_t ar[8], ai[8], xq[8];
                 tmem_ld8(acc + t8, ar);
                 tmem_ld8(acc + NT + t8, ai);
-                tmem_ld4(xhc + (t8 >> 1), xq);
+                tmem_ld8(xhc + t8, xq);
                 tmem_wait_ld();
                 if (c == 0 && t8 == 0) RGLRU_TR(TR_P1_LD, j, globaltimer());
                 uint16_t gcur[8];
@@ -782,7 +783,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 if (clean) {
 #pragma unroll
                     for (int k = 0; k < 8; k += 2) {
-                        const float2 xh = __half22float2(*reinterpret_cast<const __half2 *>(&xq[k >> 1]));
                         const f2_t zr = f2_add(f2_make(__uint_as_float(ar[k]), __uint_as_float(ar[k + 1])), hba2);
                         const f2_t zi = f2_add(f2_make(__uint_as_float(ai[k]), __uint_as_float(ai[k + 1])), hbx2);
                         const f2_t tr = f2_make(tanh_approx(f2_lo(zr)), tanh_approx(f2_hi(zr)));
@@ -796,7 +796,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                         const f2_t a2 = f2_make(a0, a1);
                         const f2_t om = f2_fma(f2_mul(a2, f2_splat(-1.f)), a2, one_2);
                         const f2_t nrm = f2_make(sqrt_approx(f2_lo(om)), sqrt_approx(f2_hi(om)));
-                        const f2_t xh2 = f2_make(xh.x, xh.y);
+                        const f2_t xh2 = f2_make(__uint_as_float(xq[k]), __uint_as_float(xq[k + 1]));
                         const f2_t v = f2_mul(nrm, f2_fma(tg, xh2, xh2));  // sqrt(1-a^2) * i * xc
                         const float h0 = fmaf(a0, hl, f2_lo(v));
                         const float P0 = P * a0;
@@ -813,8 +813,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int t = t8 + k;
-                        const __half2 xq2 = *reinterpret_cast<const __half2 *>(&xq[k >> 1]);
-                        const float xh = (k & 1) ? __high2float(xq2) : __low2float(xq2);
+                        const float xh = __uint_as_float(xq[k]);
                         const float tr = tanh_approx(__uint_as_float(ar[k]) + hba);
                         const float tg = tanh_approx(__uint_as_float(ai[k]) + hbx);
                         const float ell = fmaf(tr, hkl, hkl);
@@ -1032,20 +1031,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 
 // ---------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
 struct Layout {
     int C, G, tpg;
     size_t flags_off, flags_bytes, agg_off, prefix_off, trace_off, total;
@@ -1106,13 +1091,9 @@ rglru_status fused_prefill(const PrefillArgs &a)
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return RGLRU_ERR_CUDA;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(rglru_prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemBytes);
-    });
-    if (attr_err != cudaSuccess) return RGLRU_ERR_CUDA;
+    static PerDeviceFlag smem_set;
+    const rglru_status st = set_smem_limit_once((const void *)rglru_prefill_fused_kernel, kSmemBytes, smem_set);
+    if (st != RGLRU_OK) return st;
 
     char *ws = static_cast<char *>(a.ws);
     // tickets and flags start at zero; the status word and the test hook are kept

@@ -26,12 +26,14 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 
 static __device__ __align__(256) unsigned char g_prefill_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device; set up once per
-// device (the host symbol is only a stand-in and must never reach a kernel).
+// device index (the host symbol is only a stand-in and must never reach a
+// kernel).  The cache assumes the device's context lives as long as the
+// process: after a cudaDeviceReset the array may sit at another address, so
+// a process that resets a device must not call this entry point on it again.
 rglru_status scratch_address(void **out)
 {
     int dev = 0;

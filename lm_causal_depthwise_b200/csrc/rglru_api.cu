@@ -35,6 +35,46 @@ bool sizes_ok(int B, int T, int D)
 
 }  // namespace
 
+PFN_cuTensorMapEncodeTiled_v12000 rglru::encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool rglru::encode_bf16(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap *m, const void *base, int rank,
+                        const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box,
+                        CUtensorMapSwizzle sw)
+{
+    if (encode == nullptr) return false;
+    const cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+rglru_status rglru::set_smem_limit_once(const void *kernel, int bytes, PerDeviceFlag &flag)
+{
+    static std::mutex m;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RGLRU_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return RGLRU_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(m);
+    if (!flag.done[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return RGLRU_ERR_CUDA;
+        flag.done[dev] = true;
+    }
+    return RGLRU_OK;
+}
+
 rglru_status rglru::validate_prefill(const PrefillArgs &a, size_t need)
 {
     if (a.dt != RGLRU_IO_F32 && a.dt != RGLRU_IO_BF16) return RGLRU_ERR_INVALID_ARG;

@@ -13,6 +13,7 @@ Tolerances (fixed here, used by every parity test):
 from __future__ import annotations
 
 import concurrent.futures as cf
+import os
 
 import numpy as np
 import torch
@@ -62,9 +63,26 @@ def run_oracle(inp: dict, nthreads: int = 0):
 def oracle_units(inp: dict, units, t_end=None):
     """Oracle outputs of several (b, head) units, run concurrently (the C
     oracle releases the GIL)."""
-    with cf.ThreadPoolExecutor(max_workers=min(len(units), 16)) as ex:
+    with cf.ThreadPoolExecutor(max_workers=min(len(units), os.cpu_count() or 16)) as ex:
         futs = {u: ex.submit(oracle.prefill_unit, inp, u[0], u[1], t_end, 8.0, 1) for u in units}
         return {u: f.result() for u, f in futs.items()}
+
+
+def oracle_every_unit(inp: dict):
+    """Oracle outputs of the whole problem, computed unit by unit on all host
+    cores (memory stays at one unit's float64 copy per worker).  Returns
+    (y_units, conv_state [B,3,D], h_state [B,D]) with y_units[(b, h)] the
+    float64 [T, 256] output block of unit (b, h)."""
+    B, T, D = inp["x"].shape
+    units = [(b, h) for b in range(B) for h in range(D // 256)]
+    ref = oracle_units(inp, units)
+    cs = np.empty((B, 3, D))
+    hs = np.empty((B, D))
+    for (b, h), r in ref.items():
+        s = slice(h * 256, (h + 1) * 256)
+        cs[b, :, s] = r["conv_state"]
+        hs[b, s] = r["h_state"]
+    return {u: r["y"] for u, r in ref.items()}, cs, hs
 
 
 def check_f32(got, ref, what=""):
@@ -77,17 +95,22 @@ def check_f32(got, ref, what=""):
     return err
 
 
-def check_bf16(got, ref, what=""):
+def check_bf16(got, ref, what="", scale=1.0):
+    """Every element within atol + rtol |ref|.  ``scale`` multiplies the
+    absolute part for inputs drawn ``scale`` times larger than the workloads'
+    N(0, 1): every rounding of an intermediate (bf16 operands, the f16 stash,
+    the bf16 output) then errs ``scale`` times more in absolute terms."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     diff = np.abs(got - ref)
-    bad = diff > BF16_ATOL + BF16_RTOL * np.abs(ref)
+    atol = BF16_ATOL * scale
+    bad = ~(diff <= atol + BF16_RTOL * np.abs(ref))  # NaN or inf counts as bad
     if bad.any():
         idx = np.argwhere(bad)[0]
         raise AssertionError(
-            f"{what}: {int(bad.sum())} of {bad.size} elements outside atol {BF16_ATOL} + rtol "
+            f"{what}: {int(bad.sum())} of {bad.size} elements outside atol {atol} + rtol "
             f"{BF16_RTOL}; first at {tuple(idx)}: got {got[tuple(idx)]!r} ref {ref[tuple(idx)]!r}; "
-            f"max abs {diff.max():.3e}")
+            f"max abs {np.nanmax(diff):.3e}")
     big = np.abs(ref) >= 1.0
     max_rel = float((diff[big] / np.abs(ref[big])).max()) if big.any() else 0.0
     return float(diff.max()), max_rel

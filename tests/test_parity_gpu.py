@@ -1,8 +1,8 @@
 """GPU parity: the CUDA library against the float64 oracle on the same seeded inputs.
 
-Small cases compare every element; the full-size workloads compare every
-output of sampled (batch row, head) units, whole sequences long, computed by
-the oracle unit by unit (heads and batch rows are independent).
+Every case compares every output element.  The full-size workloads run in
+the launch configuration the benchmark times; the oracle computes them unit by
+unit on all host cores (heads and batch rows are independent).
 """
 import numpy as np
 import pytest
@@ -10,8 +10,8 @@ import torch
 
 from lm_causal_depthwise_b200 import api, workloads as W
 
-from parity_util import (check, check_bf16, check_f32, check_state, oracle_units, run_gpu,
-                         run_oracle, to_device)
+from parity_util import (check, check_bf16, check_f32, check_state, oracle_every_unit, oracle_units,
+                         run_gpu, run_oracle, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -19,9 +19,9 @@ PATHS = [False, True]  # rglru_prefill, rglru_prefill_simt
 
 
 def _case(B, T, D, io="bf16", seed=21, doc_len=None, reset_at=(0,), continue_doc=False,
-          init_state="random"):
+          init_state="random", decay="init", x_scale=1.0):
     w = W.Workload("case", B=B, T=T, D=D, io=io, seed=seed, doc_len=doc_len, reset_at=reset_at,
-                   continue_doc=continue_doc, init_state=init_state)
+                   continue_doc=continue_doc, init_state=init_state, decay=decay, x_scale=x_scale)
     return w, W.generate(w)
 
 
@@ -58,6 +58,53 @@ def test_edge_lengths(simt, io, T):
     ref = run_oracle(inp)
     check(io, got["y"], ref["y"], f"y T={T}")
     check_state(io, got, ref, f"T={T}")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_fast_decay_channels(simt, io):
+    """Lambda drawn in [-10, 6.9]: most channels have Lambda < 0
+    (sigmoid(Lambda)^8 from ~1e-35 up), the other branch of log sigmoid, and
+    decays so fast that the normaliser sqrt(1 - a^2) is ~1.  Several tiles,
+    resets, a carried initial state."""
+    _, inp = _case(2, 1000, 512, io=io, doc_len=300, decay="wide", seed=33)
+    assert (inp["lam"] < -5).any() and (inp["lam"] > 5).any() and (inp["lam"] <= 6.91).all()
+    got = run_gpu(to_device(inp, io), simt=simt)
+    ref = run_oracle(inp)
+    check(io, got["y"], ref["y"], "y")
+    check_state(io, got, ref, "state")
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_decode_fast_decay_channels(io):
+    T, D, B = 24, 512, 70
+    _, inp = _case(B, T, D, io=io, reset_at=(0, 9), decay="wide", seed=34)
+    dev = to_device(inp, io)
+    ys = []
+    for t in range(T):
+        ys.append(api.decode_step(dev["x"][:, t].contiguous(), dev["g"][:, t].contiguous(), dev["params"],
+                                  dev["segpos"][:, t].contiguous(), dev["conv_state"],
+                                  dev["h_state"]).float().cpu().numpy())
+    ref = run_oracle(inp)
+    check(io, np.stack(ys, axis=1), ref["y"], "decode y")
+    got = {"h_state": dev["h_state"].cpu().numpy(), "conv_state": dev["conv_state"].float().cpu().numpy()}
+    check_state(io, got, ref, "decode")
+
+
+@pytest.mark.parametrize("simt", PATHS)
+def test_large_magnitude_inputs(simt):
+    """x and the conv state drawn as 100 N(0, 1) (|x| up to ~500, |xc| and
+    |h| in the hundreds to thousands): every output finite and within the bf16
+    bar with its absolute part scaled by the input scale (the f16 stash of the
+    fused kernel and the bf16 operands err in proportion to the magnitudes)."""
+    s = 100.0
+    _, inp = _case(2, 1000, 512, doc_len=300, x_scale=s, seed=35)
+    got = run_gpu(to_device(inp, "bf16"), simt=simt)
+    assert np.isfinite(got["y"]).all() and np.isfinite(got["h_state"]).all()
+    ref = run_oracle(inp)
+    check_bf16(got["y"], ref["y"], "y", scale=s)
+    check_bf16(got["h_state"], ref["h_state"], "h_state", scale=s)
+    np.testing.assert_array_equal(got["conv_state"], ref["conv_state"])
 
 
 @pytest.mark.parametrize("simt", PATHS)
@@ -149,36 +196,37 @@ def test_decode_steps_match_oracle(io, B):
 
 # ------------------------------------------------------------- full-size workloads
 
-def _full_size(w, units, simt=False):
+@pytest.mark.parametrize("wname", ["prefill-2b", "prefill-long", "prefill-long-carry", "prefill-9b"])
+def test_full_size_every_element(wname):
+    """The full-size workloads in the launch configuration the benchmark
+    times, every output element (y, h_state, conv_state) against the oracle,
+    which runs every (batch row, head) unit on the host cores."""
+    w = W.ALL[wname]
     inp = W.generate(w)
     dev = to_device(inp, w.io)
     y = api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"],
-                    dev["h_state"], simt=simt)
+                    dev["h_state"])
     torch.cuda.synchronize()
-    ref = oracle_units(inp, units)
-    for (b, h), r in ref.items():
-        s = slice(h * 256, (h + 1) * 256)
-        check_bf16(y[b, :, s].float().cpu().numpy(), r["y"], f"{w.name} y unit {(b, h)}")
-        check_bf16(dev["h_state"][b, s].cpu().numpy(), r["h_state"], f"{w.name} h unit {(b, h)}")
-        np.testing.assert_array_equal(dev["conv_state"][b, :, s].float().cpu().numpy(),
-                                      r["conv_state"])
-    return y
+    del dev["x"], dev["g"]
+    ref_y, ref_cs, ref_hs = oracle_every_unit(inp)
+    yh = y.float().cpu().numpy()
+    del y
+    for (b, h), r in ref_y.items():
+        check_bf16(yh[b, :, h * 256:(h + 1) * 256], r, f"{w.name} y unit {(b, h)}")
+    check_bf16(dev["h_state"].cpu().numpy(), ref_hs, f"{w.name} h_state")
+    np.testing.assert_array_equal(dev["conv_state"].float().cpu().numpy(), ref_cs)
 
 
-@pytest.mark.parametrize("wname,units", [
-    ("prefill-2b", [(0, 0), (3, 4), (7, 9)]),
-    ("prefill-long", [(0, 0), (0, 9)]),
-    ("prefill-long-carry", [(0, 3)]),
-    ("prefill-9b", [(0, 0), (15, 15), (9, 7)]),
-])
-def test_full_size_sampled_units(wname, units):
-    _full_size(W.ALL[wname], units)
-
-
-def test_full_size_decode_sampled_units():
+def test_full_size_decode_equals_prefill_and_oracle():
+    """decode-2b: 1024 single-token steps for B = 256 sequences, against one
+    prefill over the same 1024 tokens and against the oracle, every element
+    of y and the final states."""
     w = W.DECODE_2B
     inp = W.generate(w)
     dev = to_device(inp, w.io)
+    pre = to_device(inp, w.io)
+    y_pre = api.prefill(pre["x"], pre["g"], pre["params"], pre["segpos"], pre["conv_state"],
+                        pre["h_state"])
     ys = torch.empty((w.T, w.B, w.D), dtype=torch.bfloat16, device="cuda")
     ws = api.new_workspace(api.decode_workspace_size(w.B, w.D, torch.bfloat16))
     xs = dev["x"].transpose(0, 1).contiguous()
@@ -188,11 +236,23 @@ def test_full_size_decode_sampled_units():
         api.decode_step(xs[t], gs[t], dev["params"], ss[t], dev["conv_state"], dev["h_state"],
                         workspace=ws, y=ys[t])
     torch.cuda.synchronize()
-    ref = oracle_units(inp, [(0, 0), (100, 5), (255, 9)])
-    for (b, h), r in ref.items():
+    assert api.device_status(ws) == api.OK
+    del xs, gs, pre["x"], pre["g"], dev["x"], dev["g"]
+    y_dec = ys.transpose(0, 1).float().cpu().numpy()
+    del ys
+    y_p = y_pre.float().cpu().numpy()
+    del y_pre
+    check_bf16(y_dec, y_p, "decode y vs prefill y")
+    check_bf16(dev["h_state"].cpu().numpy(), pre["h_state"].cpu().numpy(), "decode h vs prefill h")
+    np.testing.assert_array_equal(dev["conv_state"].float().cpu().numpy(),
+                                  pre["conv_state"].float().cpu().numpy())
+    ref_y, ref_cs, ref_hs = oracle_every_unit(inp)
+    for (b, h), r in ref_y.items():
         s = slice(h * 256, (h + 1) * 256)
-        check_bf16(ys[:, b, s].float().cpu().numpy(), r["y"], f"decode y unit {(b, h)}")
-        check_bf16(dev["h_state"][b, s].cpu().numpy(), r["h_state"], "decode h")
+        check_bf16(y_dec[b, :, s], r, f"decode y unit {(b, h)}")
+        check_bf16(y_p[b, :, s], r, f"prefill y unit {(b, h)}")
+    check_bf16(dev["h_state"].cpu().numpy(), ref_hs, "decode h_state")
+    np.testing.assert_array_equal(dev["conv_state"].float().cpu().numpy(), ref_cs)
 
 
 # ------------------------------------------------------------- bounded waits and cross-checks
