@@ -21,8 +21,9 @@ struct WsHeader {
     int status;            // rglru_status recorded by device code (0 = OK)
     int detail;            // first wait that gave up: (CTA << 8) | (wait site + 1), 0 = none
     int debug_unit_plus1;  // test hook: chunk that skips publishing (+1), 0 = off
-    int pad0;
-    unsigned int ticket[1000];  // per-group work counters of the fused prefill kernel
+    unsigned int epoch;    // fused prefill launches completed on this workspace (tags its scan carry)
+    unsigned int ticket[999];  // per-group work counters of the fused prefill kernel
+    unsigned int done_ctas;    // CTAs of the current fused launch that have finished
 };
 constexpr size_t kWsHeaderBytes = 4096;
 static_assert(sizeof(WsHeader) <= kWsHeaderBytes, "header too large");

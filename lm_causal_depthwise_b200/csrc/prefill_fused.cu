@@ -62,6 +62,7 @@ constexpr int NS = 6;           // stash slots in shared memory (pass 1 -> look-
 constexpr int NB = 2;           // B tiles in shared memory (conv -> MMA, both CTAs)
 constexpr int XRING = 2;        // x tiles in shared memory (TMA -> conv)
 constexpr int INFO_RING = 16;   // tile descriptors in flight
+constexpr int kClaimBatch = 4;  // consecutive tickets claimed by one atomic
 constexpr int kScanGroups = 2;  // scan warp groups, alternate tiles
 constexpr int kScanWarps = 4 * kScanGroups, kConvWarps = 4;
 constexpr int kConvWarp0 = kScanWarps;
@@ -152,8 +153,8 @@ struct FusedParams {
     __nv_bfloat16 *y;
     WsHeader *hdr;
     uint32_t *flags;   // [2 H][tiles_per_head]: one scan chain per (head, half)
-    float2 *agg;       // [2 H][tiles_per_head][128]  (prod a, h_end) from h = 0
-    float *prefix;     // [2 H][tiles_per_head][128]  h after the tile
+    uint64_t *agg;     // [2 H][tiles_per_head][128][2]  tagged (prod a), tagged h_end from h = 0
+    uint64_t *prefix;  // [2 H][tiles_per_head][128]     tagged h after the tile
     unsigned long long *trace;  // RGLRU_TRACE builds only: per-role timestamps
 };
 
@@ -236,6 +237,75 @@ __device__ __noinline__ uint32_t wait_flag(const uint32_t *f, uint32_t need, vol
     }
 }
 
+// A published float with the launch's tag in the upper half: a reader that
+// sees the tag sees the value (the 8-byte word is single-copy atomic), so the
+// scan carry crosses SMs with no fence between data and flag.
+__device__ __forceinline__ uint64_t tagged(float v, uint32_t tag)
+{
+    return ((uint64_t)tag << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ float untag(uint64_t w) { return __uint_as_float((uint32_t)w); }
+__device__ __forceinline__ bool has_tag(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
+
+// This lane's 4 channels of a tile's aggregate (A, H), spinning (bounded)
+// until every word carries `tag`; false on timeout or abort.
+__device__ __forceinline__ bool load_agg4(const uint64_t *src, uint32_t tag, float (&A)[4], float (&H)[4],
+                                       volatile int *abort_flag, WsHeader *hdr)
+{
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint64_t w[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ld_relaxed_v2_u64(src + 2 * e, w[2 * e], w[2 * e + 1]);
+        bool ok = true;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ok = ok && has_tag(w[e], tag);
+        if (ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                A[e] = untag(w[2 * e]);
+                H[e] = untag(w[2 * e + 1]);
+            }
+            return true;
+        }
+        if (t0 == 0) t0 = globaltimer();
+        __nanosleep(32);
+        if ((it & 31u) == 31u) {
+            if (*abort_flag || *(volatile int *)&hdr->status != 0) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                raise_timeout(abort_flag, hdr, 25);
+                return false;
+            }
+        }
+    }
+}
+
+// This lane's 4 channels of a tile's inclusive prefix (see load_agg4).
+__device__ __forceinline__ bool load_prefix4(const uint64_t *src, uint32_t tag, float (&h)[4], volatile int *abort_flag,
+                                          WsHeader *hdr)
+{
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint64_t w[4];
+        ld_relaxed_v2_u64(src, w[0], w[1]);
+        ld_relaxed_v2_u64(src + 2, w[2], w[3]);
+        if (has_tag(w[0], tag) && has_tag(w[1], tag) && has_tag(w[2], tag) && has_tag(w[3], tag)) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = untag(w[e]);
+            return true;
+        }
+        if (t0 == 0) t0 = globaltimer();
+        __nanosleep(32);
+        if ((it & 31u) == 31u) {
+            if (*abort_flag || *(volatile int *)&hdr->status != 0) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                raise_timeout(abort_flag, hdr, 26);
+                return false;
+            }
+        }
+    }
+}
+
 // Warp-collective forms: lane 0 waits, the result is broadcast, then every lane
 // performs its own (already satisfied) acquire so that the warp stays converged
 // for the .sync.aligned tcgen05 instructions that follow.
@@ -285,7 +355,9 @@ __device__ __forceinline__ uint32_t warp_wait_flag(const uint32_t *f, uint32_t n
 // tile holding a reset (A = 0: its prefix is its own H) -- such that every tile
 // between the anchor and `hi` has published its aggregate.  Lane l examines
 // tile hi - l, so 32 flags cost one round trip.  The first tile of the
-// sequence is an anchor only once its prefix (or its reset) is out.
+// sequence is an anchor only once its prefix (or its reset) is out.  The
+// flags are hints (set without ordering): the words they announce carry the
+// launch's tag and are validated when read.
 // Warp-collective; false on timeout or abort.
 __device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_first, int &anchor,
                                          uint32_t &anchor_flag, volatile int *abort_flag, WsHeader *hdr)
@@ -295,7 +367,7 @@ __device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_
     for (uint32_t spins = 0;;) {
         const int pu = hi - lane;
         const bool in = pu >= seq_first;
-        const uint32_t f = in ? ld_acquire_u32(flags + pu) : 0u;
+        const uint32_t f = in ? ld_relaxed_u32(flags + pu) : 0u;
         const uint32_t anchors = __ballot_sync(0xffffffffu, in && (f & (F_PREFIX | F_RESET)));
         const uint32_t ready = __ballot_sync(0xffffffffu, in && (f & F_AGG));
         if (anchors) {
@@ -440,6 +512,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     }
 #endif
     const int debug_unit = *(volatile int *)&hdr->debug_unit_plus1 - 1;
+    // this launch's tag: one more than the launches completed on this
+    // workspace (the last CTA to finish advances the count), so no word
+    // left by an earlier launch can pass for this one's
+    const uint32_t tag = *(volatile unsigned int *)&hdr->epoch + 1u;
 
     if (warp == kSchedWarp) {
         // ------------------------------------------------------------ scheduler
@@ -452,29 +528,56 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // tickets earlier and has usually published its aggregate (and its
         // prefix) by the time the tile's own look-back starts.  The look-back
         // indexes tiles by u = b C + c, their order inside the sequence.
+        // Claims come in batches of kClaimBatch consecutive tickets: one
+        // atomicAdd per batch, issued a batch ahead, and the batch's
+        // segment_pos loads issued together, so the round trips overlap the
+        // x loads instead of pacing them.
+        int k_pending = -1;  // lane 0: ticket of the next batch (atomic in flight)
+        auto fetch = [&]() {
+            if (lane == 0 && !*abort_flag) k_pending = (int)atomicAdd(&hdr->ticket[head], (unsigned)kClaimBatch);
+            else if (lane == 0) k_pending = 0x3fffffff;  // past every ticket: no more tiles
+        };
+        TileInfo batch[kClaimBatch];
+        int batch_i = kClaimBatch;
+        auto claim_batch = [&]() {
+            const int k0 = __shfl_sync(0xffffffffu, k_pending, 0);
+            fetch();
+            int sp[kClaimBatch];
+#pragma unroll
+            for (int q = 0; q < kClaimBatch; ++q) {
+                const int k = k0 + q;
+                TileInfo ti{};
+                ti.u = -1;
+                sp[q] = 3;
+                if (k >= 0 && k < p.tiles_per_head) {
+                    ti.b = k % p.B;
+                    const int c = k / p.B;
+                    ti.u = ti.b * p.C + c;
+                    ti.t0 = c * NT;
+                    ti.valid = min(NT, p.T - ti.t0);
+                    ti.first_last = (c == 0 ? 1 : 0) | (c == p.C - 1 ? 2 : 0);
+                    if (lane < ti.valid) sp[q] = p.segpos[(size_t)ti.b * p.T + ti.t0 + lane];
+                }
+                batch[q] = ti;
+            }
+#pragma unroll
+            for (int q = 0; q < kClaimBatch; ++q) {
+                batch[q].reset_mask = __ballot_sync(0xffffffffu, sp[q] < 1);
+                batch[q].m2 = __ballot_sync(0xffffffffu, sp[q] < 2);
+                batch[q].m3 = __ballot_sync(0xffffffffu, sp[q] < 3);
+            }
+            batch_i = 0;
+        };
         auto claim = [&]() -> TileInfo {
-            int k = -1;
-            if (lane == 0 && !*abort_flag) {
-                k = (int)atomicAdd(&hdr->ticket[head], 1u);
-                if (k >= p.tiles_per_head) k = -1;
-            }
-            k = __shfl_sync(0xffffffffu, k, 0);
+            if (batch_i == kClaimBatch) claim_batch();
             TileInfo ti{};
-            ti.u = -1;
-            if (k >= 0) {
-                ti.b = k % p.B;
-                const int c = k / p.B;
-                ti.u = ti.b * p.C + c;
-                ti.t0 = c * NT;
-                ti.valid = min(NT, p.T - ti.t0);
-                ti.first_last = (c == 0 ? 1 : 0) | (c == p.C - 1 ? 2 : 0);
-                const int sp = lane < ti.valid ? p.segpos[(size_t)ti.b * p.T + ti.t0 + lane] : 3;
-                ti.reset_mask = __ballot_sync(0xffffffffu, sp < 1);
-                ti.m2 = __ballot_sync(0xffffffffu, sp < 2);
-                ti.m3 = __ballot_sync(0xffffffffu, sp < 3);
-            }
+#pragma unroll
+            for (int q = 0; q < kClaimBatch; ++q)
+                if (q == batch_i) ti = batch[q];
+            ++batch_i;
             return ti;
         };
+        if (half == 0) fetch();
         TileInfo next{};
         if (half == 0) next = claim();
         int ends = 0, x_issued = 0;
@@ -664,22 +767,26 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 if (!warp_wait_bar(bar(B_W_FULL, 0), 0u, abort_flag, hdr, 11)) break;
                 w_ready = true;
             }
-            if (lane == 0) {
-                tc_fence_after();
+            // the whole (converged) warp runs the issue loop; elect.sync picks
+            // the lane that issues each MMA and commit
+            tc_fence_after();
+            {
                 const uint32_t bt = smem_u32(smem + OFF_B + sb * kBTile);
                 const uint32_t d_r = tmem + kColAcc + sa * kColsAcc, d_i = d_r + NT;
+                const uint64_t bd0 = umma_desc_mn_noswizzle(bt, kBGroup, 128);
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk) {
-                    // A (16 input channels of this half's weight rows) from TMEM
-                    // 16 input channels = two 8-channel groups of the N-major B tile
-                    const uint64_t bd = umma_desc_mn_noswizzle(bt + kk * 2 * kBGroup, kBGroup, 128);
-                    umma_ts(d_r, tmem + kColW + kk * 8, bd, idesc, kk > 0);
-                    umma_ts(d_i, tmem + kColW + kColsWGate + kk * 8, bd, idesc, kk > 0);
+                    // A (16 input channels of this half's weight rows) from TMEM;
+                    // 16 input channels = two 8-channel groups of the N-major B
+                    // tile (the descriptor's start address counts 16-byte units)
+                    const uint64_t bd = bd0 + (uint64_t)((kk * 2 * kBGroup) >> 4);
+                    umma_ts_warp(d_r, tmem + kColW + kk * 8, bd, idesc, kk > 0);
+                    umma_ts_warp(d_i, tmem + kColW + kColsWGate + kk * 8, bd, idesc, kk > 0);
                 }
-                umma_commit(bar(B_MMA, sa));
-                umma_commit_cluster(bar(B_BFREE, sb), 0x3);  // this B slot is free in both CTAs' view
-                RGLRU_TR(TR_MMA_ISSUED, j, globaltimer());
+                umma_commit_warp(bar(B_MMA, sa));
+                umma_commit_cluster_warp(bar(B_BFREE, sb), 0x3);  // this B slot is free in both CTAs' view
             }
+            if (lane == 0) RGLRU_TR(TR_MMA_ISSUED, j, globaltimer());
             __syncwarp();
             ++issued;
         }
@@ -880,12 +987,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // may combine it before this tile's own look-back has finished), find
         // the anchor, fold, publish the inclusive prefix, then pass 2 of the
         // tile: y = y_loc + q h_in from the stash, 4 channels per lane, and at
-        // a sequence end the new states.  These warps are the only ones that
-        // fence for the aggregates and prefixes.
+        // a sequence end the new states.  Aggregates and prefixes go out as
+        // tagged words with no fence; only the first tile of a sequence
+        // publishes its prefix with release (for the state write-back).
         const int ch = lane * 4;  // 4 channels per lane
         const size_t dch = (size_t)ch0 + ch;
         const size_t gbase = (size_t)group * p.tiles_per_head;
-        constexpr int kFoldBatch = 4;  // aggregates loaded per round trip
 #pragma unroll 1
         for (int j = warp - kLbWarp0;; j += kLbWarps) {
             const int ss = j % NS, ir = j % INFO_RING;
@@ -902,12 +1009,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const uint32_t rbit = ti.reset_mask ? F_RESET : 0u;
             const bool suppress = (int)gu == debug_unit;
             if (!suppress) {
-                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf + ch);
-                dst[0] = g01;
-                dst[1] = g23;
-                __threadfence();
+                // tagged words, no fence: the flag only tells readers where to look
+                uint64_t *dst = p.agg + (gu * kHalf + ch) * 2;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) st_relaxed_v2_u64(dst + 2 * e, tagged(A[e], tag), tagged(Hh[e], tag));
                 __syncwarp();
-                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | rbit);
+                if (lane == 0) red_relaxed_or_u32(p.flags + gu, F_AGG | rbit);
             }
             float hin[4];
             bool ok = true;
@@ -927,35 +1034,49 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     // sequence order from the anchor, the same order whichever
                     // prefixes happened to be published (bit-reproducible)
                     if (aflag & F_PREFIX) {
-                        const float4 pr = ld_relaxed_f4(reinterpret_cast<const float4 *>(p.prefix + (gbase + anchor) * kHalf + ch));
-                        hin[0] = pr.x; hin[1] = pr.y; hin[2] = pr.z; hin[3] = pr.w;
+                        ok = load_prefix4(p.prefix + (gbase + anchor) * kHalf + ch, tag, hin, abort_flag, hdr);
                     } else {  // a tile holding a reset: A = 0, its prefix is its H
-                        const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + anchor) * kHalf + ch);
-                        const float4 a01 = ld_relaxed_f4(src), a23 = ld_relaxed_f4(src + 1);
-                        hin[0] = a01.y; hin[1] = a01.w; hin[2] = a23.y; hin[3] = a23.w;
+                        float a4[4];
+                        ok = load_agg4(p.agg + ((gbase + anchor) * kHalf + ch) * 2, tag, a4, hin, abort_flag, hdr);
                     }
 #pragma unroll 1
-                    for (int p0 = anchor + 1; p0 < ti.u; p0 += kFoldBatch) {
-                        float4 dd[kFoldBatch][2];
+                    for (int p0 = anchor + 1; ok && p0 < ti.u; p0 += 2) {
+                        // two aggregates per round trip when both are visible
+                        const uint64_t *s0 = p.agg + ((gbase + p0) * kHalf + ch) * 2;
+                        const bool two = p0 + 1 < ti.u;
+                        uint64_t w[16];
 #pragma unroll
-                        for (int k = 0; k < kFoldBatch; ++k) {
-                            if (p0 + k < ti.u) {
-                                const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + p0 + k) * kHalf + ch);
-                                dd[k][0] = ld_relaxed_f4(src);
-                                dd[k][1] = ld_relaxed_f4(src + 1);
-                            }
+                        for (int e = 0; e < 4; ++e) ld_relaxed_v2_u64(s0 + 2 * e, w[2 * e], w[2 * e + 1]);
+                        if (two) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                ld_relaxed_v2_u64(s0 + kHalf * 2 + 2 * e, w[8 + 2 * e], w[8 + 2 * e + 1]);
                         }
+                        bool seen = true;
 #pragma unroll
-                        for (int k = 0; k < kFoldBatch; ++k) {
-                            if (p0 + k < ti.u) {
-                                hin[0] = fmaf(dd[k][0].x, hin[0], dd[k][0].y);
-                                hin[1] = fmaf(dd[k][0].z, hin[1], dd[k][0].w);
-                                hin[2] = fmaf(dd[k][1].x, hin[2], dd[k][1].y);
-                                hin[3] = fmaf(dd[k][1].z, hin[3], dd[k][1].w);
+                        for (int e = 0; e < 16; ++e) seen = seen && (has_tag(w[e], tag) || (e >= 8 && !two));
+                        float a4[4], h4[4];
+                        if (seen) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) hin[e] = fmaf(untag(w[2 * e]), hin[e], untag(w[2 * e + 1]));
+                            if (two) {
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    hin[e] = fmaf(untag(w[8 + 2 * e]), hin[e], untag(w[8 + 2 * e + 1]));
+                            }
+                        } else {
+                            ok = load_agg4(s0, tag, a4, h4, abort_flag, hdr);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) hin[e] = fmaf(a4[e], hin[e], h4[e]);
+                            if (ok && two) {
+                                ok = load_agg4(s0 + kHalf * 2, tag, a4, h4, abort_flag, hdr);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) hin[e] = fmaf(a4[e], hin[e], h4[e]);
                             }
                         }
                     }
                 }
+                ok = __all_sync(0xffffffffu, ok);
             }
             if (!ok) break;
             if (lane == 0) RGLRU_TR(TR_LB_HIN, j, globaltimer());
@@ -963,10 +1084,20 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 #pragma unroll
             for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
             if (!suppress) {
-                *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
+                uint64_t *dst = p.prefix + gu * kHalf + ch;
+                st_relaxed_v2_u64(dst, tagged(pre[0], tag), tagged(pre[1], tag));
+                st_relaxed_v2_u64(dst + 2, tagged(pre[2], tag), tagged(pre[3], tag));
+                if (ti.first_last & 1) {
+                    // the sequence's last tile overwrites the states this first
+                    // tile has read: it waits for this flag with acquire, so this
+                    // one publish is a release
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
+                } else {
+                    __syncwarp();
+                    if (lane == 0) red_relaxed_or_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
+                }
             }
             if (lane == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
             // pass 2: token t of this lane's 4 channels is one 16-byte stash word;
@@ -1027,6 +1158,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     cluster_sync();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+    if (threadIdx.x == 0 && atomicAdd(&hdr->done_ctas, 1u) == gridDim.x - 1) atomicExch(&hdr->epoch, tag);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1046,8 +1178,8 @@ Layout layout_of(int B, int T, int D)
     L.flags_off = kWsHeaderBytes;
     L.flags_bytes = align_up(tiles * 4, 256);
     L.agg_off = L.flags_off + L.flags_bytes;
-    L.prefix_off = L.agg_off + align_up(tiles * kHalf * 8, 256);
-    L.total = L.prefix_off + align_up(tiles * kHalf * 4, 256);
+    L.prefix_off = L.agg_off + align_up(tiles * kHalf * 16, 256);
+    L.total = L.prefix_off + align_up(tiles * kHalf * 8, 256);
 #ifdef RGLRU_TRACE
     L.trace_off = L.total;
     L.total += align_up((size_t)kTraceCtas * kTraceTiles * kTraceEvents * 8, 256);
@@ -1096,7 +1228,8 @@ rglru_status fused_prefill(const PrefillArgs &a)
     if (st != RGLRU_OK) return st;
 
     char *ws = static_cast<char *>(a.ws);
-    // tickets and flags start at zero; the status word and the test hook are kept
+    // tickets, the finished-CTA count and the flags start at zero; the status
+    // word, the test hook and the launch count are kept
     if (cudaMemsetAsync(ws + offsetof(WsHeader, ticket), 0,
                         L.flags_off - offsetof(WsHeader, ticket) + L.flags_bytes, a.stream) != cudaSuccess)
         return RGLRU_ERR_CUDA;
@@ -1115,8 +1248,8 @@ rglru_status fused_prefill(const PrefillArgs &a)
     p.y = static_cast<__nv_bfloat16 *>(a.y);
     p.hdr = reinterpret_cast<WsHeader *>(ws);
     p.flags = reinterpret_cast<uint32_t *>(ws + L.flags_off);
-    p.agg = reinterpret_cast<float2 *>(ws + L.agg_off);
-    p.prefix = reinterpret_cast<float *>(ws + L.prefix_off);
+    p.agg = reinterpret_cast<uint64_t *>(ws + L.agg_off);
+    p.prefix = reinterpret_cast<uint64_t *>(ws + L.prefix_off);
     p.trace = L.trace_off ? reinterpret_cast<unsigned long long *>(ws + L.trace_off) : nullptr;
 
     // one cluster of two CTAs (the two halves of a head) per SM pair; the same

@@ -56,7 +56,7 @@ def _load():
             lib.rglru_oracle_prefill.restype = ctypes.c_int
             lib.rglru_oracle_prefill.argtypes = (
                 [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double]
-                + [dp] * 8 + [dp, ip] + [dp] * 3 + [dp] * 5 + [ctypes.c_int])
+                + [dp] * 8 + [dp, ip] + [dp] * 3 + [dp] * 5 + [ctypes.c_int, ctypes.c_int])
             lib.rglru_oracle_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -84,8 +84,12 @@ def _ptr(a):
 
 def prefill(x, g, conv_w, conv_b, W_a, b_a, W_x, b_x, lam, segpos,
             conv_state, h_state, c: float = C_DEFAULT, trace: bool = False,
-            nthreads: int = 0):
+            nthreads: int = 0, gate_bf16: bool = False):
     """Run the block core over [B,T,D] inputs in float64.
+
+    ``gate_bf16=True`` rounds the conv output to bf16 where it enters the gate
+    projections (the operand precision of the tensor-core gate GEMM in bf16
+    I/O mode); everything else stays float64.
 
     Inputs may be any float dtype (they are widened exactly to float64).
     Returns a dict with ``y`` [B,T,D], ``conv_state`` [B,3,D] and ``h_state``
@@ -120,7 +124,7 @@ def prefill(x, g, conv_w, conv_b, W_a, b_a, W_x, b_x, lam, segpos,
         B, T, D, float(c), _ptr(x), _ptr(g), _ptr(conv_w), _ptr(conv_b), _ptr(W_a),
         _ptr(b_a), _ptr(W_x), _ptr(b_x), _ptr(lam), _ptr(segpos), _ptr(cs), _ptr(hs),
         _ptr(y), _ptr(tr["xc"]), _ptr(tr["r"]), _ptr(tr["i"]), _ptr(tr["a"]),
-        _ptr(tr["h"]), int(nthreads))
+        _ptr(tr["h"]), int(nthreads), 1 if gate_bf16 else 0)
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     out = {"y": y, "conv_state": cs, "h_state": hs}

@@ -42,6 +42,10 @@
  * Optional trace arrays (each [B,T,D], NULL to skip) record xc, r, i, a and
  * h per element so that the tests can pin each step separately.
  *
+ * gate_bf16 = 1 evaluates step 2 on the conv output rounded to bf16 (the
+ * operand precision of the tensor-core gate projections in bf16 I/O mode);
+ * 0, the default everywhere else, keeps it exact.
+ *
  * Independent units are the (batch row, head) pairs: heads never mix
  * (depthwise conv, block-diagonal gates, per-channel scan).  OpenMP runs the
  * units in parallel; inside a unit tokens run strictly in order.
@@ -65,6 +69,20 @@ static double log_sigmoid(double v)
 }
 
 static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* Nearest bf16 value (8 significant bits, ties to even) of v.  Used only
+ * when the caller asks for the gate projections in the precision of bf16
+ * I/O mode, where the tensor-core gate GEMM takes bf16 operands: the
+ * conv output enters the dot products rounded to bf16 (the scan and every
+ * other step keep it exact). */
+static double round_bf16(double v)
+{
+    if (v == 0.0 || !isfinite(v))
+        return v;
+    int e;
+    const double m = frexp(v, &e);        /* v = m 2^e, 0.5 <= |m| < 1 */
+    return ldexp(nearbyint(ldexp(m, 8)), e - 8);
+}
 
 static double gelu_tanh(double g)
 {
@@ -90,7 +108,7 @@ int rglru_oracle_prefill(int B, int T, int D, double c,
                          const double *lambda, const int32_t *segpos,
                          double *conv_state, double *h_state, double *y,
                          double *tr_xc, double *tr_r, double *tr_i,
-                         double *tr_a, double *tr_h, int nthreads)
+                         double *tr_a, double *tr_h, int nthreads, int gate_bf16)
 {
     if (B < 1 || T < 1 || D < HEAD || D % HEAD != 0)
         return -1;
@@ -111,7 +129,7 @@ int rglru_oracle_prefill(int B, int T, int D, double c,
             const double *gb = g + b * TD;
             const int32_t *sp = segpos + (int64_t)b * T;
             double *cs = conv_state + (int64_t)b * 3 * D;
-            double xc[HEAD], h[HEAD], newcs[3][HEAD];
+            double xc[HEAD], xg[HEAD], h[HEAD], newcs[3][HEAD];
 
             for (int j = 0; j < HEAD; ++j)
                 h[j] = h_state[(int64_t)b * D + d0 + j];
@@ -132,6 +150,7 @@ int rglru_oracle_prefill(int B, int T, int D, double c,
                         acc += conv_w[k * D + d] * xv;
                     }
                     xc[j] = acc;
+                    xg[j] = gate_bf16 ? round_bf16(acc) : acc;
                 }
                 /* steps 2-5 per output channel j of this head */
                 for (int j = 0; j < HEAD; ++j) {
@@ -140,8 +159,8 @@ int rglru_oracle_prefill(int B, int T, int D, double c,
                     const double *wx = W_x + ((int64_t)hd * HEAD + j) * HEAD;
                     double pr = b_a[d], pi = b_x[d];
                     for (int q = 0; q < HEAD; ++q) {
-                        pr += wa[q] * xc[q];
-                        pi += wx[q] * xc[q];
+                        pr += wa[q] * xg[q];
+                        pi += wx[q] * xg[q];
                     }
                     const double r = sigmoid(pr);
                     const double ig = sigmoid(pi);

@@ -295,3 +295,36 @@ def test_rejects_bad_sizes():
     inp = _inputs(B=1, T=4, D=256)
     with pytest.raises(ValueError):
         oracle.prefill(**{**inp, "x": inp["x"][:, :, :200], "g": inp["g"][:, :, :200]})
+
+
+def test_gate_operand_rounding_option():
+    """gate_bf16=True rounds the conv output to the nearest bf16 (ties to even)
+    where it enters the gate projections, and nowhere else.  Identity conv, so
+    xc = x; x is built from bf16 values v plus 0.3, 0.7 and exactly 0.5 of the
+    bf16 spacing at v, whose roundings are known: v, the next bf16 value up,
+    and (a tie) whichever of the two has an even last mantissa bit."""
+    T, D = 6, 256
+    inp = _inputs(B=1, T=T, D=D, reset_at=(0,), init_state="zero")
+    inp["conv_w"][:] = 0.0
+    inp["conv_w"][3] = 1.0
+    inp["conv_b"][:] = 0.0
+    rng = np.random.default_rng(11)
+    v = W.round_bf16(rng.standard_normal((T, D)).astype(np.float32)).astype(np.float64)
+    mant, ex = np.frexp(v)
+    ulp = np.ldexp(1.0, ex - 8)                       # bf16 spacing just above |v| (same sign)
+    frac = np.array([0.3, 0.7, 0.5, 0.3, 0.7, 0.5])[:, None]
+    x = v + np.sign(v) * frac * ulp
+    odd = (np.abs(np.ldexp(mant, 8)).astype(np.int64) & 1) == 1
+    up = (frac > 0.5) | ((frac == 0.5) & odd)
+    q = np.where(up, v + np.sign(v) * ulp, v)
+    inp["x"][0] = x
+    out = _run(inp, trace=True, gate_bf16=True)
+    np.testing.assert_array_equal(out["xc"][0], x)    # the conv itself stays exact
+    Wa, Wx = inp["W_a"][0], inp["W_x"][0]
+    np.testing.assert_allclose(out["r"][0], scipy.special.expit(q @ Wa.T + inp["b_a"]), rtol=1e-13)
+    np.testing.assert_allclose(out["i"][0], scipy.special.expit(q @ Wx.T + inp["b_x"]), rtol=1e-13)
+    # the scan uses the exact xc: at the reset token h = i * xc
+    np.testing.assert_allclose(out["h"][0, 0], out["i"][0, 0] * x[0], rtol=1e-14)
+    exact = _run(inp, trace=True)
+    np.testing.assert_allclose(exact["r"][0], scipy.special.expit(x @ Wa.T + inp["b_a"]), rtol=1e-13)
+    assert np.abs(exact["r"] - out["r"]).max() > 0
