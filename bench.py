@@ -56,6 +56,12 @@ def max_over_ranks(value: float, device="cpu") -> float:
     return float(t.item())
 
 
+def sharded_throughput(job_units: int, ms_per_step: float) -> float:
+    """Throughput of a job whose units are split across the ranks (strong
+    scaling): every unit once, divided by the (max-over-ranks) step time."""
+    return job_units / (ms_per_step * 1e-3)
+
+
 def job_throughput(units_per_rank: int, world: int, ms_per_step: float) -> float:
     """Whole-job throughput: the units every rank processed in one step, divided
     by the (max-over-ranks) step time."""
@@ -259,13 +265,13 @@ def roofline(alg_bytes: int, ms_per_launch: float, peaks: dict, peak_kind: str, 
 class PrefillCase:
     """Device buffers of one prefill workload and its timed step."""
 
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, inp=None):
         import torch
         from lm_causal_depthwise_b200 import api
         self.w, self.dev = w, dev
         bf = torch.bfloat16 if w.io == "bf16" else torch.float32
         self.bf = bf
-        self.inp = W.generate(w)
+        self.inp = W.generate(w) if inp is None else inp
         inp = self.inp
         self.x = torch.from_numpy(inp["x"]).to(dev).to(bf)
         self.g = torch.from_numpy(inp["g"]).to(dev).to(bf)
@@ -366,6 +372,194 @@ def copy_only_rates(hx, hg, hsp, hy, stream):
     return out
 
 
+def run_block(args, dev, stream, distributed, peaks, peak_kind):
+    """The whole recurrent block on the 2B shape: linear_x and linear_y in one
+    GEMM launch, the fused core, linear_out; timed as a whole (K steps) and per
+    launch, with the projections' TFLOP/s against the measured bf16 peak and
+    the same GEMM shapes through cuBLAS (torch.nn.functional.linear) for context."""
+    import torch
+    from lm_causal_depthwise_b200 import api
+    w = W.PREFILL_2B
+    inp = W.generate_block(w)
+    bf = torch.bfloat16
+    u = torch.from_numpy(inp["u"]).to(dev).to(bf)
+    sp = torch.from_numpy(inp["segpos"]).to(dev)
+    cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
+    hs = torch.from_numpy(inp["h_state"]).to(dev)
+    bp = api.BlockParams.from_arrays(inp, dev)
+    out = torch.empty_like(u)
+    ws = api.new_workspace(api.recurrent_block_workspace_size(w.B, w.T, w.D), dev)
+    M, D = w.B * w.T, w.D
+    u2 = u.view(M, D)
+    x2, g2, y2 = (torch.empty((M, D), dtype=bf, device=dev) for _ in range(3))
+    lws = api.linear_workspace(dev)
+    core_ws = api.new_workspace(api.workspace_size(w.B, w.T, w.D, bf), dev)
+    x3, g3 = x2.view(w.B, w.T, D), g2.view(w.B, w.T, D)
+
+    def block():
+        api.recurrent_block_prefill(u, bp, sp, cs, hs, out=out, workspace=ws)
+
+    def pair():
+        api.linear_pair(u2, bp.W_lin_x, bp.b_lin_x, bp.W_lin_y, bp.b_lin_y, out0=x2, out1=g2, workspace=lws)
+
+    def core():
+        api.prefill(x3, g3, bp.core, sp, cs, hs, workspace=core_ws, y=y2.view(w.B, w.T, D))
+
+    def outp():
+        api.linear(y2, bp.W_out, bp.b_out, out=out.view(M, D), workspace=lws)
+
+    bx16, by16 = bp.b_lin_x.to(bf), bp.b_lin_y.to(bf)  # torch's bf16 linear takes a bf16 bias
+
+    def cublas_pair():
+        torch.nn.functional.linear(u2, bp.W_lin_x, bx16)
+        torch.nn.functional.linear(u2, bp.W_lin_y, by16)
+
+    def timed(fn, n):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(n):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(ev0.elapsed_time(ev1), dev) / n
+
+    n = max(3, min(args.steps, 20))
+    if distributed:
+        import torch.distributed as dist
+        dist.barrier()
+    ms_block = timed(block, n)
+    st = api.device_status(ws)
+    if st != api.OK:
+        raise RuntimeError(f"recurrent block: device status {api.status_string(st)}")
+    ms_pair, ms_core, ms_out, ms_cublas = timed(pair, n), timed(core, n), timed(outp, n), timed(cublas_pair, n)
+    pair_flops, out_flops = 2 * 2 * M * D * D, 2 * M * D * D
+    world = dist.get_world_size() if distributed else 1
+    tflops = lambda f, ms: f / (ms * 1e-3) / 1e12
+    return {
+        "workload": f"recurrent block (linear_x/linear_y, core, linear_out) B={w.B} T={w.T} D={D} bf16",
+        "value": job_throughput(w.tokens, world, ms_block), "unit": "tokens/s", "ms_per_step": ms_block,
+        "steps": n, "gemm_flops_per_step": W.block_gemm_flops(w),
+        "launches": {"linear_pair_ms": ms_pair, "core_ms": ms_core, "linear_out_ms": ms_out},
+        "roofline": {"bound": "tensor", "kernel": "rglru_linear_kernel (linear_x + linear_y, one launch)",
+                     "achieved": tflops(pair_flops, ms_pair), "peak": peaks.get("bf16_tflops", 1590.0),
+                     "unit": "TFLOP/s", "frac": tflops(pair_flops, ms_pair) / peaks.get("bf16_tflops", 1590.0),
+                     "peak_source": f"{peak_kind} cuBLAS bf16 burst", "traffic": None},
+        "linear_out_tflops": tflops(out_flops, ms_out),
+        "cublas_same_pair_tflops": tflops(pair_flops, ms_cublas),
+        "core_hbm_frac": W.algorithmic_bytes(w) / (ms_core * 1e-3) / 1e9 / peaks["hbm_gbs"],
+    }
+
+
+def run_residual_block(args, dev, stream, distributed, peaks, peak_kind):
+    """The whole recurrent residual block on the 2B shape (RMSNorm, the
+    recurrent block with linear_out's residual add in its epilogue, RMSNorm,
+    the GELU-gated MLP up projection, the down projection with the residual
+    add): seven launches per step, timed as a whole, plus the MLP GEMMs alone."""
+    import torch
+    from lm_causal_depthwise_b200 import api
+    w = W.PREFILL_2B
+    inp = W.generate_residual_block(w)
+    bf = torch.bfloat16
+    u = torch.from_numpy(inp["u"]).to(dev).to(bf)
+    sp = torch.from_numpy(inp["segpos"]).to(dev)
+    cs = torch.from_numpy(inp["conv_state"]).to(dev).to(bf)
+    hs = torch.from_numpy(inp["h_state"]).to(dev)
+    rp = api.ResidualBlockParams.from_arrays(inp, dev)
+    F = rp.W_gate.shape[0]
+    out = torch.empty_like(u)
+    ws = api.new_workspace(api.residual_block_workspace_size(w.B, w.T, w.D, F), dev)
+    M, D = w.tokens, w.D
+    a2 = u.view(M, D)
+    m2 = torch.empty((M, F), dtype=bf, device=dev)
+    lws = api.linear_workspace(dev)
+
+    def step():
+        api.residual_block_prefill(u, rp, sp, cs, hs, out=out, workspace=ws)
+
+    def up():
+        api.linear_geglu(a2, rp.W_gate, rp.b_gate, rp.W_up, rp.b_up, out=m2, workspace=lws)
+
+    def down():
+        api.linear_residual(m2, rp.W_down, rp.b_down, a2, out=out.view(M, D), workspace=lws)
+
+    def timed(fn, n):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(n):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(ev0.elapsed_time(ev1), dev) / n
+
+    n = max(3, min(args.steps, 20))
+    ms = timed(step, n)
+    st = api.device_status(ws)
+    if st != api.OK:
+        raise RuntimeError(f"residual block: device status {api.status_string(st)}")
+    ms_up, ms_down = timed(up, n), timed(down, n)
+    world = torch.distributed.get_world_size() if distributed else 1
+    up_flops, down_flops = 2 * 2 * M * D * F, 2 * M * F * D
+    return {
+        "workload": f"recurrent residual block (RMSNorm, recurrent block, residual, RMSNorm, GELU-gated MLP "
+                    f"F={F}, residual) B={w.B} T={w.T} D={D} bf16",
+        "value": job_throughput(w.tokens, world, ms), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
+        "gemm_flops_per_step": W.residual_block_gemm_flops(w),
+        "gemm_tflops_whole_step": W.residual_block_gemm_flops(w) / (ms * 1e-3) / 1e12,
+        "mlp_up_geglu_tflops": up_flops / (ms_up * 1e-3) / 1e12, "mlp_up_ms": ms_up,
+        "mlp_down_residual_tflops": down_flops / (ms_down * 1e-3) / 1e12, "mlp_down_ms": ms_down,
+        "peak_bf16_tflops": peaks.get("bf16_tflops", 1590.0), "peak_source": f"{peak_kind} cuBLAS bf16 burst",
+    }
+
+
+def run_head_sharded(args, w, dev, stream, rank, world, local, distributed):
+    """--shard heads: the workload's heads split across the ranks (no
+    collective on the data path; each rank's output is a column block of the
+    whole output).  The job's work is fixed (strong scaling): its tokens once,
+    over the max-over-ranks step time."""
+    import torch
+    import torch.distributed as dist
+    from lm_causal_depthwise_b200.sharding import shard_heads, shard_inputs
+    h0, h1 = shard_heads(w.H, world, rank)
+    ms = 0.0
+    clocks = None
+    if h1 > h0:
+        part = w.scaled(D=(h1 - h0) * W.HEAD)
+        case = PrefillCase(part, dev, inp=shard_inputs(W.generate(w), h0, h1))
+        for _ in range(args.warmup):
+            case.step()
+        torch.cuda.synchronize()
+        ms, clocks = case.timed(args.steps, stream, False, local)
+    if distributed:
+        dist.barrier()
+    per_step_ms = max_over_ranks(ms, dev)
+    if distributed:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks, peak_kind = measured_peaks()
+    line = {
+        "metric": METRIC, "value": sharded_throughput(w.tokens, per_step_ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.describe(), "B": w.B, "T": w.T, "D": w.D, "tokens_per_job": w.tokens,
+                   "parallelism": f"heads split over {world} GPU(s), rank 0 has heads [{h0}, {h1})",
+                   "l2": "no flush: the shards' x, g, y exceed L2 at the sizes timed"},
+        "roofline": roofline(W.algorithmic_bytes(w), per_step_ms * world, peaks, peak_kind, None, None),
+        "roofline_note": "achieved per GPU: the job's algorithmic bytes / world over the step time",
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_cuda(args, w):
     import torch
     import torch.distributed as dist
@@ -383,6 +577,18 @@ def run_cuda(args, w):
 
     if args.profile_run and w.decode_steps:
         return profile_decode(args, w, dev, rank, distributed)
+    if args.shard == "heads":
+        return run_head_sharded(args, w, dev, stream, rank, world, local, distributed)
+    if args.profile_block:
+        # only the residual block's launches (RMSNorm, projections, core,
+        # MLP), warm-up then timed: the command an ncu launch list wraps
+        peaks0, kind0 = measured_peaks()
+        r = run_residual_block(args, dev, stream, distributed, peaks0, kind0)
+        if rank == 0:
+            print(json.dumps({"profile_block": r["workload"], "ms_per_step": r["ms_per_step"]}))
+        if distributed:
+            dist.destroy_process_group()
+        return 0
     case = PrefillCase(w, dev)
     for _ in range(args.warmup):
         case.step()
@@ -474,6 +680,17 @@ def run_cuda(args, w):
     dec = None
     if dec_setup is not None:
         dec = run_decode(dec_setup, counts[1], stream, distributed)
+        del dec_setup
+        torch.cuda.empty_cache()
+
+    # ---- the whole recurrent block (projections around the core)
+    blk = None
+    if not args.headline_only:
+        peaks0, kind0 = measured_peaks()
+        blk = run_block(args, dev, stream, distributed, peaks0, kind0)
+        torch.cuda.empty_cache()
+        blk["residual_block"] = run_residual_block(args, dev, stream, distributed, peaks0, kind0)
+        torch.cuda.empty_cache()
 
     if distributed:
         dist.barrier()
@@ -527,6 +744,8 @@ def run_cuda(args, w):
         line["prefill_workloads"] = rows
     if dec is not None:
         line["decode"] = dec
+    if blk is not None:
+        line["recurrent_block"] = blk
     if cpu_on:
         v, cores, sample = cpu_sample_run(w)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -648,6 +867,12 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-block", action="store_true",
+                    help="only the recurrent residual block's steps (the command an ncu launch list of "
+                         "the block kernels wraps)")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="none: one replica of the workload per GPU (weak scaling); heads: the workload's "
+                         "heads split across the GPUs (strong scaling)")
     ap.add_argument("--headline-only", action="store_true",
                     help="time only the headline prefill workload (not the other prefill workloads)")
     ap.add_argument("--profile-run", action="store_true",

@@ -321,6 +321,41 @@ RGLRU_API rglru_status rglru_recurrent_block_prefill(
     float *h_state, const void *W_out, const float *b_out, void *out, void *workspace, size_t workspace_bytes,
     cudaStream_t stream);
 
+/*
+ * RMSNorm of bf16 rows: out[m, :] = x[m, :] * rsqrt(mean_n(x[m, n]^2) + eps) * weight
+ * (x, out [M, N] bf16, weight [N] fp32, N a multiple of 8 up to 4096, eps > 0;
+ * out may equal x).  The decoder layer's temporal_pre_norm and
+ * channel_pre_norm (RecurrentGemmaRMSNorm in the printout; the pages give
+ * no formula, so this is the standard root-mean-square normalisation with a
+ * learned scale).
+ */
+RGLRU_API rglru_status rglru_rmsnorm(int M, int N, const void *x, const float *weight, float eps, void *out,
+                                     cudaStream_t stream);
+
+/* Workspace bytes of rglru_residual_block_prefill (0 on bad sizes). */
+RGLRU_API size_t rglru_residual_block_workspace_size(int B, int T, int D, int F);
+
+/*
+ * The recurrent residual block ("Residual block with recurrent block" and
+ * the decoder-layer printout) over T tokens of B sequences, bf16:
+ *   n   = RMSNorm(u) (w_temporal_norm)
+ *   h   = u + linear_out(GELU(linear_y(n)) * RG-LRU core(linear_x(n)))
+ *   n'  = RMSNorm(h) (w_channel_norm)
+ *   out = h + down_proj(GELU_tanh(gate_proj(n')) * up_proj(n'))
+ * u, out [B, T, D]; W_gate, W_up [F, D], W_down [D, F] bf16 (F = 3 D in the
+ * 2B model, MLP expansion factor 3); biases fp32; the recurrent block's
+ * parameters, segment_pos and states as rglru_recurrent_block_prefill.
+ * Every intermediate is a bf16 tensor in the workspace (zero-filled once),
+ * which carries one status word for all the launches.
+ */
+RGLRU_API rglru_status rglru_residual_block_prefill(
+    int B, int T, int D, int F, const void *u, const float *w_temporal_norm, const void *W_lin_x,
+    const float *b_lin_x, const void *W_lin_y, const float *b_lin_y, const float *conv_w, const float *conv_b,
+    const void *W_a, const float *b_a, const void *W_x, const float *b_x, const float *lambda, const void *W_out,
+    const float *b_out, const int32_t *segment_pos, void *conv_state, float *h_state, const float *w_channel_norm,
+    const void *W_gate, const float *b_gate, const void *W_up, const float *b_up, const void *W_down,
+    const float *b_down, float eps, void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

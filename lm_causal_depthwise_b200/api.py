@@ -26,7 +26,8 @@ SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglr
            "rglru_decode_step", "rglru_get_device_status", "rglru_debug_suppress_publish",
            "rglru_prefill_noalloc", "rglru_prefill_host_staging_size", "rglru_prefill_host",
            "rglru_linear_workspace_size", "rglru_linear", "rglru_linear_pair", "rglru_linear_residual",
-           "rglru_linear_geglu", "rglru_recurrent_block_workspace_size", "rglru_recurrent_block_prefill")
+           "rglru_linear_geglu", "rglru_recurrent_block_workspace_size", "rglru_recurrent_block_prefill",
+           "rglru_rmsnorm", "rglru_residual_block_workspace_size", "rglru_residual_block_prefill")
 
 _lib = None
 
@@ -87,6 +88,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_recurrent_block_workspace_size.argtypes = [i, i, i]
     lib.rglru_recurrent_block_prefill.restype = i
     lib.rglru_recurrent_block_prefill.argtypes = [i, i, i] + [vp] * 19 + [sz, vp]
+    lib.rglru_rmsnorm.restype = i
+    lib.rglru_rmsnorm.argtypes = [i, i, vp, vp, ctypes.c_float, vp, vp]
+    lib.rglru_residual_block_workspace_size.restype = sz
+    lib.rglru_residual_block_workspace_size.argtypes = [i, i, i, i]
+    lib.rglru_residual_block_prefill.restype = i
+    lib.rglru_residual_block_prefill.argtypes = [i, i, i, i] + [vp] * 25 + [ctypes.c_float, vp, vp, sz, vp]
     _lib = lib
     return lib
 
@@ -477,4 +484,99 @@ def recurrent_block_prefill(u, bp: BlockParams, segment_pos, conv_state, h_state
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
     if st != OK:
         raise RGLRUError(st, "rglru_recurrent_block_prefill")
+    return out
+
+
+def rmsnorm(x, weight, eps: float = 1e-6, out=None) -> torch.Tensor:
+    """out = x * rsqrt(mean(x^2) + eps) * weight over the last dimension (rglru_rmsnorm)."""
+    N = x.shape[-1]
+    M = x.numel() // N
+    _check(x, "x", x.shape, torch.bfloat16, x.device)
+    _check(weight, "weight", (N,), torch.float32, x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    _check(out, "out", x.shape, torch.bfloat16, x.device)
+    st = load().rglru_rmsnorm(M, N, _ptr(x), _ptr(weight), ctypes.c_float(eps), _ptr(out), _stream(x.device))
+    if st != OK:
+        raise RGLRUError(st, "rglru_rmsnorm")
+    return out
+
+
+@dataclass
+class ResidualBlockParams:
+    """The recurrent residual block: both RMSNorm scales, the recurrent block
+    and the MLP (gate/up [F, D], down [D, F] bf16; biases fp32)."""
+    w_temporal_norm: torch.Tensor
+    block: BlockParams
+    w_channel_norm: torch.Tensor
+    W_gate: torch.Tensor
+    b_gate: torch.Tensor
+    W_up: torch.Tensor
+    b_up: torch.Tensor
+    W_down: torch.Tensor
+    b_down: torch.Tensor
+
+    @staticmethod
+    def from_arrays(inp: dict, device="cuda") -> "ResidualBlockParams":
+        def w(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).to(torch.bfloat16).contiguous()
+
+        def f32(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).contiguous()
+        return ResidualBlockParams(f32(inp["w_temporal_norm"]), BlockParams.from_arrays(inp, device),
+                                   f32(inp["w_channel_norm"]), w(inp["W_gate"]), f32(inp["b_gate"]), w(inp["W_up"]),
+                                   f32(inp["b_up"]), w(inp["W_down"]), f32(inp["b_down"]))
+
+
+def residual_block_workspace_size(B: int, T: int, D: int, F: int) -> int:
+    n = int(load().rglru_residual_block_workspace_size(B, T, D, F))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "residual_block_workspace_size")
+    return n
+
+
+def residual_block_prefill(u, rp: ResidualBlockParams, segment_pos, conv_state, h_state, eps: float = 1e-6,
+                           out=None, workspace=None) -> torch.Tensor:
+    """The recurrent residual block over u [B,T,D] bf16 (rglru_residual_block_prefill)."""
+    if u.dim() != 3:
+        raise ValueError("u must be [B,T,D]")
+    B, T, D = u.shape
+    F = rp.W_gate.shape[0]
+    dev = u.device
+    _check(u, "u", (B, T, D), torch.bfloat16, dev)
+    _check(rp.w_temporal_norm, "w_temporal_norm", (D,), torch.float32, dev)
+    _check(rp.w_channel_norm, "w_channel_norm", (D,), torch.float32, dev)
+    _check(rp.W_gate, "W_gate", (F, D), torch.bfloat16, dev)
+    _check(rp.W_up, "W_up", (F, D), torch.bfloat16, dev)
+    _check(rp.W_down, "W_down", (D, F), torch.bfloat16, dev)
+    for n_, t in (("b_gate", rp.b_gate), ("b_up", rp.b_up)):
+        _check(t, n_, (F,), torch.float32, dev)
+    _check(rp.b_down, "b_down", (D,), torch.float32, dev)
+    bp, p = rp.block, rp.block.core
+    for n_ in ("W_lin_x", "W_lin_y", "W_out"):
+        _check(getattr(bp, n_), n_, (D, D), torch.bfloat16, dev)
+    for n_ in ("b_lin_x", "b_lin_y", "b_out"):
+        _check(getattr(bp, n_), n_, (D,), torch.float32, dev)
+    _check(p.conv_w, "conv_w", (4, D), torch.float32, dev)
+    for n_ in ("conv_b", "b_a", "b_x", "lam"):
+        _check(getattr(p, n_), n_, (D,), torch.float32, dev)
+    _check(p.W_a, "W_a", (D // 256, 256, 256), torch.bfloat16, dev)
+    _check(p.W_x, "W_x", (D // 256, 256, 256), torch.bfloat16, dev)
+    _check(segment_pos, "segment_pos", (B, T), torch.int32, dev)
+    _check(conv_state, "conv_state", (B, 3, D), torch.bfloat16, dev)
+    _check(h_state, "h_state", (B, D), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(u)
+    _check(out, "out", (B, T, D), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(residual_block_workspace_size(B, T, D, F), dev)
+    st = load().rglru_residual_block_prefill(
+        B, T, D, F, _ptr(u), _ptr(rp.w_temporal_norm), _ptr(bp.W_lin_x), _ptr(bp.b_lin_x), _ptr(bp.W_lin_y),
+        _ptr(bp.b_lin_y), _ptr(p.conv_w), _ptr(p.conv_b), _ptr(p.W_a), _ptr(p.b_a), _ptr(p.W_x), _ptr(p.b_x),
+        _ptr(p.lam), _ptr(bp.W_out), _ptr(bp.b_out), _ptr(segment_pos), _ptr(conv_state), _ptr(h_state),
+        _ptr(rp.w_channel_norm), _ptr(rp.W_gate), _ptr(rp.b_gate), _ptr(rp.W_up), _ptr(rp.b_up), _ptr(rp.W_down),
+        _ptr(rp.b_down), ctypes.c_float(eps), _ptr(out), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_residual_block_prefill")
     return out

@@ -1,5 +1,7 @@
-// block_api.cu -- C ABI of the dense projections and of the whole recurrent
-// block (linear_x / linear_y -> conv + RG-LRU core -> linear_out).
+// block_api.cu -- C ABI of the dense projections, RMSNorm, the whole
+// recurrent block (linear_x / linear_y -> conv + RG-LRU core -> linear_out)
+// and the whole recurrent residual block (RMSNorm, recurrent block, residual,
+// RMSNorm, GELU-gated MLP, residual).
 //
 // Structure: "Gemma explained: RecurrentGemma architecture", the
 // RecurrentGemmaRecurrentBlock printout (linear_y, linear_x, linear_out, each
@@ -184,6 +186,72 @@ RGLRU_API rglru_status rglru_recurrent_block_prefill(
                        conv_state, h_state, y, ws, core, stream);
     if (st != RGLRU_OK) return st;
     return rglru_linear(M, D, D, y, W_out, b_out, out, ws, kWsHeaderBytes, stream);
+}
+
+RGLRU_API rglru_status rglru_rmsnorm(int M, int N, const void *x, const float *weight, float eps, void *out,
+                                     cudaStream_t stream)
+{
+    if (M < 1 || N < 8 || N % 8 != 0 || (int64_t)M > kMaxRows || !(eps > 0.f)) return RGLRU_ERR_UNSUPPORTED;
+    if (!al16(x) || !al16(weight) || !al16(out)) return RGLRU_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)M * N * 2;
+    if (out != x && meet(span(out, bytes), span(x, bytes))) return RGLRU_ERR_INVALID_ARG;
+    if (meet(span(out, bytes), span(weight, (size_t)N * 4))) return RGLRU_ERR_INVALID_ARG;
+    return rmsnorm_launch(M, N, x, weight, eps, out, stream);
+}
+
+// Workspace of the residual block: the fused core's workspace first (its
+// header is shared by every launch), then x, the gate branch, the core's
+// output, the normalised rows, h (the recurrent block's residual output),
+// all [B, T, D] bf16, then the MLP's hidden rows [B, T, F] bf16.
+RGLRU_API size_t rglru_residual_block_workspace_size(int B, int T, int D, int F)
+{
+    const size_t core = rglru_workspace_size(B, T, D, RGLRU_IO_BF16);
+    if (core == 0 || F < 128 || F % 128 != 0 || F > (1 << 20)) return 0;
+    return align_up(core, 256) + 5 * align_up((size_t)B * T * D * 2, 256) + align_up((size_t)B * T * F * 2, 256);
+}
+
+RGLRU_API rglru_status rglru_residual_block_prefill(
+    int B, int T, int D, int F, const void *u, const float *w_temporal_norm, const void *W_lin_x,
+    const float *b_lin_x, const void *W_lin_y, const float *b_lin_y, const float *conv_w, const float *conv_b,
+    const void *W_a, const float *b_a, const void *W_x, const float *b_x, const float *lambda, const void *W_out,
+    const float *b_out, const int32_t *segment_pos, void *conv_state, float *h_state, const float *w_channel_norm,
+    const void *W_gate, const float *b_gate, const void *W_up, const float *b_up, const void *W_down,
+    const float *b_down, float eps, void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    const size_t need = rglru_residual_block_workspace_size(B, T, D, F);
+    if (need == 0) return RGLRU_ERR_INVALID_ARG;
+    if ((int64_t)B * T > kMaxRows || !(eps > 0.f)) return RGLRU_ERR_UNSUPPORTED;
+    if (workspace == nullptr || !al16(workspace) || workspace_bytes < need) return RGLRU_ERR_WORKSPACE;
+    const size_t act = (size_t)B * T * D * 2;
+    if (!al16(u) || !al16(out) || !al16(w_temporal_norm) || !al16(w_channel_norm)) return RGLRU_ERR_INVALID_ARG;
+    const Span ins[] = {span(u, act), span(workspace, workspace_bytes), span(conv_state, (size_t)B * 3 * D * 2),
+                        span(h_state, (size_t)B * D * 4), span(W_lin_x, (size_t)D * D * 2),
+                        span(W_lin_y, (size_t)D * D * 2), span(W_out, (size_t)D * D * 2),
+                        span(W_gate, (size_t)F * D * 2), span(W_up, (size_t)F * D * 2),
+                        span(W_down, (size_t)D * F * 2)};
+    for (const Span &s : ins)
+        if (meet(span(out, act), s)) return RGLRU_ERR_INVALID_ARG;
+    if (meet(span(u, act), span(workspace, workspace_bytes))) return RGLRU_ERR_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const size_t core = align_up(rglru_workspace_size(B, T, D, RGLRU_IO_BF16), 256);
+    const size_t a = align_up(act, 256);
+    void *x = ws + core, *g = ws + core + a, *y = ws + core + 2 * a, *n = ws + core + 3 * a, *h = ws + core + 4 * a;
+    void *m = ws + core + 5 * a;
+    const int M = B * T;
+    // temporal_pre_norm -> linear_x / linear_y -> conv + RG-LRU core -> linear_out + residual
+    rglru_status st = rglru_rmsnorm(M, D, u, w_temporal_norm, eps, n, stream);
+    if (st == RGLRU_OK)
+        st = rglru_linear_pair(M, D, D, n, W_lin_x, b_lin_x, x, W_lin_y, b_lin_y, g, ws, kWsHeaderBytes, stream);
+    if (st == RGLRU_OK)
+        st = rglru_prefill(B, T, D, RGLRU_IO_BF16, x, g, conv_w, conv_b, W_a, b_a, W_x, b_x, lambda, segment_pos,
+                           conv_state, h_state, y, ws, core, stream);
+    if (st == RGLRU_OK) st = rglru_linear_residual(M, D, D, y, W_out, b_out, u, h, ws, kWsHeaderBytes, stream);
+    // channel_pre_norm -> GELU-gated up projection -> down projection + residual
+    if (st == RGLRU_OK) st = rglru_rmsnorm(M, D, h, w_channel_norm, eps, n, stream);
+    if (st == RGLRU_OK)
+        st = rglru_linear_geglu(M, F, D, n, W_gate, b_gate, W_up, b_up, m, ws, kWsHeaderBytes, stream);
+    if (st == RGLRU_OK) st = rglru_linear_residual(M, D, F, m, W_down, b_down, h, out, ws, kWsHeaderBytes, stream);
+    return st;
 }
 
 }  // extern "C"

@@ -7,17 +7,18 @@
 // y[b, d] = GELU_tanh(g[b, d]) * h.  With one token per sequence the B rows of
 // a head are the token dimension of its gate GEMM.
 //
-// Grid: one cluster of two CTAs per (head, block of kTok batch rows); CTA rank r
-// owns channels [128 r, 128 r + 128) of the head.  Thread = one channel (its
-// TMEM lane) and 16 rows, for the conv and the epilogue alike:
+// Grid: one cluster of two CTAs per (head, block of kTok = 48 batch rows); CTA
+// rank r owns channels [128 r, 128 r + 128) of the head.  Thread = one channel
+// (its TMEM lane) and 16 rows, for the conv and the epilogue alike:
 //   1. one thread TMA-loads this half's x and conv_state tiles and its 128 rows
 //      of W_a and W_x (128-byte swizzled, K-major: the tensor core's A
 //      operands); every thread prefetches the h_state and GELU-branch values
 //      of its rows into registers;
 //   2. the conv of the thread's channel keeps xc / 2 in registers, writes its
-//      bf16 copy into the B tile of both CTAs of the cluster, and shifts the
-//      conv_state tile in shared memory (rows 1, 2, x become rows 0, 1, 2),
-//      which a TMA store writes back; a cluster barrier completes both B tiles;
+//      bf16 copy into this CTA's half of the B tile, and shifts the conv_state
+//      tile in shared memory (rows 1, 2, x become rows 0, 1, 2), which a TMA
+//      store writes back; one bulk copy sends the half to the peer CTA, whose
+//      mbarrier counts its bytes;
 //   3. one thread issues the 2 x 16 MMAs D[128 out x kTok rows] = W * xc^T;
 //   4. the epilogue applies the gates, a = sigmoid(Lambda)^(8 r), the
 //      normalised one-step update (a reset when segment_pos == 0) and the GELU
@@ -28,8 +29,9 @@
 // every other global access follows griddepcontrol.wait.
 // Each CTA reads and writes only its own channels of the states, so the two
 // CTAs never race.  Waits on mbarriers are bounded (RGLRU_ERR_TIMEOUT in the
-// workspace header); the two cluster barriers are reached exactly once by every
-// thread of both CTAs.
+// workspace header); the cluster barrier at set-up and the split one at the
+// end (arrive once the peer's copy has landed, wait before exiting) are reached
+// exactly once by every thread of both CTAs.
 //
 // Block structure: "Gemma explained: RecurrentGemma architecture",
 // RecurrentGemmaRecurrentBlock printout (Conv1d k=4, groups=D; GELU tanh) and
@@ -47,27 +49,31 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTok = 64;        // batch rows per cluster: the MMA N
+constexpr int kTok = 48;        // batch rows per cluster: the MMA N (B = 256: 6 blocks, 120 CTAs)
 constexpr int kHalfCh = 128;    // channels per CTA: the MMA M and TMEM lanes
-constexpr int kThreads = 512;   // 16 warps: lane quarter (warp & 3), row group (warp >> 2)
-constexpr int kRows = kTok / 4;  // rows per thread
+constexpr int kRows = 16;                  // rows per thread
+constexpr int kRowGroups = kTok / kRows;   // 3
+constexpr int kThreads = 128 * kRowGroups;  // 12 warps: lane quarter (warp & 3), row group (warp >> 2)
+static_assert(kTok % kRows == 0 && kTok % 16 == 0, "row blocks");
 
 constexpr int kWBlock = kHalfCh * 128;          // 128 weight rows x 64 channels (bf16): 16 KB
 constexpr int kWGate = 4 * kWBlock;             // one gate, K = 256: 64 KB
-constexpr int kBBlock = kTok * 128;             // kTok rows x 64 channels (bf16): 8 KB
-constexpr int kXTile = kTok * kHalfCh * 2;      // [kTok][128] bf16: 16 KB
-constexpr int kCsTile = 3 * kXTile;             // [kTok][3][128] bf16: 48 KB
+constexpr int kBBlock = kTok * 128;             // kTok rows x 64 channels (bf16): 6 KB
+static_assert(kBBlock % 1024 == 0, "B blocks are whole 128-byte swizzle atoms");
+constexpr int kXTile = kTok * kHalfCh * 2;      // [kTok][128] bf16: 12 KB
+constexpr int kCsTile = 3 * kXTile;             // [kTok][3][128] bf16: 36 KB
 constexpr int OFF_W = 0;                        // W_a rows, then W_x rows
 constexpr int OFF_B = OFF_W + 2 * kWGate;       // B tile: 4 K-blocks (all 256 channels of the head)
 constexpr int OFF_X = OFF_B + 4 * kBBlock;      // x tile, later the y tile
 constexpr int OFF_CS = OFF_X + kXTile;          // conv_state tile
 constexpr int OFF_SP = OFF_CS + kCsTile;        // segment_pos of the block's rows
-constexpr int OFF_BAR = OFF_SP + kTok * 4;      // x and conv_state loaded, W loaded, MMA done
+constexpr int OFF_BAR = OFF_SP + kTok * 4;      // x and conv_state loaded, W loaded, MMA done, peer's B half in
 constexpr int OFF_MISC = OFF_BAR + 4 * 8;       // TMEM base address
 constexpr int kSmemUsed = OFF_MISC + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;    // slack for the 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-constexpr uint32_t kTmemCols = 2 * kTok;        // D_r then D_i
+constexpr uint32_t kTmemCols = 128;             // D_r at column 0, D_i at column kTok (2 kTok <= 128)
+static_assert(2 * kTok <= (int)kTmemCols, "TMEM columns");
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Tracing (compiled in with -DRGLRU_TRACE only): CTAs below kTraceCtas record
@@ -158,6 +164,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const int nb = min(kTok, p.B - b0);                // valid rows of this block
     const int ch0 = head * 256 + (int)half * kHalfCh;  // first channel of this CTA
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(smem + OFF_BAR), *bar_w = bar_in + 1, *bar_mma = bar_in + 2;
+    uint64_t *bar_bx = bar_in + 3;  // the peer's half of the B tile has landed (bulk copy)
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     int32_t *sp_s = reinterpret_cast<int32_t *>(smem + OFF_SP);
     const __nv_bfloat16 *x_s = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_X);  // [kTok][128]
@@ -175,7 +182,10 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         mbar_init(bar_in, 1);
         mbar_init(bar_w, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_bx, 1);
         mbar_fence_init();
+        // the peer's 128 channels of the B tile arrive as one bulk copy
+        mbar_arrive_expect_tx(bar_bx, 2 * kBBlock);
         // this half's rows of W_a and W_x (parameters: read before the wait)
         mbar_arrive_expect_tx(bar_w, 2 * kWGate);
 #pragma unroll
@@ -224,7 +234,6 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     {
         const int k = (int)half * kHalfCh + c;  // channel within the head = K index of the B tile
         const uint32_t b_local = smem_u32(smem + OFF_B + (k >> 6) * kBBlock);
-        const uint32_t b_peer = mapa_shared(b_local, half ^ 1u);
         const int j = k & 63;
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
@@ -246,14 +255,19 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             const uint32_t off = n * 128 + (((j >> 3) ^ (n & 7)) << 4) + (j & 7) * 2;
             const uint16_t bv = __bfloat16_as_ushort(__float2bfloat16_rn(v));
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(b_local + off), "h"(bv) : "memory");
-            asm volatile("st.shared::cluster.b16 [%0], %1;" ::"r"(b_peer + off), "h"(bv) : "memory");
         }
     }
     if (tid == 0) DEC_TR(DT_CONV);
-    fence_proxy_async_cluster();  // B tiles (both CTAs) and the conv_state tile, for the async proxy
+    fence_proxy_async_smem();  // this half of the B tile and the conv_state tile, for the async proxy
     tc_fence_before();
-    cluster_sync();               // both halves of both B tiles written
+    __syncthreads();           // this CTA's half of the B tile written
     tc_fence_after();
+    if (tid == 32) {
+        // this half (K blocks 2 half, 2 half + 1: contiguous) into the peer's B tile
+        uint8_t *src = smem + OFF_B + (int)half * 2 * kBBlock;
+        bulk_copy_to_cluster(mapa_shared(smem_u32(src), half ^ 1u), src, 2 * kBBlock,
+                             mapa_shared(smem_u32(bar_bx), half ^ 1u));
+    }
     if (tid == 0) DEC_TR(DT_CLUSTER);
 
     // ---- 3. conv_state write-back and the gate projections
@@ -263,6 +277,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             bulk_commit();
         }
         ok = dec_wait(bar_w, 0, p.hdr, 1) && ok;
+        ok = dec_wait(bar_bx, 0, p.hdr, 3) && ok;  // the peer's half of the B tile
         if (lane == 0) DEC_TR(DT_WEIGHTS);
         if (ok && lane == 0) {
             tc_fence_after();
@@ -283,6 +298,15 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 
     // ---- 4. epilogue
     ok = dec_wait(bar_mma, 0, p.hdr, 2) && ok;
+    {
+        // the peer's copy into this CTA has landed (the MMA waited for it;
+        // bounded here for the timeout path): tell the peer, whose exit waits
+        // for it, and wait for the same news before this CTA exits
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar_bx, 0) && globaltimer() - t0 < kTimeoutNs) {
+        }
+        cluster_arrive();
+    }
     if (tid == 0) DEC_TR(DT_EPI0);
     tc_fence_after();
     __nv_bfloat16 *y_s = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_X);  // the x tile is dead
@@ -337,6 +361,7 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         }
         tmem_dealloc(tmem, kTmemCols);
     }
+    cluster_wait();  // this CTA's copy into the peer has landed before it exits
 }
 
 }  // namespace

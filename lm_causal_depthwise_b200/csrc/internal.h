@@ -21,9 +21,8 @@ struct WsHeader {
     int status;            // rglru_status recorded by device code (0 = OK)
     int detail;            // first wait that gave up: (CTA << 8) | (wait site + 1), 0 = none
     int debug_unit_plus1;  // test hook: chunk that skips publishing (+1), 0 = off
-    unsigned int epoch;    // fused prefill launches completed on this workspace (tags its scan carry)
-    unsigned int ticket[999];  // per-group work counters of the fused prefill kernel
-    unsigned int done_ctas;    // CTAs of the current fused launch that have finished
+    int pad0;
+    unsigned int ticket[1000];  // per-group work counters of the fused prefill kernel
 };
 constexpr size_t kWsHeaderBytes = 4096;
 static_assert(sizeof(WsHeader) <= kWsHeaderBytes, "header too large");
@@ -77,6 +76,9 @@ struct LinearArgs {
 };
 size_t linear_workspace_bytes();
 rglru_status linear_launch(const LinearArgs &a);
+
+// RMSNorm of bf16 rows (rmsnorm.cu): out = x * rsqrt(mean(x^2) + eps) * w.
+rglru_status rmsnorm_launch(int M, int N, const void *x, const float *w, float eps, void *out, cudaStream_t stream);
 
 // Batched decode step (decode.cu)
 size_t decode_workspace_bytes(int B, int D);

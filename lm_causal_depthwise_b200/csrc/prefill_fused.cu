@@ -153,8 +153,8 @@ struct FusedParams {
     __nv_bfloat16 *y;
     WsHeader *hdr;
     uint32_t *flags;   // [2 H][tiles_per_head]: one scan chain per (head, half)
-    uint64_t *agg;     // [2 H][tiles_per_head][128][2]  tagged (prod a), tagged h_end from h = 0
-    uint64_t *prefix;  // [2 H][tiles_per_head][128]     tagged h after the tile
+    float2 *agg;       // [2 H][tiles_per_head][128]  (prod a, h_end) from h = 0
+    float *prefix;     // [2 H][tiles_per_head][128]  h after the tile
     unsigned long long *trace;  // RGLRU_TRACE builds only: per-role timestamps
 };
 
@@ -237,75 +237,6 @@ __device__ __noinline__ uint32_t wait_flag(const uint32_t *f, uint32_t need, vol
     }
 }
 
-// A published float with the launch's tag in the upper half: a reader that
-// sees the tag sees the value (the 8-byte word is single-copy atomic), so the
-// scan carry crosses SMs with no fence between data and flag.
-__device__ __forceinline__ uint64_t tagged(float v, uint32_t tag)
-{
-    return ((uint64_t)tag << 32) | __float_as_uint(v);
-}
-__device__ __forceinline__ float untag(uint64_t w) { return __uint_as_float((uint32_t)w); }
-__device__ __forceinline__ bool has_tag(uint64_t w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
-
-// This lane's 4 channels of a tile's aggregate (A, H), spinning (bounded)
-// until every word carries `tag`; false on timeout or abort.
-__device__ __forceinline__ bool load_agg4(const uint64_t *src, uint32_t tag, float (&A)[4], float (&H)[4],
-                                       volatile int *abort_flag, WsHeader *hdr)
-{
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        uint64_t w[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ld_relaxed_v2_u64(src + 2 * e, w[2 * e], w[2 * e + 1]);
-        bool ok = true;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ok = ok && has_tag(w[e], tag);
-        if (ok) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                A[e] = untag(w[2 * e]);
-                H[e] = untag(w[2 * e + 1]);
-            }
-            return true;
-        }
-        if (t0 == 0) t0 = globaltimer();
-        __nanosleep(32);
-        if ((it & 31u) == 31u) {
-            if (*abort_flag || *(volatile int *)&hdr->status != 0) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
-                raise_timeout(abort_flag, hdr, 25);
-                return false;
-            }
-        }
-    }
-}
-
-// This lane's 4 channels of a tile's inclusive prefix (see load_agg4).
-__device__ __forceinline__ bool load_prefix4(const uint64_t *src, uint32_t tag, float (&h)[4], volatile int *abort_flag,
-                                          WsHeader *hdr)
-{
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        uint64_t w[4];
-        ld_relaxed_v2_u64(src, w[0], w[1]);
-        ld_relaxed_v2_u64(src + 2, w[2], w[3]);
-        if (has_tag(w[0], tag) && has_tag(w[1], tag) && has_tag(w[2], tag) && has_tag(w[3], tag)) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) h[e] = untag(w[e]);
-            return true;
-        }
-        if (t0 == 0) t0 = globaltimer();
-        __nanosleep(32);
-        if ((it & 31u) == 31u) {
-            if (*abort_flag || *(volatile int *)&hdr->status != 0) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
-                raise_timeout(abort_flag, hdr, 26);
-                return false;
-            }
-        }
-    }
-}
-
 // Warp-collective forms: lane 0 waits, the result is broadcast, then every lane
 // performs its own (already satisfied) acquire so that the warp stays converged
 // for the .sync.aligned tcgen05 instructions that follow.
@@ -355,9 +286,7 @@ __device__ __forceinline__ uint32_t warp_wait_flag(const uint32_t *f, uint32_t n
 // tile holding a reset (A = 0: its prefix is its own H) -- such that every tile
 // between the anchor and `hi` has published its aggregate.  Lane l examines
 // tile hi - l, so 32 flags cost one round trip.  The first tile of the
-// sequence is an anchor only once its prefix (or its reset) is out.  The
-// flags are hints (set without ordering): the words they announce carry the
-// launch's tag and are validated when read.
+// sequence is an anchor only once its prefix (or its reset) is out.
 // Warp-collective; false on timeout or abort.
 __device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_first, int &anchor,
                                          uint32_t &anchor_flag, volatile int *abort_flag, WsHeader *hdr)
@@ -367,7 +296,7 @@ __device__ __noinline__ bool find_anchor(const uint32_t *flags, int hi, int seq_
     for (uint32_t spins = 0;;) {
         const int pu = hi - lane;
         const bool in = pu >= seq_first;
-        const uint32_t f = in ? ld_relaxed_u32(flags + pu) : 0u;
+        const uint32_t f = in ? ld_acquire_u32(flags + pu) : 0u;
         const uint32_t anchors = __ballot_sync(0xffffffffu, in && (f & (F_PREFIX | F_RESET)));
         const uint32_t ready = __ballot_sync(0xffffffffu, in && (f & F_AGG));
         if (anchors) {
@@ -512,10 +441,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     }
 #endif
     const int debug_unit = *(volatile int *)&hdr->debug_unit_plus1 - 1;
-    // this launch's tag: one more than the launches completed on this
-    // workspace (the last CTA to finish advances the count), so no word
-    // left by an earlier launch can pass for this one's
-    const uint32_t tag = *(volatile unsigned int *)&hdr->epoch + 1u;
 
     if (warp == kSchedWarp) {
         // ------------------------------------------------------------ scheduler
@@ -533,8 +458,9 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // segment_pos loads issued together, so the round trips overlap the
         // x loads instead of pacing them.
         int k_pending = -1;  // lane 0: ticket of the next batch (atomic in flight)
+        const int nbatch = min(kClaimBatch, p.B);
         auto fetch = [&]() {
-            if (lane == 0 && !*abort_flag) k_pending = (int)atomicAdd(&hdr->ticket[head], (unsigned)kClaimBatch);
+            if (lane == 0 && !*abort_flag) k_pending = (int)atomicAdd(&hdr->ticket[head], (unsigned)nbatch);
             else if (lane == 0) k_pending = 0x3fffffff;  // past every ticket: no more tiles
         };
         TileInfo batch[kClaimBatch];
@@ -549,7 +475,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                 TileInfo ti{};
                 ti.u = -1;
                 sp[q] = 3;
-                if (k >= 0 && k < p.tiles_per_head) {
+                if (q < nbatch && k >= 0 && k < p.tiles_per_head) {
                     ti.b = k % p.B;
                     const int c = k / p.B;
                     ti.u = ti.b * p.C + c;
@@ -569,7 +495,7 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             batch_i = 0;
         };
         auto claim = [&]() -> TileInfo {
-            if (batch_i == kClaimBatch) claim_batch();
+            if (batch_i >= nbatch) claim_batch();
             TileInfo ti{};
 #pragma unroll
             for (int q = 0; q < kClaimBatch; ++q)
@@ -987,12 +913,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
         // may combine it before this tile's own look-back has finished), find
         // the anchor, fold, publish the inclusive prefix, then pass 2 of the
         // tile: y = y_loc + q h_in from the stash, 4 channels per lane, and at
-        // a sequence end the new states.  Aggregates and prefixes go out as
-        // tagged words with no fence; only the first tile of a sequence
-        // publishes its prefix with release (for the state write-back).
+        // a sequence end the new states.  These warps are the only ones that
+        // fence for the aggregates and prefixes.
         const int ch = lane * 4;  // 4 channels per lane
         const size_t dch = (size_t)ch0 + ch;
         const size_t gbase = (size_t)group * p.tiles_per_head;
+        constexpr int kFoldBatch = 4;  // aggregates loaded per round trip
 #pragma unroll 1
         for (int j = warp - kLbWarp0;; j += kLbWarps) {
             const int ss = j % NS, ir = j % INFO_RING;
@@ -1009,12 +935,12 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
             const uint32_t rbit = ti.reset_mask ? F_RESET : 0u;
             const bool suppress = (int)gu == debug_unit;
             if (!suppress) {
-                // tagged words, no fence: the flag only tells readers where to look
-                uint64_t *dst = p.agg + (gu * kHalf + ch) * 2;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) st_relaxed_v2_u64(dst + 2 * e, tagged(A[e], tag), tagged(Hh[e], tag));
+                float4 *dst = reinterpret_cast<float4 *>(p.agg + gu * kHalf + ch);
+                dst[0] = g01;
+                dst[1] = g23;
+                __threadfence();
                 __syncwarp();
-                if (lane == 0) red_relaxed_or_u32(p.flags + gu, F_AGG | rbit);
+                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | rbit);
             }
             float hin[4];
             bool ok = true;
@@ -1034,49 +960,35 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
                     // sequence order from the anchor, the same order whichever
                     // prefixes happened to be published (bit-reproducible)
                     if (aflag & F_PREFIX) {
-                        ok = load_prefix4(p.prefix + (gbase + anchor) * kHalf + ch, tag, hin, abort_flag, hdr);
+                        const float4 pr = ld_relaxed_f4(reinterpret_cast<const float4 *>(p.prefix + (gbase + anchor) * kHalf + ch));
+                        hin[0] = pr.x; hin[1] = pr.y; hin[2] = pr.z; hin[3] = pr.w;
                     } else {  // a tile holding a reset: A = 0, its prefix is its H
-                        float a4[4];
-                        ok = load_agg4(p.agg + ((gbase + anchor) * kHalf + ch) * 2, tag, a4, hin, abort_flag, hdr);
+                        const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + anchor) * kHalf + ch);
+                        const float4 a01 = ld_relaxed_f4(src), a23 = ld_relaxed_f4(src + 1);
+                        hin[0] = a01.y; hin[1] = a01.w; hin[2] = a23.y; hin[3] = a23.w;
                     }
 #pragma unroll 1
-                    for (int p0 = anchor + 1; ok && p0 < ti.u; p0 += 2) {
-                        // two aggregates per round trip when both are visible
-                        const uint64_t *s0 = p.agg + ((gbase + p0) * kHalf + ch) * 2;
-                        const bool two = p0 + 1 < ti.u;
-                        uint64_t w[16];
+                    for (int p0 = anchor + 1; p0 < ti.u; p0 += kFoldBatch) {
+                        float4 dd[kFoldBatch][2];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) ld_relaxed_v2_u64(s0 + 2 * e, w[2 * e], w[2 * e + 1]);
-                        if (two) {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                ld_relaxed_v2_u64(s0 + kHalf * 2 + 2 * e, w[8 + 2 * e], w[8 + 2 * e + 1]);
-                        }
-                        bool seen = true;
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) seen = seen && (has_tag(w[e], tag) || (e >= 8 && !two));
-                        float a4[4], h4[4];
-                        if (seen) {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) hin[e] = fmaf(untag(w[2 * e]), hin[e], untag(w[2 * e + 1]));
-                            if (two) {
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    hin[e] = fmaf(untag(w[8 + 2 * e]), hin[e], untag(w[8 + 2 * e + 1]));
+                        for (int k = 0; k < kFoldBatch; ++k) {
+                            if (p0 + k < ti.u) {
+                                const float4 *src = reinterpret_cast<const float4 *>(p.agg + (gbase + p0 + k) * kHalf + ch);
+                                dd[k][0] = ld_relaxed_f4(src);
+                                dd[k][1] = ld_relaxed_f4(src + 1);
                             }
-                        } else {
-                            ok = load_agg4(s0, tag, a4, h4, abort_flag, hdr);
+                        }
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) hin[e] = fmaf(a4[e], hin[e], h4[e]);
-                            if (ok && two) {
-                                ok = load_agg4(s0 + kHalf * 2, tag, a4, h4, abort_flag, hdr);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) hin[e] = fmaf(a4[e], hin[e], h4[e]);
+                        for (int k = 0; k < kFoldBatch; ++k) {
+                            if (p0 + k < ti.u) {
+                                hin[0] = fmaf(dd[k][0].x, hin[0], dd[k][0].y);
+                                hin[1] = fmaf(dd[k][0].z, hin[1], dd[k][0].w);
+                                hin[2] = fmaf(dd[k][1].x, hin[2], dd[k][1].y);
+                                hin[3] = fmaf(dd[k][1].z, hin[3], dd[k][1].w);
                             }
                         }
                     }
                 }
-                ok = __all_sync(0xffffffffu, ok);
             }
             if (!ok) break;
             if (lane == 0) RGLRU_TR(TR_LB_HIN, j, globaltimer());
@@ -1084,20 +996,10 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
 #pragma unroll
             for (int e = 0; e < 4; ++e) pre[e] = fmaf(A[e], hin[e], Hh[e]);
             if (!suppress) {
-                uint64_t *dst = p.prefix + gu * kHalf + ch;
-                st_relaxed_v2_u64(dst, tagged(pre[0], tag), tagged(pre[1], tag));
-                st_relaxed_v2_u64(dst + 2, tagged(pre[2], tag), tagged(pre[3], tag));
-                if (ti.first_last & 1) {
-                    // the sequence's last tile overwrites the states this first
-                    // tile has read: it waits for this flag with acquire, so this
-                    // one publish is a release
-                    __threadfence();
-                    __syncwarp();
-                    if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
-                } else {
-                    __syncwarp();
-                    if (lane == 0) red_relaxed_or_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
-                }
+                *reinterpret_cast<float4 *>(p.prefix + gu * kHalf + ch) = make_float4(pre[0], pre[1], pre[2], pre[3]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atom_or_release_u32(p.flags + gu, F_AGG | F_PREFIX | rbit);
             }
             if (lane == 0) RGLRU_TR(TR_P2_START, j, globaltimer());
             // pass 2: token t of this lane's 4 channels is one 16-byte stash word;
@@ -1158,7 +1060,6 @@ rglru_prefill_fused_kernel(const FusedParams p, const __grid_constant__ CUtensor
     cluster_sync();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
-    if (threadIdx.x == 0 && atomicAdd(&hdr->done_ctas, 1u) == gridDim.x - 1) atomicExch(&hdr->epoch, tag);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1178,8 +1079,8 @@ Layout layout_of(int B, int T, int D)
     L.flags_off = kWsHeaderBytes;
     L.flags_bytes = align_up(tiles * 4, 256);
     L.agg_off = L.flags_off + L.flags_bytes;
-    L.prefix_off = L.agg_off + align_up(tiles * kHalf * 16, 256);
-    L.total = L.prefix_off + align_up(tiles * kHalf * 8, 256);
+    L.prefix_off = L.agg_off + align_up(tiles * kHalf * 8, 256);
+    L.total = L.prefix_off + align_up(tiles * kHalf * 4, 256);
 #ifdef RGLRU_TRACE
     L.trace_off = L.total;
     L.total += align_up((size_t)kTraceCtas * kTraceTiles * kTraceEvents * 8, 256);
@@ -1228,8 +1129,7 @@ rglru_status fused_prefill(const PrefillArgs &a)
     if (st != RGLRU_OK) return st;
 
     char *ws = static_cast<char *>(a.ws);
-    // tickets, the finished-CTA count and the flags start at zero; the status
-    // word, the test hook and the launch count are kept
+    // tickets and flags start at zero; the status word and the test hook are kept
     if (cudaMemsetAsync(ws + offsetof(WsHeader, ticket), 0,
                         L.flags_off - offsetof(WsHeader, ticket) + L.flags_bytes, a.stream) != cudaSuccess)
         return RGLRU_ERR_CUDA;
@@ -1248,8 +1148,8 @@ rglru_status fused_prefill(const PrefillArgs &a)
     p.y = static_cast<__nv_bfloat16 *>(a.y);
     p.hdr = reinterpret_cast<WsHeader *>(ws);
     p.flags = reinterpret_cast<uint32_t *>(ws + L.flags_off);
-    p.agg = reinterpret_cast<uint64_t *>(ws + L.agg_off);
-    p.prefix = reinterpret_cast<uint64_t *>(ws + L.prefix_off);
+    p.agg = reinterpret_cast<float2 *>(ws + L.agg_off);
+    p.prefix = reinterpret_cast<float *>(ws + L.prefix_off);
     p.trace = L.trace_off ? reinterpret_cast<unsigned long long *>(ws + L.trace_off) : nullptr;
 
     // one cluster of two CTAs (the two halves of a head) per SM pair; the same

@@ -70,9 +70,8 @@ extern "C" RGLRU_API rglru_status rglru_prefill_noalloc(int B, int T, int D, rgl
     const rglru_status st = scratch_address(&scratch);
     if (st != RGLRU_OK) return st;
     // status word, wait record and test hook from any earlier call back to zero
-    // (the prefill itself zeroes the tickets and the tile flags; the launch
-    // counter that tags the scan carry is kept)
-    if (cudaMemsetAsync(scratch, 0, 3 * sizeof(int), stream) != cudaSuccess) return RGLRU_ERR_CUDA;
+    // (the prefill itself zeroes the tickets and the tile flags)
+    if (cudaMemsetAsync(scratch, 0, 4 * sizeof(int), stream) != cudaSuccess) return RGLRU_ERR_CUDA;
     return rglru_prefill(B, T, D, dt, x, gate_branch, conv_w, conv_b, W_a, b_a, W_x, b_x, lambda, segment_pos,
                          conv_state, h_state, y, scratch, kNoAllocScratchBytes, stream);
 }

@@ -148,10 +148,7 @@ template <typename IO>
 rglru_status launch(const PrefillArgs &a)
 {
     const size_t n = (size_t)a.B * a.T * a.D;
-    // the intermediates sit past the fused prefill's region of the same shape,
-    // so a workspace shared by both paths never holds stray words where the
-    // fused kernel looks for its tagged scan carry
-    char *base = static_cast<char *>(a.ws) + align_up(fused_workspace_bytes(a.B, a.T, a.D), 256);
+    char *base = static_cast<char *>(a.ws) + kWsHeaderBytes;
     float *xc_ws = reinterpret_cast<float *>(base);
     float *pr_ws = xc_ws + n;
     float *pi_ws = pr_ws + n;
@@ -173,7 +170,7 @@ rglru_status launch(const PrefillArgs &a)
 
 size_t simt_workspace_bytes(int B, int T, int D)
 {
-    return align_up(fused_workspace_bytes(B, T, D), 256) + align_up(3 * (size_t)B * T * D * sizeof(float), 256);
+    return kWsHeaderBytes + align_up(3 * (size_t)B * T * D * sizeof(float), 256);
 }
 
 rglru_status simt_prefill(const PrefillArgs &a)

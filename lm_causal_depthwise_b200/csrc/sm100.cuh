@@ -124,27 +124,6 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// Relaxed (strong, unordered) GPU-scope accesses for self-validating words:
-// each 8-byte element of a v2.b64 access is single-copy atomic, so a reader
-// that sees a word's tag also sees the value stored with it.
-__device__ __forceinline__ void red_relaxed_or_u32(uint32_t *p, uint32_t v)
-{
-    asm volatile("red.relaxed.gpu.global.or.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_relaxed_v2_u64(uint64_t *p, uint64_t a, uint64_t b)
-{
-    asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
-}
-__device__ __forceinline__ void ld_relaxed_v2_u64(const uint64_t *p, uint64_t &a, uint64_t &b)
-{
-    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
-}
 __device__ __forceinline__ float4 ld_relaxed_f4(const float4 *p)
 {
     float4 v;
@@ -408,6 +387,15 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v)
 __device__ __forceinline__ void fence_proxy_async_cluster()
 {
     asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+// the two halves of cluster_sync, for a barrier whose wait comes later
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // all threads of all CTAs of the cluster; release/acquire for shared memory
 __device__ __forceinline__ void cluster_sync()

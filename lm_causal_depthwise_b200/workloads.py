@@ -222,3 +222,35 @@ def generate_block(w: Workload) -> dict:
 def block_gemm_flops(w: Workload) -> int:
     """Dense flops of the block's three D x D projections over its tokens."""
     return 3 * 2 * w.tokens * w.D * w.D
+
+
+MLP_EXPANSION = 3  # MLP width 3 D (7680 for D = 2560)
+
+
+def generate_residual_block(w: Workload) -> dict:
+    """Inputs of the whole recurrent residual block: ``generate_block(w)`` plus,
+    from ``default_rng((seed, 2))`` in this order:
+      w_temporal_norm, w_channel_norm [D] ~ 1 + N(0, 0.01)   fp32 (RMSNorm scales)
+      W_gate, W_up [F, D] ~ N(0, 1/D), b_gate, b_up [F] ~ N(0, 0.1)
+      W_down [D, F] ~ N(0, 1/F),      b_down [D]       ~ N(0, 0.1)
+    with F = 3 D (bf16 weights, fp32 biases)."""
+    inp = generate_block(w)
+    rng = np.random.default_rng((w.seed, 2))
+    D = w.D
+    F = MLP_EXPANSION * D
+    inp["w_temporal_norm"] = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    inp["w_channel_norm"] = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    inp["W_gate"] = round_bf16((rng.standard_normal((F, D)) / np.sqrt(D)).astype(np.float32))
+    inp["b_gate"] = (np.sqrt(0.1) * rng.standard_normal(F)).astype(np.float32)
+    inp["W_up"] = round_bf16((rng.standard_normal((F, D)) / np.sqrt(D)).astype(np.float32))
+    inp["b_up"] = (np.sqrt(0.1) * rng.standard_normal(F)).astype(np.float32)
+    inp["W_down"] = round_bf16((rng.standard_normal((D, F)) / np.sqrt(F)).astype(np.float32))
+    inp["b_down"] = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
+    return inp
+
+
+def residual_block_gemm_flops(w: Workload) -> int:
+    """Dense flops of the residual block: three D x D projections and the
+    MLP's three D x 3D ones."""
+    F = MLP_EXPANSION * w.D
+    return 2 * w.tokens * (3 * w.D * w.D + 3 * w.D * F)

@@ -16,6 +16,12 @@ RecurrentGemma architecture"):
     bias=True) each (MLP expansion factor 3, section "MLP expansion
     factor"); the tanh GELU (PytorchGELUTanh) on the gate; their product
     feeds down_proj, Linear(3 D, D, bias=True).
+  * The decoder layer (printout: temporal_pre_norm, temporal block,
+    channel_pre_norm, mlp_block; section "Residual block with recurrent
+    block"): RMSNorm, the recurrent block, a residual add, RMSNorm, the MLP,
+    a residual add.  The pages name RecurrentGemmaRMSNorm without a formula;
+    this is the standard root-mean-square normalisation with a learned scale,
+    x / sqrt(mean(x^2) + eps) * w (reading stated here; eps = 1e-6).
 
 A Linear layer is ``y = x W^T + b`` with W stored [out, in] (torch's layout,
 the one the printout's modules use).  The product with numpy's matmul in
@@ -80,3 +86,29 @@ def mlp(v, W_gate, b_gate, W_up, b_up, W_down, b_down, round_io: bool = True) ->
     rnd = round_bf16 if round_io else (lambda a: np.asarray(a, np.float64))
     h = rnd(gelu_tanh(linear(v, W_gate, b_gate)) * linear(v, W_up, b_up))
     return rnd(linear(h, W_down, b_down))
+
+
+def rmsnorm(x, w, eps: float = 1e-6) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * w over the last axis, float64."""
+    x = np.asarray(x, np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * np.asarray(w, np.float64)
+
+
+def residual_block(u, w_temporal_norm, W_lin_x, b_lin_x, W_lin_y, b_lin_y, W_out, b_out, conv_w, conv_b, W_a,
+                   b_a, W_x, b_x, lam, segpos, conv_state, h_state, w_channel_norm, W_gate, b_gate, W_up, b_up,
+                   W_down, b_down, eps: float = 1e-6, round_io: bool = True) -> dict:
+    """The recurrent residual block over u [B, T, D] in float64, each layer's
+    output rounded to bf16 once (``round_io``): returns out, the new states and
+    the intermediates n (normalised u), h (after the first residual add)."""
+    rnd = round_bf16 if round_io else (lambda a: np.asarray(a, np.float64))
+    u = np.asarray(u, np.float64)
+    n = rnd(rmsnorm(u, w_temporal_norm, eps))
+    x = rnd(linear(n, W_lin_x, b_lin_x))
+    g = rnd(linear(n, W_lin_y, b_lin_y))
+    c = core.prefill(x, g, conv_w, conv_b, W_a, b_a, W_x, b_x, lam, segpos, conv_state, h_state)
+    y = rnd(c["y"])
+    h = rnd(linear(y, W_out, b_out) + u)
+    n2 = rnd(rmsnorm(h, w_channel_norm, eps))
+    m = rnd(gelu_tanh(linear(n2, W_gate, b_gate)) * linear(n2, W_up, b_up))
+    out = rnd(linear(m, W_down, b_down) + h)
+    return {"out": out, "conv_state": c["conv_state"], "h_state": c["h_state"], "n": n, "h": h}

@@ -73,3 +73,65 @@ def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
     args = argparse.Namespace(steps=1, warmup=0)
     assert bench.run_reference(args, W.TINY_F32) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_shard_heads_covers_every_head_once():
+    sys.path.insert(0, ROOT)
+    from lm_causal_depthwise_b200.sharding import shard_heads
+    for H in (1, 10, 16):
+        for world in (1, 2, 3, 4, 8, 12):
+            got = [shard_heads(H, world, r) for r in range(world)]
+            heads = [h for a, b in got for h in range(a, b)]
+            assert heads == list(range(H))
+            sizes = [b - a for a, b in got]
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+
+
+def _shard_rank_main(rank: int, world: int, port: int, out_dir: str):
+    """Each gloo rank slices its heads of one workload and times a fake step;
+    the job's throughput counts the tokens once (strong scaling)."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+
+    import numpy as np
+    import torch.distributed as dist
+
+    import bench
+    from lm_causal_depthwise_b200 import workloads as W
+    from lm_causal_depthwise_b200.sharding import shard_heads, shard_inputs
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = W.Workload("s", B=2, T=40, D=768, io="bf16", seed=3, init_state="random")
+        inp = W.generate(w)
+        h0, h1 = shard_heads(w.H, world, rank)
+        part = shard_inputs(inp, h0, h1)
+        ms = bench.max_over_ranks(1.0 + rank)
+        value = bench.sharded_throughput(w.tokens, ms)
+        np.save(os.path.join(out_dir, f"x{rank}.npy"), part["x"])
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"h": [h0, h1], "ms": ms, "value": value}, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_job_gloo(tmp_path):
+    """Two ranks take heads [0, 2) and [2, 3) of a 3-head workload; their
+    slices of x put back together are the whole x, and the job's time is the
+    slower rank's."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    from lm_causal_depthwise_b200 import workloads as W
+    world = 2
+    mp.start_processes(_shard_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    got = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert [g["h"] for g in got] == [[0, 2], [2, 3]]
+    for g in got:
+        assert g["ms"] == pytest.approx(2.0)
+        assert g["value"] == pytest.approx(2 * 40 / 2.0e-3)
+    whole = W.generate(W.Workload("s", B=2, T=40, D=768, io="bf16", seed=3, init_state="random"))["x"]
+    parts = [np.load(tmp_path / f"x{r}.npy") for r in range(world)]
+    np.testing.assert_array_equal(np.concatenate(parts, axis=2), whole)

@@ -84,3 +84,43 @@ def test_mlp_matches_torch_modules():
     want = F_.linear(F_.gelu(F_.linear(t["v"], t["Wg"], t["bg"]), approximate="tanh")
                      * F_.linear(t["v"], t["Wu"], t["bu"]), t["Wd"], t["bd"]).numpy()
     np.testing.assert_allclose(block.mlp(v, Wg, bg, Wu, bu, Wd, bd, round_io=False), want, rtol=1e-12, atol=1e-12)
+
+
+def test_rmsnorm_matches_torch():
+    rng = np.random.default_rng(7)
+    x, w = rng.standard_normal((6, 40)) * 3.0, rng.standard_normal(40)
+    want = torch.nn.functional.rms_norm(torch.from_numpy(x), (40,), torch.from_numpy(w), eps=1e-6).numpy()
+    np.testing.assert_allclose(block.rmsnorm(x, w, 1e-6), want, rtol=1e-13, atol=1e-13)
+    # a constant row normalises to w (sign kept): x / |x| * w
+    np.testing.assert_allclose(block.rmsnorm(np.full((1, 40), -2.5), w, 0.0)[0], -w, rtol=1e-15)
+
+
+def _res_args(inp):
+    keys = ("u", "w_temporal_norm", "W_lin_x", "b_lin_x", "W_lin_y", "b_lin_y", "W_out", "b_out", "conv_w",
+            "conv_b", "W_a", "b_a", "W_x", "b_x", "lam", "segpos", "conv_state", "h_state", "w_channel_norm",
+            "W_gate", "b_gate", "W_up", "b_up", "W_down", "b_down")
+    return [inp[k] for k in keys]
+
+
+def test_residual_block_wiring():
+    """Zero linear_out and down_proj (weights and biases): both residual adds
+    pass their input through, out = u.  Zero down_proj only: out = h, the
+    recurrent block's residual output, which equals u + the recurrent block
+    applied to RMSNorm(u)."""
+    w = W.Workload("pin", B=1, T=30, D=256, io="bf16", seed=8, init_state="zero")
+    inp = W.generate_residual_block(w)
+    z = dict(inp)
+    z["W_out"] = np.zeros_like(inp["W_out"]); z["b_out"] = np.zeros_like(inp["b_out"])
+    z["W_down"] = np.zeros_like(inp["W_down"]); z["b_down"] = np.zeros_like(inp["b_down"])
+    np.testing.assert_array_equal(block.residual_block(*_res_args(z))["out"], inp["u"])
+    z2 = dict(inp)
+    z2["W_down"] = z["W_down"]; z2["b_down"] = z["b_down"]
+    o = block.residual_block(*_res_args(z2))
+    n = block.round_bf16(block.rmsnorm(inp["u"], inp["w_temporal_norm"]))
+    rb = block.recurrent_block(n, inp["W_lin_x"], inp["b_lin_x"], inp["W_lin_y"], inp["b_lin_y"],
+                               np.zeros_like(inp["W_out"]), np.zeros(256), inp["conv_w"], inp["conv_b"],
+                               inp["W_a"], inp["b_a"], inp["W_x"], inp["b_x"], inp["lam"], inp["segpos"],
+                               inp["conv_state"], inp["h_state"])
+    want_h = block.round_bf16(block.linear(rb["y"], inp["W_out"], inp["b_out"]) + inp["u"])
+    np.testing.assert_array_equal(o["h"], want_h)
+    np.testing.assert_array_equal(o["out"], want_h)

@@ -339,3 +339,22 @@ def test_prefill_from_host_buffers_equals_device_call(io, rows):
     np.testing.assert_array_equal(dev["h_state"].cpu().numpy(), want["h_state"])
     ref = run_oracle(inp)
     check(io, hy.float().numpy(), ref["y"], "y")
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_shards_equal_the_whole_run(world):
+    """The core run on each rank's head range (run one after another here, on
+    one GPU) gives the whole run's output column blocks and states bit for bit:
+    heads never mix and each head's result does not depend on the others."""
+    from lm_causal_depthwise_b200.sharding import shard_heads, shard_inputs
+    _, inp = _case(2, 700, 768, doc_len=250)
+    whole = run_gpu(to_device(inp, "bf16"))
+    for r in range(world):
+        h0, h1 = shard_heads(3, world, r)
+        if h1 == h0:
+            continue
+        got = run_gpu(to_device(shard_inputs(inp, h0, h1), "bf16"))
+        c = slice(h0 * 256, h1 * 256)
+        np.testing.assert_array_equal(got["y"], whole["y"][:, :, c])
+        np.testing.assert_array_equal(got["h_state"], whole["h_state"][:, c])
+        np.testing.assert_array_equal(got["conv_state"], whole["conv_state"][:, :, c])
