@@ -1,0 +1,87 @@
+"""float64 CPU oracle of the local sliding-window MQA temporal block --
+TEST INFRASTRUCTURE (only tests/, the smoke check and the benchmark's
+CPU-baseline leg may import it; the product path never does).
+
+What it computes, from "Gemma explained: RecurrentGemma architecture", the
+RecurrentGemmaSdpaAttention printout (q_proj Linear(2560, 2560, bias=False),
+k_proj and v_proj Linear(2560, 256, bias=False), o_proj Linear(2560, 2560,
+bias=True), rotary_emb) and section "Residual block with local MQA" (10 query
+heads of 256 share one key/value head of 256; local sliding-window attention
+lets each position attend only a fixed number of past tokens; the window is
+2k tokens, section "Local attention window size"; RoPE as in the base Gemma
+model).
+
+Readings where the pages are silent (stated here and in the design notes):
+  * RoPE: the rotate-half form on the full head dimension, frequencies
+    base^(-2i/d) for i < d/2 with base 10000, rotating the pairs
+    (x[i], x[i + d/2]); the position of a token is its position inside its
+    document (segment_pos), so a document starts at position 0.
+  * Scores are scaled by 1/sqrt(d) (d = 256) before the softmax.
+  * Query t attends key s when t - W < s <= t (W = 2048, itself included) and
+    s lies in t's document (s >= t - segment_pos[t]).
+  * In bf16 I/O every tensor between layers (q, k, v after RoPE, the
+    attention output, the block output) is bf16: rounded once, here as on the
+    GPU.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import block
+
+HEAD = 256
+WINDOW = 2048
+ROPE_BASE = 10000.0
+
+
+def rope(x, pos, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotate-half RoPE of x [..., T, n, d] (or [..., T, d]) at positions pos
+    [..., T]: pairs (x[i], x[i + d/2]) rotated by pos * base^(-2i/d)."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    inv = base ** (-np.arange(half, dtype=np.float64) * 2.0 / d)
+    ang = np.asarray(pos, np.float64)[..., None] * inv          # [..., T, half]
+    if x.ndim == ang.ndim + 1:                                   # a head axis between T and d
+        ang = ang[..., None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def attention(q, k, v, segpos, window: int = WINDOW) -> np.ndarray:
+    """Local MQA: q [B, T, H, d], k and v [B, T, d], segpos [B, T] ->
+    [B, T, H, d].  Query t attends keys s with t - window < s <= t inside t's
+    document, scores scaled by 1/sqrt(d), softmax over those keys."""
+    q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+    B, T, H, d = q.shape
+    out = np.empty_like(q)
+    idx = np.arange(T)
+    for b in range(B):
+        start = idx - np.asarray(segpos[b], np.int64)              # document start of each query
+        lo = np.maximum(start, idx - window + 1)
+        for t in range(T):
+            ks = k[b, lo[t]:t + 1]                                  # [n, d]
+            vs = v[b, lo[t]:t + 1]
+            sc = q[b, t] @ ks.T / np.sqrt(d)                        # [H, n]
+            sc = sc - sc.max(axis=1, keepdims=True)
+            p = np.exp(sc)
+            out[b, t] = (p / p.sum(axis=1, keepdims=True)) @ vs
+    return out
+
+
+def mqa_block(u, W_q, W_k, W_v, W_o, b_o, segpos, window: int = WINDOW, round_io: bool = True) -> dict:
+    """The local MQA temporal block over u [B, T, D]: projections (q_proj,
+    k_proj, v_proj without bias), RoPE on q and k, local attention, o_proj
+    with bias.  Returns out and the intermediates q, k, v (after RoPE) and a
+    (the attention output)."""
+    rnd = block.round_bf16 if round_io else (lambda a: np.asarray(a, np.float64))
+    u = np.asarray(u, np.float64)
+    B, T, D = u.shape
+    H = np.asarray(W_q).shape[0] // HEAD
+    q = rnd(rope(block.linear(u, W_q).reshape(B, T, H, HEAD), segpos))
+    k = rnd(rope(block.linear(u, W_k), segpos))
+    v = rnd(block.linear(u, W_v))
+    a = rnd(attention(q, k, v, segpos, window))
+    out = rnd(block.linear(a.reshape(B, T, H * HEAD), W_o, b_o))
+    return {"out": out, "q": q, "k": k, "v": v, "a": a}

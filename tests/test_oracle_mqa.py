@@ -1,0 +1,69 @@
+"""Pins of the local MQA oracle (oracle/mqa.py) against facts from outside it:
+RoPE as a complex rotation, attention against torch's float64
+scaled_dot_product_attention with an explicit mask and against a brute-force
+loop, and the window and document limits by perturbation."""
+import numpy as np
+import torch
+
+from oracle import mqa
+
+
+def test_rope_is_a_complex_rotation():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((5, 3, 16))
+    pos = np.array([0, 1, 7, 100, 3])
+    got = mqa.rope(x, pos, base=100.0)
+    z = x[..., :8] + 1j * x[..., 8:]
+    theta = pos[:, None, None] * 100.0 ** (-np.arange(8) * 2.0 / 16)
+    w = z * np.exp(1j * theta)
+    np.testing.assert_allclose(got, np.concatenate([w.real, w.imag], axis=-1), rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(mqa.rope(x[:1], [0]), x[:1])      # position 0: no rotation
+    # rotations preserve norms and relative position: <R(p)q, R(p+m)k> depends on m only
+    q, k = rng.standard_normal(16), rng.standard_normal(16)
+    dots = [mqa.rope(q[None], [p])[0] @ mqa.rope(k[None], [p + 5])[0] for p in (0, 3, 40)]
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-12)
+
+
+def _inputs(B=2, T=40, H=3, d=16, seed=2):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, T, H, d)), rng.standard_normal((B, T, d)), rng.standard_normal((B, T, d)))
+
+
+def test_attention_matches_torch_sdpa_with_explicit_mask():
+    q, k, v = _inputs()
+    B, T, H, d = q.shape
+    seg = np.stack([np.arange(T), np.where(np.arange(T) < 13, np.arange(T), np.arange(T) - 13)]).astype(np.int32)
+    window = 9
+    got = mqa.attention(q, k, v, seg, window)
+    for b in range(B):
+        t, s = np.arange(T)[:, None], np.arange(T)[None, :]
+        allowed = (s <= t) & (s > t - window) & (s >= t - seg[b][:, None])
+        qt = torch.from_numpy(q[b]).permute(1, 0, 2)                     # [H, T, d]
+        kt = torch.from_numpy(k[b])[None].expand(H, T, d)
+        vt = torch.from_numpy(v[b])[None].expand(H, T, d)
+        want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(allowed))
+        np.testing.assert_allclose(got[b], want.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_window_and_document_limits():
+    """Changing a key just outside a query's window, or before its document
+    start, leaves that query's output unchanged; changing one inside moves it."""
+    q, k, v = _inputs(B=1, T=30)
+    seg = np.where(np.arange(30) < 20, np.arange(30), np.arange(30) - 20)[None].astype(np.int32)
+    base = mqa.attention(q, k, v, seg, window=6)
+    # query 18: window keys 13..18; query 25 (its document starts at 20): keys 20..25
+    for key, query, moves in ((12, 18, False), (13, 18, True), (19, 18, False), (19, 25, False),
+                              (20, 25, True)):
+        k2, v2 = k.copy(), v.copy()
+        k2[0, key] += 1.0
+        v2[0, key] += 1.0
+        alt = mqa.attention(q, k2, v2, seg, window=6)
+        assert (not np.allclose(alt[0, query], base[0, query])) == moves, (key, query, moves)
+
+
+def test_single_key_copies_its_value():
+    """A query at a document start attends only itself: the output is its v."""
+    q, k, v = _inputs(B=1, T=5)
+    seg = np.zeros((1, 5), np.int32)
+    out = mqa.attention(q, k, v, seg)
+    np.testing.assert_allclose(out[0], np.broadcast_to(v[0][:, None, :], out[0].shape), rtol=1e-14)
