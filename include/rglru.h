@@ -214,8 +214,11 @@ RGLRU_API rglru_status rglru_get_device_status(void *workspace, cudaStream_t str
  * Test hook for the bounded waits (never used by a normal call): makes chunk
  * `unit` of the next rglru_prefill calls on this workspace skip publishing
  * its scan carry, so that its successor's wait runs out and records
- * RGLRU_ERR_TIMEOUT instead of hanging.  unit = -1 turns it off.  The flag
- * lives in the workspace header and is enqueued on `stream`.
+ * RGLRU_ERR_TIMEOUT instead of hanging; on a decode workspace, CTA `unit` of
+ * the next rglru_decode_step calls keeps its half of the gate GEMM's operand
+ * from its peer CTA, whose wait runs out the same way (the call then takes a
+ * few seconds).  unit = -1 turns it off.  The flag lives in the workspace
+ * header and is enqueued on `stream`.
  */
 RGLRU_API rglru_status rglru_debug_suppress_publish(void *workspace, int unit, cudaStream_t stream);
 

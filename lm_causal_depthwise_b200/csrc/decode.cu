@@ -262,7 +262,10 @@ rglru_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     tc_fence_before();
     __syncthreads();           // this CTA's half of the B tile written
     tc_fence_after();
-    if (tid == 32) {
+    // test hook (rglru_debug_suppress_publish): the CTA it names keeps its half,
+    // so that its peer's bounded wait for it runs out
+    const bool suppress = *(volatile int *)&p.hdr->debug_unit_plus1 == (int)blockIdx.x + 1;
+    if (tid == 32 && !suppress) {
         // this half (K blocks 2 half, 2 half + 1: contiguous) into the peer's B tile
         uint8_t *src = smem + OFF_B + (int)half * 2 * kBBlock;
         bulk_copy_to_cluster(mapa_shared(smem_u32(src), half ^ 1u), src, 2 * kBBlock,

@@ -358,3 +358,30 @@ def test_head_shards_equal_the_whole_run(world):
         np.testing.assert_array_equal(got["y"], whole["y"][:, :, c])
         np.testing.assert_array_equal(got["h_state"], whole["h_state"][:, c])
         np.testing.assert_array_equal(got["conv_state"], whole["conv_state"][:, :, c])
+
+
+def test_decode_bounded_wait_reports_timeout_and_context_survives():
+    """The test hook makes CTA 0 of the decode grid keep its half of the gate
+    GEMM's operand from its peer: the peer's bounded wait runs out, the call
+    ends with RGLRU_ERR_TIMEOUT in the device status within seconds, and the
+    next step on the same context and workspace is correct."""
+    import time
+    _, inp = _case(64, 2, 512, reset_at=(0,))
+    dev = to_device(inp, "bf16")
+    ws = api.new_workspace(api.decode_workspace_size(64, 512, torch.bfloat16))
+    api.debug_suppress_publish(ws, 0)
+    t0 = time.time()
+    api.decode_step(dev["x"][:, 0].contiguous(), dev["g"][:, 0].contiguous(), dev["params"],
+                    dev["segpos"][:, 0].contiguous(), dev["conv_state"], dev["h_state"], workspace=ws)
+    assert api.device_status(ws) == api.ERR_TIMEOUT
+    assert time.time() - t0 < 60
+    api.debug_suppress_publish(ws, -1)
+    dev = to_device(inp, "bf16")
+    ys = []
+    for t in range(2):
+        ys.append(api.decode_step(dev["x"][:, t].contiguous(), dev["g"][:, t].contiguous(), dev["params"],
+                                  dev["segpos"][:, t].contiguous(), dev["conv_state"], dev["h_state"],
+                                  workspace=ws).float().cpu().numpy())
+    assert api.device_status(ws) == api.OK
+    ref = run_oracle(inp)
+    check_bf16(np.stack(ys, axis=1), ref["y"], "decode y after timeout")
