@@ -18,7 +18,9 @@ Readings where the pages are silent (stated here and in the design notes):
     document (segment_pos), so a document starts at position 0.
   * Scores are scaled by 1/sqrt(d) (d = 256) before the softmax.
   * Query t attends key s when t - W < s <= t (W = 2048, itself included) and
-    s lies in t's document (s >= t - segment_pos[t]).
+    s lies in t's document (s >= t - segment_pos[t]).  A prefill sees the keys
+    of its own tokens only: a document that began before the first token
+    (segment_pos[t] > t) attends from token 0.
   * In bf16 I/O every tensor between layers (q, k, v after RoPE, the
     attention output, the block output) is bf16: rounded once, here as on the
     GPU.
@@ -59,7 +61,7 @@ def attention(q, k, v, segpos, window: int = WINDOW) -> np.ndarray:
     idx = np.arange(T)
     for b in range(B):
         start = idx - np.asarray(segpos[b], np.int64)              # document start of each query
-        lo = np.maximum(start, idx - window + 1)
+        lo = np.maximum(np.maximum(start, idx - window + 1), 0)    # keys of this call only
         for t in range(T):
             ks = k[b, lo[t]:t + 1]                                  # [n, d]
             vs = v[b, lo[t]:t + 1]
@@ -68,6 +70,20 @@ def attention(q, k, v, segpos, window: int = WINDOW) -> np.ndarray:
             p = np.exp(sc)
             out[b, t] = (p / p.sum(axis=1, keepdims=True)) @ vs
     return out
+
+
+def attention_rows(q, k, v, segpos, rows, window: int = WINDOW) -> np.ndarray:
+    """attention() for the query rows ``rows`` [(b, t), ...] only: [len(rows), H, d],
+    so that a sample of rows of a large case costs only those rows."""
+    q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+    d = q.shape[-1]
+    out = []
+    for b, t in rows:
+        lo = max(t - int(segpos[b][t]), t - window + 1, 0)
+        sc = q[b, t] @ k[b, lo:t + 1].T / np.sqrt(d)                # [H, n]
+        p = np.exp(sc - sc.max(axis=1, keepdims=True))
+        out.append((p / p.sum(axis=1, keepdims=True)) @ v[b, lo:t + 1])
+    return np.stack(out)
 
 
 def mqa_block(u, W_q, W_k, W_v, W_o, b_o, segpos, window: int = WINDOW, round_io: bool = True) -> dict:

@@ -67,3 +67,30 @@ def test_single_key_copies_its_value():
     seg = np.zeros((1, 5), np.int32)
     out = mqa.attention(q, k, v, seg)
     np.testing.assert_allclose(out[0], np.broadcast_to(v[0][:, None, :], out[0].shape), rtol=1e-14)
+
+
+def test_attention_rows_equal_the_full_evaluation():
+    """The row-sampled form (used at full sizes) gives the rows of attention()."""
+    q, k, v = _inputs(B=2, T=50)
+    seg = np.stack([np.arange(50), np.where(np.arange(50) < 31, np.arange(50), np.arange(50) - 31)]).astype(np.int32)
+    full = mqa.attention(q, k, v, seg, window=11)
+    rows = [(0, 0), (0, 10), (0, 49), (1, 30), (1, 31), (1, 45)]
+    got = mqa.attention_rows(q, k, v, seg, rows, window=11)
+    for n, (b, t) in enumerate(rows):
+        np.testing.assert_allclose(got[n], full[b, t], rtol=1e-13, atol=1e-13)
+
+
+def test_document_begun_before_the_call_attends_from_token_zero():
+    """segment_pos above t (a document continuing from before the call): the
+    keys are those of the call, so the result equals a document starting at
+    token 0 (torch SDPA with the causal mask alone, window wider than T)."""
+    q, k, v = _inputs(B=1, T=20)
+    seg = (np.arange(20) + 7)[None].astype(np.int32)
+    got = mqa.attention(q, k, v, seg, window=64)
+    allowed = np.tril(np.ones((20, 20), bool))
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[0]).permute(1, 0, 2), torch.from_numpy(k[0])[None].expand(3, 20, 16),
+        torch.from_numpy(v[0])[None].expand(3, 20, 16), attn_mask=torch.from_numpy(allowed))
+    np.testing.assert_allclose(got[0], want.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(mqa.attention_rows(q, k, v, seg, [(0, 5), (0, 19)], window=64),
+                               got[0, [5, 19]], rtol=1e-13, atol=1e-13)
