@@ -453,6 +453,103 @@ def run_block(args, dev, stream, distributed, peaks, peak_kind):
     }
 
 
+def mqa_valid_pairs(segpos, window: int = 2048) -> int:
+    """(query, key) pairs the local MQA attends over: for query t the keys from
+    max(t - segment_pos[t], t - window + 1, 0) to t (the attention's
+    algorithmic work is 4 * 256 flops per pair and head)."""
+    import numpy as np
+    t = np.arange(segpos.shape[1])[None, :]
+    lo = np.maximum(np.maximum(t - segpos.astype(np.int64), t - window + 1), 0)
+    return int((t - lo + 1).sum())
+
+
+def run_mqa(args, dev, stream, distributed, peaks, peak_kind):
+    """The local MQA temporal block on the 2B shape (B=8, T=4096, D=2560: 10
+    query heads, one key/value head, window 2048, documents of mean length
+    1024): the QKV projection, RoPE, the attention kernel and o_proj, timed as a
+    whole and per launch; the attention kernel against the measured bf16 peak."""
+    import torch
+    from lm_causal_depthwise_b200 import api
+    w = W.PREFILL_2B
+    inp = W.generate_mqa(w)
+    bf = torch.bfloat16
+    B, T, D = w.B, w.T, w.D
+    H, M = D // 256, B * T
+    u = torch.from_numpy(inp["u"]).to(dev).to(bf)
+    sp = torch.from_numpy(inp["segpos"]).to(dev)
+    mp = api.MQAParams.from_arrays(inp, dev)
+    out = torch.empty_like(u)
+    ws = api.new_workspace(api.mqa_block_workspace_size(B, T, D), dev)
+    qkv = torch.empty((B, T, D + 512), dtype=bf, device=dev)
+    vt = api.mqa_vt(B, T, dev)
+    att = torch.empty((B, T, D), dtype=bf, device=dev)
+    lws = api.linear_workspace(dev)
+    api.linear(u.view(M, D), mp.W_qkv, None, out=qkv.view(M, D + 512), workspace=lws)
+    api.mqa_rope(qkv, sp, vt)
+
+    def block():
+        api.mqa_block_prefill(u, mp, sp, out=out, workspace=ws)
+
+    def proj():
+        api.linear(u.view(M, D), mp.W_qkv, None, out=qkv.view(M, D + 512), workspace=lws)
+
+    def rope():
+        api.mqa_rope(qkv, sp, vt)
+
+    def attention():
+        api.mqa_attention(qkv, vt, sp, out=att, workspace=lws)
+
+    def oproj():
+        api.linear(att.view(M, D), mp.W_o, mp.b_o, out=out.view(M, D), workspace=lws)
+
+    def timed(fn, n):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(n):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(ev0.elapsed_time(ev1), dev) / n
+
+    n = max(3, min(args.steps, 20))
+    if distributed:
+        import torch.distributed as dist
+        dist.barrier()
+    ms_block = timed(block, n)
+    for wsp, what in ((ws, "mqa block"), (lws, "mqa launches")):
+        st = api.device_status(wsp)
+        if st != api.OK:
+            raise RuntimeError(f"{what}: device status {api.status_string(st)}")
+    ms_attn = timed(attention, n)
+    ms_proj, ms_rope, ms_o = timed(proj, n), timed(rope, n), timed(oproj, n)
+    st = api.device_status(lws)
+    if st != api.OK:
+        raise RuntimeError(f"mqa launches: device status {api.status_string(st)}")
+    pairs = mqa_valid_pairs(inp["segpos"])
+    attn_flops = 4 * 256 * H * pairs
+    peak = peaks.get("bf16_tflops", 1590.0)
+    achieved = attn_flops / (ms_attn * 1e-3) / 1e12
+    world = dist.get_world_size() if distributed else 1
+    rope_bytes = M * (2 * (D + 256) * 2 + 2 * 256 * 2)   # q, k read and written; v read, v_t written
+    return {
+        "workload": f"local MQA block (QKV projection, RoPE, attention, o_proj) B={B} T={T} D={D} H={H} "
+                    f"window 2048, documents of mean length {w.doc_len}, bf16",
+        "value": job_throughput(w.tokens, world, ms_block), "unit": "tokens/s", "ms_per_step": ms_block,
+        "steps": n,
+        "launches": {"qkv_proj_ms": ms_proj, "rope_ms": ms_rope, "attention_ms": ms_attn, "o_proj_ms": ms_o},
+        "attention_pairs": pairs, "attention_flops": attn_flops,
+        "roofline": {"bound": "tensor", "kernel": "rglru_mqa_attention_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} cuBLAS bf16 burst", "traffic": None},
+        "qkv_proj_tflops": 2 * M * D * (D + 512) / (ms_proj * 1e-3) / 1e12,
+        "o_proj_tflops": 2 * M * D * D / (ms_o * 1e-3) / 1e12,
+        "rope_hbm_frac": rope_bytes / (ms_rope * 1e-3) / 1e9 / peaks["hbm_gbs"],
+    }
+
+
 def run_residual_block(args, dev, stream, distributed, peaks, peak_kind):
     """The whole recurrent residual block on the 2B shape (RMSNorm, the
     recurrent block with linear_out's residual add in its epilogue, RMSNorm,
@@ -579,6 +676,16 @@ def run_cuda(args, w):
         return profile_decode(args, w, dev, rank, distributed)
     if args.shard == "heads":
         return run_head_sharded(args, w, dev, stream, rank, world, local, distributed)
+    if args.profile_mqa:
+        # only the local MQA block's launches, warm-up then timed
+        peaks0, kind0 = measured_peaks()
+        r = run_mqa(args, dev, stream, distributed, peaks0, kind0)
+        if rank == 0:
+            print(json.dumps({"profile_mqa": r["workload"], "ms_per_step": r["ms_per_step"],
+                              "attention_ms": r["launches"]["attention_ms"], "roofline": r["roofline"]}))
+        if distributed:
+            dist.destroy_process_group()
+        return 0
     if args.profile_block:
         # only the residual block's launches (RMSNorm, projections, core,
         # MLP), warm-up then timed: the command an ncu launch list wraps
@@ -690,6 +797,8 @@ def run_cuda(args, w):
         blk = run_block(args, dev, stream, distributed, peaks0, kind0)
         torch.cuda.empty_cache()
         blk["residual_block"] = run_residual_block(args, dev, stream, distributed, peaks0, kind0)
+        torch.cuda.empty_cache()
+        blk["mqa_block"] = run_mqa(args, dev, stream, distributed, peaks0, kind0)
         torch.cuda.empty_cache()
 
     if distributed:
@@ -867,6 +976,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-mqa", action="store_true",
+                    help="run only the local MQA block's launches (for an ncu launch list)")
     ap.add_argument("--profile-block", action="store_true",
                     help="only the recurrent residual block's steps (the command an ncu launch list of "
                          "the block kernels wraps)")

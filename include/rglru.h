@@ -359,6 +359,74 @@ RGLRU_API rglru_status rglru_residual_block_prefill(
     const void *W_gate, const float *b_gate, const void *W_up, const float *b_up, const void *W_down,
     const float *b_down, float eps, void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Local sliding-window MQA: the other temporal block.
+ *
+ * "Gemma explained: RecurrentGemma architecture", the
+ * RecurrentGemmaSdpaAttention printout (q_proj D -> D and k_proj, v_proj
+ * D -> 256 without bias, o_proj D -> D with bias, rotary_emb) and sections
+ * "Residual block with local MQA" (H = D / 256 query heads of 256 share one
+ * key/value head of 256; each position attends a fixed number of past tokens)
+ * and "Local attention window size" (2048 tokens).  Readings where the pages
+ * are silent: rotate-half RoPE over the whole head, the pairs (x[i],
+ * x[i + 128]) turned by segment_pos * 10000^(-2i/256); scores scaled by 1/16;
+ * query t attends key s when t - window < s <= t, s >= t - segment_pos[t]
+ * (same document) and s >= 0 (a call sees the keys of its own tokens only).
+ *
+ * Layouts (bf16, row-major): qkv [B, T, (H + 2) * 256] holds the H query
+ * heads, then k, then v of each token; v_t [B, 256, Tp] is v transposed,
+ * Tp = T rounded up to a multiple of 8 (rglru_mqa_vt_size bytes);
+ * segment_pos [B, T] int32 (>= 0); out [B, T, H * 256].  Every pointer is
+ * device memory, 16-byte aligned; calls enqueue on `stream` and return after
+ * synchronous argument checks (RGLRU_ERR_INVALID_ARG on null, misaligned or
+ * overlapping arguments, RGLRU_ERR_UNSUPPORTED on sizes outside B <= 65535,
+ * H <= 64, B * T <= 2^30).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of v_t for B sequences of T tokens (0 on bad sizes). */
+RGLRU_API size_t rglru_mqa_vt_size(int B, int T);
+
+/*
+ * RoPE of the query heads and the key in place in qkv, at the positions
+ * segment_pos, and v_t = the v columns of qkv transposed (its tokens past T
+ * up to Tp are written as zeros).  qkv and v_t must not overlap.
+ */
+RGLRU_API rglru_status rglru_mqa_rope(int B, int T, int H, void *qkv, const int32_t *segment_pos, void *v_t,
+                                      cudaStream_t stream);
+
+/*
+ * out[b, t, h] = sum_s softmax_s(q[b, t, h] . k[b, s] / 16) v[b, s] over the
+ * keys s query t attends (see above), from qkv and v_t after rglru_mqa_rope.
+ * fp32 scores and accumulation on the tensor cores, the probabilities rounded
+ * to bf16 as the operand of the second product, out rounded to bf16.
+ * window >= 1 (2048 in the 2B and 9B models).  The workspace (at least
+ * rglru_linear_workspace_size() bytes, zero-filled once) carries the device
+ * status: a wait inside the kernel that runs out (2 s) records
+ * RGLRU_ERR_TIMEOUT there instead of hanging.  out must not overlap the inputs.
+ */
+RGLRU_API rglru_status rglru_mqa_attention(int B, int T, int H, int window, const void *qkv, const void *v_t,
+                                           const int32_t *segment_pos, void *out, void *workspace,
+                                           size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes of rglru_mqa_block_prefill (0 on bad sizes). */
+RGLRU_API size_t rglru_mqa_block_workspace_size(int B, int T, int D);
+
+/*
+ * The local MQA temporal block over T tokens of B sequences, bf16:
+ *   qkv = u W_qkv^T                       (q_proj, k_proj, v_proj in one launch)
+ *   RoPE on q and k, v transposed          (rglru_mqa_rope)
+ *   a   = local MQA(q, k, v)               (rglru_mqa_attention)
+ *   out = a W_o^T + b_o                    (o_proj)
+ * u, out [B, T, D]; W_qkv [D + 512, D] = the rows of W_q [D, D], then W_k
+ * [256, D], then W_v [256, D]; W_o [D, D]; b_o [D] fp32 (may be NULL).  qkv,
+ * v_t and a live in the workspace (zero-filled once), which carries one status
+ * word for all four launches.
+ */
+RGLRU_API rglru_status rglru_mqa_block_prefill(int B, int T, int D, int window, const void *u, const void *W_qkv,
+                                               const void *W_o, const float *b_o, const int32_t *segment_pos,
+                                               void *out, void *workspace, size_t workspace_bytes,
+                                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

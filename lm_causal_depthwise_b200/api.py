@@ -27,7 +27,9 @@ SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglr
            "rglru_prefill_noalloc", "rglru_prefill_host_staging_size", "rglru_prefill_host",
            "rglru_linear_workspace_size", "rglru_linear", "rglru_linear_pair", "rglru_linear_residual",
            "rglru_linear_geglu", "rglru_recurrent_block_workspace_size", "rglru_recurrent_block_prefill",
-           "rglru_rmsnorm", "rglru_residual_block_workspace_size", "rglru_residual_block_prefill")
+           "rglru_rmsnorm", "rglru_residual_block_workspace_size", "rglru_residual_block_prefill",
+           "rglru_mqa_vt_size", "rglru_mqa_rope", "rglru_mqa_attention", "rglru_mqa_block_workspace_size",
+           "rglru_mqa_block_prefill")
 
 _lib = None
 
@@ -94,6 +96,16 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_residual_block_workspace_size.argtypes = [i, i, i, i]
     lib.rglru_residual_block_prefill.restype = i
     lib.rglru_residual_block_prefill.argtypes = [i, i, i, i] + [vp] * 25 + [ctypes.c_float, vp, vp, sz, vp]
+    lib.rglru_mqa_vt_size.restype = sz
+    lib.rglru_mqa_vt_size.argtypes = [i, i]
+    lib.rglru_mqa_rope.restype = i
+    lib.rglru_mqa_rope.argtypes = [i, i, i, vp, vp, vp, vp]
+    lib.rglru_mqa_attention.restype = i
+    lib.rglru_mqa_attention.argtypes = [i, i, i, i] + [vp] * 5 + [sz, vp]
+    lib.rglru_mqa_block_workspace_size.restype = sz
+    lib.rglru_mqa_block_workspace_size.argtypes = [i, i, i]
+    lib.rglru_mqa_block_prefill.restype = i
+    lib.rglru_mqa_block_prefill.argtypes = [i, i, i, i] + [vp] * 7 + [sz, vp]
     _lib = lib
     return lib
 
@@ -579,4 +591,104 @@ def residual_block_prefill(u, rp: ResidualBlockParams, segment_pos, conv_state, 
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
     if st != OK:
         raise RGLRUError(st, "rglru_residual_block_prefill")
+    return out
+
+
+# ---------------------------------------------------------------- local MQA
+MQA_WINDOW = 2048
+
+
+def mqa_vt(B: int, T: int, device="cuda") -> torch.Tensor:
+    """v transposed, [B, 256, Tp] bf16 with Tp = T rounded up to 8."""
+    if int(load().rglru_mqa_vt_size(B, T)) == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "mqa_vt_size")
+    return torch.empty((B, 256, (T + 7) // 8 * 8), dtype=torch.bfloat16, device=device)
+
+
+def mqa_rope(qkv, segment_pos, v_t=None) -> torch.Tensor:
+    """RoPE on the query heads and the key of qkv [B, T, (H + 2) * 256] in
+    place (rglru_mqa_rope); returns v_t, the v columns transposed."""
+    if qkv.dim() != 3 or qkv.shape[2] % 256 != 0 or qkv.shape[2] < 768:
+        raise ValueError("qkv must be [B, T, (H + 2) * 256]")
+    B, T, C = qkv.shape
+    dev = qkv.device
+    _check(qkv, "qkv", (B, T, C), torch.bfloat16, dev)
+    _check(segment_pos, "segment_pos", (B, T), torch.int32, dev)
+    if v_t is None:
+        v_t = mqa_vt(B, T, dev)
+    _check(v_t, "v_t", (B, 256, (T + 7) // 8 * 8), torch.bfloat16, dev)
+    st = load().rglru_mqa_rope(B, T, C // 256 - 2, _ptr(qkv), _ptr(segment_pos), _ptr(v_t), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_mqa_rope")
+    return v_t
+
+
+def mqa_attention(qkv, v_t, segment_pos, window: int = MQA_WINDOW, out=None, workspace=None) -> torch.Tensor:
+    """Local MQA over qkv (after mqa_rope) and v_t (rglru_mqa_attention):
+    out [B, T, H * 256] bf16."""
+    if qkv.dim() != 3 or qkv.shape[2] % 256 != 0 or qkv.shape[2] < 768:
+        raise ValueError("qkv must be [B, T, (H + 2) * 256]")
+    B, T, C = qkv.shape
+    H = C // 256 - 2
+    dev = qkv.device
+    _check(qkv, "qkv", (B, T, C), torch.bfloat16, dev)
+    _check(v_t, "v_t", (B, 256, (T + 7) // 8 * 8), torch.bfloat16, dev)
+    _check(segment_pos, "segment_pos", (B, T), torch.int32, dev)
+    if out is None:
+        out = torch.empty((B, T, H * 256), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", (B, T, H * 256), torch.bfloat16, dev)
+    workspace, nb = _ws(workspace, dev)
+    st = load().rglru_mqa_attention(B, T, H, int(window), _ptr(qkv), _ptr(v_t), _ptr(segment_pos), _ptr(out),
+                                    _ptr(workspace), nb, _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_mqa_attention")
+    return out
+
+
+@dataclass
+class MQAParams:
+    """Projections of the local MQA block: W_qkv [D + 512, D] (the rows of
+    W_q, then W_k, then W_v), W_o [D, D] bf16 and b_o [D] fp32."""
+    W_qkv: torch.Tensor
+    W_o: torch.Tensor
+    b_o: torch.Tensor
+
+    @staticmethod
+    def from_arrays(inp: dict, device="cuda") -> "MQAParams":
+        def w(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).to(torch.bfloat16).contiguous()
+        W_qkv = torch.cat([w(inp["W_q"]), w(inp["W_k"]), w(inp["W_v"])], dim=0).contiguous()
+        return MQAParams(W_qkv, w(inp["W_o"]), torch.as_tensor(inp["b_o"], dtype=torch.float32).to(device).contiguous())
+
+
+def mqa_block_workspace_size(B: int, T: int, D: int) -> int:
+    n = int(load().rglru_mqa_block_workspace_size(B, T, D))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "mqa_block_workspace_size")
+    return n
+
+
+def mqa_block_prefill(u, mp: MQAParams, segment_pos, window: int = MQA_WINDOW, out=None,
+                      workspace=None) -> torch.Tensor:
+    """out = o_proj(local MQA(RoPE(q_proj u), RoPE(k_proj u), v_proj u)) over u [B,T,D] bf16
+    (rglru_mqa_block_prefill)."""
+    if u.dim() != 3:
+        raise ValueError("u must be [B,T,D]")
+    B, T, D = u.shape
+    dev = u.device
+    _check(u, "u", (B, T, D), torch.bfloat16, dev)
+    _check(mp.W_qkv, "W_qkv", (D + 512, D), torch.bfloat16, dev)
+    _check(mp.W_o, "W_o", (D, D), torch.bfloat16, dev)
+    _check(mp.b_o, "b_o", (D,), torch.float32, dev)
+    _check(segment_pos, "segment_pos", (B, T), torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(u)
+    _check(out, "out", (B, T, D), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(mqa_block_workspace_size(B, T, D), dev)
+    st = load().rglru_mqa_block_prefill(B, T, D, int(window), _ptr(u), _ptr(mp.W_qkv), _ptr(mp.W_o), _ptr(mp.b_o),
+                                        _ptr(segment_pos), _ptr(out), _ptr(workspace),
+                                        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_mqa_block_prefill")
     return out

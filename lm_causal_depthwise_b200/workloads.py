@@ -254,3 +254,24 @@ def residual_block_gemm_flops(w: Workload) -> int:
     MLP's three D x 3D ones."""
     F = MLP_EXPANSION * w.D
     return 2 * w.tokens * (3 * w.D * w.D + 3 * w.D * F)
+
+
+def generate_mqa(w: Workload) -> dict:
+    """Inputs of the local MQA temporal block, from ``default_rng((seed, 3))``
+    in this order:
+      segpos [B, T]   as ``segment_positions`` (the workload's documents)
+      u [B, T, D]     ~ N(0, 1)                 bf16 values
+      W_q [D, D], W_k [256, D], W_v [256, D], W_o [D, D] ~ N(0, 1/D)  bf16
+      b_o [D]         ~ N(0, 0.1)               fp32
+    With these scales q and k have unit-variance entries and the scaled scores
+    q.k / 16 are about N(0, 1)."""
+    rng = np.random.default_rng((w.seed, 3))
+    B, T, D = w.B, w.T, w.D
+    seg = segment_positions(rng, w)
+    u = round_bf16(rng.standard_normal((B, T, D), dtype=np.float32))
+
+    def weight(n, k):
+        return round_bf16((rng.standard_normal((n, k), dtype=np.float32) / np.sqrt(k)).astype(np.float32))
+    W_q, W_k, W_v, W_o = weight(D, D), weight(HEAD, D), weight(HEAD, D), weight(D, D)
+    b_o = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
+    return {"u": u, "W_q": W_q, "W_k": W_k, "W_v": W_v, "W_o": W_o, "b_o": b_o, "segpos": seg}
