@@ -550,6 +550,75 @@ def run_mqa(args, dev, stream, distributed, peaks, peak_kind):
     }
 
 
+def run_mqa_decode(args, dev, stream, distributed, peaks, peak_kind):
+    """One local-MQA decode step for B=256 sequences (10 query heads, window
+    2048): RoPE, the cache write, the split-KV attention and the combine, timed
+    as a 64-step CUDA graph.  Positions: the decode-2b recipe's document
+    positions at its last step; the rings hold synthetic bf16 keys and values.
+    HBM roofline: every attended key and value (512 B each) read once, the
+    token's qkv read, its cache slot and output written."""
+    import numpy as np
+    import torch
+    from lm_causal_depthwise_b200 import api
+    wd = W.DECODE_2B
+    B, H, window = wd.B, wd.H, 2048
+    rng = np.random.default_rng((wd.seed, 4))
+    seg = W.segment_positions(rng, wd)[:, -1].astype(np.int32)
+    bf = torch.bfloat16
+    g = torch.Generator(device="cpu").manual_seed(wd.seed)
+    qkv = torch.randn((B, (H + 2) * 256), generator=g).to(bf).to(dev)
+    kc = torch.randn((B, window, 256), generator=g).to(bf).to(dev)
+    vc = torch.randn((B, window, 256), generator=g).to(bf).to(dev)
+    sp = torch.from_numpy(seg).to(dev)
+    out = torch.empty((B, H * 256), dtype=bf, device=dev)
+    ws = api.new_workspace(api.mqa_decode_workspace_size(B, H, window), dev)
+    steps = 64
+
+    def step():
+        api.mqa_decode_step(qkv, sp, kc, vc, out=out, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    s2 = torch.cuda.Stream(dev)
+    s2.wait_stream(torch.cuda.current_stream(dev))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s2):
+        step()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=s2):
+            for _ in range(steps):
+                step()
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    if distributed:
+        import torch.distributed as dist
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(3, min(args.steps, 10))
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev) / (reps * steps)
+    del graph
+    n = np.minimum(seg.astype(np.int64) + 1, window)
+    alg = int(n.sum()) * 2 * 512 + B * (H + 2) * 512 + B * 2 * 512 + B * H * 512
+    world = dist.get_world_size() if distributed else 1
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {
+        "workload": f"local MQA decode step B={B} H={H} window {window}, positions of the decode-2b recipe "
+                    f"(mean {float(n.mean()):.0f} keys per sequence), bf16",
+        "value": job_throughput(B, world, ms), "unit": "tokens/s", "us_per_step": ms * 1e3,
+        "graph_steps": steps, "algorithmic_bytes_per_step": alg,
+        "roofline": {"bound": "hbm", "kernel": "rglru_mqa_decode_kernel + combine", "achieved": gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "peak_source": "measured copy bandwidth", "traffic": None},
+    }
+
+
 def run_residual_block(args, dev, stream, distributed, peaks, peak_kind):
     """The whole recurrent residual block on the 2B shape (RMSNorm, the
     recurrent block with linear_out's residual add in its epilogue, RMSNorm,
@@ -680,9 +749,12 @@ def run_cuda(args, w):
         # only the local MQA block's launches, warm-up then timed
         peaks0, kind0 = measured_peaks()
         r = run_mqa(args, dev, stream, distributed, peaks0, kind0)
+        rd = run_mqa_decode(args, dev, stream, distributed, peaks0, kind0)
         if rank == 0:
             print(json.dumps({"profile_mqa": r["workload"], "ms_per_step": r["ms_per_step"],
-                              "attention_ms": r["launches"]["attention_ms"], "roofline": r["roofline"]}))
+                              "attention_ms": r["launches"]["attention_ms"], "roofline": r["roofline"],
+                              "decode": {"us_per_step": rd["us_per_step"], "roofline": rd["roofline"],
+                                         "workload": rd["workload"]}}))
         if distributed:
             dist.destroy_process_group()
         return 0
@@ -799,6 +871,8 @@ def run_cuda(args, w):
         blk["residual_block"] = run_residual_block(args, dev, stream, distributed, peaks0, kind0)
         torch.cuda.empty_cache()
         blk["mqa_block"] = run_mqa(args, dev, stream, distributed, peaks0, kind0)
+        torch.cuda.empty_cache()
+        blk["mqa_decode"] = run_mqa_decode(args, dev, stream, distributed, peaks0, kind0)
         torch.cuda.empty_cache()
 
     if distributed:

@@ -427,6 +427,31 @@ RGLRU_API rglru_status rglru_mqa_block_prefill(int B, int T, int D, int window, 
                                                void *out, void *workspace, size_t workspace_bytes,
                                                cudaStream_t stream);
 
+/* Workspace bytes of rglru_mqa_decode_step (0 on unsupported sizes:
+ * 1 <= B <= 65535, 1 <= H <= 16, 1 <= window <= 2^20). */
+RGLRU_API size_t rglru_mqa_decode_workspace_size(int B, int H, int window);
+
+/*
+ * One decode step of the local MQA attention for B sequences (one token
+ * each), after the QKV projection of that token:
+ *   qkv         [B, (H + 2) * 256] bf16, read only: q heads, k, v of the token;
+ *   segment_pos [B] int32 >= 0: the token's position in its document;
+ *   k_cache, v_cache [B, window, 256] bf16, in/out: a ring per sequence, the
+ *               rotated key and the value of document position p at slot
+ *               p % window.  The step writes this token's slot, then attends
+ *               positions max(0, p - window + 1) .. p of the cache (earlier
+ *               steps of the same document must have written them);
+ *   out         [B, H * 256] bf16.
+ * q and k are rotated (RoPE at segment_pos) and rounded to bf16 as in
+ * rglru_mqa_rope; scores and sums in fp32; out rounded to bf16.  Two kernels:
+ * per (256-key chunk, sequence) partial maxima, sums and outputs in the
+ * workspace, then their combination.  No buffer may overlap another one that
+ * the step writes.
+ */
+RGLRU_API rglru_status rglru_mqa_decode_step(int B, int H, int window, const void *qkv, const int32_t *segment_pos,
+                                             void *k_cache, void *v_cache, void *out, void *workspace,
+                                             size_t workspace_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,7 +29,7 @@ SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglr
            "rglru_linear_geglu", "rglru_recurrent_block_workspace_size", "rglru_recurrent_block_prefill",
            "rglru_rmsnorm", "rglru_residual_block_workspace_size", "rglru_residual_block_prefill",
            "rglru_mqa_vt_size", "rglru_mqa_rope", "rglru_mqa_attention", "rglru_mqa_block_workspace_size",
-           "rglru_mqa_block_prefill")
+           "rglru_mqa_block_prefill", "rglru_mqa_decode_workspace_size", "rglru_mqa_decode_step")
 
 _lib = None
 
@@ -106,6 +106,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_mqa_block_workspace_size.argtypes = [i, i, i]
     lib.rglru_mqa_block_prefill.restype = i
     lib.rglru_mqa_block_prefill.argtypes = [i, i, i, i] + [vp] * 7 + [sz, vp]
+    lib.rglru_mqa_decode_workspace_size.restype = sz
+    lib.rglru_mqa_decode_workspace_size.argtypes = [i, i, i]
+    lib.rglru_mqa_decode_step.restype = i
+    lib.rglru_mqa_decode_step.argtypes = [i, i, i] + [vp] * 6 + [sz, vp]
     _lib = lib
     return lib
 
@@ -691,4 +695,44 @@ def mqa_block_prefill(u, mp: MQAParams, segment_pos, window: int = MQA_WINDOW, o
                                         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
     if st != OK:
         raise RGLRUError(st, "rglru_mqa_block_prefill")
+    return out
+
+
+def mqa_decode_workspace_size(B: int, H: int, window: int = MQA_WINDOW) -> int:
+    n = int(load().rglru_mqa_decode_workspace_size(B, H, window))
+    if n == 0:
+        raise RGLRUError(ERR_UNSUPPORTED, "mqa_decode_workspace_size")
+    return n
+
+
+def mqa_cache(B: int, window: int = MQA_WINDOW, device="cuda"):
+    """Zero-filled key and value rings [B, window, 256] bf16."""
+    return (torch.zeros((B, window, 256), dtype=torch.bfloat16, device=device),
+            torch.zeros((B, window, 256), dtype=torch.bfloat16, device=device))
+
+
+def mqa_decode_step(qkv, segment_pos, k_cache, v_cache, out=None, workspace=None) -> torch.Tensor:
+    """One local-MQA decode step (rglru_mqa_decode_step): qkv [B, (H + 2) * 256]
+    bf16 of the new token, segment_pos [B] int32, the rings k_cache / v_cache
+    [B, window, 256] (updated in place); returns out [B, H * 256] bf16."""
+    if qkv.dim() != 2 or qkv.shape[1] % 256 != 0 or qkv.shape[1] < 768:
+        raise ValueError("qkv must be [B, (H + 2) * 256]")
+    B, C = qkv.shape
+    H = C // 256 - 2
+    dev = qkv.device
+    window = k_cache.shape[1] if k_cache.dim() == 3 else -1
+    _check(qkv, "qkv", (B, C), torch.bfloat16, dev)
+    _check(segment_pos, "segment_pos", (B,), torch.int32, dev)
+    _check(k_cache, "k_cache", (B, window, 256), torch.bfloat16, dev)
+    _check(v_cache, "v_cache", (B, window, 256), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty((B, H * 256), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", (B, H * 256), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(mqa_decode_workspace_size(B, H, window), dev)
+    st = load().rglru_mqa_decode_step(B, H, window, _ptr(qkv), _ptr(segment_pos), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(out), _ptr(workspace),
+                                      ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_mqa_decode_step")
     return out

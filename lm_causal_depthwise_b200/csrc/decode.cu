@@ -112,7 +112,7 @@ struct DecodeMaps {
 
 // Bounded wait on an mbarrier phase by every lane of a warp; false (and the
 // status recorded) if it does not complete within kTimeoutNs.
-__device__ __noinline__ bool dec_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
+__device__ __noinline__ bool dec_wait_slow(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
 {
     bool seen = mbar_try_wait(bar, parity);
     if (!seen) {
@@ -128,6 +128,13 @@ __device__ __noinline__ bool dec_wait(uint64_t *bar, uint32_t parity, WsHeader *
         return false;
     }
     return true;
+}
+
+// A phase that is already complete costs one inline test per lane and a vote.
+__device__ __forceinline__ bool dec_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
+{
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    return dec_wait_slow(bar, parity, hdr, where);
 }
 
 // 1 - exp(2l) for -1/8 < l <= 0 by its Taylor series -2l (1 + l + 2/3 l^2 + 1/3 l^3),

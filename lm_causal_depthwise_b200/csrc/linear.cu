@@ -69,9 +69,8 @@ struct LinearParams {
     WsHeader *hdr;
 };
 
-__device__ __noinline__ bool lin_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
+__device__ __noinline__ bool lin_wait_slow(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
@@ -86,9 +85,18 @@ __device__ __noinline__ bool lin_wait(uint64_t *bar, uint32_t parity, WsHeader *
     }
 }
 
+// a phase that is already complete costs one inline test; only a wait that
+// has to poll calls out
+__device__ __forceinline__ bool lin_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return lin_wait_slow(bar, parity, hdr, where);
+}
+
 // every lane of the warp waits; the warp's verdict is unanimous
 __device__ __forceinline__ bool lin_warp_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
 {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = lin_wait(bar, parity, hdr, where);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;

@@ -25,24 +25,26 @@
 //
 // rglru_mqa_attention_kernel: one CTA per (head, 128-query tile, sequence),
 // 192 threads:
-//   warp 4     TMA producer: the Q tile once (4 boxes [128 x 64], 128-byte
-//              swizzle), then per 64-key tile the K tile (4 boxes [64 x 64])
-//              and the V^T tile ([256 x 64]) into 2-deep rings;
-//   warp 5     MMA issuer (one thread): S = Q K^T (M=128, N=64, 16 K-steps)
-//              into one of two TMEM score buffers, then O += P V (M=128,
-//              N=256, 4 K-steps) with P read from TMEM (bf16 pairs); S of
-//              tile j + 1 is issued before O of tile j, so the softmax of tile
-//              j overlaps the tensor cores;
-//   warps 0-3  softmax: thread = query row = TMEM lane.  Scores in log2
-//              units, the window / document / causal limits applied only on
-//              tiles that cross them; the running max used for the
+//   warp 4     TMA producer: lane 0 the K tiles (4 boxes [64 keys x 64
+//              channels], 128-byte swizzle), lane 1 the V^T tiles ([256 x 64
+//              keys]), each into a 3-deep ring;
+//   warp 5     MMA issuer (the converged warp, one lane elected per MMA):
+//              S = Q K^T (M=128, N=64, 16 K-steps) with Q read from TMEM,
+//              then O += P V (M=128, N=256, 4 K-steps) with P read from TMEM;
+//              S of tile j + 1 is issued as soon as the softmax has read S of
+//              tile j, so it runs under the softmax of tile j;
+//   warps 0-3  softmax: thread = query row = TMEM lane.  Each first writes its
+//              row of the Q tile into TMEM (the A operand of S).  Scores in
+//              log2 units, the window / document / causal limits applied only
+//              on tiles that cross them; the running max used for the
 //              exponentials is raised only when a row's max grows by more
 //              than 8 (a factor 256), and only then is O (in TMEM) rescaled,
 //              after the MMAs that wrote it have completed.  P goes to TMEM as
 //              bf16 pairs; at the end O / l is written as bf16.
-// TMEM: O 256 columns, S 2 x 64, P 2 x 32 (512 allocated, one CTA per SM).
+// TMEM: O 256 columns, Q 128, S 64, P 2 x 32 (all 512, one CTA per SM).
 // Every mbarrier wait is bounded (2 s): one that runs out records
-// RGLRU_ERR_TIMEOUT in the workspace header and the CTA unwinds.
+// RGLRU_ERR_TIMEOUT in the workspace header and the CTA unwinds.  A wait whose
+// phase is already complete costs one inline test.
 #include <climits>
 #include <cmath>
 
@@ -58,23 +60,21 @@ constexpr int kHd = 256;             // head dimension
 constexpr int kQT = 128;             // query rows per CTA
 constexpr int kKT = 64;              // keys per tile
 constexpr int kThreads = 192;
-constexpr int kQBox = kQT * 64 * 2;  // 16 KB: [128 rows x 64 channels]
-constexpr int kQBytes = 4 * kQBox;   // 64 KB
 constexpr int kKBox = kKT * 64 * 2;  // 8 KB: [64 keys x 64 channels]
 constexpr int kKBytes = 4 * kKBox;   // 32 KB
 constexpr int kVBytes = kHd * kKT * 2;  // 32 KB: [256 channels x 64 keys]
-constexpr int kStages = 2;
-constexpr int OFF_Q = 0, OFF_K = OFF_Q + kQBytes, OFF_V = OFF_K + kStages * kKBytes;
+constexpr int kStages = 3;
+constexpr int OFF_K = 0, OFF_V = OFF_K + kStages * kKBytes;
 constexpr int OFF_BAR = OFF_V + kStages * kVBytes;
 enum {
-    B_Q = 0,
+    B_QFULL = 0,                  // the Q tile is in TMEM (128 arrivals)
     B_KFULL = 1,
     B_KFREE = B_KFULL + kStages,
     B_VFULL = B_KFREE + kStages,
     B_VFREE = B_VFULL + kStages,
-    B_SFULL = B_VFREE + kStages,  // scores of tile j in buffer j % 2
-    B_SFREE = B_SFULL + 2,        // ... read by the softmax warps
-    B_PFULL = B_SFREE + 2,        // P of tile j in buffer j % 2
+    B_SFULL = B_VFREE + kStages,  // scores of tile j complete
+    B_SFREE = B_SFULL + 1,        // ... read by the softmax warps (128 arrivals)
+    B_PFULL = B_SFREE + 1,        // P of tile j in buffer j % 2 (128 arrivals)
     B_PVDONE = B_PFULL + 2,       // O += P V of tile j complete (P buffer free, O settled)
     B_DRAIN = B_PVDONE + 2,
     B_N = B_DRAIN + 1
@@ -82,20 +82,22 @@ enum {
 constexpr int OFF_MISC = OFF_BAR + B_N * 8;
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 384;
+// TMEM columns: O (fp32) 256, the Q tile (bf16 pairs, the A operand of S) 128,
+// S (fp32) 64, P (bf16 pairs, the A operand of O) 2 x 32
+constexpr uint32_t kColO = 0, kColQ = 256, kColS = 384, kColP = 448;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.f;  // raise the reference max when the row max exceeds it by 2^8
 
 struct AttnParams {
     int B, T, H, window, ntiles;
+    const __nv_bfloat16 *qkv;
     const int32_t *segpos;
     __nv_bfloat16 *out;
     WsHeader *hdr;
 };
 
-__device__ __noinline__ bool attn_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
+__device__ __noinline__ bool attn_wait_slow(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
@@ -110,9 +112,18 @@ __device__ __noinline__ bool attn_wait(uint64_t *bar, uint32_t parity, WsHeader 
     }
 }
 
+// a phase that is already complete costs one inline test; only a wait that
+// has to poll calls out
+__device__ __forceinline__ bool attn_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return attn_wait_slow(bar, parity, hdr, where);
+}
+
 // every lane of the warp waits; the warp's verdict is unanimous
 __device__ __forceinline__ bool attn_warp_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
 {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = attn_wait(bar, parity, hdr, where);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -146,8 +157,8 @@ __device__ __forceinline__ int row_lo(const AttnParams &p, int b, int t)
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
-                           const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v)
+rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -174,16 +185,16 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
     if (warp == 5) {
         tmem_alloc(tmem_holder, 512);
         if (lane == 0) {
-            mbar_init(bars + B_Q, 1);
+            mbar_init(bars + B_QFULL, 4 * 32);
             for (int s = 0; s < kStages; ++s) {
                 mbar_init(bars + B_KFULL + s, 1);
                 mbar_init(bars + B_KFREE + s, 1);
                 mbar_init(bars + B_VFULL + s, 1);
                 mbar_init(bars + B_VFREE + s, 1);
             }
+            mbar_init(bars + B_SFULL, 1);
+            mbar_init(bars + B_SFREE, 4 * 32);
             for (int s = 0; s < 2; ++s) {
-                mbar_init(bars + B_SFULL + s, 1);
-                mbar_init(bars + B_SFREE + s, 4 * 32);
                 mbar_init(bars + B_PFULL + s, 4 * 32);
                 mbar_init(bars + B_PVDONE + s, 1);
             }
@@ -198,79 +209,80 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
 
     if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bars + B_Q, kQBytes);
-            for (int kb = 0; kb < 4; ++kb)
-                tma_load_3d(smem + OFF_Q + kb * kQBox, &tm_q, bars + B_Q, h * kHd + kb * 64, t0, b);
+        // lane 0 loads the K tiles, lane 1 the V tiles: a wait for a V slot
+        // never holds back the next K load
+        if (lane < 2) {
+            const bool is_k = lane == 0;
+            const int full = is_k ? B_KFULL : B_VFULL, freeb = is_k ? B_KFREE : B_VFREE;
             bool ok = true;
-            int jk = 0, jv = 0;  // K and V tiles issued
+            int issued = 0;
             for (int j = 0; j < n && ok; ++j) {
                 const int s = j % kStages, s0 = (j0 + j) * kKT;
-                const uint32_t ph = (uint32_t)((j / kStages) - 1) & 1u;
-                if (j >= kStages && !(ok = attn_wait(bars + B_KFREE + s, ph, p.hdr, 0))) break;
-                mbar_arrive_expect_tx(bars + B_KFULL + s, kKBytes);
-                for (int kb = 0; kb < 4; ++kb)
-                    tma_load_3d(smem + OFF_K + s * kKBytes + kb * kKBox, &tm_k, bars + B_KFULL + s,
-                                p.H * kHd + kb * 64, s0, b);
-                ++jk;
-                if (j >= kStages && !(ok = attn_wait(bars + B_VFREE + s, ph, p.hdr, 1))) break;
-                mbar_arrive_expect_tx(bars + B_VFULL + s, kVBytes);
-                tma_load_3d(smem + OFF_V + s * kVBytes, &tm_v, bars + B_VFULL + s, s0, 0, b);
-                ++jv;
+                if (j >= kStages &&
+                    !(ok = attn_wait(bars + freeb + s, (uint32_t)((j / kStages) - 1) & 1u, p.hdr, is_k ? 0 : 1)))
+                    break;
+                if (is_k) {
+                    mbar_arrive_expect_tx(bars + full + s, kKBytes);
+                    for (int kb = 0; kb < 4; ++kb)
+                        tma_load_3d(smem + OFF_K + s * kKBytes + kb * kKBox, &tm_k, bars + full + s,
+                                    p.H * kHd + kb * 64, s0, b);
+                } else {
+                    mbar_arrive_expect_tx(bars + full + s, kVBytes);
+                    tma_load_3d(smem + OFF_V + s * kVBytes, &tm_v, bars + full + s, s0, 0, b);
+                }
+                ++issued;
             }
             if (!ok) {
                 // the loads already issued land before the CTA exits
-                drain_wait(bars + B_Q, 0);
-                for (int k = max(0, jk - kStages); k < jk; ++k)
-                    drain_wait(bars + B_KFULL + k % kStages, (uint32_t)(k / kStages) & 1u);
-                for (int k = max(0, jv - kStages); k < jv; ++k)
-                    drain_wait(bars + B_VFULL + k % kStages, (uint32_t)(k / kStages) & 1u);
+                for (int k = max(0, issued - kStages); k < issued; ++k)
+                    drain_wait(bars + full + k % kStages, (uint32_t)(k / kStages) & 1u);
             }
         }
         __syncwarp();
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc_s = umma_idesc_bf16(kQT, kKT), idesc_o = umma_idesc_bf16(kQT, kHd);
-            const uint32_t q_base = smem_u32(smem + OFF_Q);
-            bool ok = attn_wait(bars + B_Q, 0, p.hdr, 2);
-            for (int j = 0; ok && j <= n; ++j) {
-                if (j < n) {
-                    const int s = j % 2;
-                    if (!(ok = attn_wait(bars + B_KFULL + s, (uint32_t)(j / 2) & 1u, p.hdr, 3))) break;
-                    if (j >= 2 && !(ok = attn_wait(bars + B_SFREE + s, (uint32_t)((j / 2) - 1) & 1u, p.hdr, 4)))
-                        break;
-                    tc_fence_after();
-                    const uint32_t k_base = smem_u32(smem + OFF_K + s * kKBytes);
+        // the whole (converged) warp runs the loop, so descriptors and TMEM
+        // addresses stay warp-uniform; elect.sync picks the lane that issues
+        const uint32_t idesc_s = umma_idesc_bf16(kQT, kKT), idesc_o = umma_idesc_bf16(kQT, kHd);
+        bool ok = attn_warp_wait(bars + B_QFULL, 0, p.hdr, 2);
+        for (int j = 0; ok && j <= n; ++j) {
+            if (j < n) {
+                const int s = j % kStages;
+                if (!(ok = attn_warp_wait(bars + B_KFULL + s, (uint32_t)(j / kStages) & 1u, p.hdr, 3))) break;
+                // the single score buffer: tile j - 1 has been read
+                if (j >= 1 && !(ok = attn_warp_wait(bars + B_SFREE, (uint32_t)(j - 1) & 1u, p.hdr, 4))) break;
+                tc_fence_after();
+                const uint64_t kd0 = umma_desc_sw128(smem_u32(smem + OFF_K + s * kKBytes));
 #pragma unroll
-                    for (int kk = 0; kk < kHd / 16; ++kk) {
-                        // 64-channel box kk / 4, 16-channel step kk % 4 (32 bytes into each swizzled row)
-                        const uint32_t off = (uint32_t)(kk >> 2), in = (uint32_t)(kk & 3) * 32;
-                        umma_ss(tmem + kColS + (uint32_t)(s * kKT), umma_desc_sw128(q_base + off * kQBox + in),
-                                umma_desc_sw128(k_base + off * kKBox + in), idesc_s, kk > 0);
-                    }
-                    umma_commit(bars + B_SFULL + s);
-                    umma_commit(bars + B_KFREE + s);
+                for (int kk = 0; kk < kHd / 16; ++kk) {
+                    // A: 16 channels of Q from TMEM (8 columns); B: 64-channel box kk / 4,
+                    // 16-channel step kk % 4 (32 bytes into each swizzled row; the
+                    // descriptor's start field counts 16-byte units)
+                    const uint32_t off = (uint32_t)(kk >> 2) * kKBox + (uint32_t)(kk & 3) * 32;
+                    umma_ts_warp(tmem + kColS, tmem + kColQ + (uint32_t)kk * 8, kd0 + (off >> 4), idesc_s, kk > 0);
                 }
-                if (j >= 1) {
-                    const int i = j - 1, s = i % 2;
-                    if (!(ok = attn_wait(bars + B_PFULL + s, (uint32_t)(i / 2) & 1u, p.hdr, 5))) break;
-                    if (!(ok = attn_wait(bars + B_VFULL + s, (uint32_t)(i / 2) & 1u, p.hdr, 6))) break;
-                    tc_fence_after();
-                    const uint32_t v_base = smem_u32(smem + OFF_V + s * kVBytes);
+                umma_commit_warp(bars + B_SFULL);
+                umma_commit_warp(bars + B_KFREE + s);
+            }
+            if (j >= 1) {
+                const int i = j - 1, pb = i % 2, s = i % kStages;
+                if (!(ok = attn_warp_wait(bars + B_PFULL + pb, (uint32_t)(i / 2) & 1u, p.hdr, 5))) break;
+                if (!(ok = attn_warp_wait(bars + B_VFULL + s, (uint32_t)(i / kStages) & 1u, p.hdr, 6))) break;
+                tc_fence_after();
+                const uint64_t vd0 = umma_desc_sw128(smem_u32(smem + OFF_V + s * kVBytes));
 #pragma unroll
-                    for (int kk = 0; kk < kKT / 16; ++kk)
-                        umma_ts(tmem + kColO, tmem + kColP + (uint32_t)(s * 32 + kk * 8),
-                                umma_desc_sw128(v_base + (uint32_t)kk * 32), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(bars + B_PVDONE + s);
-                    umma_commit(bars + B_VFREE + s);
-                }
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    umma_ts_warp(tmem + kColO, tmem + kColP + (uint32_t)(pb * 32 + kk * 8), vd0 + (uint64_t)(kk * 2),
+                                 idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+                umma_commit_warp(bars + B_PVDONE + pb);
+                umma_commit_warp(bars + B_VFREE + s);
             }
-            if (!ok) {
-                // the MMAs in flight finish before TMEM is freed
-                umma_commit(bars + B_DRAIN);
-                drain_wait(bars + B_DRAIN, 0);
-            }
+            __syncwarp();
+        }
+        if (!ok) {
+            // the MMAs in flight finish before TMEM is freed
+            umma_commit_warp(bars + B_DRAIN);
+            if (lane == 0) drain_wait(bars + B_DRAIN, 0);
         }
         __syncwarp();
     } else {
@@ -281,25 +293,46 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
         const int lo = live ? row_lo(p, b, t) : INT_MAX;
         const int hi = live ? t : -1;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        {
+            // this row of the Q tile into its TMEM lane: 256 bf16 = 128 columns
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.qkv + ((size_t)b * p.T + (live ? t : 0)) * (size_t)((p.H + 2) * kHd) + (size_t)h * kHd);
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t r[32];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 v = live ? __ldg(src + q * 8 + k) : make_uint4(0, 0, 0, 0);
+                    r[4 * k] = v.x;
+                    r[4 * k + 1] = v.y;
+                    r[4 * k + 2] = v.z;
+                    r[4 * k + 3] = v.w;
+                }
+                tmem_st32(tmem + lane_off + kColQ + (uint32_t)(q * 32), r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bars + B_QFULL);
+        }
         const float kScale = 1.4426950408889634f / 16.f;  // log2(e) / sqrt(256)
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
 #pragma unroll 1
         for (int j = 0; j < n; ++j) {
-            const int s = j % 2, s0 = (j0 + j) * kKT;
-            if (!(ok = attn_warp_wait(bars + B_SFULL + s, (uint32_t)(j / 2) & 1u, p.hdr, 7))) break;
+            const int pb = j % 2, s0 = (j0 + j) * kKT;
+            if (!(ok = attn_warp_wait(bars + B_SFULL, (uint32_t)j & 1u, p.hdr, 7))) break;
             tc_fence_after();
             uint32_t ra[32], rb[32];
-            tmem_ld32(tmem + lane_off + kColS + (uint32_t)(s * kKT), ra);
-            tmem_ld32(tmem + lane_off + kColS + (uint32_t)(s * kKT + 32), rb);
+            tmem_ld32(tmem + lane_off + kColS, ra);
+            tmem_ld32(tmem + lane_off + kColS + 32, rb);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(bars + B_SFREE + s);
-            float v[64];
+            mbar_arrive(bars + B_SFREE);
+            float v[64];  // raw scores; the scale is folded into the exponent below
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                v[e] = __uint_as_float(ra[e]) * kScale;
-                v[e + 32] = __uint_as_float(rb[e]) * kScale;
+                v[e] = __uint_as_float(ra[e]);
+                v[e + 32] = __uint_as_float(rb[e]);
             }
             const bool inside = s0 >= lo && s0 + kKT - 1 <= hi;
             if (!__all_sync(0xffffffffu, inside)) {
@@ -307,9 +340,13 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
                 for (int e = 0; e < 64; ++e)
                     if (s0 + e < lo || s0 + e > hi) v[e] = -INFINITY;
             }
-            float mt = v[0];
+            float m8[8];
 #pragma unroll
-            for (int e = 1; e < 64; ++e) mt = fmaxf(mt, v[e]);
+            for (int e = 0; e < 8; ++e) m8[e] = v[e];
+#pragma unroll
+            for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], v[e]);
+            const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * kScale;
             const float m_new = fmaxf(m_ref, mt);
             const bool grow = m_new > m_ref + kRescaleLog2;  // false while the row has no key yet
             const bool rescale = grow && m_ref != -INFINITY;
@@ -337,19 +374,23 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
             }
             const float mu = m_ref == -INFINITY ? 0.f : m_ref;
             uint32_t pk[32];
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const float p0 = ex2_approx(v[2 * e] - mu), p1 = ex2_approx(v[2 * e + 1] - mu);
-                l += p0 + p1;
+                const float p0 = ex2_approx(fmaf(v[2 * e], kScale, -mu));
+                const float p1 = ex2_approx(fmaf(v[2 * e + 1], kScale, -mu));
+                l4[e & 3] += p0 + p1;
                 pk[e] = pack_bf16(p0, p1);
             }
-            // P buffer s was last read by the MMAs of tile j - 2
-            if (j >= 2 && !(ok = attn_warp_wait(bars + B_PVDONE + s, (uint32_t)((j / 2) - 1) & 1u, p.hdr, 9))) break;
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            // P buffer pb was last read by the MMAs of tile j - 2
+            if (j >= 2 && !(ok = attn_warp_wait(bars + B_PVDONE + pb, (uint32_t)((j / 2) - 1) & 1u, p.hdr, 9)))
+                break;
             tc_fence_after();
-            tmem_st32(tmem + lane_off + kColP + (uint32_t)(s * 32), pk);
+            tmem_st32(tmem + lane_off + kColP + (uint32_t)(pb * 32), pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bars + B_PFULL + s);
+            mbar_arrive(bars + B_PFULL + pb);
         }
         if (ok && n > 0 && attn_warp_wait(bars + B_PVDONE + (n - 1) % 2, (uint32_t)((n - 1) / 2) & 1u, p.hdr, 10)) {
             tc_fence_after();
@@ -438,6 +479,217 @@ rglru_mqa_rope_kernel(int T, int H, int Tp, __nv_bfloat16 *__restrict__ qkv, con
 }
 static_assert(kRopeThreads == kHd, "one thread per v channel");
 
+// ---------------------------------------------------------------- decode step
+// One token per sequence at document position pos attends the cached keys of
+// positions max(0, pos - window + 1) .. pos; the cache keeps position q at
+// slot q % window.  HBM bound (1 KB of K and V per key and sequence), so it
+// runs on the CUDA cores: a split over 256-key chunks, one CTA per (chunk,
+// sequence), then a combine kernel.  Every CTA of a sequence rotates q and k
+// itself; the CTA whose chunk holds pos first writes this token's rotated k
+// and its v into the cache slot, and only it reads that slot.
+constexpr int kDecKeys = 256;   // keys per CTA
+constexpr int kDecThreads = 256;
+constexpr int kDecMaxH = 16;
+
+struct DecParams {
+    int B, H, window, nch;
+    const __nv_bfloat16 *qkv;   // [B, (H + 2) * 256]
+    const int32_t *segpos;      // [B]
+    __nv_bfloat16 *kc, *vc;     // [B, window, 256]
+    float *part_o;              // [B, nch, H, 256]
+    float *part_ml;             // [B, nch, H, 2]: chunk max (log2 units) and sum
+    __nv_bfloat16 *out;         // [B, H * 256]
+};
+
+__device__ __forceinline__ f2_t bf16x2_to_f2(uint32_t w)
+{
+    return f2_make(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__global__ void __launch_bounds__(kDecThreads)
+rglru_mqa_decode_kernel(const DecParams p)
+{
+    __shared__ __align__(16) float qs[kDecMaxH][kHd];       // rotated q (bf16 values) in fp32
+    __shared__ __align__(16) float ps[kDecMaxH][kDecKeys];  // probabilities; later the second half's O
+    __shared__ float red[kDecThreads / 32][kDecMaxH];
+    __shared__ float mch[kDecMaxH], lch[kDecMaxH];
+    __shared__ float2 cs[kHd / 2];
+    const int b = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H, W = p.window;
+    const int pos = max(p.segpos[b], 0);
+    const int n = min(pos + 1, W);
+    const int i0 = c * kDecKeys;
+    if (i0 >= n) return;  // the whole CTA
+    const int lo = pos - n + 1;
+    const size_t C = (size_t)(H + 2) * kHd;
+    const __nv_bfloat16 *row = p.qkv + (size_t)b * C;
+    if (tid < kHd / 2) {
+        const double inv = exp2(-(double)tid * (13.287712379549449 / 128.0));
+        double turns = (double)pos * inv * 0.15915494309189535;
+        turns -= floor(turns);
+        float sn, co;
+        sincospif((float)(2.0 * turns), &sn, &co);
+        cs[tid] = make_float2(co, sn);
+    }
+    __syncthreads();
+    const bool owner = c == (n - 1) / kDecKeys;  // this CTA's chunk holds position pos
+    __nv_bfloat16 *kslot = p.kc + ((size_t)b * W + pos % W) * kHd;
+    for (int e = tid; e < (H + 1) * (kHd / 2); e += kDecThreads) {
+        const int hh = e / (kHd / 2), i = e % (kHd / 2);
+        const float x1 = __bfloat162float(row[hh * kHd + i]), x2 = __bfloat162float(row[hh * kHd + i + kHd / 2]);
+        const float2 r = cs[i];
+        const __nv_bfloat16 y1 = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
+        const __nv_bfloat16 y2 = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
+        if (hh < H) {
+            qs[hh][i] = __bfloat162float(y1);
+            qs[hh][i + kHd / 2] = __bfloat162float(y2);
+        } else if (owner) {
+            kslot[i] = y1;
+            kslot[i + kHd / 2] = y2;
+        }
+    }
+    if (owner) p.vc[((size_t)b * W + pos % W) * kHd + tid] = row[(H + 1) * kHd + tid];
+    __syncthreads();  // the slot's k and v (global) and q (shared) are visible to the CTA
+
+    // scores: thread = key
+    const float kScale = 1.4426950408889634f / 16.f;
+    const int key = i0 + tid;
+    const bool have = key < n;
+    float sc[kDecMaxH];
+    {
+        f2_t acc[kDecMaxH];
+#pragma unroll
+        for (int h = 0; h < kDecMaxH; ++h) acc[h] = 0ull;
+        if (have) {
+            const uint4 *kr = reinterpret_cast<const uint4 *>(p.kc + ((size_t)b * W + (lo + key) % W) * kHd);
+#pragma unroll 2
+            for (int c8 = 0; c8 < kHd / 8; ++c8) {
+                const uint4 kv = kr[c8];
+                const f2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
+                const f2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
+#pragma unroll
+                for (int h = 0; h < kDecMaxH; ++h) {
+                    if (h < H) {
+                        const float4 qa = *reinterpret_cast<const float4 *>(&qs[h][c8 * 8]);
+                        const float4 qb = *reinterpret_cast<const float4 *>(&qs[h][c8 * 8 + 4]);
+                        acc[h] = f2_fma(k01, f2_make(qa.x, qa.y), acc[h]);
+                        acc[h] = f2_fma(k23, f2_make(qa.z, qa.w), acc[h]);
+                        acc[h] = f2_fma(k45, f2_make(qb.x, qb.y), acc[h]);
+                        acc[h] = f2_fma(k67, f2_make(qb.z, qb.w), acc[h]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < kDecMaxH; ++h) sc[h] = have ? (f2_lo(acc[h]) + f2_hi(acc[h])) * kScale : -INFINITY;
+    }
+    // chunk max and sum per head
+#pragma unroll
+    for (int h = 0; h < kDecMaxH; ++h) {
+        if (h < H) {
+            float m = sc[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) red[warp][h] = m;
+        }
+    }
+    __syncthreads();
+    if (tid < H) {
+        float m = red[0][tid];
+        for (int w = 1; w < kDecThreads / 32; ++w) m = fmaxf(m, red[w][tid]);
+        mch[tid] = m;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < kDecMaxH; ++h) {
+        if (h < H) {
+            const float pr = have ? ex2_approx(sc[h] - mch[h]) : 0.f;
+            ps[h][tid] = pr;
+            float l = pr;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+            if (lane == 0) red[warp][h] = l;
+        }
+    }
+    __syncthreads();
+    if (tid < H) {
+        float l = 0.f;
+        for (int w = 0; w < kDecThreads / 32; ++w) l += red[w][tid];
+        lch[tid] = l;
+    }
+
+    // O partial: thread = (channel pair dp, half of the chunk's keys)
+    const int dp = tid % (kHd / 2), half = tid / (kHd / 2);
+    const int kb = half * (kDecKeys / 2), ke = min(kb + kDecKeys / 2, n - i0);
+    f2_t o[kDecMaxH];
+#pragma unroll
+    for (int h = 0; h < kDecMaxH; ++h) o[h] = 0ull;
+    if (kb < ke) {
+        int slot = (lo + i0 + kb) % W;
+#pragma unroll 2
+        for (int kk = kb; kk < ke; ++kk) {
+            const uint32_t vv = *reinterpret_cast<const uint32_t *>(p.vc + ((size_t)b * W + slot) * kHd + 2 * dp);
+            const f2_t v2 = bf16x2_to_f2(vv);
+#pragma unroll
+            for (int h = 0; h < kDecMaxH; ++h)
+                if (h < H) o[h] = f2_fma(f2_splat(ps[h][kk]), v2, o[h]);
+            slot = slot + 1 == W ? 0 : slot + 1;
+        }
+    }
+    __syncthreads();  // every thread is done with ps: the second half's O goes there
+    float2 *oh = reinterpret_cast<float2 *>(&ps[0][0]);  // [kDecMaxH][128] float2
+    if (half == 1) {
+#pragma unroll
+        for (int h = 0; h < kDecMaxH; ++h)
+            if (h < H) oh[h * (kHd / 2) + dp] = make_float2(f2_lo(o[h]), f2_hi(o[h]));
+    }
+    __syncthreads();
+    if (half == 0) {
+        const size_t base = ((size_t)b * p.nch + c) * H;
+#pragma unroll
+        for (int h = 0; h < kDecMaxH; ++h) {
+            if (h < H) {
+                const float2 q2 = oh[h * (kHd / 2) + dp];
+                reinterpret_cast<float2 *>(p.part_o + (base + h) * kHd)[dp] =
+                    make_float2(f2_lo(o[h]) + q2.x, f2_hi(o[h]) + q2.y);
+            }
+        }
+    }
+    if (tid < H) {
+        const size_t base = ((size_t)b * p.nch + c) * H + tid;
+        p.part_ml[2 * base] = mch[tid];
+        p.part_ml[2 * base + 1] = lch[tid];
+    }
+}
+
+// out[b, h] = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c over the chunks of sequence b
+__global__ void __launch_bounds__(kHd)
+rglru_mqa_decode_combine_kernel(const DecParams p)
+{
+    const int b = blockIdx.x, d = threadIdx.x, H = p.H;
+    const int pos = max(p.segpos[b], 0);
+    const int n = min(pos + 1, p.window);
+    const int nc = (n + kDecKeys - 1) / kDecKeys;
+    for (int h = 0; h < H; ++h) {
+        float M = -INFINITY;
+        for (int c = 0; c < nc; ++c) M = fmaxf(M, p.part_ml[2 * (((size_t)b * p.nch + c) * H + h)]);
+        float num = 0.f, den = 0.f;
+        for (int c = 0; c < nc; ++c) {
+            const size_t base = ((size_t)b * p.nch + c) * H + h;
+            const float f = ex2_approx(p.part_ml[2 * base] - M);
+            num = fmaf(f, p.part_o[base * kHd + d], num);
+            den = fmaf(f, p.part_ml[2 * base + 1], den);
+        }
+        p.out[(size_t)b * H * kHd + (size_t)h * kHd + d] = __float2bfloat16_rn(num / den);
+    }
+}
+
+size_t dec_part_bytes(int B, int H, int window)
+{
+    const size_t nch = (size_t)((window + kDecKeys - 1) / kDecKeys);
+    return align_up((size_t)B * nch * H * kHd * 4, 256) + align_up((size_t)B * nch * H * 2 * 4, 256);
+}
+
 bool al16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 constexpr int64_t kMaxRows = int64_t(1) << 30;
 
@@ -466,12 +718,11 @@ rglru_status mqa_attention_launch(int B, int T, int H, int window, const void *q
     if (!encode) return RGLRU_ERR_CUDA;
     const int Tp = (T + 7) / 8 * 8;
     const cuuint64_t cols = (cuuint64_t)(H + 2) * kHd;
-    CUtensorMap tm_q, tm_k, tm_v;
-    const cuuint64_t qdim[3] = {cols, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t qstride[2] = {cols * 2, cols * 2 * (cuuint64_t)T};
-    const cuuint32_t qbox[3] = {64, kQT, 1}, kbox[3] = {64, kKT, 1};
-    if (!encode_bf16(encode, &tm_q, qkv, 3, qdim, qstride, qbox, CU_TENSOR_MAP_SWIZZLE_128B)) return RGLRU_ERR_CUDA;
-    if (!encode_bf16(encode, &tm_k, qkv, 3, qdim, qstride, kbox, CU_TENSOR_MAP_SWIZZLE_128B)) return RGLRU_ERR_CUDA;
+    CUtensorMap tm_k, tm_v;
+    const cuuint64_t kdim[3] = {cols, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t kstride[2] = {cols * 2, cols * 2 * (cuuint64_t)T};
+    const cuuint32_t kbox[3] = {64, kKT, 1};
+    if (!encode_bf16(encode, &tm_k, qkv, 3, kdim, kstride, kbox, CU_TENSOR_MAP_SWIZZLE_128B)) return RGLRU_ERR_CUDA;
     const cuuint64_t vdim[3] = {(cuuint64_t)Tp, (cuuint64_t)kHd, (cuuint64_t)B};
     const cuuint64_t vstride[2] = {(cuuint64_t)Tp * 2, (cuuint64_t)Tp * 2 * kHd};
     const cuuint32_t vbox[3] = {kKT, kHd, 1};
@@ -483,6 +734,7 @@ rglru_status mqa_attention_launch(int B, int T, int H, int window, const void *q
     p.H = H;
     p.window = window;
     p.ntiles = (T + kQT - 1) / kQT;
+    p.qkv = static_cast<const __nv_bfloat16 *>(qkv);
     p.segpos = segpos;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.hdr = static_cast<WsHeader *>(ws);
@@ -490,7 +742,7 @@ rglru_status mqa_attention_launch(int B, int T, int H, int window, const void *q
     const rglru_status st = set_smem_limit_once((const void *)rglru_mqa_attention_kernel, kSmemBytes, smem_set);
     if (st != RGLRU_OK) return st;
     const unsigned grid = (unsigned)((int64_t)B * p.ntiles * H);
-    rglru_mqa_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p, tm_q, tm_k, tm_v);
+    rglru_mqa_attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p, tm_k, tm_v);
     return cuda_status(cudaGetLastError());
 }
 
@@ -585,6 +837,55 @@ RGLRU_API rglru_status rglru_mqa_block_prefill(int B, int T, int D, int window, 
     st = mqa_attention_launch(B, T, H, window, qkv, vt, segment_pos, att, ws, stream);
     if (st != RGLRU_OK) return st;
     return rglru_linear((int)M, D, D, att, W_o, b_o, out, ws, kWsHeaderBytes, stream);
+}
+
+RGLRU_API size_t rglru_mqa_decode_workspace_size(int B, int H, int window)
+{
+    if (B < 1 || B > 65535 || H < 1 || H > kDecMaxH || window < 1 || window > (1 << 20)) return 0;
+    return kWsHeaderBytes + dec_part_bytes(B, H, window);
+}
+
+RGLRU_API rglru_status rglru_mqa_decode_step(int B, int H, int window, const void *qkv, const int32_t *segment_pos,
+                                             void *k_cache, void *v_cache, void *out, void *workspace,
+                                             size_t workspace_bytes, cudaStream_t stream)
+{
+    const size_t need = rglru_mqa_decode_workspace_size(B, H, window);
+    if (need == 0) return RGLRU_ERR_UNSUPPORTED;
+    if (!al16(qkv) || !al16(k_cache) || !al16(v_cache) || !al16(out) || segment_pos == nullptr)
+        return RGLRU_ERR_INVALID_ARG;
+    if (workspace == nullptr || !al16(workspace) || workspace_bytes < need) return RGLRU_ERR_WORKSPACE;
+    const size_t cache = (size_t)B * window * kHd * 2;
+    const struct {
+        const void *p;
+        size_t n;
+    } bufs[] = {{qkv, (size_t)B * (H + 2) * kHd * 2}, {segment_pos, (size_t)B * 4}, {k_cache, cache},
+                {v_cache, cache}, {out, (size_t)B * H * kHd * 2}, {workspace, workspace_bytes}};
+    // the caches, out and the workspace are written: none may overlap another buffer
+    for (int i = 0; i < 6; ++i)
+        for (int j = i + 1; j < 6; ++j) {
+            const bool written = i >= 2 || j >= 2;
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(bufs[i].p), a1 = a0 + bufs[i].n;
+            const uintptr_t b0 = reinterpret_cast<uintptr_t>(bufs[j].p), b1 = b0 + bufs[j].n;
+            if (written && a0 < b1 && b0 < a1) return RGLRU_ERR_INVALID_ARG;
+        }
+    DecParams p;
+    p.B = B;
+    p.H = H;
+    p.window = window;
+    p.nch = (window + kDecKeys - 1) / kDecKeys;
+    p.qkv = static_cast<const __nv_bfloat16 *>(qkv);
+    p.segpos = segment_pos;
+    p.kc = static_cast<__nv_bfloat16 *>(k_cache);
+    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
+    char *ws = static_cast<char *>(workspace) + kWsHeaderBytes;
+    p.part_o = reinterpret_cast<float *>(ws);
+    p.part_ml = reinterpret_cast<float *>(ws + align_up((size_t)B * p.nch * H * kHd * 4, 256));
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    rglru_mqa_decode_kernel<<<dim3((unsigned)p.nch, (unsigned)B), kDecThreads, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return RGLRU_ERR_CUDA;
+    rglru_mqa_decode_combine_kernel<<<(unsigned)B, kHd, 0, stream>>>(p);
+    return cuda_status(cudaGetLastError());
 }
 
 }  // extern "C"

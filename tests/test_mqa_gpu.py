@@ -178,3 +178,58 @@ def test_mqa_block_matches_oracle(B, T, D, doc_len, window):
     assert api.device_status(ws) == api.OK
     ref = _oracle_block(inp, window)
     check_bf16(out.float().cpu().numpy(), ref["out"], "mqa block out")
+
+
+@pytest.mark.parametrize("B,T,H,window,doc_len", [(2, 300, 2, 64, None), (3, 200, 10, 2048, 60),
+                                                  (1, 600, 3, 300, 250), (2, 70, 16, 256, None)])
+def test_decode_steps_match_oracle(B, T, H, window, doc_len):
+    """T decode steps from empty rings (window 64 and 300 wrap the ring; 16
+    heads is the 9B shape's count): each step's output against the oracle's
+    attention over the same rotated, bf16-rounded q, k and v; the rings hold
+    the rotated keys and the values at slot position % window."""
+    qkv, seg = _qkv(B, T, H, seed=7, doc_len=doc_len)
+    dq = torch.from_numpy(qkv).to(dev).to(bf)
+    ds = torch.from_numpy(seg).to(dev)
+    kc, vc = api.mqa_cache(B, window, dev)
+    ws = api.new_workspace(api.mqa_decode_workspace_size(B, H, window), dev)
+    outs = []
+    for t in range(T):
+        outs.append(api.mqa_decode_step(dq[:, t].contiguous(), ds[:, t].contiguous(), kc, vc, workspace=ws))
+    got = torch.stack(outs, 1).float().cpu().numpy()
+    q, k, v = _split(qkv, H)
+    from oracle import block as oblock
+    qr, kr = oblock.round_bf16(omqa.rope(q, seg)), oblock.round_bf16(omqa.rope(k, seg))
+    want = omqa.attention(qr, kr, v, seg, window).reshape(B, T, H * 256)
+    _attn_bar(got, want, np.abs(v).max(), f"decode B={B} T={T} H={H} window={window}")
+    # the ring after the last step: slot p % window holds position p of the last document
+    kcn, vcn = kc.float().cpu().numpy(), vc.float().cpu().numpy()
+    for b in range(B):
+        t_last = T - 1
+        p_last = int(seg[b, t_last])
+        for back in range(min(p_last + 1, window)):
+            t = t_last - back
+            slot = (p_last - back) % window
+            np.testing.assert_array_equal(vcn[b, slot], v[b, t])
+            err = np.abs(kcn[b, slot] - kr[b, t])
+            assert (err <= 2.0 ** -8 * np.abs(kr[b, t]) + 1e-5).all(), (b, t, float(err.max()))
+
+
+def test_decode_equals_prefill_rows():
+    """The decode step and the prefill kernels compute the same attention: the
+    last tokens of a sequence decoded one by one against the prefill's rows."""
+    B, T, H = 2, 400, 4
+    qkv, seg = _qkv(B, T, H, seed=8, doc_len=150)
+    dq = torch.from_numpy(qkv).to(dev).to(bf)
+    ds = torch.from_numpy(seg).to(dev)
+    pre_q = dq.clone()
+    vt = api.mqa_rope(pre_q, ds)
+    pre = api.mqa_attention(pre_q, vt, ds).float().cpu().numpy()
+    kc, vc = api.mqa_cache(B, 2048, dev)
+    dec = [api.mqa_decode_step(dq[:, t].contiguous(), ds[:, t].contiguous(), kc, vc).float().cpu().numpy()
+           for t in range(T)]
+    dec = np.stack(dec, 1)
+    _, _, v = _split(qkv, H)
+    # each side is within the attention bar of the exact value: twice the bar between them
+    err = np.abs(dec - pre)
+    bad = ~(err <= 2.0 ** -8 * np.abs(v).max() + 2.0 ** -7 * np.abs(pre) + 2e-6)
+    assert not bad.any(), f"decode vs prefill: {int(bad.sum())} outside, max err {err.max():.3e}"
