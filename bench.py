@@ -568,7 +568,7 @@ def run_mqa_decode(args, dev, stream, distributed, peaks, peak_kind):
     g = torch.Generator(device="cpu").manual_seed(wd.seed)
     qkv = torch.randn((B, (H + 2) * 256), generator=g).to(bf).to(dev)
     kc = torch.randn((B, window, 256), generator=g).to(bf).to(dev)
-    vc = torch.randn((B, window, 256), generator=g).to(bf).to(dev)
+    vc = torch.randn((B, 256, window), generator=g).to(bf).to(dev)
     sp = torch.from_numpy(seg).to(dev)
     out = torch.empty((B, H * 256), dtype=bf, device=dev)
     ws = api.new_workspace(api.mqa_decode_workspace_size(B, H, window), dev)

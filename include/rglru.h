@@ -428,7 +428,7 @@ RGLRU_API rglru_status rglru_mqa_block_prefill(int B, int T, int D, int window, 
                                                cudaStream_t stream);
 
 /* Workspace bytes of rglru_mqa_decode_step (0 on unsupported sizes:
- * 1 <= B <= 65535, 1 <= H <= 16, 1 <= window <= 2^20). */
+ * 1 <= B <= 65535, 1 <= H <= 16, window a multiple of 128 up to 2048). */
 RGLRU_API size_t rglru_mqa_decode_workspace_size(int B, int H, int window);
 
 /*
@@ -436,21 +436,47 @@ RGLRU_API size_t rglru_mqa_decode_workspace_size(int B, int H, int window);
  * each), after the QKV projection of that token:
  *   qkv         [B, (H + 2) * 256] bf16, read only: q heads, k, v of the token;
  *   segment_pos [B] int32 >= 0: the token's position in its document;
- *   k_cache, v_cache [B, window, 256] bf16, in/out: a ring per sequence, the
- *               rotated key and the value of document position p at slot
- *               p % window.  The step writes this token's slot, then attends
- *               positions max(0, p - window + 1) .. p of the cache (earlier
- *               steps of the same document must have written them);
+ *   k_cache     [B, window, 256] bf16, in/out: a ring per sequence, the rotated
+ *               key of document position q at slot q % window;
+ *   v_cache_t   [B, 256, window] bf16, in/out: the values, transposed (value
+ *               of position q in column q % window);
  *   out         [B, H * 256] bf16.
- * q and k are rotated (RoPE at segment_pos) and rounded to bf16 as in
- * rglru_mqa_rope; scores and sums in fp32; out rounded to bf16.  Two kernels:
- * per (256-key chunk, sequence) partial maxima, sums and outputs in the
- * workspace, then their combination.  No buffer may overlap another one that
- * the step writes.
+ * The step writes this token's slot, then attends positions
+ * max(0, p - window + 1) .. p (earlier steps of the same document must have
+ * written them).  Every slot of both rings must hold finite values (zero-fill
+ * them before first use): slots outside the attended range enter the
+ * products with probability 0.  q and k are rotated (RoPE at segment_pos) and
+ * rounded to bf16 as in rglru_mqa_rope; scores on the tensor cores in fp32,
+ * probabilities as bf16 operands, sums in fp32, out rounded to bf16.  Two
+ * kernels: per (sequence, block of 128 positions) partial maxima, sums and
+ * outputs in the workspace, then their combination.  No buffer may overlap
+ * another one that the step writes.
  */
 RGLRU_API rglru_status rglru_mqa_decode_step(int B, int H, int window, const void *qkv, const int32_t *segment_pos,
-                                             void *k_cache, void *v_cache, void *out, void *workspace,
+                                             void *k_cache, void *v_cache_t, void *out, void *workspace,
                                              size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes of rglru_mqa_residual_block_prefill (0 on bad sizes). */
+RGLRU_API size_t rglru_mqa_residual_block_workspace_size(int B, int T, int D, int F);
+
+/*
+ * The residual block with local MQA ("Residual block with local MQA" and the
+ * decoder-layer printout: norm, temporal block, residual, norm, MLP,
+ * residual) over T tokens of B sequences, bf16:
+ *   n   = RMSNorm(u) (w_temporal_norm)
+ *   h   = u + o_proj(local MQA(RoPE(q_proj n), RoPE(k_proj n), v_proj n))
+ *   n'  = RMSNorm(h) (w_channel_norm)
+ *   out = h + down_proj(GELU_tanh(gate_proj(n')) * up_proj(n'))
+ * W_qkv, W_o, b_o as rglru_mqa_block_prefill; the MLP as
+ * rglru_residual_block_prefill (W_gate, W_up [F, D], W_down [D, F]); every
+ * intermediate is a bf16 tensor in the workspace (zero-filled once), which
+ * carries one status word for all the launches.
+ */
+RGLRU_API rglru_status rglru_mqa_residual_block_prefill(
+    int B, int T, int D, int F, int window, const void *u, const float *w_temporal_norm, const void *W_qkv,
+    const void *W_o, const float *b_o, const int32_t *segment_pos, const float *w_channel_norm, const void *W_gate,
+    const float *b_gate, const void *W_up, const float *b_up, const void *W_down, const float *b_down, float eps,
+    void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

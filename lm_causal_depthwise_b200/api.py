@@ -29,7 +29,8 @@ SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglr
            "rglru_linear_geglu", "rglru_recurrent_block_workspace_size", "rglru_recurrent_block_prefill",
            "rglru_rmsnorm", "rglru_residual_block_workspace_size", "rglru_residual_block_prefill",
            "rglru_mqa_vt_size", "rglru_mqa_rope", "rglru_mqa_attention", "rglru_mqa_block_workspace_size",
-           "rglru_mqa_block_prefill", "rglru_mqa_decode_workspace_size", "rglru_mqa_decode_step")
+           "rglru_mqa_block_prefill", "rglru_mqa_decode_workspace_size", "rglru_mqa_decode_step",
+           "rglru_mqa_residual_block_workspace_size", "rglru_mqa_residual_block_prefill")
 
 _lib = None
 
@@ -110,6 +111,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_mqa_decode_workspace_size.argtypes = [i, i, i]
     lib.rglru_mqa_decode_step.restype = i
     lib.rglru_mqa_decode_step.argtypes = [i, i, i] + [vp] * 6 + [sz, vp]
+    lib.rglru_mqa_residual_block_workspace_size.restype = sz
+    lib.rglru_mqa_residual_block_workspace_size.argtypes = [i, i, i, i]
+    lib.rglru_mqa_residual_block_prefill.restype = i
+    lib.rglru_mqa_residual_block_prefill.argtypes = [i, i, i, i, i] + [vp] * 13 + [ctypes.c_float, vp, vp, sz, vp]
     _lib = lib
     return lib
 
@@ -706,15 +711,16 @@ def mqa_decode_workspace_size(B: int, H: int, window: int = MQA_WINDOW) -> int:
 
 
 def mqa_cache(B: int, window: int = MQA_WINDOW, device="cuda"):
-    """Zero-filled key and value rings [B, window, 256] bf16."""
+    """Zero-filled rings: keys [B, window, 256] and values transposed [B, 256, window], bf16."""
     return (torch.zeros((B, window, 256), dtype=torch.bfloat16, device=device),
-            torch.zeros((B, window, 256), dtype=torch.bfloat16, device=device))
+            torch.zeros((B, 256, window), dtype=torch.bfloat16, device=device))
 
 
-def mqa_decode_step(qkv, segment_pos, k_cache, v_cache, out=None, workspace=None) -> torch.Tensor:
+def mqa_decode_step(qkv, segment_pos, k_cache, v_cache_t, out=None, workspace=None) -> torch.Tensor:
     """One local-MQA decode step (rglru_mqa_decode_step): qkv [B, (H + 2) * 256]
-    bf16 of the new token, segment_pos [B] int32, the rings k_cache / v_cache
-    [B, window, 256] (updated in place); returns out [B, H * 256] bf16."""
+    bf16 of the new token, segment_pos [B] int32, the rings k_cache [B, window,
+    256] and v_cache_t [B, 256, window] (updated in place); returns out
+    [B, H * 256] bf16."""
     if qkv.dim() != 2 or qkv.shape[1] % 256 != 0 or qkv.shape[1] < 768:
         raise ValueError("qkv must be [B, (H + 2) * 256]")
     B, C = qkv.shape
@@ -724,15 +730,83 @@ def mqa_decode_step(qkv, segment_pos, k_cache, v_cache, out=None, workspace=None
     _check(qkv, "qkv", (B, C), torch.bfloat16, dev)
     _check(segment_pos, "segment_pos", (B,), torch.int32, dev)
     _check(k_cache, "k_cache", (B, window, 256), torch.bfloat16, dev)
-    _check(v_cache, "v_cache", (B, window, 256), torch.bfloat16, dev)
+    _check(v_cache_t, "v_cache_t", (B, 256, window), torch.bfloat16, dev)
     if out is None:
         out = torch.empty((B, H * 256), dtype=torch.bfloat16, device=dev)
     _check(out, "out", (B, H * 256), torch.bfloat16, dev)
     if workspace is None:
         workspace = new_workspace(mqa_decode_workspace_size(B, H, window), dev)
-    st = load().rglru_mqa_decode_step(B, H, window, _ptr(qkv), _ptr(segment_pos), _ptr(k_cache), _ptr(v_cache),
+    st = load().rglru_mqa_decode_step(B, H, window, _ptr(qkv), _ptr(segment_pos), _ptr(k_cache), _ptr(v_cache_t),
                                       _ptr(out), _ptr(workspace),
                                       ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
     if st != OK:
         raise RGLRUError(st, "rglru_mqa_decode_step")
+    return out
+
+
+@dataclass
+class MQAResidualParams:
+    """The residual block with local MQA: RMSNorm scales [D] fp32, the MQA
+    projections (MQAParams) and the MLP (bf16 weights, fp32 biases)."""
+    w_temporal_norm: torch.Tensor
+    mqa: MQAParams
+    w_channel_norm: torch.Tensor
+    W_gate: torch.Tensor
+    b_gate: torch.Tensor
+    W_up: torch.Tensor
+    b_up: torch.Tensor
+    W_down: torch.Tensor
+    b_down: torch.Tensor
+
+    @staticmethod
+    def from_arrays(inp: dict, device="cuda") -> "MQAResidualParams":
+        def w(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).to(torch.bfloat16).contiguous()
+
+        def f32(a):
+            return torch.as_tensor(a, dtype=torch.float32).to(device).contiguous()
+        return MQAResidualParams(f32(inp["w_temporal_norm"]), MQAParams.from_arrays(inp, device),
+                                 f32(inp["w_channel_norm"]), w(inp["W_gate"]), f32(inp["b_gate"]), w(inp["W_up"]),
+                                 f32(inp["b_up"]), w(inp["W_down"]), f32(inp["b_down"]))
+
+
+def mqa_residual_block_workspace_size(B: int, T: int, D: int, F: int) -> int:
+    n = int(load().rglru_mqa_residual_block_workspace_size(B, T, D, F))
+    if n == 0:
+        raise RGLRUError(ERR_INVALID_ARG, "mqa_residual_block_workspace_size")
+    return n
+
+
+def mqa_residual_block_prefill(u, rp: MQAResidualParams, segment_pos, window: int = MQA_WINDOW, eps: float = 1e-6,
+                               out=None, workspace=None) -> torch.Tensor:
+    """The residual block with local MQA over u [B,T,D] bf16 (rglru_mqa_residual_block_prefill)."""
+    if u.dim() != 3:
+        raise ValueError("u must be [B,T,D]")
+    B, T, D = u.shape
+    dev = u.device
+    F = rp.W_gate.shape[0]
+    _check(u, "u", (B, T, D), torch.bfloat16, dev)
+    for n in ("w_temporal_norm", "w_channel_norm"):
+        _check(getattr(rp, n), n, (D,), torch.float32, dev)
+    _check(rp.mqa.W_qkv, "W_qkv", (D + 512, D), torch.bfloat16, dev)
+    _check(rp.mqa.W_o, "W_o", (D, D), torch.bfloat16, dev)
+    _check(rp.mqa.b_o, "b_o", (D,), torch.float32, dev)
+    _check(rp.W_gate, "W_gate", (F, D), torch.bfloat16, dev)
+    _check(rp.W_up, "W_up", (F, D), torch.bfloat16, dev)
+    _check(rp.W_down, "W_down", (D, F), torch.bfloat16, dev)
+    for n, k in (("b_gate", F), ("b_up", F), ("b_down", D)):
+        _check(getattr(rp, n), n, (k,), torch.float32, dev)
+    _check(segment_pos, "segment_pos", (B, T), torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(u)
+    _check(out, "out", (B, T, D), torch.bfloat16, dev)
+    if workspace is None:
+        workspace = new_workspace(mqa_residual_block_workspace_size(B, T, D, F), dev)
+    st = load().rglru_mqa_residual_block_prefill(
+        B, T, D, F, int(window), _ptr(u), _ptr(rp.w_temporal_norm), _ptr(rp.mqa.W_qkv), _ptr(rp.mqa.W_o),
+        _ptr(rp.mqa.b_o), _ptr(segment_pos), _ptr(rp.w_channel_norm), _ptr(rp.W_gate), _ptr(rp.b_gate), _ptr(rp.W_up),
+        _ptr(rp.b_up), _ptr(rp.W_down), _ptr(rp.b_down), ctypes.c_float(eps), _ptr(out), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_mqa_residual_block_prefill")
     return out

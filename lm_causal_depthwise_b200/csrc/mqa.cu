@@ -481,212 +481,319 @@ static_assert(kRopeThreads == kHd, "one thread per v channel");
 
 // ---------------------------------------------------------------- decode step
 // One token per sequence at document position pos attends the cached keys of
-// positions max(0, pos - window + 1) .. pos; the cache keeps position q at
-// slot q % window.  HBM bound (1 KB of K and V per key and sequence), so it
-// runs on the CUDA cores: a split over 256-key chunks, one CTA per (chunk,
-// sequence), then a combine kernel.  Every CTA of a sequence rotates q and k
-// itself; the CTA whose chunk holds pos first writes this token's rotated k
-// and its v into the cache slot, and only it reads that slot.
-constexpr int kDecKeys = 256;   // keys per CTA
-constexpr int kDecThreads = 256;
-constexpr int kDecMaxH = 16;
+// positions lo = max(0, pos - window + 1) .. pos.  The rings keep position q
+// at slot q % window: k_cache [B, window, 256] (rotated keys) and v_cache
+// transposed, [B, 256, window], so that both tiles below are K-major operands.
+// One CTA per (sequence, block of 128 positions aligned to 128), 128 threads:
+//   TMA loads the block's K tile (4 boxes [128 keys x 64 channels], 128-byte
+//   swizzle) while the threads rotate q and write it (heads padded to 16,
+//   bf16) into a swizzled tile;
+//   S^T = K Q^T        M = 128 keys, N = 16 heads, K = 256   (tcgen05, TMEM);
+//   once S is done the same 64 KB buffer receives the V^T tile (4 boxes
+//   [128 channels x 64 keys]) while the softmax runs over the block's keys
+//   per head (thread = key, keys outside [lo, pos] masked; P^T written bf16
+//   into a swizzled tile);
+//   O^T = V^T P^T      M = 128 channels (two halves), N = 16, K = 128 keys;
+// one 64 KB tile buffer per CTA lets two CTAs share an SM, so one CTA's loads
+// run under the other's arithmetic;
+// then the block's (max, sum, O) per head go to the workspace and a combine
+// kernel merges the blocks.  The CTA whose block holds pos writes this token's
+// rotated k and its v into its tiles (after the loads land) and into the rings.
+// The rings must hold finite values in every slot (zero-filled at first use):
+// masked keys enter the products with probability 0.
+constexpr int kDecKeys = 128;                    // keys per CTA (TMEM lanes)
+constexpr int kDecThreads = 128;
+constexpr int kDecMaxH = 16;                     // heads padded to the MMA's N
+constexpr int kDecKBox = kDecKeys * 64 * 2;      // 16 KB: [128 keys x 64 channels]
+constexpr int kDecVBox = 128 * 64 * 2;           // 16 KB: [128 channels x 64 keys]
+constexpr int kDecQBox = kDecMaxH * 128;         // 2 KB:  [16 heads x 64 channels]
+constexpr int kDecPBox = kDecMaxH * 128;         // 2 KB:  [16 heads x 64 keys]
+static_assert(kDecKBox == kDecVBox, "K and V^T tiles share one buffer");
+constexpr int DOFF_K = 0, DOFF_V = 0, DOFF_Q = DOFF_K + 4 * kDecKBox;
+constexpr int DOFF_P = DOFF_Q + 4 * kDecQBox, DOFF_BAR = DOFF_P + 2 * kDecPBox, DOFF_MISC = DOFF_BAR + 4 * 8;
+constexpr int kDecSmem = DOFF_MISC + 16 + 1024;
+static_assert(kDecSmem <= 227 * 1024, "shared memory budget");
+constexpr uint32_t kDecCols = 64;                // TMEM: S^T 16 columns, O^T 2 x 16
+constexpr uint64_t kDecTimeoutNs = 2000000000ull;
 
 struct DecParams {
     int B, H, window, nch;
     const __nv_bfloat16 *qkv;   // [B, (H + 2) * 256]
     const int32_t *segpos;      // [B]
-    __nv_bfloat16 *kc, *vc;     // [B, window, 256]
+    __nv_bfloat16 *kc;          // [B, window, 256]
+    __nv_bfloat16 *vtc;         // [B, 256, window]
     float *part_o;              // [B, nch, H, 256]
-    float *part_ml;             // [B, nch, H, 2]: chunk max (log2 units) and sum
+    float *part_ml;             // [B, nch, H, 2]: block max (log2 units) and sum
     __nv_bfloat16 *out;         // [B, H * 256]
+    WsHeader *hdr;
 };
 
-__device__ __forceinline__ f2_t bf16x2_to_f2(uint32_t w)
+// Byte offset of element (row, k) of a K-major tile of 64-element (128-byte)
+// rows in the 128-byte swizzled layout a TMA load writes: the 16-byte chunk
+// index is XORed with the row's index within its 8-row atom.
+__device__ __forceinline__ uint32_t sw128(int row, int k)
 {
-    return f2_make(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    return (uint32_t)row * 128u + ((uint32_t)(((k >> 3) ^ row) & 7) << 4) + (uint32_t)(k & 7) * 2u;
 }
 
-__global__ void __launch_bounds__(kDecThreads)
-rglru_mqa_decode_kernel(const DecParams p)
+// bounded wait by every thread of the CTA; false (status recorded) on timeout
+__device__ bool mqd_wait(uint64_t *bar, uint32_t parity, WsHeader *hdr, int where)
 {
-    __shared__ __align__(16) float qs[kDecMaxH][kHd];       // rotated q (bf16 values) in fp32
-    __shared__ __align__(16) float ps[kDecMaxH][kDecKeys];  // probabilities; later the second half's O
-    __shared__ float red[kDecThreads / 32][kDecMaxH];
-    __shared__ float mch[kDecMaxH], lch[kDecMaxH];
-    __shared__ float2 cs[kHd / 2];
-    const int b = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = p.H, W = p.window;
-    const int pos = max(p.segpos[b], 0);
-    const int n = min(pos + 1, W);
-    const int i0 = c * kDecKeys;
-    if (i0 >= n) return;  // the whole CTA
-    const int lo = pos - n + 1;
-    const size_t C = (size_t)(H + 2) * kHd;
-    const __nv_bfloat16 *row = p.qkv + (size_t)b * C;
-    if (tid < kHd / 2) {
-        const double inv = exp2(-(double)tid * (13.287712379549449 / 128.0));
-        double turns = (double)pos * inv * 0.15915494309189535;
-        turns -= floor(turns);
-        float sn, co;
-        sincospif((float)(2.0 * turns), &sn, &co);
-        cs[tid] = make_float2(co, sn);
-    }
-    __syncthreads();
-    const bool owner = c == (n - 1) / kDecKeys;  // this CTA's chunk holds position pos
-    __nv_bfloat16 *kslot = p.kc + ((size_t)b * W + pos % W) * kHd;
-    for (int e = tid; e < (H + 1) * (kHd / 2); e += kDecThreads) {
-        const int hh = e / (kHd / 2), i = e % (kHd / 2);
-        const float x1 = __bfloat162float(row[hh * kHd + i]), x2 = __bfloat162float(row[hh * kHd + i + kHd / 2]);
-        const float2 r = cs[i];
-        const __nv_bfloat16 y1 = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
-        const __nv_bfloat16 y2 = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
-        if (hh < H) {
-            qs[hh][i] = __bfloat162float(y1);
-            qs[hh][i + kHd / 2] = __bfloat162float(y2);
-        } else if (owner) {
-            kslot[i] = y1;
-            kslot[i + kHd / 2] = y2;
+    bool done = mbar_try_wait(bar, parity);
+    if (!done) {
+        const uint64_t t0 = globaltimer();
+        while (!(done = mbar_try_wait_sleep(bar, parity, 20000u)) && globaltimer() - t0 < kDecTimeoutNs) {
         }
     }
-    if (owner) p.vc[((size_t)b * W + pos % W) * kHd + tid] = row[(H + 1) * kHd + tid];
-    __syncthreads();  // the slot's k and v (global) and q (shared) are visible to the CTA
+    if (!__syncthreads_and(done ? 1 : 0)) {
+        if (threadIdx.x == 0) {
+            atomicCAS(&hdr->status, 0, (int)RGLRU_ERR_TIMEOUT);
+            atomicCAS(&hdr->detail, 0, (int)((blockIdx.y * gridDim.x + blockIdx.x) << 8) | (where + 1));
+        }
+        return false;
+    }
+    return true;
+}
 
-    // scores: thread = key
+__global__ void __launch_bounds__(kDecThreads, 2)
+rglru_mqa_decode_kernel(const DecParams p, const __grid_constant__ CUtensorMap tm_kc,
+                        const __grid_constant__ CUtensorMap tm_vt)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DOFF_BAR);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + DOFF_MISC);
+    __shared__ float2 cs[kHd / 2];
+    __shared__ __align__(16) __nv_bfloat16 kv_tok[2][kHd];  // this token's rotated k and its v
+    __shared__ float red[kDecThreads / 32][kDecMaxH];
+    __shared__ float mh[kDecMaxH], lh[kDecMaxH];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H, W = p.window;
+
+    if (warp == 0) {
+        tmem_alloc(tmem_holder, kDecCols);
+        if (lane == 0) {
+            for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+            mbar_fence_init();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    uint8_t *Kt = smem + DOFF_K, *Vt = smem + DOFF_V, *Qt = smem + DOFF_Q, *Pt = smem + DOFF_P;
+    const uint32_t idesc = umma_idesc_bf16(kDecKeys, kDecMaxH);
     const float kScale = 1.4426950408889634f / 16.f;
-    const int key = i0 + tid;
-    const bool have = key < n;
-    float sc[kDecMaxH];
-    {
-        f2_t acc[kDecMaxH];
-#pragma unroll
-        for (int h = 0; h < kDecMaxH; ++h) acc[h] = 0ull;
-        if (have) {
-            const uint4 *kr = reinterpret_cast<const uint4 *>(p.kc + ((size_t)b * W + (lo + key) % W) * kHd);
-#pragma unroll 2
-            for (int c8 = 0; c8 < kHd / 8; ++c8) {
-                const uint4 kv = kr[c8];
-                const f2_t k01 = bf16x2_to_f2(kv.x), k23 = bf16x2_to_f2(kv.y);
-                const f2_t k45 = bf16x2_to_f2(kv.z), k67 = bf16x2_to_f2(kv.w);
-#pragma unroll
-                for (int h = 0; h < kDecMaxH; ++h) {
-                    if (h < H) {
-                        const float4 qa = *reinterpret_cast<const float4 *>(&qs[h][c8 * 8]);
-                        const float4 qb = *reinterpret_cast<const float4 *>(&qs[h][c8 * 8 + 4]);
-                        acc[h] = f2_fma(k01, f2_make(qa.x, qa.y), acc[h]);
-                        acc[h] = f2_fma(k23, f2_make(qa.z, qa.w), acc[h]);
-                        acc[h] = f2_fma(k45, f2_make(qb.x, qb.y), acc[h]);
-                        acc[h] = f2_fma(k67, f2_make(qb.z, qb.w), acc[h]);
-                    }
-                }
+
+    // items (block c, sequence b), block-major; the CTA's k-th processed item
+    // uses phase k & 1 of each of its four barriers
+    bool ok = true;
+    uint32_t ph = 0;
+    for (int w = blockIdx.x; ok && w < p.B * p.nch; w += gridDim.x) {
+        const int b = w % p.B, c = w / p.B;
+        const int pos = max(p.segpos[b], 0);
+        const int n = min(pos + 1, W);
+        const int lo = pos - n + 1;
+        const int mblk = (lo >> 7) + c;  // this item's block of 128 positions
+        if (mblk > (pos >> 7)) continue;  // (uniform in the CTA)
+        const int p0 = mblk << 7;
+        const int slot0 = p0 % W;  // window is a multiple of 128: the block's slots are contiguous
+        const bool owner = mblk == (pos >> 7);
+
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bars + 0, 4 * kDecKBox);
+            for (int kb = 0; kb < 4; ++kb) tma_load_2d(Kt + kb * kDecKBox, &tm_kc, bars + 0, kb * 64, b * W + slot0);
+        }
+        // RoPE angles of this position (reduced modulo 2 pi in fp64), one pair per thread
+        {
+            const double inv = exp2(-(double)tid * (13.287712379549449 / 128.0));
+            double turns = (double)pos * inv * 0.15915494309189535;
+            turns -= floor(turns);
+            float sn, co;
+            sincospif((float)(2.0 * turns), &sn, &co);
+            cs[tid] = make_float2(co, sn);
+        }
+        __syncthreads();
+        const __nv_bfloat16 *row = p.qkv + (size_t)b * (H + 2) * kHd;
+        // Q^T tile: rows = heads (16, zero past H), K = channels, 4 boxes of 64
+        // channels; row H of the token is its key (into kv_tok; with 16 heads that
+        // row lies past the tile)
+        for (int e = tid; e < (kDecMaxH + 1) * (kHd / 2); e += kDecThreads) {
+            const int hh = e / (kHd / 2), i = e % (kHd / 2);
+            __nv_bfloat16 y1 = __float2bfloat16_rn(0.f), y2 = y1;
+            if (hh <= H) {
+                const float x1 = __bfloat162float(row[hh * kHd + i]), x2 = __bfloat162float(row[hh * kHd + i + kHd / 2]);
+                const float2 r = cs[i];
+                y1 = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
+                y2 = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
+            }
+            if (hh == H) {  // the key
+                kv_tok[0][i] = y1;
+                kv_tok[0][i + kHd / 2] = y2;
+                y1 = y2 = __float2bfloat16_rn(0.f);
+            }
+            if (hh < kDecMaxH) {
+                const int d1 = i, d2 = i + kHd / 2;
+                *reinterpret_cast<__nv_bfloat16 *>(Qt + (d1 >> 6) * kDecQBox + sw128(hh, d1 & 63)) = y1;
+                *reinterpret_cast<__nv_bfloat16 *>(Qt + (d2 >> 6) * kDecQBox + sw128(hh, d2 & 63)) = y2;
             }
         }
+        kv_tok[1][tid] = row[(H + 1) * kHd + tid];
+        kv_tok[1][tid + 128] = row[(H + 1) * kHd + tid + 128];
+        // the K tile has landed (a timeout ends the loop; TMEM is freed below)
+        if (!(ok = mqd_wait(bars + 0, ph, p.hdr, 0))) break;
+        if (owner) {
+            // this token's key into the tile (over the ring's stale slot) and both into the rings
+            const int r = pos - p0, sl = pos % W;
+            for (int d = tid; d < kHd; d += kDecThreads) {
+                const __nv_bfloat16 kk = kv_tok[0][d];
+                *reinterpret_cast<__nv_bfloat16 *>(Kt + (d >> 6) * kDecKBox + sw128(r, d & 63)) = kk;
+                p.kc[((size_t)b * W + sl) * kHd + d] = kk;
+                p.vtc[((size_t)b * kHd + d) * W + sl] = kv_tok[1][d];
+            }
+        }
+        fence_proxy_async_smem();  // the generic writes of the tiles, before the tensor cores read them
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t kd = umma_desc_sw128(smem_u32(Kt)), qd = umma_desc_sw128(smem_u32(Qt));
 #pragma unroll
-        for (int h = 0; h < kDecMaxH; ++h) sc[h] = have ? (f2_lo(acc[h]) + f2_hi(acc[h])) * kScale : -INFINITY;
-    }
-    // chunk max and sum per head
+            for (int kk = 0; kk < kHd / 16; ++kk) {
+                const uint32_t off_k = (uint32_t)(kk >> 2) * kDecKBox + (uint32_t)(kk & 3) * 32;
+                const uint32_t off_q = (uint32_t)(kk >> 2) * kDecQBox + (uint32_t)(kk & 3) * 32;
+                umma_ss(tmem, kd + (off_k >> 4), qd + (off_q >> 4), idesc, kk > 0);
+            }
+            umma_commit(bars + 1);
+        }
+        if (!(ok = mqd_wait(bars + 1, ph, p.hdr, 1))) break;
+        tc_fence_after();
+        // S is complete, so the K tile has been read: the V^T tile goes into the same buffer
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bars + 3, 4 * kDecVBox);
+            for (int dh = 0; dh < 2; ++dh)
+                for (int kh = 0; kh < 2; ++kh)
+                    tma_load_3d(Vt + (dh * 2 + kh) * kDecVBox, &tm_vt, bars + 3, slot0 + 64 * kh, 128 * dh, b);
+        }
+        uint32_t sr[16];
+        tmem_ld16(lane_base, sr);
+        tmem_wait_ld();
+        const int kp = p0 + tid;  // this thread's key position
+        const bool valid = kp >= lo && kp <= pos;
+        float sc[kDecMaxH];
 #pragma unroll
-    for (int h = 0; h < kDecMaxH; ++h) {
-        if (h < H) {
+        for (int h = 0; h < kDecMaxH; ++h) sc[h] = (valid && h < H) ? __uint_as_float(sr[h]) * kScale : -INFINITY;
+#pragma unroll
+        for (int h = 0; h < kDecMaxH; ++h) {
             float m = sc[h];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (lane == 0) red[warp][h] = m;
         }
-    }
-    __syncthreads();
-    if (tid < H) {
-        float m = red[0][tid];
-        for (int w = 1; w < kDecThreads / 32; ++w) m = fmaxf(m, red[w][tid]);
-        mch[tid] = m;
-    }
-    __syncthreads();
+        __syncthreads();
+        if (tid < kDecMaxH) mh[tid] = fmaxf(fmaxf(red[0][tid], red[1][tid]), fmaxf(red[2][tid], red[3][tid]));
+        __syncthreads();
+        float pr[kDecMaxH];
 #pragma unroll
-    for (int h = 0; h < kDecMaxH; ++h) {
-        if (h < H) {
-            const float pr = have ? ex2_approx(sc[h] - mch[h]) : 0.f;
-            ps[h][tid] = pr;
-            float l = pr;
+        for (int h = 0; h < kDecMaxH; ++h) {
+            pr[h] = (valid && h < H) ? ex2_approx(sc[h] - mh[h]) : 0.f;
+            float l = pr[h];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
             if (lane == 0) red[warp][h] = l;
         }
-    }
-    __syncthreads();
-    if (tid < H) {
-        float l = 0.f;
-        for (int w = 0; w < kDecThreads / 32; ++w) l += red[w][tid];
-        lch[tid] = l;
-    }
-
-    // O partial: thread = (channel pair dp, half of the chunk's keys)
-    const int dp = tid % (kHd / 2), half = tid / (kHd / 2);
-    const int kb = half * (kDecKeys / 2), ke = min(kb + kDecKeys / 2, n - i0);
-    f2_t o[kDecMaxH];
-#pragma unroll
-    for (int h = 0; h < kDecMaxH; ++h) o[h] = 0ull;
-    if (kb < ke) {
-        int slot = (lo + i0 + kb) % W;
-#pragma unroll 2
-        for (int kk = kb; kk < ke; ++kk) {
-            const uint32_t vv = *reinterpret_cast<const uint32_t *>(p.vc + ((size_t)b * W + slot) * kHd + 2 * dp);
-            const f2_t v2 = bf16x2_to_f2(vv);
-#pragma unroll
-            for (int h = 0; h < kDecMaxH; ++h)
-                if (h < H) o[h] = f2_fma(f2_splat(ps[h][kk]), v2, o[h]);
-            slot = slot + 1 == W ? 0 : slot + 1;
-        }
-    }
-    __syncthreads();  // every thread is done with ps: the second half's O goes there
-    float2 *oh = reinterpret_cast<float2 *>(&ps[0][0]);  // [kDecMaxH][128] float2
-    if (half == 1) {
+        // P^T tile: rows = heads, K = this block's keys (2 boxes of 64)
 #pragma unroll
         for (int h = 0; h < kDecMaxH; ++h)
-            if (h < H) oh[h * (kHd / 2) + dp] = make_float2(f2_lo(o[h]), f2_hi(o[h]));
-    }
-    __syncthreads();
-    if (half == 0) {
+            *reinterpret_cast<__nv_bfloat16 *>(Pt + (tid >> 6) * kDecPBox + sw128(h, tid & 63)) =
+                __float2bfloat16_rn(pr[h]);
+        __syncthreads();
+        if (tid < kDecMaxH) lh[tid] = (red[0][tid] + red[1][tid]) + (red[2][tid] + red[3][tid]);
+        if (!(ok = mqd_wait(bars + 3, ph, p.hdr, 3))) break;  // the V^T tile has landed
+        if (owner) {
+            const int r = pos - p0;
+            for (int d = tid; d < kHd; d += kDecThreads)
+                *reinterpret_cast<__nv_bfloat16 *>(Vt + ((d >> 7) * 2 + (r >> 6)) * kDecVBox + sw128(d & 127, r & 63)) =
+                    kv_tok[1][d];
+        }
+        fence_proxy_async_smem();  // P^T and the token's value, before the tensor cores read them
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t pd = umma_desc_sw128(smem_u32(Pt));
+#pragma unroll
+            for (int dh = 0; dh < 2; ++dh) {
+                const uint64_t vd = umma_desc_sw128(smem_u32(Vt + dh * 2 * kDecVBox));
+#pragma unroll
+                for (int kk = 0; kk < kDecKeys / 16; ++kk) {
+                    const uint32_t off_v = (uint32_t)(kk >> 2) * kDecVBox + (uint32_t)(kk & 3) * 32;
+                    const uint32_t off_p = (uint32_t)(kk >> 2) * kDecPBox + (uint32_t)(kk & 3) * 32;
+                    umma_ss(tmem + 16 + 16 * dh, vd + (off_v >> 4), pd + (off_p >> 4), idesc, kk > 0);
+                }
+            }
+            umma_commit(bars + 2);
+        }
+        if (!(ok = mqd_wait(bars + 2, ph, p.hdr, 2))) break;
+        tc_fence_after();
+        uint32_t o0[16], o1[16];
+        tmem_ld16(lane_base + 16, o0);
+        tmem_ld16(lane_base + 32, o1);
+        tmem_wait_ld();
         const size_t base = ((size_t)b * p.nch + c) * H;
 #pragma unroll
         for (int h = 0; h < kDecMaxH; ++h) {
             if (h < H) {
-                const float2 q2 = oh[h * (kHd / 2) + dp];
-                reinterpret_cast<float2 *>(p.part_o + (base + h) * kHd)[dp] =
-                    make_float2(f2_lo(o[h]) + q2.x, f2_hi(o[h]) + q2.y);
+                p.part_o[(base + h) * kHd + tid] = __uint_as_float(o0[h]);
+                p.part_o[(base + h) * kHd + 128 + tid] = __uint_as_float(o1[h]);
             }
         }
+        if (tid < H) {
+            p.part_ml[2 * (base + tid)] = mh[tid];
+            p.part_ml[2 * (base + tid) + 1] = lh[tid];
+        }
+        // the next item rewrites the tiles, cs, kv_tok and TMEM only after every
+        // thread has finished with this one
+        tc_fence_before();
+        __syncthreads();
+        ph ^= 1u;
     }
-    if (tid < H) {
-        const size_t base = ((size_t)b * p.nch + c) * H + tid;
-        p.part_ml[2 * base] = mch[tid];
-        p.part_ml[2 * base + 1] = lch[tid];
-    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kDecCols);
 }
 
-// out[b, h] = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c over the chunks of sequence b
+// out[b, h] = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c over the blocks of
+// sequence b (at most 17: window <= 2048).  One CTA per (sequence, head):
+// every warp finds the weights (lane c holds block c's max and sum), then each
+// thread (= channel) sums its channel over the blocks.
 __global__ void __launch_bounds__(kHd)
 rglru_mqa_decode_combine_kernel(const DecParams p)
 {
-    const int b = blockIdx.x, d = threadIdx.x, H = p.H;
+    const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x, H = p.H, lane = d & 31;
     const int pos = max(p.segpos[b], 0);
-    const int n = min(pos + 1, p.window);
-    const int nc = (n + kDecKeys - 1) / kDecKeys;
-    for (int h = 0; h < H; ++h) {
-        float M = -INFINITY;
-        for (int c = 0; c < nc; ++c) M = fmaxf(M, p.part_ml[2 * (((size_t)b * p.nch + c) * H + h)]);
-        float num = 0.f, den = 0.f;
-        for (int c = 0; c < nc; ++c) {
-            const size_t base = ((size_t)b * p.nch + c) * H + h;
-            const float f = ex2_approx(p.part_ml[2 * base] - M);
-            num = fmaf(f, p.part_o[base * kHd + d], num);
-            den = fmaf(f, p.part_ml[2 * base + 1], den);
-        }
-        p.out[(size_t)b * H * kHd + (size_t)h * kHd + d] = __float2bfloat16_rn(num / den);
-    }
+    const int lo = pos - min(pos + 1, p.window) + 1;
+    const int nc = (pos >> 7) - (lo >> 7) + 1;
+    const bool in = lane < nc;
+    const size_t base = ((size_t)b * p.nch + lane) * H + h;
+    const float m = in ? p.part_ml[2 * base] : -INFINITY, l = in ? p.part_ml[2 * base + 1] : 0.f;
+    float M = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float f = in ? ex2_approx(m - M) : 0.f;
+    float den = f * l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float *po = p.part_o + ((size_t)b * p.nch * H + h) * kHd + d;
+    const size_t cstride = (size_t)H * kHd;
+    float num = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < nc; ++c) num = fmaf(__shfl_sync(0xffffffffu, f, c), po[c * cstride], num);
+    p.out[(size_t)b * H * kHd + (size_t)h * kHd + d] = __float2bfloat16_rn(num / den);
 }
 
 size_t dec_part_bytes(int B, int H, int window)
 {
-    const size_t nch = (size_t)((window + kDecKeys - 1) / kDecKeys);
+    const size_t nch = (size_t)(window / kDecKeys + 1);
     return align_up((size_t)B * nch * H * kHd * 4, 256) + align_up((size_t)B * nch * H * 2 * 4, 256);
 }
 
@@ -841,17 +948,19 @@ RGLRU_API rglru_status rglru_mqa_block_prefill(int B, int T, int D, int window, 
 
 RGLRU_API size_t rglru_mqa_decode_workspace_size(int B, int H, int window)
 {
-    if (B < 1 || B > 65535 || H < 1 || H > kDecMaxH || window < 1 || window > (1 << 20)) return 0;
+    if (B < 1 || B > 65535 || H < 1 || H > kDecMaxH || window < kDecKeys || window % kDecKeys != 0 ||
+        window > 16 * kDecKeys)
+        return 0;
     return kWsHeaderBytes + dec_part_bytes(B, H, window);
 }
 
 RGLRU_API rglru_status rglru_mqa_decode_step(int B, int H, int window, const void *qkv, const int32_t *segment_pos,
-                                             void *k_cache, void *v_cache, void *out, void *workspace,
+                                             void *k_cache, void *v_cache_t, void *out, void *workspace,
                                              size_t workspace_bytes, cudaStream_t stream)
 {
     const size_t need = rglru_mqa_decode_workspace_size(B, H, window);
     if (need == 0) return RGLRU_ERR_UNSUPPORTED;
-    if (!al16(qkv) || !al16(k_cache) || !al16(v_cache) || !al16(out) || segment_pos == nullptr)
+    if (!al16(qkv) || !al16(k_cache) || !al16(v_cache_t) || !al16(out) || segment_pos == nullptr)
         return RGLRU_ERR_INVALID_ARG;
     if (workspace == nullptr || !al16(workspace) || workspace_bytes < need) return RGLRU_ERR_WORKSPACE;
     const size_t cache = (size_t)B * window * kHd * 2;
@@ -859,8 +968,8 @@ RGLRU_API rglru_status rglru_mqa_decode_step(int B, int H, int window, const voi
         const void *p;
         size_t n;
     } bufs[] = {{qkv, (size_t)B * (H + 2) * kHd * 2}, {segment_pos, (size_t)B * 4}, {k_cache, cache},
-                {v_cache, cache}, {out, (size_t)B * H * kHd * 2}, {workspace, workspace_bytes}};
-    // the caches, out and the workspace are written: none may overlap another buffer
+                {v_cache_t, cache}, {out, (size_t)B * H * kHd * 2}, {workspace, workspace_bytes}};
+    // the rings, out and the workspace are written: none may overlap another buffer
     for (int i = 0; i < 6; ++i)
         for (int j = i + 1; j < 6; ++j) {
             const bool written = i >= 2 || j >= 2;
@@ -868,24 +977,103 @@ RGLRU_API rglru_status rglru_mqa_decode_step(int B, int H, int window, const voi
             const uintptr_t b0 = reinterpret_cast<uintptr_t>(bufs[j].p), b1 = b0 + bufs[j].n;
             if (written && a0 < b1 && b0 < a1) return RGLRU_ERR_INVALID_ARG;
         }
+    auto encode = encode_fn();
+    if (!encode) return RGLRU_ERR_CUDA;
+    CUtensorMap tm_kc, tm_vt;
+    const cuuint64_t kdim[2] = {(cuuint64_t)kHd, (cuuint64_t)B * window}, kstride[1] = {(cuuint64_t)kHd * 2};
+    const cuuint32_t kbox[2] = {64, kDecKeys};
+    if (!encode_bf16(encode, &tm_kc, k_cache, 2, kdim, kstride, kbox, CU_TENSOR_MAP_SWIZZLE_128B)) return RGLRU_ERR_CUDA;
+    const cuuint64_t vdim[3] = {(cuuint64_t)window, (cuuint64_t)kHd, (cuuint64_t)B};
+    const cuuint64_t vstride[2] = {(cuuint64_t)window * 2, (cuuint64_t)window * 2 * kHd};
+    const cuuint32_t vbox[3] = {64, 128, 1};
+    if (!encode_bf16(encode, &tm_vt, v_cache_t, 3, vdim, vstride, vbox, CU_TENSOR_MAP_SWIZZLE_128B))
+        return RGLRU_ERR_CUDA;
     DecParams p;
     p.B = B;
     p.H = H;
     p.window = window;
-    p.nch = (window + kDecKeys - 1) / kDecKeys;
+    p.nch = window / kDecKeys + 1;
     p.qkv = static_cast<const __nv_bfloat16 *>(qkv);
     p.segpos = segment_pos;
     p.kc = static_cast<__nv_bfloat16 *>(k_cache);
-    p.vc = static_cast<__nv_bfloat16 *>(v_cache);
+    p.vtc = static_cast<__nv_bfloat16 *>(v_cache_t);
     char *ws = static_cast<char *>(workspace) + kWsHeaderBytes;
     p.part_o = reinterpret_cast<float *>(ws);
     p.part_ml = reinterpret_cast<float *>(ws + align_up((size_t)B * p.nch * H * kHd * 4, 256));
     p.out = static_cast<__nv_bfloat16 *>(out);
-    rglru_mqa_decode_kernel<<<dim3((unsigned)p.nch, (unsigned)B), kDecThreads, 0, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return RGLRU_ERR_CUDA;
-    rglru_mqa_decode_combine_kernel<<<(unsigned)B, kHd, 0, stream>>>(p);
+    p.hdr = static_cast<WsHeader *>(workspace);
+    static PerDeviceFlag smem_set;
+    const rglru_status st = set_smem_limit_once((const void *)rglru_mqa_decode_kernel, kDecSmem, smem_set);
+    if (st != RGLRU_OK) return st;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return RGLRU_ERR_CUDA;
+    const long long items = (long long)B * p.nch;
+    const unsigned grid = (unsigned)(items < 2LL * sms ? items : 2LL * sms);  // two per SM, persistent
+    rglru_mqa_decode_kernel<<<grid, kDecThreads, kDecSmem, stream>>>(p, tm_kc, tm_vt);
+    if (cudaGetLastError() != cudaSuccess) return RGLRU_ERR_CUDA;
+    rglru_mqa_decode_combine_kernel<<<dim3((unsigned)B, (unsigned)H), kHd, 0, stream>>>(p);
     return cuda_status(cudaGetLastError());
+}
+
+RGLRU_API size_t rglru_mqa_residual_block_workspace_size(int B, int T, int D, int F)
+{
+    if (B < 1 || T < 1 || D < kHd || D % kHd != 0 || F < 128 || F % 128 != 0 || F > (1 << 20)) return 0;
+    const size_t M = (size_t)B * T, act = align_up(M * D * 2, 256);
+    return kWsHeaderBytes + 3 * act + align_up(M * (D + 2 * kHd) * 2, 256) + align_up(vt_elems(B, T) * 2, 256) +
+           align_up(M * F * 2, 256);
+}
+
+RGLRU_API rglru_status rglru_mqa_residual_block_prefill(
+    int B, int T, int D, int F, int window, const void *u, const float *w_temporal_norm, const void *W_qkv,
+    const void *W_o, const float *b_o, const int32_t *segment_pos, const float *w_channel_norm, const void *W_gate,
+    const float *b_gate, const void *W_up, const float *b_up, const void *W_down, const float *b_down, float eps,
+    void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    const size_t need = rglru_mqa_residual_block_workspace_size(B, T, D, F);
+    if (need == 0) return RGLRU_ERR_INVALID_ARG;
+    const int H = D / kHd;
+    if (!mqa_sizes_ok(B, T, H) || !(eps > 0.f)) return RGLRU_ERR_UNSUPPORTED;
+    if (window < 1) return RGLRU_ERR_INVALID_ARG;
+    if (workspace == nullptr || !al16(workspace) || workspace_bytes < need) return RGLRU_ERR_WORKSPACE;
+    if (!al16(u) || !al16(out) || !al16(W_qkv) || !al16(W_o) || !al16(w_temporal_norm) || !al16(w_channel_norm) ||
+        segment_pos == nullptr)
+        return RGLRU_ERR_INVALID_ARG;
+    const size_t M = (size_t)B * T, act = M * D * 2;
+    const struct {
+        const void *p;
+        size_t n;
+    } ins[] = {{u, act}, {workspace, workspace_bytes}, {W_qkv, (size_t)(D + 2 * kHd) * D * 2},
+               {W_o, (size_t)D * D * 2}, {W_gate, (size_t)F * D * 2}, {W_up, (size_t)F * D * 2},
+               {W_down, (size_t)D * F * 2}, {segment_pos, M * 4}};
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out), o1 = o0 + act;
+    for (const auto &b : ins) {
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(b.p), a1 = a0 + b.n;
+        if (a0 < o1 && o0 < a1) return RGLRU_ERR_INVALID_ARG;
+    }
+    {
+        const uintptr_t u0 = reinterpret_cast<uintptr_t>(u), w0 = reinterpret_cast<uintptr_t>(workspace);
+        if (u0 < w0 + workspace_bytes && w0 < u0 + act) return RGLRU_ERR_INVALID_ARG;
+    }
+    char *ws = static_cast<char *>(workspace);
+    const size_t a = align_up(act, 256);
+    char *n = ws + kWsHeaderBytes, *h = n + a, *att = h + a;
+    char *qkv = att + a;
+    char *vt = qkv + align_up(M * (D + 2 * kHd) * 2, 256);
+    char *m = vt + align_up(vt_elems(B, T) * 2, 256);
+    // temporal_pre_norm -> q/k/v projections -> RoPE -> local MQA -> o_proj + residual
+    rglru_status st = rglru_rmsnorm((int)M, D, u, w_temporal_norm, eps, n, stream);
+    if (st == RGLRU_OK) st = rglru_linear((int)M, D + 2 * kHd, D, n, W_qkv, nullptr, qkv, ws, kWsHeaderBytes, stream);
+    if (st == RGLRU_OK) st = mqa_rope_launch(B, T, H, qkv, segment_pos, vt, stream);
+    if (st == RGLRU_OK) st = mqa_attention_launch(B, T, H, window, qkv, vt, segment_pos, att, ws, stream);
+    if (st == RGLRU_OK) st = rglru_linear_residual((int)M, D, D, att, W_o, b_o, u, h, ws, kWsHeaderBytes, stream);
+    // channel_pre_norm -> GELU-gated up projection -> down projection + residual
+    if (st == RGLRU_OK) st = rglru_rmsnorm((int)M, D, h, w_channel_norm, eps, n, stream);
+    if (st == RGLRU_OK)
+        st = rglru_linear_geglu((int)M, F, D, n, W_gate, b_gate, W_up, b_up, m, ws, kWsHeaderBytes, stream);
+    if (st == RGLRU_OK) st = rglru_linear_residual((int)M, D, F, m, W_down, b_down, h, out, ws, kWsHeaderBytes, stream);
+    return st;
 }
 
 }  // extern "C"

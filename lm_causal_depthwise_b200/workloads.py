@@ -275,3 +275,22 @@ def generate_mqa(w: Workload) -> dict:
     W_q, W_k, W_v, W_o = weight(D, D), weight(HEAD, D), weight(HEAD, D), weight(D, D)
     b_o = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
     return {"u": u, "W_q": W_q, "W_k": W_k, "W_v": W_v, "W_o": W_o, "b_o": b_o, "segpos": seg}
+
+
+def generate_mqa_residual(w: Workload) -> dict:
+    """Inputs of the residual block with local MQA: ``generate_mqa(w)`` plus,
+    from ``default_rng((seed, 5))`` in this order, the RMSNorm scales and the
+    MLP drawn as in ``generate_residual_block`` (F = 3 D)."""
+    inp = generate_mqa(w)
+    rng = np.random.default_rng((w.seed, 5))
+    D = w.D
+    F = MLP_EXPANSION * D
+    inp["w_temporal_norm"] = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    inp["w_channel_norm"] = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    inp["W_gate"] = round_bf16((rng.standard_normal((F, D)) / np.sqrt(D)).astype(np.float32))
+    inp["b_gate"] = (np.sqrt(0.1) * rng.standard_normal(F)).astype(np.float32)
+    inp["W_up"] = round_bf16((rng.standard_normal((F, D)) / np.sqrt(D)).astype(np.float32))
+    inp["b_up"] = (np.sqrt(0.1) * rng.standard_normal(F)).astype(np.float32)
+    inp["W_down"] = round_bf16((rng.standard_normal((D, F)) / np.sqrt(F)).astype(np.float32))
+    inp["b_down"] = (np.sqrt(0.1) * rng.standard_normal(D)).astype(np.float32)
+    return inp

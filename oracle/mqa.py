@@ -86,6 +86,18 @@ def attention_rows(q, k, v, segpos, rows, window: int = WINDOW) -> np.ndarray:
     return np.stack(out)
 
 
+def _attend(n, W_q, W_k, W_v, segpos, window, rnd) -> dict:
+    """q_proj, k_proj, v_proj of n [B, T, D], RoPE on q and k, local attention;
+    each result rounded by ``rnd``."""
+    B, T, D = n.shape
+    H = np.asarray(W_q).shape[0] // HEAD
+    q = rnd(rope(block.linear(n, W_q).reshape(B, T, H, HEAD), segpos))
+    k = rnd(rope(block.linear(n, W_k), segpos))
+    v = rnd(block.linear(n, W_v))
+    a = rnd(attention(q, k, v, segpos, window))
+    return {"q": q, "k": k, "v": v, "a": a}
+
+
 def mqa_block(u, W_q, W_k, W_v, W_o, b_o, segpos, window: int = WINDOW, round_io: bool = True) -> dict:
     """The local MQA temporal block over u [B, T, D]: projections (q_proj,
     k_proj, v_proj without bias), RoPE on q and k, local attention, o_proj
@@ -94,10 +106,25 @@ def mqa_block(u, W_q, W_k, W_v, W_o, b_o, segpos, window: int = WINDOW, round_io
     rnd = block.round_bf16 if round_io else (lambda a: np.asarray(a, np.float64))
     u = np.asarray(u, np.float64)
     B, T, D = u.shape
-    H = np.asarray(W_q).shape[0] // HEAD
-    q = rnd(rope(block.linear(u, W_q).reshape(B, T, H, HEAD), segpos))
-    k = rnd(rope(block.linear(u, W_k), segpos))
-    v = rnd(block.linear(u, W_v))
-    a = rnd(attention(q, k, v, segpos, window))
-    out = rnd(block.linear(a.reshape(B, T, H * HEAD), W_o, b_o))
-    return {"out": out, "q": q, "k": k, "v": v, "a": a}
+    r = _attend(u, W_q, W_k, W_v, segpos, window, rnd)
+    r["out"] = rnd(block.linear(r["a"].reshape(B, T, -1), W_o, b_o))
+    return r
+
+
+def mqa_residual_block(u, w_temporal_norm, W_q, W_k, W_v, W_o, b_o, segpos, w_channel_norm, W_gate, b_gate, W_up,
+                       b_up, W_down, b_down, eps: float = 1e-6, window: int = WINDOW) -> dict:
+    """The residual block with local MQA ("Residual block with local MQA" and
+    the decoder-layer printout): h = u + o_proj(MQA(RMSNorm(u))), out = h +
+    MLP(RMSNorm(h)); every layer's output a bf16 tensor (the residual adds
+    belong to the projection before them, rounded once with it).  Returns out
+    and the intermediates n (normalised u) and h."""
+    rnd = block.round_bf16
+    u = np.asarray(u, np.float64)
+    B, T, D = u.shape
+    n = rnd(block.rmsnorm(u, w_temporal_norm, eps))
+    a = _attend(n, W_q, W_k, W_v, segpos, window, rnd)["a"]
+    h = rnd(block.linear(a.reshape(B, T, -1), W_o, b_o) + u)
+    n2 = rnd(block.rmsnorm(h, w_channel_norm, eps))
+    m = rnd(block.gelu_tanh(block.linear(n2, W_gate, b_gate)) * block.linear(n2, W_up, b_up))
+    out = rnd(block.linear(m, W_down, b_down) + h)
+    return {"out": out, "n": n, "h": h}

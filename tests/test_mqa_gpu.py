@@ -180,11 +180,11 @@ def test_mqa_block_matches_oracle(B, T, D, doc_len, window):
     check_bf16(out.float().cpu().numpy(), ref["out"], "mqa block out")
 
 
-@pytest.mark.parametrize("B,T,H,window,doc_len", [(2, 300, 2, 64, None), (3, 200, 10, 2048, 60),
-                                                  (1, 600, 3, 300, 250), (2, 70, 16, 256, None)])
+@pytest.mark.parametrize("B,T,H,window,doc_len", [(2, 300, 2, 128, None), (3, 200, 10, 2048, 60),
+                                                  (1, 700, 3, 256, 300), (2, 140, 16, 128, None)])
 def test_decode_steps_match_oracle(B, T, H, window, doc_len):
-    """T decode steps from empty rings (window 64 and 300 wrap the ring; 16
-    heads is the 9B shape's count): each step's output against the oracle's
+    """T decode steps from empty rings (windows of 128 and 256 wrap the ring;
+    16 heads is the 9B shape's count): each step's output against the oracle's
     attention over the same rotated, bf16-rounded q, k and v; the rings hold
     the rotated keys and the values at slot position % window."""
     qkv, seg = _qkv(B, T, H, seed=7, doc_len=doc_len)
@@ -202,6 +202,9 @@ def test_decode_steps_match_oracle(B, T, H, window, doc_len):
     want = omqa.attention(qr, kr, v, seg, window).reshape(B, T, H * 256)
     _attn_bar(got, want, np.abs(v).max(), f"decode B={B} T={T} H={H} window={window}")
     # the ring after the last step: slot p % window holds position p of the last document
+    # (k against the unrounded rotation: the kernel's fp32 rotation may round
+    # to the other neighbour of a tie, which the RoPE bar allows)
+    k_exact = omqa.rope(k, seg)
     kcn, vcn = kc.float().cpu().numpy(), vc.float().cpu().numpy()
     for b in range(B):
         t_last = T - 1
@@ -209,9 +212,9 @@ def test_decode_steps_match_oracle(B, T, H, window, doc_len):
         for back in range(min(p_last + 1, window)):
             t = t_last - back
             slot = (p_last - back) % window
-            np.testing.assert_array_equal(vcn[b, slot], v[b, t])
-            err = np.abs(kcn[b, slot] - kr[b, t])
-            assert (err <= 2.0 ** -8 * np.abs(kr[b, t]) + 1e-5).all(), (b, t, float(err.max()))
+            np.testing.assert_array_equal(vcn[b, :, slot], v[b, t])
+            err = np.abs(kcn[b, slot] - k_exact[b, t])
+            assert (err <= 2.0 ** -8 * np.abs(k_exact[b, t]) + 1e-5).all(), (b, t, float(err.max()))
 
 
 def test_decode_equals_prefill_rows():
@@ -233,3 +236,56 @@ def test_decode_equals_prefill_rows():
     err = np.abs(dec - pre)
     bad = ~(err <= 2.0 ** -8 * np.abs(v).max() + 2.0 ** -7 * np.abs(pre) + 2e-6)
     assert not bad.any(), f"decode vs prefill: {int(bad.sum())} outside, max err {err.max():.3e}"
+
+
+def test_mqa_write_coverage_and_canaries():
+    """RoPE, attention and the decode step write every element of their
+    outputs and nothing past the end of out, v_t or the rings."""
+    B, T, H, pad = 2, 333, 3, 2048
+    qkv, seg = _qkv(B, T, H, seed=9, doc_len=100)
+    dq = torch.from_numpy(qkv).to(dev).to(bf)
+    ds = torch.from_numpy(seg).to(dev)
+    Tp = (T + 7) // 8 * 8
+    vtb = torch.full((B * 256 * Tp + pad,), float("nan"), dtype=bf, device=dev)
+    vt = api.mqa_rope(dq, ds, vtb[:B * 256 * Tp].view(B, 256, Tp))
+    outb = torch.full((B * T * H * 256 + pad,), float("nan"), dtype=bf, device=dev)
+    out = api.mqa_attention(dq, vt, ds, out=outb[:B * T * H * 256].view(B, T, H * 256))
+    torch.cuda.synchronize()
+    assert not torch.isnan(vt).any() and torch.isnan(vtb[B * 256 * Tp:]).all()
+    assert not torch.isnan(out).any() and torch.isnan(outb[B * T * H * 256:]).all()
+    W = 128
+    kcb = torch.full((B * W * 256 + pad,), float("nan"), dtype=bf, device=dev)
+    vcb = torch.full((B * W * 256 + pad,), float("nan"), dtype=bf, device=dev)
+    kc, vc = kcb[:B * W * 256].view(B, W, 256), vcb[:B * W * 256].view(B, 256, W)
+    kc.zero_()
+    vc.zero_()
+    dob = torch.full((B * H * 256 + pad,), float("nan"), dtype=bf, device=dev)
+    raw = torch.from_numpy(qkv).to(dev).to(bf)
+    for t in range(160):
+        o = api.mqa_decode_step(raw[:, t].contiguous(), ds[:, t].contiguous(), kc, vc,
+                                out=dob[:B * H * 256].view(B, H * 256))
+    torch.cuda.synchronize()
+    assert not torch.isnan(o).any() and torch.isnan(dob[B * H * 256:]).all()
+    assert torch.isnan(kcb[B * W * 256:]).all() and torch.isnan(vcb[B * W * 256:]).all()
+
+
+@pytest.mark.parametrize("B,T,D,doc_len,window", [(2, 300, 512, 100, 2048), (1, 500, 2560, 200, 128)])
+def test_mqa_residual_block_matches_oracle(B, T, D, doc_len, window):
+    """The residual block with local MQA against the oracle.  As for the
+    recurrent residual block, an error of the temporal block's size passes
+    through o_proj into h and again through the MLP into out: out is held to
+    twice the bf16 bar (atol 4e-2, rtol 2e-2)."""
+    w = W.Workload("mqa-res", B=B, T=T, D=D, io="bf16", seed=10, doc_len=doc_len)
+    inp = W.generate_mqa_residual(w)
+    rp = api.MQAResidualParams.from_arrays(inp, dev)
+    u = torch.from_numpy(inp["u"]).to(dev).to(bf)
+    sp = torch.from_numpy(inp["segpos"]).to(dev)
+    ws = api.new_workspace(api.mqa_residual_block_workspace_size(B, T, D, rp.W_gate.shape[0]), dev)
+    out = api.mqa_residual_block_prefill(u, rp, sp, window, workspace=ws)
+    assert api.device_status(ws) == api.OK
+    keys = ("u", "w_temporal_norm", "W_q", "W_k", "W_v", "W_o", "b_o", "segpos", "w_channel_norm", "W_gate",
+            "b_gate", "W_up", "b_up", "W_down", "b_down")
+    ref = omqa.mqa_residual_block(*[inp[k] for k in keys], window=window)
+    got, want = out.float().cpu().numpy().astype(np.float64), ref["out"]
+    bad = ~(np.abs(got - want) <= 4e-2 + 2e-2 * np.abs(want))
+    assert not bad.any(), f"mqa residual block: {int(bad.sum())} of {bad.size} outside, max {np.abs(got - want).max():.3e}"

@@ -94,3 +94,39 @@ def test_document_begun_before_the_call_attends_from_token_zero():
     np.testing.assert_allclose(got[0], want.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(mqa.attention_rows(q, k, v, seg, [(0, 5), (0, 19)], window=64),
                                got[0, [5, 19]], rtol=1e-13, atol=1e-13)
+
+
+def _res_inputs(seed=11, B=1, T=24, D=512):
+    from lm_causal_depthwise_b200 import workloads as W
+    w = W.Workload("res-mqa", B=B, T=T, D=D, io="bf16", seed=seed, doc_len=10)
+    return W.generate_mqa_residual(w)
+
+
+def _res(inp, **over):
+    keys = ("u", "w_temporal_norm", "W_q", "W_k", "W_v", "W_o", "b_o", "segpos", "w_channel_norm", "W_gate",
+            "b_gate", "W_up", "b_up", "W_down", "b_down")
+    args = [over.get(k, inp[k]) for k in keys]
+    return mqa.mqa_residual_block(*args, window=16)
+
+
+def test_mqa_residual_block_wiring():
+    """Zero projections leave the residual paths: out = u; with a zero MLP,
+    out = h = u + o_proj(attention of the normalised u) (the MQA block's own
+    pinned pieces); with a zero o_proj, h = u and out = u + MLP(RMSNorm(u))."""
+    from oracle import block
+    inp = _res_inputs()
+    D, F = inp["W_o"].shape[0], inp["W_gate"].shape[0]
+    zD, zDD, zDF, zF = np.zeros(D), np.zeros((D, D)), np.zeros((D, F)), np.zeros(F)
+    r = _res(inp, W_o=zDD, b_o=zD, W_down=zDF, b_down=zD)
+    np.testing.assert_array_equal(r["out"], inp["u"])
+    r = _res(inp, W_down=zDF, b_down=zD)
+    n = block.round_bf16(block.rmsnorm(inp["u"], inp["w_temporal_norm"], 1e-6))
+    a = mqa.mqa_block(n, inp["W_q"], inp["W_k"], inp["W_v"], inp["W_o"], inp["b_o"], inp["segpos"], 16)["a"]
+    B, T, _ = inp["u"].shape
+    h = block.round_bf16(block.linear(a.reshape(B, T, -1), inp["W_o"], inp["b_o"]) + inp["u"])
+    np.testing.assert_array_equal(r["out"], h)
+    r = _res(inp, W_o=zDD, b_o=zD)
+    n2 = block.round_bf16(block.rmsnorm(inp["u"], inp["w_channel_norm"], 1e-6))
+    m = block.round_bf16(block.gelu_tanh(block.linear(n2, inp["W_gate"], inp["b_gate"]))
+                         * block.linear(n2, inp["W_up"], inp["b_up"]))
+    np.testing.assert_array_equal(r["out"], block.round_bf16(block.linear(m, inp["W_down"], inp["b_down"]) + inp["u"]))

@@ -134,17 +134,28 @@ def test_short_documents(simt):
 
 def test_write_coverage_and_canaries():
     """Every output element is written (NaN sentinels gone) and nothing past
-    the end of y is touched."""
+    the end of y, the two states or the workspace is touched."""
     _, inp = _case(2, 777, 512, doc_len=200)
     dev = to_device(inp, "bf16")
     B, T, D = 2, 777, 512
-    buf = torch.full((B * T * D + 4096,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    pad = 4096
+    buf = torch.full((B * T * D + pad,), float("nan"), dtype=torch.bfloat16, device="cuda")
     y = buf[:B * T * D].view(B, T, D)
-    api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], dev["conv_state"],
-                dev["h_state"], y=y)
+    csb = torch.full((B * 3 * D + pad,), 7.0, dtype=torch.bfloat16, device="cuda")
+    csb[:B * 3 * D].copy_(dev["conv_state"].view(-1))
+    hsb = torch.full((B * D + pad,), 7.0, dtype=torch.float32, device="cuda")
+    hsb[:B * D].copy_(dev["h_state"].view(-1))
+    need = api.workspace_size(B, T, D, torch.bfloat16)
+    wsb = torch.full((need + pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    wsb[:need].zero_()
+    api.prefill(dev["x"], dev["g"], dev["params"], dev["segpos"], csb[:B * 3 * D].view(B, 3, D),
+                hsb[:B * D].view(B, D), y=y, workspace=wsb[:need])
     torch.cuda.synchronize()
+    assert api.device_status(wsb[:need]) == api.OK
     assert not torch.isnan(y).any()
     assert torch.isnan(buf[B * T * D:]).all()
+    assert (csb[B * 3 * D:] == 7.0).all() and (hsb[B * D:] == 7.0).all()
+    assert (wsb[need:] == 0xA5).all()
 
 
 @pytest.mark.parametrize("simt", PATHS)
