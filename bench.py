@@ -928,7 +928,9 @@ def run_cuda(args, w):
     if dec is not None:
         line["decode"] = dec
     if blk is not None:
+        mqa = {"prefill_block": blk.pop("mqa_block", None), "decode_step": blk.pop("mqa_decode", None)}
         line["recurrent_block"] = blk
+        line["local_mqa"] = mqa
     if cpu_on:
         v, cores, sample = cpu_sample_run(w)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",

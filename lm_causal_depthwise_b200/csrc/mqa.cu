@@ -32,7 +32,8 @@
 //              S = Q K^T (M=128, N=64, 16 K-steps) with Q read from TMEM,
 //              then O += P V (M=128, N=256, 4 K-steps) with P read from TMEM;
 //              S of tile j + 1 is issued as soon as the softmax has read S of
-//              tile j, so it runs under the softmax of tile j;
+//              tile j (ahead of O += P V of tile j - 1), so it runs under the
+//              softmax of tile j;
 //   warps 0-3  softmax: thread = query row = TMEM lane.  Each first writes its
 //              row of the Q tile into TMEM (the A operand of S).  Scores in
 //              log2 units, the window / document / causal limits applied only
@@ -245,7 +246,10 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
         // addresses stay warp-uniform; elect.sync picks the lane that issues
         const uint32_t idesc_s = umma_idesc_bf16(kQT, kKT), idesc_o = umma_idesc_bf16(kQT, kHd);
         bool ok = attn_warp_wait(bars + B_QFULL, 0, p.hdr, 2);
-        for (int j = 0; ok && j <= n; ++j) {
+        // S of tile j goes out as soon as the score buffer is free, ahead of
+        // O += P V of tile j - 2, so the softmax of tile j starts as soon as
+        // that of tile j - 1 is done
+        for (int j = 0; ok && j <= n + 1; ++j) {
             if (j < n) {
                 const int s = j % kStages;
                 if (!(ok = attn_warp_wait(bars + B_KFULL + s, (uint32_t)(j / kStages) & 1u, p.hdr, 3))) break;
@@ -264,8 +268,8 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
                 umma_commit_warp(bars + B_SFULL);
                 umma_commit_warp(bars + B_KFREE + s);
             }
-            if (j >= 1) {
-                const int i = j - 1, pb = i % 2, s = i % kStages;
+            if (j >= 2) {
+                const int i = j - 2, pb = i % 2, s = i % kStages;
                 if (!(ok = attn_warp_wait(bars + B_PFULL + pb, (uint32_t)(i / 2) & 1u, p.hdr, 5))) break;
                 if (!(ok = attn_warp_wait(bars + B_VFULL + s, (uint32_t)(i / kStages) & 1u, p.hdr, 6))) break;
                 tc_fence_after();
@@ -564,11 +568,14 @@ rglru_mqa_decode_kernel(const DecParams p, const __grid_constant__ CUtensorMap t
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DOFF_BAR);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + DOFF_MISC);
     __shared__ float2 cs[kHd / 2];
+    __shared__ double inv_freq[kHd / 2];
+    __shared__ __align__(16) __nv_bfloat16 rowbuf[(kDecMaxH + 2) * kHd];  // the token's q, k, v
     __shared__ __align__(16) __nv_bfloat16 kv_tok[2][kHd];  // this token's rotated k and its v
     __shared__ float red[kDecThreads / 32][kDecMaxH];
     __shared__ float mh[kDecMaxH], lh[kDecMaxH];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = p.H, W = p.window;
+    inv_freq[tid] = exp2(-(double)tid * (13.287712379549449 / 128.0));  // 10000^(-2i/256)
 
     if (warp == 0) {
         tmem_alloc(tmem_holder, kDecCols);
@@ -605,17 +612,33 @@ rglru_mqa_decode_kernel(const DecParams p, const __grid_constant__ CUtensorMap t
             mbar_arrive_expect_tx(bars + 0, 4 * kDecKBox);
             for (int kb = 0; kb < 4; ++kb) tma_load_2d(Kt + kb * kDecKBox, &tm_kc, bars + 0, kb * 64, b * W + slot0);
         }
+        // the token's qkv row into shared memory: all 16-byte loads issued at once
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.qkv + (size_t)b * (H + 2) * kHd);
+            uint4 *dst = reinterpret_cast<uint4 *>(rowbuf);
+            const int nv = (H + 2) * kHd / 8;
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0, v2 = v0, v3 = v0, v4 = v0;
+            if (tid < nv) v0 = __ldg(src + tid);
+            if (tid + 128 < nv) v1 = __ldg(src + tid + 128);
+            if (tid + 256 < nv) v2 = __ldg(src + tid + 256);
+            if (tid + 384 < nv) v3 = __ldg(src + tid + 384);
+            if (tid + 512 < nv) v4 = __ldg(src + tid + 512);
+            if (tid < nv) dst[tid] = v0;
+            if (tid + 128 < nv) dst[tid + 128] = v1;
+            if (tid + 256 < nv) dst[tid + 256] = v2;
+            if (tid + 384 < nv) dst[tid + 384] = v3;
+            if (tid + 512 < nv) dst[tid + 512] = v4;
+        }
         // RoPE angles of this position (reduced modulo 2 pi in fp64), one pair per thread
         {
-            const double inv = exp2(-(double)tid * (13.287712379549449 / 128.0));
-            double turns = (double)pos * inv * 0.15915494309189535;
+            double turns = (double)pos * inv_freq[tid] * 0.15915494309189535;
             turns -= floor(turns);
             float sn, co;
             sincospif((float)(2.0 * turns), &sn, &co);
             cs[tid] = make_float2(co, sn);
         }
         __syncthreads();
-        const __nv_bfloat16 *row = p.qkv + (size_t)b * (H + 2) * kHd;
+        const __nv_bfloat16 *row = rowbuf;
         // Q^T tile: rows = heads (16, zero past H), K = channels, 4 boxes of 64
         // channels; row H of the token is its key (into kv_tok; with 16 heads that
         // row lies past the tile)
