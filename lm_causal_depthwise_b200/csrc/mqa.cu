@@ -425,20 +425,46 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
 }
 
 // ---------------------------------------------------------------- RoPE and v_t
-constexpr int kRopeTok = 32;  // tokens per CTA
+constexpr int kRopeTok = 16;  // tokens per CTA
 constexpr int kRopeThreads = 256;
+
+__device__ __forceinline__ uint32_t rot_pair(uint32_t a, uint32_t c, float2 r0, float2 r1, bool second)
+{
+    // elements 2e, 2e+1 of the first half (a) or of the second half (c)
+    const float a0 = __uint_as_float(a << 16), a1 = __uint_as_float(a & 0xffff0000u);
+    const float c0 = __uint_as_float(c << 16), c1 = __uint_as_float(c & 0xffff0000u);
+    float y0, y1;
+    if (!second) {
+        y0 = a0 * r0.x - c0 * r0.y;
+        y1 = a1 * r1.x - c1 * r1.y;
+    } else {
+        y0 = c0 * r0.x + a0 * r0.y;
+        y1 = c1 * r1.x + a1 * r1.y;
+    }
+    uint32_t o;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o) : "f"(y1), "f"(y0));
+    return o;
+}
 
 __global__ void __launch_bounds__(kRopeThreads)
 rglru_mqa_rope_kernel(int T, int H, int Tp, __nv_bfloat16 *__restrict__ qkv, const int32_t *__restrict__ segpos,
                       __nv_bfloat16 *__restrict__ vt)
 {
     __shared__ double inv_freq[kHd / 2];
-    __shared__ float2 cs[kRopeTok][kHd / 2];  // (cos, sin) per token and pair
-    const int b = blockIdx.y, tb = blockIdx.x * kRopeTok;
+    __shared__ __align__(16) float2 cs[kRopeTok][kHd / 2];            // (cos, sin) per token and pair
+    __shared__ __align__(16) __nv_bfloat16 vs[kRopeTok][kHd + 8];     // the v rows, padded
+    const int b = blockIdx.y, tb = blockIdx.x * kRopeTok, tid = threadIdx.x;
     const size_t W = (size_t)(H + 2) * kHd;
-    if (threadIdx.x < kHd / 2) inv_freq[threadIdx.x] = exp2(-(double)threadIdx.x * (13.287712379549449 / 128.0));
+    if (tid < kHd / 2) inv_freq[tid] = exp2(-(double)tid * (13.287712379549449 / 128.0));
+    // the v rows of the CTA's tokens into shared memory (16-byte loads, all in flight)
+    for (int e = tid; e < kRopeTok * (kHd / 8); e += kRopeThreads) {
+        const int tt = e / (kHd / 8), c = e % (kHd / 8), t = tb + tt;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (t < T) v = *reinterpret_cast<const uint4 *>(qkv + ((size_t)b * T + t) * W + (size_t)(H + 1) * kHd + c * 8);
+        *reinterpret_cast<uint4 *>(&vs[tt][c * 8]) = v;
+    }
     __syncthreads();
-    for (int e = threadIdx.x; e < kRopeTok * (kHd / 2); e += kRopeThreads) {
+    for (int e = tid; e < kRopeTok * (kHd / 2); e += kRopeThreads) {
         const int tt = e / (kHd / 2), i = e % (kHd / 2), t = tb + tt;
         float c = 1.f, s = 0.f;
         if (t < T) {
@@ -450,34 +476,41 @@ rglru_mqa_rope_kernel(int T, int H, int Tp, __nv_bfloat16 *__restrict__ qkv, con
         cs[tt][i] = make_float2(c, s);
     }
     __syncthreads();
-    // q heads and k: thread = (token, pair), pairs (x[i], x[i + 128]) of every head
-    for (int e = threadIdx.x; e < kRopeTok * (kHd / 2); e += kRopeThreads) {
-        const int tt = e / (kHd / 2), i = e % (kHd / 2), t = tb + tt;
+    // q heads and k: unit = (token, head, 8 pairs): 16-byte loads of x[i..i+8] and
+    // x[i+128..i+136], rotated, 16-byte stores back
+    const int units = kRopeTok * (H + 1) * 16;
+    for (int u = tid; u < units; u += kRopeThreads) {
+        const int c8 = u % 16, rest = u / 16, hh = rest % (H + 1), tt = rest / (H + 1), t = tb + tt;
         if (t >= T) continue;
-        const float2 r = cs[tt][i];
-        __nv_bfloat16 *row = qkv + ((size_t)b * T + t) * W + i;
-#pragma unroll 1
-        for (int hh = 0; hh <= H; ++hh) {
-            const float x1 = __bfloat162float(row[hh * kHd]), x2 = __bfloat162float(row[hh * kHd + kHd / 2]);
-            row[hh * kHd] = __float2bfloat16_rn(x1 * r.x - x2 * r.y);
-            row[hh * kHd + kHd / 2] = __float2bfloat16_rn(x2 * r.x + x1 * r.y);
+        __nv_bfloat16 *rowp = qkv + ((size_t)b * T + t) * W + (size_t)hh * kHd + c8 * 8;
+        const uint4 a = *reinterpret_cast<const uint4 *>(rowp);
+        const uint4 c = *reinterpret_cast<const uint4 *>(rowp + kHd / 2);
+        const float4 *cp = reinterpret_cast<const float4 *>(&cs[tt][c8 * 8]);
+        const float4 r01 = cp[0], r23 = cp[1], r45 = cp[2], r67 = cp[3];
+        const float2 r[8] = {make_float2(r01.x, r01.y), make_float2(r01.z, r01.w), make_float2(r23.x, r23.y),
+                             make_float2(r23.z, r23.w), make_float2(r45.x, r45.y), make_float2(r45.z, r45.w),
+                             make_float2(r67.x, r67.y), make_float2(r67.z, r67.w)};
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+        uint32_t o1[4], o2[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            o1[q] = rot_pair(aw[q], cw[q], r[2 * q], r[2 * q + 1], false);
+            o2[q] = rot_pair(aw[q], cw[q], r[2 * q], r[2 * q + 1], true);
         }
+        *reinterpret_cast<uint4 *>(rowp) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+        *reinterpret_cast<uint4 *>(rowp + kHd / 2) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
     }
     // v transposed: thread = channel, 8 tokens per 16-byte store
-    const int d = threadIdx.x;
-    const __nv_bfloat16 *vcol = qkv + (size_t)(H + 1) * kHd + d;
+    const int d = tid;
 #pragma unroll 1
     for (int g = 0; g < kRopeTok; g += 8) {
         const int tg = tb + g;
         if (tg >= T) break;
         uint32_t w[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int ta = tg + 2 * q, tb2 = ta + 1;
-            const uint32_t lo = ta < T ? __bfloat16_as_ushort(vcol[((size_t)b * T + ta) * W]) : 0u;
-            const uint32_t hi = tb2 < T ? __bfloat16_as_ushort(vcol[((size_t)b * T + tb2) * W]) : 0u;
-            w[q] = lo | (hi << 16);
-        }
+        for (int q = 0; q < 4; ++q)
+            w[q] = (uint32_t)__bfloat16_as_ushort(vs[g + 2 * q][d]) |
+                   ((uint32_t)__bfloat16_as_ushort(vs[g + 2 * q + 1][d]) << 16);
         *reinterpret_cast<uint4 *>(vt + ((size_t)b * kHd + d) * Tp + tg) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
