@@ -24,16 +24,17 @@
 // beyond any position), then sine and cosine in fp32.
 //
 // rglru_mqa_attention_kernel: one CTA per (head, 128-query tile, sequence),
-// 192 threads:
+// 224 threads:
 //   warp 4     TMA producer: lane 0 the K tiles (4 boxes [64 keys x 64
 //              channels], 128-byte swizzle), lane 1 the V^T tiles ([256 x 64
 //              keys]), each into a 3-deep ring;
-//   warp 5     MMA issuer (the converged warp, one lane elected per MMA):
-//              S = Q K^T (M=128, N=64, 16 K-steps) with Q read from TMEM,
-//              then O += P V (M=128, N=256, 4 K-steps) with P read from TMEM;
-//              S of tile j + 1 is issued as soon as the softmax has read S of
-//              tile j (ahead of O += P V of tile j - 1), so it runs under the
-//              softmax of tile j;
+//   warp 5     S issuer (the converged warp, one lane elected per MMA):
+//              S = Q K^T (M=128, N=64, 16 K-steps) with Q read from TMEM; S of
+//              tile j + 1 goes out as soon as the softmax has read S of tile j,
+//              so it runs under the softmax of tile j;
+//   warp 6     P V issuer: O += P V (M=128, N=256, 4 K-steps) with P read from
+//              TMEM, as soon as P of the tile is written (two issuing warps, so
+//              neither kind of MMA waits behind the other's barriers);
 //   warps 0-3  softmax: thread = query row = TMEM lane.  Each first writes its
 //              row of the Q tile into TMEM (the A operand of S).  Scores in
 //              log2 units, the window / document / causal limits applied only
@@ -60,7 +61,7 @@ using namespace sm100;
 constexpr int kHd = 256;             // head dimension
 constexpr int kQT = 128;             // query rows per CTA
 constexpr int kKT = 64;              // keys per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kKBox = kKT * 64 * 2;  // 8 KB: [64 keys x 64 channels]
 constexpr int kKBytes = 4 * kKBox;   // 32 KB
 constexpr int kVBytes = kHd * kKT * 2;  // 32 KB: [256 channels x 64 keys]
@@ -77,8 +78,8 @@ enum {
     B_SFREE = B_SFULL + 1,        // ... read by the softmax warps (128 arrivals)
     B_PFULL = B_SFREE + 1,        // P of tile j in buffer j % 2 (128 arrivals)
     B_PVDONE = B_PFULL + 2,       // O += P V of tile j complete (P buffer free, O settled)
-    B_DRAIN = B_PVDONE + 2,
-    B_N = B_DRAIN + 1
+    B_DRAIN = B_PVDONE + 2,       // per issuing warp: its MMAs have finished (error path)
+    B_N = B_DRAIN + 2
 };
 constexpr int OFF_MISC = OFF_BAR + B_N * 8;
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;
@@ -174,6 +175,16 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
     const int b = y % p.B;
     const int t0 = (p.ntiles - 1 - y / p.B) * kQT;
     const int t_last = min(t0 + kQT, p.T) - 1;
+    // the softmax warps' rows of the Q tile: every 16-byte load in flight now,
+    // under the key-range scan, the barrier setup and the TMEM allocation
+    uint4 qv[32];
+    if (warp < 4) {
+        const int tq = t0 + warp * 32 + lane;
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            p.qkv + ((size_t)b * p.T + (tq < p.T ? tq : 0)) * (size_t)((p.H + 2) * kHd) + (size_t)h * kHd);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) qv[k] = tq < p.T ? __ldg(src + k) : make_uint4(0, 0, 0, 0);
+    }
     // key tiles j0 .. j0 + n - 1 cover every key of every row of the tile
     int lo_min = INT_MAX;
     for (int r = lane; r < kQT; r += 32)
@@ -200,6 +211,7 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
                 mbar_init(bars + B_PVDONE + s, 1);
             }
             mbar_init(bars + B_DRAIN, 1);
+            mbar_init(bars + B_DRAIN + 1, 1);
             mbar_fence_init();
         }
     }
@@ -241,52 +253,57 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
         }
         __syncwarp();
     } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA issuer
-        // the whole (converged) warp runs the loop, so descriptors and TMEM
-        // addresses stay warp-uniform; elect.sync picks the lane that issues
-        const uint32_t idesc_s = umma_idesc_bf16(kQT, kKT), idesc_o = umma_idesc_bf16(kQT, kHd);
+        // ------------------------------------------------------------ S issuer
+        // S of tile j as soon as K_j has landed and the score buffer is free
+        // (the converged warp runs the loop; elect.sync picks the issuing lane)
+        const uint32_t idesc_s = umma_idesc_bf16(kQT, kKT);
         bool ok = attn_warp_wait(bars + B_QFULL, 0, p.hdr, 2);
-        // S of tile j goes out as soon as the score buffer is free, ahead of
-        // O += P V of tile j - 2, so the softmax of tile j starts as soon as
-        // that of tile j - 1 is done
-        for (int j = 0; ok && j <= n + 1; ++j) {
-            if (j < n) {
-                const int s = j % kStages;
-                if (!(ok = attn_warp_wait(bars + B_KFULL + s, (uint32_t)(j / kStages) & 1u, p.hdr, 3))) break;
-                // the single score buffer: tile j - 1 has been read
-                if (j >= 1 && !(ok = attn_warp_wait(bars + B_SFREE, (uint32_t)(j - 1) & 1u, p.hdr, 4))) break;
-                tc_fence_after();
-                const uint64_t kd0 = umma_desc_sw128(smem_u32(smem + OFF_K + s * kKBytes));
+        for (int j = 0; ok && j < n; ++j) {
+            const int s = j % kStages;
+            if (!(ok = attn_warp_wait(bars + B_KFULL + s, (uint32_t)(j / kStages) & 1u, p.hdr, 3))) break;
+            if (j >= 1 && !(ok = attn_warp_wait(bars + B_SFREE, (uint32_t)(j - 1) & 1u, p.hdr, 4))) break;
+            tc_fence_after();
+            const uint64_t kd0 = umma_desc_sw128(smem_u32(smem + OFF_K + s * kKBytes));
 #pragma unroll
-                for (int kk = 0; kk < kHd / 16; ++kk) {
-                    // A: 16 channels of Q from TMEM (8 columns); B: 64-channel box kk / 4,
-                    // 16-channel step kk % 4 (32 bytes into each swizzled row; the
-                    // descriptor's start field counts 16-byte units)
-                    const uint32_t off = (uint32_t)(kk >> 2) * kKBox + (uint32_t)(kk & 3) * 32;
-                    umma_ts_warp(tmem + kColS, tmem + kColQ + (uint32_t)kk * 8, kd0 + (off >> 4), idesc_s, kk > 0);
-                }
-                umma_commit_warp(bars + B_SFULL);
-                umma_commit_warp(bars + B_KFREE + s);
+            for (int kk = 0; kk < kHd / 16; ++kk) {
+                // A: 16 channels of Q from TMEM (8 columns); B: 64-channel box kk / 4,
+                // 16-channel step kk % 4 (32 bytes into each swizzled row; the
+                // descriptor's start field counts 16-byte units)
+                const uint32_t off = (uint32_t)(kk >> 2) * kKBox + (uint32_t)(kk & 3) * 32;
+                umma_ts_warp(tmem + kColS, tmem + kColQ + (uint32_t)kk * 8, kd0 + (off >> 4), idesc_s, kk > 0);
             }
-            if (j >= 2) {
-                const int i = j - 2, pb = i % 2, s = i % kStages;
-                if (!(ok = attn_warp_wait(bars + B_PFULL + pb, (uint32_t)(i / 2) & 1u, p.hdr, 5))) break;
-                if (!(ok = attn_warp_wait(bars + B_VFULL + s, (uint32_t)(i / kStages) & 1u, p.hdr, 6))) break;
-                tc_fence_after();
-                const uint64_t vd0 = umma_desc_sw128(smem_u32(smem + OFF_V + s * kVBytes));
-#pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_ts_warp(tmem + kColO, tmem + kColP + (uint32_t)(pb * 32 + kk * 8), vd0 + (uint64_t)(kk * 2),
-                                 idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-                umma_commit_warp(bars + B_PVDONE + pb);
-                umma_commit_warp(bars + B_VFREE + s);
-            }
+            umma_commit_warp(bars + B_SFULL);
+            umma_commit_warp(bars + B_KFREE + s);
             __syncwarp();
         }
         if (!ok) {
-            // the MMAs in flight finish before TMEM is freed
+            // this warp's MMAs finish before TMEM is freed
             umma_commit_warp(bars + B_DRAIN);
             if (lane == 0) drain_wait(bars + B_DRAIN, 0);
+        }
+        __syncwarp();
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ P V issuer
+        // O += P_i V_i as soon as P_i is in TMEM and V_i has landed
+        const uint32_t idesc_o = umma_idesc_bf16(kQT, kHd);
+        bool ok = true;
+        for (int i = 0; ok && i < n; ++i) {
+            const int pb = i % 2, s = i % kStages;
+            if (!(ok = attn_warp_wait(bars + B_PFULL + pb, (uint32_t)(i / 2) & 1u, p.hdr, 5))) break;
+            if (!(ok = attn_warp_wait(bars + B_VFULL + s, (uint32_t)(i / kStages) & 1u, p.hdr, 6))) break;
+            tc_fence_after();
+            const uint64_t vd0 = umma_desc_sw128(smem_u32(smem + OFF_V + s * kVBytes));
+#pragma unroll
+            for (int kk = 0; kk < kKT / 16; ++kk)
+                umma_ts_warp(tmem + kColO, tmem + kColP + (uint32_t)(pb * 32 + kk * 8), vd0 + (uint64_t)(kk * 2),
+                             idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+            umma_commit_warp(bars + B_PVDONE + pb);
+            umma_commit_warp(bars + B_VFREE + s);
+            __syncwarp();
+        }
+        if (!ok) {
+            umma_commit_warp(bars + B_DRAIN + 1);
+            if (lane == 0) drain_wait(bars + B_DRAIN + 1, 0);
         }
         __syncwarp();
     } else {
@@ -298,19 +315,16 @@ rglru_mqa_attention_kernel(const AttnParams p, const __grid_constant__ CUtensorM
         const int hi = live ? t : -1;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         {
-            // this row of the Q tile into its TMEM lane: 256 bf16 = 128 columns
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.qkv + ((size_t)b * p.T + (live ? t : 0)) * (size_t)((p.H + 2) * kHd) + (size_t)h * kHd);
-#pragma unroll 1
+            // this row of the Q tile (loaded at the start) into its TMEM lane: 128 columns
+#pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t r[32];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint4 v = live ? __ldg(src + q * 8 + k) : make_uint4(0, 0, 0, 0);
-                    r[4 * k] = v.x;
-                    r[4 * k + 1] = v.y;
-                    r[4 * k + 2] = v.z;
-                    r[4 * k + 3] = v.w;
+                    r[4 * k] = qv[q * 8 + k].x;
+                    r[4 * k + 1] = qv[q * 8 + k].y;
+                    r[4 * k + 2] = qv[q * 8 + k].z;
+                    r[4 * k + 3] = qv[q * 8 + k].w;
                 }
                 tmem_st32(tmem + lane_off + kColQ + (uint32_t)(q * 32), r);
             }
