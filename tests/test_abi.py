@@ -192,3 +192,72 @@ def test_host_prefill_rejects_overlaps_before_any_cuda_call(lib):
     par_bad[4] = ctypes.c_void_p(staging + 64)  # W_x
     assert lib.rglru_prefill_host(B, T, D, dt, hx, hg, *par_bad, hsp, cs_ok, hs_ok, hy, rows,
                                   ctypes.c_void_p(staging), st_need, ws, ws_need, None) == api.ERR_INVALID_ARG
+
+
+def test_mqa_sizes(lib):
+    assert lib.rglru_mqa_vt_size(2, 13) == 2 * 256 * 16 * 2          # T rounded up to 8
+    assert lib.rglru_mqa_vt_size(0, 5) == 0 and lib.rglru_mqa_vt_size(1, 0) == 0
+    assert lib.rglru_mqa_decode_workspace_size(256, 10, 2048) > 4096
+    for window in (0, 64, 100, 2176, 4096):                             # a multiple of 128 up to 2048
+        assert lib.rglru_mqa_decode_workspace_size(4, 10, window) == 0, window
+    assert lib.rglru_mqa_decode_workspace_size(4, 17, 2048) == 0       # at most 16 heads
+    assert lib.rglru_mqa_block_workspace_size(2, 100, 255) == 0
+    assert lib.rglru_mqa_block_workspace_size(2, 100, 512) > 4096
+    assert lib.rglru_mqa_residual_block_workspace_size(2, 100, 512, 100) == 0   # F a multiple of 128
+    assert lib.rglru_mqa_residual_block_workspace_size(2, 100, 512, 1536) > 4096
+
+
+def _fake(k, off=0):
+    """Distinct, aligned, non-overlapping fake device addresses (never used:
+    every call below fails validation first)."""
+    return ctypes.c_void_p((1 << 24) * (k + 1) + off)
+
+
+def test_mqa_attention_and_rope_reject_before_launch(lib):
+    ws, wsb = _fake(9), ctypes.c_size_t(4096)
+    att = lib.rglru_mqa_attention
+    assert att(1, 8, 1, 0, _fake(0), _fake(1), _fake(2), _fake(3), ws, wsb, None) == api.ERR_INVALID_ARG  # window 0
+    assert att(1, 8, 1, 16, _fake(0, 4), _fake(1), _fake(2), _fake(3), ws, wsb, None) == api.ERR_INVALID_ARG
+    assert att(1, 8, 1, 16, _fake(0), _fake(1), None, _fake(3), ws, wsb, None) == api.ERR_INVALID_ARG
+    assert att(1, 8, 1, 16, _fake(0), _fake(1), _fake(2), _fake(3), ws, ctypes.c_size_t(64), None) == api.ERR_WORKSPACE
+    assert att(1, 8, 1, 16, _fake(0), _fake(1), _fake(2), _fake(0), ws, wsb, None) == api.ERR_INVALID_ARG  # out = qkv
+    assert att(1, 8, 65, 16, _fake(0), _fake(1), _fake(2), _fake(3), ws, wsb, None) == api.ERR_UNSUPPORTED
+    rope = lib.rglru_mqa_rope
+    assert rope(1, 8, 1, _fake(0), _fake(2), _fake(0), None) == api.ERR_INVALID_ARG   # v_t overlaps qkv
+    assert rope(1, 8, 1, _fake(0, 8), _fake(2), _fake(1), None) == api.ERR_INVALID_ARG
+    assert rope(0, 8, 1, _fake(0), _fake(2), _fake(1), None) == api.ERR_UNSUPPORTED
+
+
+def test_mqa_decode_and_blocks_reject_before_launch(lib):
+    dec = lib.rglru_mqa_decode_step
+    need = lib.rglru_mqa_decode_workspace_size(2, 2, 128)
+    ws = _fake(9)
+    ok_args = dict(qkv=_fake(0), sp=_fake(1), kc=_fake(2), vc=_fake(3), out=_fake(4))
+
+    def call(window=128, wsb=need, **kw):
+        a = {**ok_args, **kw}
+        return dec(2, 2, window, a["qkv"], a["sp"], a["kc"], a["vc"], a["out"], ws, ctypes.c_size_t(wsb), None)
+    assert call(window=100) == api.ERR_UNSUPPORTED
+    assert call(kc=_fake(2, 2)) == api.ERR_INVALID_ARG
+    assert call(sp=None) == api.ERR_INVALID_ARG
+    assert call(wsb=16) == api.ERR_WORKSPACE
+    assert call(vc=_fake(2)) == api.ERR_INVALID_ARG       # the two rings overlap
+    assert call(out=_fake(0)) == api.ERR_INVALID_ARG      # out overlaps qkv
+    blk = lib.rglru_mqa_block_prefill
+    bneed = lib.rglru_mqa_block_workspace_size(1, 8, 256)
+    assert blk(1, 8, 255, 2048, _fake(0), _fake(1), _fake(2), None, _fake(4), _fake(5), ws,
+               ctypes.c_size_t(bneed), None) == api.ERR_INVALID_ARG
+    assert blk(1, 8, 256, 2048, _fake(0), _fake(1), _fake(2), None, _fake(4), _fake(5), ws,
+               ctypes.c_size_t(64), None) == api.ERR_WORKSPACE
+    assert blk(1, 8, 256, 2048, _fake(0), _fake(1), _fake(2), None, _fake(4), _fake(0), ws,
+               ctypes.c_size_t(bneed), None) == api.ERR_INVALID_ARG   # out = u
+    res = lib.rglru_mqa_residual_block_prefill
+    rneed = lib.rglru_mqa_residual_block_workspace_size(1, 8, 256, 768)
+    args = [_fake(k) for k in range(13)]  # u, the norms, the projections and their biases, segment_pos
+    ws2 = _fake(20)
+    assert res(1, 8, 256, 768, 2048, *args, ctypes.c_float(1e-6), _fake(14), ws2, ctypes.c_size_t(16),
+               None) == api.ERR_WORKSPACE
+    assert res(1, 8, 256, 768, 2048, *args, ctypes.c_float(0.0), _fake(14), ws2, ctypes.c_size_t(rneed),
+               None) == api.ERR_UNSUPPORTED    # eps must be positive
+    assert res(1, 8, 256, 768, 2048, *args, ctypes.c_float(1e-6), _fake(0), ws2, ctypes.c_size_t(rneed),
+               None) == api.ERR_INVALID_ARG    # out = u
