@@ -35,8 +35,9 @@
 //   warp 6     P V issuer: O += P V (M=128, N=256, 4 K-steps) with P read from
 //              TMEM, as soon as P of the tile is written (two issuing warps, so
 //              neither kind of MMA waits behind the other's barriers);
-//   warps 0-3  softmax: thread = query row = TMEM lane.  Each first writes its
-//              row of the Q tile into TMEM (the A operand of S).  Scores in
+//   warps 0-3  softmax: thread = query row = TMEM lane.  Each loads its row of
+//              the Q tile at kernel start (all 32 loads in flight under the
+//              setup) and writes it into TMEM (the A operand of S).  Scores in
 //              log2 units, the window / document / causal limits applied only
 //              on tiles that cross them; the running max used for the
 //              exponentials is raised only when a row's max grows by more
@@ -44,6 +45,7 @@
 //              after the MMAs that wrote it have completed.  P goes to TMEM as
 //              bf16 pairs; at the end O / l is written as bf16.
 // TMEM: O 256 columns, Q 128, S 64, P 2 x 32 (all 512, one CTA per SM).
+// The decode step (rglru_mqa_decode_kernel, further down) has its own notes.
 // Every mbarrier wait is bounded (2 s): one that runs out records
 // RGLRU_ERR_TIMEOUT in the workspace header and the CTA unwinds.  A wait whose
 // phase is already complete costs one inline test.
