@@ -683,6 +683,92 @@ def run_residual_block(args, dev, stream, distributed, peaks, peak_kind):
     }
 
 
+def run_time_sharded(args, w, dev, stream, rank, world, local, distributed):
+    """--shard time: each sequence of the workload split along time over the
+    ranks, one contiguous chunk of tokens per rank.  A step: the chunk from h = 0
+    and from h = 1 (its end states H0, H1), one all-gather of those end states,
+    rglru_carry_scan for the state every chunk starts from, the chunk once more
+    from its own carried state.  Three passes over each chunk, so the job runs
+    at most world / 3 times faster than one GPU (head sharding, where there are
+    heads to spread, has no such factor).  Strong scaling: the job's tokens once
+    over the max-over-ranks step time."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from lm_causal_depthwise_b200 import api
+    from lm_causal_depthwise_b200.sharding import shard_time, shard_time_inputs
+    t0, t1 = shard_time(w.T, world, rank)
+    inp = W.generate(w)
+    part = w.scaled(T=t1 - t0)
+    case = PrefillCase(part, dev, inp=shard_time_inputs(inp, t0, t1))
+    h_first = torch.from_numpy(inp["h_state"]).to(dev)
+    cs0 = case.cs.clone()
+    ends = torch.empty((2, w.B, w.D), dtype=torch.float32, device=dev)  # this chunk's H0, H1
+    gathered = torch.empty((world, 2, w.B, w.D), dtype=torch.float32, device=dev)
+    H0 = torch.empty((world, w.B, w.D), dtype=torch.float32, device=dev)
+    H1 = torch.empty_like(H0)
+    h_in = torch.empty_like(H0)
+
+    def step():
+        for k, h in enumerate((0.0, 1.0)):
+            case.hs.fill_(h)
+            case.cs.copy_(cs0)
+            case.step()
+            ends[k].copy_(case.hs)
+        if distributed:
+            dist.all_gather_into_tensor(gathered, ends)
+        else:
+            gathered[0].copy_(ends)
+        H0.copy_(gathered[:, 0])
+        H1.copy_(gathered[:, 1])
+        api.carry_scan(H0, H1, h_first, h_in)
+        case.hs.copy_(h_in[rank])
+        case.cs.copy_(cs0)
+        case.step()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if distributed:
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if distributed:
+        dist.barrier()
+    per_step_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+    st = case.status()
+    if st != api.OK:
+        raise RuntimeError(f"time-sharded prefill: device status {api.status_string(st)}")
+    if distributed:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks, peak_kind = measured_peaks()
+    line = {
+        "metric": METRIC, "value": sharded_throughput(w.tokens, per_step_ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.describe(), "B": w.B, "T": w.T, "D": w.D, "tokens_per_job": w.tokens,
+                   "parallelism": f"time split over {world} GPU(s): three passes per chunk and one all-gather "
+                                  f"of the chunks' end states; rank 0 has tokens [{t0}, {t1})",
+                   "l2": "no flush: on prefill-long a chunk's x, g and y together exceed L2 (126 MB) "
+                         "up to 8 GPUs"},
+        "roofline": roofline(W.algorithmic_bytes(w), per_step_ms * world, peaks, peak_kind, None, None),
+        "roofline_note": "achieved per GPU: the job's algorithmic bytes / world over the step time (each chunk "
+                         "is read three times)",
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_head_sharded(args, w, dev, stream, rank, world, local, distributed):
     """--shard heads: the workload's heads split across the ranks (no
     collective on the data path; each rank's output is a column block of the
@@ -743,6 +829,8 @@ def run_cuda(args, w):
 
     if args.profile_run and w.decode_steps:
         return profile_decode(args, w, dev, rank, distributed)
+    if args.shard == "time":
+        return run_time_sharded(args, w, dev, stream, rank, world, local, distributed)
     if args.shard == "heads":
         return run_head_sharded(args, w, dev, stream, rank, world, local, distributed)
     if args.profile_mqa:
@@ -1057,9 +1145,10 @@ def main():
     ap.add_argument("--profile-block", action="store_true",
                     help="only the recurrent residual block's steps (the command an ncu launch list of "
                          "the block kernels wraps)")
-    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+    ap.add_argument("--shard", default="none", choices=["none", "heads", "time"],
                     help="none: one replica of the workload per GPU (weak scaling); heads: the workload's "
-                         "heads split across the GPUs (strong scaling)")
+                         "heads split across the GPUs (strong scaling); time: each sequence split along "
+                         "time, one all-gather of the chunks' end states per step (strong scaling)")
     ap.add_argument("--headline-only", action="store_true",
                     help="time only the headline prefill workload (not the other prefill workloads)")
     ap.add_argument("--profile-run", action="store_true",

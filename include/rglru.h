@@ -478,6 +478,24 @@ RGLRU_API rglru_status rglru_mqa_residual_block_prefill(
     const float *b_gate, const void *W_up, const float *b_up, const void *W_down, const float *b_down, float eps,
     void *out, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * The carried scan state of a long sequence split into N time chunks (one per
+ * rank), from one exchange.  The recurrence is affine in the state a chunk
+ * starts from: the chunk ends in A h_in + H0 per channel.  Each rank runs
+ * rglru_prefill on its chunk from h_state = 0 and from h_state = 1, giving the
+ * end states H0 and H1 (so A = H1 - H0); the ranks all-gather them; then
+ *   h_in[0] = h0,   h_in[r + 1] = (H1[r] - H0[r]) h_in[r] + H0[r]
+ * and each rank runs its chunk once more from h_in[rank], with conv_state =
+ * the three raw inputs before its first token.
+ *   H0, H1   [N, B, D] fp32, rank-major (the gathered end states);
+ *   h0       [B, D] fp32: the state before the first chunk;
+ *   h_in     [N, B, D] fp32 out: the state each chunk starts from.
+ * Device pointers; h_in must not overlap the inputs.  In fp32 the subtraction
+ * H1 - H0 carries the rounding of the end states (about 1e-7 of their size).
+ */
+RGLRU_API rglru_status rglru_carry_scan(int N, int B, int D, const float *H0, const float *H1, const float *h0,
+                                        float *h_in, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

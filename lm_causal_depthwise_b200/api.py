@@ -30,7 +30,7 @@ SYMBOLS = ("rglru_version", "rglru_status_string", "rglru_workspace_size", "rglr
            "rglru_rmsnorm", "rglru_residual_block_workspace_size", "rglru_residual_block_prefill",
            "rglru_mqa_vt_size", "rglru_mqa_rope", "rglru_mqa_attention", "rglru_mqa_block_workspace_size",
            "rglru_mqa_block_prefill", "rglru_mqa_decode_workspace_size", "rglru_mqa_decode_step",
-           "rglru_mqa_residual_block_workspace_size", "rglru_mqa_residual_block_prefill")
+           "rglru_mqa_residual_block_workspace_size", "rglru_mqa_residual_block_prefill", "rglru_carry_scan")
 
 _lib = None
 
@@ -115,6 +115,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rglru_mqa_residual_block_workspace_size.argtypes = [i, i, i, i]
     lib.rglru_mqa_residual_block_prefill.restype = i
     lib.rglru_mqa_residual_block_prefill.argtypes = [i, i, i, i, i] + [vp] * 13 + [ctypes.c_float, vp, vp, sz, vp]
+    lib.rglru_carry_scan.restype = i
+    lib.rglru_carry_scan.argtypes = [i, i, i] + [vp] * 4 + [vp]
     _lib = lib
     return lib
 
@@ -810,3 +812,23 @@ def mqa_residual_block_prefill(u, rp: MQAResidualParams, segment_pos, window: in
     if st != OK:
         raise RGLRUError(st, "rglru_mqa_residual_block_prefill")
     return out
+
+
+def carry_scan(H0, H1, h0, h_in=None) -> torch.Tensor:
+    """rglru_carry_scan: the state each of N time chunks starts from, given the
+    chunks' end states from 0 (H0) and from 1 (H1), [N, B, D] fp32, and the
+    state h0 [B, D] before the first chunk.  Returns h_in [N, B, D]."""
+    if H0.dim() != 3:
+        raise ValueError("H0 must be [N, B, D]")
+    N, B, D = H0.shape
+    dev = H0.device
+    _check(H0, "H0", (N, B, D), torch.float32, dev)
+    _check(H1, "H1", (N, B, D), torch.float32, dev)
+    _check(h0, "h0", (B, D), torch.float32, dev)
+    if h_in is None:
+        h_in = torch.empty_like(H0)
+    _check(h_in, "h_in", (N, B, D), torch.float32, dev)
+    st = load().rglru_carry_scan(N, B, D, _ptr(H0), _ptr(H1), _ptr(h0), _ptr(h_in), _stream(dev))
+    if st != OK:
+        raise RGLRUError(st, "rglru_carry_scan")
+    return h_in

@@ -1,4 +1,5 @@
-"""Head sharding of the block core across GPUs (one process per GPU).
+"""Head sharding and time sharding of the block core across GPUs (one
+process per GPU).
 
 Heads never mix in the core: the conv is depthwise, the gate projections are
 block-diagonal per head of 256 channels and the scan is per channel.  A rank
@@ -8,7 +9,12 @@ to them -- with no collective on the data path; the outputs of the ranks are
 the full output's column blocks.  (In a tensor-parallel model these blocks are
 what a column-parallel linear_x / linear_y leaves on each rank.)
 
-This module only computes the assignment and slices arrays; it holds none of
+Time sharding splits one long sequence into contiguous chunks of tokens, one
+per rank.  A chunk needs the three raw inputs before its first token (the
+conv taps) and the scan state there, which the ranks obtain from one
+exchange of their chunks' end states (rglru_carry_scan).
+
+This module only computes the assignments and slices arrays; it holds none of
 the method's arithmetic.
 """
 from __future__ import annotations
@@ -45,4 +51,34 @@ def shard_inputs(inp: dict, h0: int, h1: int) -> dict:
         out[k] = np.ascontiguousarray(inp[k][h0:h1])
     out["conv_state"] = np.ascontiguousarray(inp["conv_state"][:, :, c])
     out["h_state"] = np.ascontiguousarray(inp["h_state"][:, c])
+    return out
+
+
+def shard_time(T: int, world: int, rank: int) -> Tuple[int, int]:
+    """Contiguous token range [t0, t1) of ``rank`` in a sequence of T tokens:
+    sizes differ by at most one, the larger ranges first."""
+    if T < 1 or world < 1 or not 0 <= rank < world:
+        raise ValueError("bad shard arguments")
+    base, extra = divmod(T, world)
+    t0 = rank * base + min(rank, extra)
+    return t0, t0 + base + (1 if rank < extra else 0)
+
+
+def conv_halo(x: np.ndarray, conv_state: np.ndarray, t0: int) -> np.ndarray:
+    """The conv state a chunk starting at token t0 begins with: the three raw
+    inputs before t0, oldest first ([B, 3, D]), taken from the carried conv
+    state where t0 < 3."""
+    prev = np.concatenate([np.asarray(conv_state), np.asarray(x)[:, :t0]], axis=1)
+    return np.ascontiguousarray(prev[:, -3:])
+
+
+def shard_time_inputs(inp: dict, t0: int, t1: int) -> dict:
+    """The core's inputs for tokens [t0, t1): the time slices of x, the gate
+    branch and segment_pos, and the conv state at t0.  h_state is left as
+    given (each pass sets its own)."""
+    out = dict(inp)
+    for k in ("x", "g"):
+        out[k] = np.ascontiguousarray(inp[k][:, t0:t1])
+    out["segpos"] = np.ascontiguousarray(inp["segpos"][:, t0:t1])
+    out["conv_state"] = conv_halo(inp["x"], inp["conv_state"], t0)
     return out

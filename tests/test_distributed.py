@@ -135,3 +135,70 @@ def test_head_sharded_job_gloo(tmp_path):
     whole = W.generate(W.Workload("s", B=2, T=40, D=768, io="bf16", seed=3, init_state="random"))["x"]
     parts = [np.load(tmp_path / f"x{r}.npy") for r in range(world)]
     np.testing.assert_array_equal(np.concatenate(parts, axis=2), whole)
+
+
+def test_shard_time_covers_every_token_once():
+    sys.path.insert(0, ROOT)
+    from lm_causal_depthwise_b200.sharding import shard_time
+    for T in (1, 5, 131072, 4097):
+        for world in (1, 2, 3, 8):
+            got = [shard_time(T, world, r) for r in range(world)]
+            assert got[0][0] == 0 and got[-1][1] == T
+            assert all(a[1] == b[0] for a, b in zip(got, got[1:]))
+            sizes = [t1 - t0 for t0, t1 in got]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_conv_halo_takes_the_three_inputs_before_the_chunk():
+    """Chunks starting at 0, 1, 2 take (some of) the carried conv state, later
+    ones the last three tokens of x before them, oldest first."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    from lm_causal_depthwise_b200.sharding import conv_halo
+    x = np.arange(2 * 10 * 4, dtype=np.float32).reshape(2, 10, 4)
+    cs = -np.arange(2 * 3 * 4, dtype=np.float32).reshape(2, 3, 4) - 1
+    np.testing.assert_array_equal(conv_halo(x, cs, 0), cs)
+    np.testing.assert_array_equal(conv_halo(x, cs, 1), np.concatenate([cs[:, 1:], x[:, :1]], axis=1))
+    np.testing.assert_array_equal(conv_halo(x, cs, 2), np.concatenate([cs[:, 2:], x[:, :2]], axis=1))
+    np.testing.assert_array_equal(conv_halo(x, cs, 7), x[:, 4:7])
+
+
+def _time_rank_main(rank: int, world: int, port: int, out_dir: str):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from lm_causal_depthwise_b200.sharding import shard_time
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # each rank's chunk end states (stand-ins); the one exchange gathers them in rank order
+        t0, t1 = shard_time(1000, world, rank)
+        H0 = torch.full((2, 8), float(rank), dtype=torch.float32)
+        H1 = H0 + 0.5
+        g0 = [torch.empty_like(H0) for _ in range(world)]
+        g1 = [torch.empty_like(H1) for _ in range(world)]
+        dist.all_gather(g0, H0)
+        dist.all_gather(g1, H1)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"t": [t0, t1], "H0": [float(g[0, 0]) for g in g0], "A": [float(a[0, 0] - b[0, 0])
+                                                                                  for a, b in zip(g1, g0)]}, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_time_sharded_exchange_gloo(tmp_path):
+    """Two ranks split 1000 tokens and gather each other's chunk end states in
+    rank order (the input of rglru_carry_scan on every rank)."""
+    world = 2
+    mp.start_processes(_time_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    got = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert [g["t"] for g in got] == [[0, 500], [500, 1000]]
+    for g in got:
+        assert g["H0"] == [0.0, 1.0]
+        assert g["A"] == [0.5, 0.5]

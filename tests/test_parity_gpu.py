@@ -399,3 +399,40 @@ def test_decode_bounded_wait_reports_timeout_and_context_survives():
     assert api.device_status(ws) == api.OK
     ref = run_oracle(inp)
     check_bf16(np.stack(ys, axis=1), ref["y"], "decode y after timeout")
+
+
+@pytest.mark.parametrize("world,kw", [(2, dict(continue_doc=True)), (4, dict(continue_doc=True)),
+                                      (3, dict(doc_len=700))])
+def test_time_shards_with_one_exchange_match_oracle(world, kw):
+    """One long sequence split in time over `world` ranks, emulated one after
+    another on this GPU: each rank runs its chunk from h = 0 and from h = 1,
+    rglru_carry_scan folds the gathered end states into every chunk's starting
+    state, each rank runs its chunk again from it (conv state = the three raw
+    inputs before the chunk).  The joined outputs and the final states against
+    the oracle of the whole sequence; with documents carried across every chunk
+    boundary (continue_doc) and with resets inside the chunks."""
+    from lm_causal_depthwise_b200.sharding import shard_time, shard_time_inputs
+    B, T, D = 2, 2000, 512
+    _, inp = _case(B, T, D, **kw)
+    bf = torch.bfloat16
+    ends = {0.0: [], 1.0: []}
+    for r in range(world):
+        t0, t1 = shard_time(T, world, r)
+        part = shard_time_inputs(inp, t0, t1)
+        for h in (0.0, 1.0):
+            dev = to_device({**part, "h_state": np.full((B, D), h, np.float32)}, "bf16")
+            run_gpu(dev)
+            ends[h].append(dev["h_state"])
+    H0, H1 = torch.stack(ends[0.0]).contiguous(), torch.stack(ends[1.0]).contiguous()
+    h_in = api.carry_scan(H0, H1, torch.from_numpy(inp["h_state"]).cuda())
+    ys = []
+    for r in range(world):
+        t0, t1 = shard_time(T, world, r)
+        dev = to_device(shard_time_inputs(inp, t0, t1), "bf16")
+        dev["h_state"].copy_(h_in[r])
+        got = run_gpu(dev)
+        ys.append(got["y"])
+    ref = run_oracle(inp)
+    check_bf16(np.concatenate(ys, axis=1), ref["y"], f"time shards x{world} y")
+    check_bf16(got["h_state"], ref["h_state"], f"time shards x{world} h_state")
+    np.testing.assert_array_equal(got["conv_state"], ref["conv_state"])
