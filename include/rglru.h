@@ -100,6 +100,10 @@ RGLRU_API size_t rglru_workspace_size(int B, int T, int D, rglru_io_dtype dt);
  * the plain SIMT kernels of rglru_prefill_simt.
  * Outputs: y [B,T,D]; conv_state and h_state updated to their values after
  * token T-1.
+ * Range (bf16 mode): the fused kernel keeps each token's GELU(g)*h_local
+ * and GELU(g)*prod(a) between its two scan passes as f16, so it requires
+ * |GELU(g)*h| and |GELU(g)| below 65504; beyond that y may be inf where the
+ * recurrence is finite.  fp32 mode and rglru_prefill_simt have no such limit.
  */
 RGLRU_API rglru_status rglru_prefill(int B, int T, int D, rglru_io_dtype dt,
                            const void *x, const void *gate_branch,
