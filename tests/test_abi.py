@@ -261,3 +261,11 @@ def test_mqa_decode_and_blocks_reject_before_launch(lib):
                None) == api.ERR_UNSUPPORTED    # eps must be positive
     assert res(1, 8, 256, 768, 2048, *args, ctypes.c_float(1e-6), _fake(0), ws2, ctypes.c_size_t(rneed),
                None) == api.ERR_INVALID_ARG    # out = u
+    for k in (7, 9, 11):  # W_gate, W_up, W_down: checked before the first launch
+        bad = list(args)
+        bad[k] = None
+        assert res(1, 8, 256, 768, 2048, *bad, ctypes.c_float(1e-6), _fake(14), ws2, ctypes.c_size_t(rneed),
+                   None) == api.ERR_INVALID_ARG
+        bad[k] = _fake(k, 2)
+        assert res(1, 8, 256, 768, 2048, *bad, ctypes.c_float(1e-6), _fake(14), ws2, ctypes.c_size_t(rneed),
+                   None) == api.ERR_INVALID_ARG
