@@ -352,6 +352,9 @@ RGLRU_API size_t rglru_residual_block_workspace_size(int B, int T, int D, int F)
  * u, out [B, T, D]; W_gate, W_up [F, D], W_down [D, F] bf16 (F = 3 D in the
  * 2B model, MLP expansion factor 3); biases fp32; the recurrent block's
  * parameters, segment_pos and states as rglru_recurrent_block_prefill.
+ * b_gate and b_up are required; b_lin_x, b_lin_y, b_out and b_down may be
+ * NULL.  Every operand is checked before the first launch: on
+ * RGLRU_ERR_INVALID_ARG nothing ran and the states and out are untouched.
  * Every intermediate is a bf16 tensor in the workspace (zero-filled once),
  * which carries one status word for all the launches.
  */
@@ -472,9 +475,10 @@ RGLRU_API size_t rglru_mqa_residual_block_workspace_size(int B, int T, int D, in
  *   n'  = RMSNorm(h) (w_channel_norm)
  *   out = h + down_proj(GELU_tanh(gate_proj(n')) * up_proj(n'))
  * W_qkv, W_o, b_o as rglru_mqa_block_prefill; the MLP as
- * rglru_residual_block_prefill (W_gate, W_up [F, D], W_down [D, F]); every
- * intermediate is a bf16 tensor in the workspace (zero-filled once), which
- * carries one status word for all the launches.
+ * rglru_residual_block_prefill (W_gate, W_up [F, D], W_down [D, F]; b_gate
+ * and b_up required, b_down may be NULL); every operand is checked before the
+ * first launch.  Every intermediate is a bf16 tensor in the workspace
+ * (zero-filled once), which carries one status word for all the launches.
  */
 RGLRU_API rglru_status rglru_mqa_residual_block_prefill(
     int B, int T, int D, int F, int window, const void *u, const float *w_temporal_norm, const void *W_qkv,

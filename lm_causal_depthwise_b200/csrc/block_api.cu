@@ -224,6 +224,13 @@ RGLRU_API rglru_status rglru_residual_block_prefill(
     if (workspace == nullptr || !al16(workspace) || workspace_bytes < need) return RGLRU_ERR_WORKSPACE;
     const size_t act = (size_t)B * T * D * 2;
     if (!al16(u) || !al16(out) || !al16(w_temporal_norm) || !al16(w_channel_norm)) return RGLRU_ERR_INVALID_ARG;
+    // the operands of the steps after the core, checked before the core updates the states: a bad
+    // argument leaves conv_state, h_state and out untouched
+    if (!al16(W_lin_x) || !al16(W_lin_y) || !al16(W_out) || !al16(W_gate) || !al16(b_gate) || !al16(W_up) ||
+        !al16(b_up) || !al16(W_down))
+        return RGLRU_ERR_INVALID_ARG;
+    for (const float *bias : {b_lin_x, b_lin_y, b_out, b_down})
+        if (bias != nullptr && !al16(bias)) return RGLRU_ERR_INVALID_ARG;
     const Span ins[] = {span(u, act), span(workspace, workspace_bytes), span(conv_state, (size_t)B * 3 * D * 2),
                         span(h_state, (size_t)B * D * 4), span(W_lin_x, (size_t)D * D * 2),
                         span(W_lin_y, (size_t)D * D * 2), span(W_out, (size_t)D * D * 2),

@@ -1111,8 +1111,10 @@ RGLRU_API rglru_status rglru_mqa_residual_block_prefill(
     if (workspace == nullptr || !al16(workspace) || workspace_bytes < need) return RGLRU_ERR_WORKSPACE;
     // every operand checked before the first launch, so that a bad argument leaves out untouched
     if (!al16(u) || !al16(out) || !al16(W_qkv) || !al16(W_o) || !al16(w_temporal_norm) || !al16(w_channel_norm) ||
-        !al16(W_gate) || !al16(W_up) || !al16(W_down) || segment_pos == nullptr)
+        !al16(W_gate) || !al16(b_gate) || !al16(W_up) || !al16(b_up) || !al16(W_down) || segment_pos == nullptr)
         return RGLRU_ERR_INVALID_ARG;
+    for (const float *bias : {b_o, b_down})
+        if (bias != nullptr && !al16(bias)) return RGLRU_ERR_INVALID_ARG;
     const size_t M = (size_t)B * T, act = M * D * 2;
     const struct {
         const void *p;

@@ -261,7 +261,7 @@ def test_mqa_decode_and_blocks_reject_before_launch(lib):
                None) == api.ERR_UNSUPPORTED    # eps must be positive
     assert res(1, 8, 256, 768, 2048, *args, ctypes.c_float(1e-6), _fake(0), ws2, ctypes.c_size_t(rneed),
                None) == api.ERR_INVALID_ARG    # out = u
-    for k in (7, 9, 11):  # W_gate, W_up, W_down: checked before the first launch
+    for k in (7, 8, 9, 10, 11):  # W_gate, b_gate, W_up, b_up, W_down: checked before the first launch
         bad = list(args)
         bad[k] = None
         assert res(1, 8, 256, 768, 2048, *bad, ctypes.c_float(1e-6), _fake(14), ws2, ctypes.c_size_t(rneed),
@@ -269,3 +269,28 @@ def test_mqa_decode_and_blocks_reject_before_launch(lib):
         bad[k] = _fake(k, 2)
         assert res(1, 8, 256, 768, 2048, *bad, ctypes.c_float(1e-6), _fake(14), ws2, ctypes.c_size_t(rneed),
                    None) == api.ERR_INVALID_ARG
+
+
+def test_residual_block_checks_every_operand_before_the_core(lib):
+    """rglru_residual_block_prefill updates the states in its core step: an
+    operand of a later step that is missing or misaligned must be rejected
+    before anything is enqueued (the states and out stay untouched)."""
+    res = lib.rglru_residual_block_prefill
+    need = lib.rglru_residual_block_workspace_size(1, 8, 256, 768)
+    assert need > 0
+    # u, w_temporal_norm, W_lin_x, b_lin_x, W_lin_y, b_lin_y, conv_w, conv_b, W_a, b_a, W_x, b_x, lambda,
+    # W_out, b_out, segment_pos, conv_state, h_state, w_channel_norm, W_gate, b_gate, W_up, b_up, W_down, b_down
+    args = [_fake(k) for k in range(25)]
+    names = {13: "W_out", 19: "W_gate", 20: "b_gate", 21: "W_up", 22: "b_up", 23: "W_down"}
+
+    def call(a):
+        return res(1, 8, 256, 768, *a, ctypes.c_float(1e-6), _fake(26), _fake(27), ctypes.c_size_t(need), None)
+    for k, name in names.items():
+        for bad in (None, _fake(k, 2)):
+            a = list(args)
+            a[k] = bad
+            assert call(a) == api.ERR_INVALID_ARG, name
+    for k in (3, 5, 14, 24):  # optional biases: NULL passes this check, misaligned does not
+        a = list(args)
+        a[k] = _fake(k, 4)
+        assert call(a) == api.ERR_INVALID_ARG
