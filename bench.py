@@ -829,6 +829,8 @@ def run_cuda(args, w):
 
     if args.profile_run and w.decode_steps:
         return profile_decode(args, w, dev, rank, distributed)
+    if args.shard != "none" and w.decode_steps:
+        raise SystemExit(f"--shard {args.shard} times prefill workloads; {w.name} is a decode workload")
     if args.shard == "time":
         return run_time_sharded(args, w, dev, stream, rank, world, local, distributed)
     if args.shard == "heads":

@@ -374,6 +374,32 @@ def test_head_shards_equal_the_whole_run(world):
         np.testing.assert_array_equal(got["conv_state"], whole["conv_state"][:, :, c])
 
 
+@pytest.mark.parametrize("world", [2, 3])
+def test_decode_head_shards_equal_the_whole_run(world):
+    """Decode steps on each rank's head range (run one after another here)
+    give the whole decode's output columns and states bit for bit; B = 100
+    leaves the second 64-row block of every head partial."""
+    from lm_causal_depthwise_b200.sharding import shard_heads, shard_inputs
+    B, T, D = 100, 12, 768
+    _, inp = _case(B, T, D, reset_at=(0, 5))
+
+    def decode(part):
+        dev = to_device(part, "bf16")
+        ys = [api.decode_step(dev["x"][:, t].contiguous(), dev["g"][:, t].contiguous(), dev["params"],
+                              dev["segpos"][:, t].contiguous(), dev["conv_state"], dev["h_state"])
+              for t in range(T)]
+        return (torch.stack(ys, 1).float().cpu().numpy(), dev["h_state"].cpu().numpy(),
+                dev["conv_state"].float().cpu().numpy())
+    y, h, cs = decode(inp)
+    for r in range(world):
+        h0, h1 = shard_heads(D // 256, world, r)
+        c = slice(h0 * 256, h1 * 256)
+        ys, hs, css = decode(shard_inputs(inp, h0, h1))
+        np.testing.assert_array_equal(ys, y[:, :, c])
+        np.testing.assert_array_equal(hs, h[:, c])
+        np.testing.assert_array_equal(css, cs[:, :, c])
+
+
 def test_decode_bounded_wait_reports_timeout_and_context_survives():
     """The test hook makes CTA 0 of the decode grid keep its half of the gate
     GEMM's operand from its peer: the peer's bounded wait runs out, the call
