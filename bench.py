@@ -697,6 +697,8 @@ def run_time_sharded(args, w, dev, stream, rank, world, local, distributed):
     import torch.distributed as dist
     from lm_causal_depthwise_b200 import api
     from lm_causal_depthwise_b200.sharding import shard_time, shard_time_inputs
+    if world > w.T:
+        raise SystemExit(f"--shard time needs at least one token per GPU: T = {w.T}, {world} GPUs")
     t0, t1 = shard_time(w.T, world, rank)
     inp = W.generate(w)
     part = w.scaled(T=t1 - t0)

@@ -56,7 +56,8 @@ def shard_inputs(inp: dict, h0: int, h1: int) -> dict:
 
 def shard_time(T: int, world: int, rank: int) -> Tuple[int, int]:
     """Contiguous token range [t0, t1) of ``rank`` in a sequence of T tokens:
-    sizes differ by at most one, the larger ranges first."""
+    sizes differ by at most one, the larger ranges first (empty for the last
+    ranks when world > T)."""
     if T < 1 or world < 1 or not 0 <= rank < world:
         raise ValueError("bad shard arguments")
     base, extra = divmod(T, world)
@@ -68,7 +69,7 @@ def conv_halo(x: np.ndarray, conv_state: np.ndarray, t0: int) -> np.ndarray:
     """The conv state a chunk starting at token t0 begins with: the three raw
     inputs before t0, oldest first ([B, 3, D]), taken from the carried conv
     state where t0 < 3."""
-    prev = np.concatenate([np.asarray(conv_state), np.asarray(x)[:, :t0]], axis=1)
+    prev = np.concatenate([np.asarray(conv_state), np.asarray(x)[:, max(0, t0 - 3):t0]], axis=1)
     return np.ascontiguousarray(prev[:, -3:])
 
 
