@@ -69,7 +69,7 @@ extern "C" {
 typedef enum {
     RGLRU_OK = 0,
     RGLRU_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, overlap */
-    RGLRU_ERR_UNSUPPORTED = 2,  /* shape or dtype this build does not handle */
+    RGLRU_ERR_UNSUPPORTED = 2,  /* shape or dtype the library does not handle */
     RGLRU_ERR_WORKSPACE = 3,    /* workspace missing or too small */
     RGLRU_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
     RGLRU_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
