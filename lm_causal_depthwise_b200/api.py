@@ -174,6 +174,12 @@ def _check(t: torch.Tensor, name: str, shape, dtype, device):
 
 
 def _stream(device) -> ctypes.c_void_p:
+    """The current stream of ``device``; every call that enqueues work takes
+    its device from its tensors, so host tensors stop here, before the
+    library sees a host pointer as device memory."""
+    device = torch.device(device)
+    if device.type != "cuda":
+        raise ValueError(f"the tensors must be CUDA tensors, got device {device}")
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 

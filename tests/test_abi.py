@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from lm_causal_depthwise_b200 import api, build
 
@@ -294,3 +295,17 @@ def test_residual_block_checks_every_operand_before_the_core(lib):
         a = list(args)
         a[k] = _fake(k, 4)
         assert call(a) == api.ERR_INVALID_ARG
+
+
+def test_bindings_reject_host_tensors_before_the_library_runs():
+    """Every call that enqueues work takes its stream from its tensors'
+    device: host tensors raise in the binding, so no host pointer reaches a
+    kernel as device memory."""
+    H = torch.zeros(2, 1, 256)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        api.carry_scan(H, H.clone(), torch.zeros(1, 256))
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        api.rmsnorm(x, torch.ones(256))
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        api.linear(x, torch.zeros(256, 256, dtype=torch.bfloat16), workspace=torch.zeros(1 << 16, dtype=torch.uint8))
